@@ -1,0 +1,481 @@
+#!/usr/bin/env python3
+"""Benchmark of the head-split attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Default workload ``mha_decode_32k``: a Llama-2-7B-shaped MHA attention layer
+(32 heads, head_dim 128, bf16, batch 1), 8 of 32 heads retrieval (chosen by
+seed), sink 16 / recent 64, context 32,768 tokens, one token appended and
+attended per decode step.  A step is one pass of the path: duo_append_kv then
+duo_decode_attn (both caches, both head types, output concatenated in model
+head order).  Inputs are resident in HBM before timing starts; L2 is flushed
+(a 256 MiB write) before every timed step, outside the timed interval.
+
+Other workloads: gqa_decode_128k, gqa_decode_1m (Llama-3-8B-shaped GQA, 4 of
+8 KV heads retrieval), batch64_paged_decode (64 sequences, lengths U[4096,
+32768], 64-token pages), gqa_prefill_128k (one 131,072-token prompt in 32
+chunks of 4,096; a step is one chunk's duo_prefill_chunk + duo_append_kv).
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs an independent
+replica of the workload on its own GPU (the path has no exchange step); the
+time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from head_split_kv_b200 import synthetic as S  # noqa: E402
+
+METRIC = "decode attn µs/step/layer & HBM GB/s; chunked-prefill TFLOP/s; % of roofline"
+
+WORKLOADS = {
+    "mha_decode_32k": dict(kind="decode", hq=32, hkv=32, d=128, n_ret=8, lengths=[32768], steps=256, sigma=False),
+    "gqa_decode_128k": dict(kind="decode", hq=32, hkv=8, d=128, n_ret=4, lengths=[131072], steps=64, sigma=True),
+    "gqa_decode_1m": dict(kind="decode", hq=32, hkv=8, d=128, n_ret=4, lengths=[1048576], steps=64, sigma=True),
+    "batch64_paged_decode": dict(kind="decode", hq=32, hkv=32, d=128, n_ret=8, batch=64, lo=4096, hi=32768,
+                                 steps=32, sigma=False, paged=True),
+    "gqa_prefill_128k": dict(kind="prefill", hq=32, hkv=8, d=128, n_ret=4, n=131072, chunk=4096, sigma=False),
+}
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1590.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas)
+# ---------------------------------------------------------------------------
+
+def _dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def _barrier(world):
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        dist.barrier(device_ids=[torch.cuda.current_device()])
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# decode workloads
+# ---------------------------------------------------------------------------
+
+def _decode_setup(duo, wl, total_steps, seed=0):
+    import torch
+    sh = S.LayerShape(wl["hq"], wl["hkv"], wl["d"], "bf16")
+    retrieval = S.retrieval_heads_by_seed(wl["hkv"], wl["n_ret"], seed=1)
+    if "batch" in wl:
+        lengths = S.context_lengths(wl["batch"], wl["lo"], wl["hi"], seed=seed)
+    else:
+        lengths = np.asarray(wl["lengths"], dtype=np.int64)
+    B = len(lengths)
+    sigma = S.head_sigma(wl["hkv"], seed=seed) if wl.get("sigma") else None
+    alpha = S.binary_alpha(wl["hkv"], retrieval)
+    gate, perm, inv, R = duo.partition_heads(alpha, 0.5)
+    paged = wl.get("paged", False)
+    if paged:
+        table, n_pages = S.page_assignment(lengths, total_steps, 64, seed=seed)
+        desc = duo.desc_init(B, sh.n_q_heads, sh.n_kv_heads, sh.head_dim, duo.BF16, perm, R, page_size=64)
+        caches = duo.LayerCaches(desc, 0, table, n_pages)
+    else:
+        table = None
+        desc = duo.desc_init(B, sh.n_q_heads, sh.n_kv_heads, sh.head_dim, duo.BF16, perm, R)
+        caches = duo.LayerCaches(desc, int(lengths.max()) + total_steps)
+    st = S.decode_state(sh, retrieval, lengths, seed=seed, sigma=sigma)
+    _load_decode_state(caches, st, inv, R, sh, table)
+    ws = duo.Workspace(desc, duo.OP_DECODE, caches.capacity)
+    qs, ks, vs = S.decode_steps(sh, B, total_steps, seed=seed, sigma=sigma)
+    torch.cuda.synchronize()
+    return dict(sh=sh, desc=desc, caches=caches, ws=ws, qs=qs, ks=ks, vs=vs, lengths=lengths, B=B, R=R,
+                retrieval=retrieval, gate=gate, state=st, sigma=sigma)
+
+
+def _to_dev(a):
+    import torch
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(a).cuda()
+
+
+def _load_decode_state(caches, st, inv, R, sh, table):
+    """Write a seeded cache state into the documented device layout."""
+    import torch
+    ring_pos = np.full((caches.ring_pos.shape[0], sh.sink + sh.recent), -1, dtype=np.int32)
+    for (b, h), (k, v) in st["full"].items():
+        r = inv[h]
+        L = k.shape[0]
+        if table is None:
+            caches.k_full[b, r, :L] = _to_dev(k)
+            caches.v_full[b, r, :L] = _to_dev(v)
+        else:
+            pos = np.arange(L)
+            pages = torch.from_numpy(table[b, pos // 64].astype(np.int64)).cuda()
+            rows = torch.from_numpy(pos % 64).cuda()
+            caches.k_full[pages, r, rows] = _to_dev(k)
+            caches.v_full[pages, r, rows] = _to_dev(v)
+    for (b, h), (pos, k, v) in st["stream"].items():
+        s = inv[h] - R
+        slots = np.array([p if p < sh.sink else sh.sink + (p - sh.sink) % sh.recent for p in pos], dtype=np.int64)
+        if len(slots):
+            idx = torch.from_numpy(slots).cuda()
+            caches.k_ring[b, s, idx] = _to_dev(k)
+            caches.v_ring[b, s, idx] = _to_dev(v)
+            ring_pos[b, slots] = pos
+    caches.ring_pos.copy_(torch.from_numpy(ring_pos))
+    caches.seq_len.copy_(torch.from_numpy(st["lengths"].astype(np.int32)))
+
+
+def _decode_bytes(sh, R, lengths_after):
+    """Algorithmic HBM bytes of one decode launch: every cached K/V row of
+    every retrieval head once, the ring rows of the streaming heads, q and out."""
+    S_ = sh.n_kv_heads - R
+    row = sh.head_dim * 2
+    total = 0
+    for L in lengths_after:
+        total += R * L * row * 2
+        total += S_ * min(L, sh.sink + sh.recent) * row * 2
+    total += len(lengths_after) * sh.n_q_heads * sh.head_dim * 2 * 2
+    return total
+
+
+def run_decode(args, wl, world, rank):
+    import torch
+    from head_split_kv_b200 import duo
+    steps, warm = args.steps, args.warmup
+    total = warm + steps
+    # capacity for the warm-up, the timed steps and the end-to-end steps
+    env = _decode_setup(duo, wl, max(total + 32, wl["steps"]) + 1)
+    sh, desc, caches, ws, B, R = env["sh"], env["desc"], env["caches"], env["ws"], env["B"], env["R"]
+    qd = [_to_dev(env["qs"][i]) for i in range(total)]
+    kd = [_to_dev(env["ks"][i][:, None]) for i in range(total)]
+    vd = [_to_dev(env["vs"][i][:, None]) for i in range(total)]
+    out = torch.empty_like(qd[0])
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    sp = int(stream.cuda_stream)
+
+    def step(i):
+        duo.append_kv(desc, caches.state, kd[i], vd[i], 1, sp)
+        duo.decode_attn(desc, caches.state, qd[i], out, ws.ptr, ws.nbytes, sp)
+
+    for i in range(warm):
+        flush.zero_()
+        step(i)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    lengths_seen = []
+    base = env["lengths"] + warm
+    _barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(int(os.environ.get("LOCAL_RANK", "0"))) as clk:
+        for j in range(steps):
+            flush.zero_()
+            e0, e1, e2 = ev[j]
+            e0.record(stream)
+            duo.append_kv(desc, caches.state, kd[warm + j], vd[warm + j], 1, sp)
+            e1.record(stream)
+            duo.decode_attn(desc, caches.state, qd[warm + j], out, ws.ptr, ws.nbytes, sp)
+            e2.record(stream)
+            lengths_seen.append(base + j + 1)
+        torch.cuda.synchronize()
+    _barrier(world)
+    step_ms = [e0.elapsed_time(e2) for e0, _, e2 in ev]
+    dec_ms = [e1.elapsed_time(e2) for _, e1, e2 in ev]
+    app_ms = [e0.elapsed_time(e1) for e0, e1, _ in ev]
+    total_ms = _max_over_ranks(sum(step_ms), world)
+    st_code = duo.check_status(caches.state)
+    if st_code:
+        raise RuntimeError(f"device status 0x{st_code:x} after the timed steps")
+
+    # end to end through the public API with host buffers
+    e2e = _decode_e2e(duo, env, args, world)
+
+    hbm, _, peak_kind = _peaks()
+    bytes_per_launch = statistics.mean(_decode_bytes(sh, R, L) for L in lengths_seen)
+    dec_avg_s = statistics.mean(dec_ms) * 1e-3
+    achieved = bytes_per_launch / dec_avg_s / 1e9
+    us_step = total_ms * 1e3 / (steps * world)
+    res = {
+        "metric": METRIC, "value": round(us_step, 3), "unit": "us/step/layer", "n_gpus": world, "steps": steps,
+        "warmup": warm, "ms_per_step": round(total_ms / steps, 6), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "batch": B, "n_q_heads": sh.n_q_heads, "n_kv_heads": sh.n_kv_heads,
+                   "head_dim": sh.head_dim, "n_retrieval": R, "sink": sh.sink, "recent": sh.recent,
+                   "context": [int(env["lengths"].min()), int(env["lengths"].max())],
+                   "paged": bool(wl.get("paged", False)), "parallelism": f"replicas{world}",
+                   "l2": "flushed (256 MiB write) before every timed step, outside the timed interval"},
+        "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": round(achieved, 1), "peak": hbm,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                     "traffic": None, "algorithmic_bytes_per_launch": int(bytes_per_launch),
+                     "decode_us": round(statistics.mean(dec_ms) * 1e3, 3),
+                     "append_us": round(statistics.mean(app_ms) * 1e3, 3)},
+        "e2e": e2e,
+        "gpu_launches": 2 * steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = _decode_cpu_baseline(env, budget_s=args.cpu_budget)
+    return res
+
+
+def _decode_e2e(duo, env, args, world):
+    """Same steps through the binding with pinned host buffers: per step the
+    new token's q/k/v go host->device and the output comes back."""
+    import torch
+    sh, desc, caches, ws, B = env["sh"], env["desc"], env["caches"], env["ws"], env["B"]
+    n = min(args.steps, 32)
+    h_q = [torch.from_numpy(env["qs"][i].view(np.int16)).view(torch.bfloat16).pin_memory() for i in range(n)]
+    h_k = [torch.from_numpy(env["ks"][i][:, None].copy().view(np.int16)).view(torch.bfloat16).pin_memory()
+           for i in range(n)]
+    h_v = [torch.from_numpy(env["vs"][i][:, None].copy().view(np.int16)).view(torch.bfloat16).pin_memory()
+           for i in range(n)]
+    h_out = torch.empty_like(h_q[0]).pin_memory()
+    dq, dk, dv = torch.empty_like(h_q[0], device="cuda"), torch.empty_like(h_k[0], device="cuda"), \
+        torch.empty_like(h_v[0], device="cuda")
+    dout = torch.empty_like(dq)
+    stream = torch.cuda.current_stream()
+    sp = int(stream.cuda_stream)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    times = []
+    _barrier(world)
+    for i in range(n):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        dq.copy_(h_q[i], non_blocking=True)
+        dk.copy_(h_k[i], non_blocking=True)
+        dv.copy_(h_v[i], non_blocking=True)
+        duo.append_kv(desc, caches.state, dk, dv, 1, sp)
+        duo.decode_attn(desc, caches.state, dq, dout, ws.ptr, ws.nbytes, sp)
+        h_out.copy_(dout, non_blocking=True)
+        e1.record(stream)
+        times.append((e0, e1))
+    torch.cuda.synchronize()
+    _barrier(world)
+    tot = _max_over_ranks(sum(a.elapsed_time(b) for a, b in times), world)
+    h2d = (h_q[0].numel() + h_k[0].numel() + h_v[0].numel()) * 2
+    return {"value": round(tot * 1e3 / (n * world), 3), "unit": "us/step/layer", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": h_out.numel() * 2, "steps": n}
+
+
+def _decode_cpu_baseline(env, budget_s=15.0):
+    """The oracle, as it stands, on this host's cores: decode steps from the
+    same seeded state until the time budget is used."""
+    import oracle as O
+    sh, B = env["sh"], env["B"]
+    cache = O.HeadSplitCache(B, sh.n_kv_heads, sh.head_dim, gate=env["gate"], sink=sh.sink, recent=sh.recent)
+    st = env["state"]
+    for (b, h), (k, v) in st["full"].items():
+        cache.load_state(b, h, np.arange(k.shape[0]), k, v)
+    for (b, h), (pos, k, v) in st["stream"].items():
+        cache.load_state(b, h, pos, k, v)
+    for b, L in enumerate(st["lengths"]):
+        cache.set_length(b, int(L))
+    t0 = time.perf_counter()
+    n = 0
+    while n < len(env["qs"]) and (time.perf_counter() - t0 < budget_s or n < 1):
+        cache.decode(env["qs"][n], env["ks"][n], env["vs"][n])
+        n += 1
+    dt = time.perf_counter() - t0
+    return {"value": round(dt * 1e6 / n, 1), "unit": "us/step/layer", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{n} decode steps of the same workload from the same seeded state (fp64 NumPy oracle)"}
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def run_prefill(args, wl, world, rank):
+    raise NotImplementedError("pre-fill workload not wired yet")
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the oracle, timed on the host cores
+# ---------------------------------------------------------------------------
+
+def run_reference(args, wl):
+    import oracle as O
+    sh = S.LayerShape(wl["hq"], wl["hkv"], wl["d"], "bf16")
+    if wl["kind"] != "decode":
+        return {"impl": "reference", "unavailable": "the reference arm is timed on decode workloads only"}
+    retrieval = S.retrieval_heads_by_seed(wl["hkv"], wl["n_ret"], seed=1)
+    lengths = (S.context_lengths(wl["batch"], wl["lo"], wl["hi"]) if "batch" in wl
+               else np.asarray(wl["lengths"], dtype=np.int64))
+    B = len(lengths)
+    sigma = S.head_sigma(wl["hkv"]) if wl.get("sigma") else None
+    gate, _, _, R = O.partition_heads(S.binary_alpha(wl["hkv"], retrieval).astype(np.float64), 0.5)
+    st = S.decode_state(sh, retrieval, lengths, sigma=sigma)
+    cache = O.HeadSplitCache(B, sh.n_kv_heads, sh.head_dim, gate=gate, sink=sh.sink, recent=sh.recent)
+    for (b, h), (k, v) in st["full"].items():
+        cache.load_state(b, h, np.arange(k.shape[0]), k, v)
+    for (b, h), (pos, k, v) in st["stream"].items():
+        cache.load_state(b, h, pos, k, v)
+    for b, L in enumerate(lengths):
+        cache.set_length(b, int(L))
+    total = args.warmup + args.steps
+    qs, ks, vs = S.decode_steps(sh, B, total, sigma=sigma)
+    for i in range(args.warmup):
+        cache.decode(qs[i], ks[i], vs[i])
+    t0 = time.perf_counter()
+    for i in range(args.warmup, total):
+        cache.decode(qs[i], ks[i], vs[i])
+    dt = time.perf_counter() - t0
+    v = round(dt * 1e6 / args.steps, 1)
+    cores = _blas_threads()
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "us/step/layer", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 3),
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "batch": B, "n_q_heads": sh.n_q_heads,
+                       "n_kv_heads": sh.n_kv_heads, "head_dim": sh.head_dim, "n_retrieval": R,
+                       "context": [int(lengths.min()), int(lengths.max())]},
+            "cpu_baseline": {"value": v, "unit": "us/step/layer", "cores": cores, "kind": "oracle",
+                             "sample": f"{args.steps} timed decode steps after {args.warmup} warm-up steps"},
+            "e2e": {"value": v, "unit": "us/step/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------------------
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mha_decode_32k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, wl)), flush=True)
+        return 0
+
+    import torch
+    world, rank, local = _dist_init()
+    torch.cuda.set_device(local)
+    from head_split_kv_b200 import duo  # noqa: F401  (fails loudly without libduo.so)
+    try:
+        if wl["kind"] == "decode":
+            res = run_decode(args, wl, world, rank)
+        else:
+            res = run_prefill(args, wl, world, rank)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,383 @@
+// duo_abi.cu -- the extern "C" entry points of libduo.so: argument checks,
+// the host-side gate binarisation / head partition, workspace planning, and
+// dispatch to the kernels.  See include/duo.h for the contract of each call.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+duo_status fail(duo_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+duo_status fail(duo_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+duo_status ok() {
+    g_last_error.clear();
+    return DUO_OK;
+}
+
+duo_status cuda_fail(cudaError_t e, const char* where) {
+    return fail(DUO_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+duo_status check_desc(const duo_layer_desc* d) {
+    if (!d) return fail(DUO_ERR_INVALID_ARG, "desc is NULL");
+    if (d->batch < 1) return fail(DUO_ERR_SHAPE, "batch must be >= 1 (got %d)", d->batch);
+    if (d->n_kv_heads < 1 || d->n_kv_heads > DUO_MAX_KV_HEADS)
+        return fail(DUO_ERR_INVALID_ARG, "n_kv_heads must be in 1..%d (got %d)", DUO_MAX_KV_HEADS, d->n_kv_heads);
+    if (d->n_q_heads < 1 || d->n_q_heads % d->n_kv_heads)
+        return fail(DUO_ERR_SHAPE, "n_q_heads (%d) must be a positive multiple of n_kv_heads (%d)", d->n_q_heads,
+                    d->n_kv_heads);
+    const int g = d->n_q_heads / d->n_kv_heads;
+    if (g != 1 && g != 2 && g != 4 && g != 8)
+        return fail(DUO_ERR_UNSUPPORTED, "query group size %d is not built (1, 2, 4 or 8)", g);
+    if (d->head_dim <= 0) return fail(DUO_ERR_SHAPE, "head_dim must be positive (got %d)", d->head_dim);
+    if (d->head_dim != 64 && d->head_dim != 128)
+        return fail(DUO_ERR_UNSUPPORTED, "head_dim %d is not built (64 or 128)", d->head_dim);
+    if (d->dtype != DUO_BF16 && d->dtype != DUO_FP32) return fail(DUO_ERR_DTYPE, "unknown dtype %d", d->dtype);
+    if (d->sink < 0 || d->recent < 1 || d->sink + d->recent > 1024)
+        return fail(DUO_ERR_SHAPE, "need sink >= 0, recent >= 1, sink + recent <= 1024 (got %d, %d)", d->sink,
+                    d->recent);
+    if (d->page_size != 0 && d->page_size != 64)
+        return fail(DUO_ERR_UNSUPPORTED, "page_size must be 0 or 64 (got %d)", d->page_size);
+    if (d->n_retrieval < 0 || d->n_retrieval > d->n_kv_heads)
+        return fail(DUO_ERR_SHAPE, "n_retrieval %d outside 0..%d", d->n_retrieval, d->n_kv_heads);
+    if (d->io_order != DUO_ORDER_MODEL && d->io_order != DUO_ORDER_BLOCK)
+        return fail(DUO_ERR_INVALID_ARG, "unknown io_order %d", d->io_order);
+    if (!std::isfinite(d->scale)) return fail(DUO_ERR_INVALID_ARG, "scale is not finite");
+    bool seen[DUO_MAX_KV_HEADS] = {};
+    for (int i = 0; i < d->n_kv_heads; ++i) {
+        const int h = d->kv_perm[i];
+        if (h < 0 || h >= d->n_kv_heads || seen[h])
+            return fail(DUO_ERR_INVALID_ARG, "kv_perm is not a permutation of 0..%d (slot %d holds %d)",
+                        d->n_kv_heads - 1, i, h);
+        seen[h] = true;
+    }
+    return DUO_OK;
+}
+
+void fill_args(const duo_layer_desc* d, duo::LayerArgs& a) {
+    a.B = d->batch;
+    a.Hq = d->n_q_heads;
+    a.Hkv = d->n_kv_heads;
+    a.G = a.Hq / a.Hkv;
+    a.D = d->head_dim;
+    a.R = d->n_retrieval;
+    a.S = a.Hkv - a.R;
+    a.sink = d->sink;
+    a.recent = d->recent;
+    a.W = d->sink + d->recent;
+    a.dtype = d->dtype;
+    a.page_size = d->page_size;
+    a.capacity = a.max_pages = a.n_pages = 0;
+    a.scale = d->scale > 0.f ? d->scale : 1.0f / std::sqrt(static_cast<float>(d->head_dim));
+    for (int i = 0; i < DUO_MAX_KV_HEADS; ++i) {
+        a.q_head0[i] = 0;
+        a.kv_head[i] = 0;
+        a.slot_of[i] = 0;
+    }
+    for (int i = 0; i < a.Hkv; ++i) {
+        const int h = d->io_order == DUO_ORDER_MODEL ? d->kv_perm[i] : i;
+        a.kv_head[i] = h;
+        a.q_head0[i] = h * a.G;
+        a.slot_of[h] = i;
+    }
+}
+
+duo_status check_state(const duo_layer_desc* d, const duo_kv_state* st, duo::LayerArgs& a, duo::CacheArgs& c) {
+    if (!st) return fail(DUO_ERR_INVALID_ARG, "state is NULL");
+    if (!st->seq_len || !st->counters || !st->status)
+        return fail(DUO_ERR_INVALID_ARG, "state.seq_len, state.counters and state.status are required");
+    const int R = d->n_retrieval, S = d->n_kv_heads - d->n_retrieval;
+    if (R > 0) {
+        if (!st->k_full || !st->v_full) return fail(DUO_ERR_INVALID_ARG, "full cache pointers are NULL");
+        if (!aligned16(st->k_full) || !aligned16(st->v_full))
+            return fail(DUO_ERR_INVALID_ARG, "full cache pointers must be 16-byte aligned");
+        if (st->capacity < 1) return fail(DUO_ERR_SHAPE, "capacity must be >= 1 (got %d)", st->capacity);
+        if (d->page_size) {
+            if (!st->page_table) return fail(DUO_ERR_INVALID_ARG, "paged cache needs page_table");
+            if (st->max_pages < 1 || st->n_pages < 1)
+                return fail(DUO_ERR_SHAPE, "paged cache needs max_pages >= 1 and n_pages >= 1");
+            if ((int64_t)st->max_pages * d->page_size != st->capacity)
+                return fail(DUO_ERR_SHAPE, "capacity (%d) must equal max_pages * page_size (%d * %d)", st->capacity,
+                            st->max_pages, d->page_size);
+        }
+    }
+    if (S > 0) {
+        if (!st->k_ring || !st->v_ring || !st->ring_pos)
+            return fail(DUO_ERR_INVALID_ARG, "ring pointers are NULL");
+        if (!aligned16(st->k_ring) || !aligned16(st->v_ring))
+            return fail(DUO_ERR_INVALID_ARG, "ring pointers must be 16-byte aligned");
+    }
+    a.capacity = R > 0 ? st->capacity : 0;
+    a.max_pages = st->max_pages;
+    a.n_pages = st->n_pages;
+    c.k_full = st->k_full;
+    c.v_full = st->v_full;
+    c.page_table = st->page_table;
+    c.k_ring = st->k_ring;
+    c.v_ring = st->v_ring;
+    c.ring_pos = st->ring_pos;
+    c.seq_len = st->seq_len;
+    c.counters = st->counters;
+    c.status = st->status;
+    return DUO_OK;
+}
+
+}  // namespace
+
+// ===========================================================================
+// Split-K plan (host): enough CTAs to keep every SM streaming, and no split
+// longer than 16K tokens.
+// ===========================================================================
+namespace duo {
+DecodePlan decode_plan(const LayerArgs& a) {
+    DecodePlan p{};
+    const long pairs = (long)a.B * a.R;
+    int ns = 1;
+    if (pairs > 0) {
+        const long target_ctas = 296;  // 148 SMs x 2 resident CTAs
+        ns = (int)((target_ctas + pairs - 1) / pairs);
+        const int by_len = (a.capacity + 16383) / 16384;
+        if (by_len > ns) ns = by_len;
+        if (ns > 256) ns = 256;
+        if (ns < 1) ns = 1;
+    }
+    p.nsplit = ns;
+    p.partial_floats = (size_t)pairs * ns * a.G * (a.D + 2);
+    p.ticket_offset = ((p.partial_floats * sizeof(float)) + 255) / 256 * 256;
+    p.bytes = p.ticket_offset + ((size_t)pairs * sizeof(uint32_t) + 255) / 256 * 256;
+    if (pairs == 0) p.bytes = 256;
+    return p;
+}
+}  // namespace duo
+
+// ===========================================================================
+// extern "C"
+// ===========================================================================
+extern "C" {
+
+const char* duo_last_error(void) { return g_last_error.c_str(); }
+
+const char* duo_status_string(duo_status s) {
+    switch (s) {
+        case DUO_OK: return "DUO_OK";
+        case DUO_ERR_INVALID_ARG: return "DUO_ERR_INVALID_ARG";
+        case DUO_ERR_SHAPE: return "DUO_ERR_SHAPE";
+        case DUO_ERR_DTYPE: return "DUO_ERR_DTYPE";
+        case DUO_ERR_CAPACITY: return "DUO_ERR_CAPACITY";
+        case DUO_ERR_UNSUPPORTED: return "DUO_ERR_UNSUPPORTED";
+        case DUO_ERR_CUDA: return "DUO_ERR_CUDA";
+        case DUO_ERR_DEVICE: return "DUO_ERR_DEVICE";
+    }
+    return "DUO_ERR_UNKNOWN";
+}
+
+int32_t duo_abi_version(void) { return 1; }
+
+duo_status duo_partition_heads(const float* alpha, int32_t n_kv_heads, float tau, int32_t target_n_retrieval,
+                               uint8_t* gate, int32_t* kv_perm, int32_t* kv_inv_perm, int32_t* n_retrieval) {
+    if (!alpha || !gate || !kv_perm || !kv_inv_perm || !n_retrieval)
+        return fail(DUO_ERR_INVALID_ARG, "duo_partition_heads: NULL argument");
+    if (n_kv_heads < 1 || n_kv_heads > DUO_MAX_KV_HEADS)
+        return fail(DUO_ERR_INVALID_ARG, "n_kv_heads must be in 1..%d (got %d)", DUO_MAX_KV_HEADS, n_kv_heads);
+    for (int h = 0; h < n_kv_heads; ++h)
+        if (std::isnan(alpha[h])) return fail(DUO_ERR_INVALID_ARG, "alpha[%d] is NaN", h);
+    if (target_n_retrieval > n_kv_heads)
+        return fail(DUO_ERR_SHAPE, "target_n_retrieval %d exceeds n_kv_heads %d", target_n_retrieval, n_kv_heads);
+    if (target_n_retrieval < 0) {
+        if (std::isnan(tau)) return fail(DUO_ERR_INVALID_ARG, "tau is NaN");
+        for (int h = 0; h < n_kv_heads; ++h) gate[h] = alpha[h] >= tau ? 1 : 0;
+    } else {
+        // exactly k heads: the largest alpha, ties to the lower index
+        for (int h = 0; h < n_kv_heads; ++h) gate[h] = 0;
+        for (int k = 0; k < target_n_retrieval; ++k) {
+            int best = -1;
+            for (int h = 0; h < n_kv_heads; ++h)
+                if (!gate[h] && (best < 0 || alpha[h] > alpha[best])) best = h;
+            gate[best] = 1;
+        }
+    }
+    int n = 0;
+    for (int h = 0; h < n_kv_heads; ++h)
+        if (gate[h]) kv_perm[n++] = h;
+    *n_retrieval = n;
+    for (int h = 0; h < n_kv_heads; ++h)
+        if (!gate[h]) kv_perm[n++] = h;
+    for (int i = 0; i < n_kv_heads; ++i) kv_inv_perm[kv_perm[i]] = i;
+    return ok();
+}
+
+duo_status duo_desc_init(duo_layer_desc* desc, int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
+                         int32_t head_dim, int32_t dtype, const int32_t* kv_perm, int32_t n_retrieval) {
+    if (!desc || !kv_perm) return fail(DUO_ERR_INVALID_ARG, "duo_desc_init: NULL argument");
+    std::memset(desc, 0, sizeof(*desc));
+    desc->batch = batch;
+    desc->n_q_heads = n_q_heads;
+    desc->n_kv_heads = n_kv_heads;
+    desc->head_dim = head_dim;
+    desc->sink = 16;
+    desc->recent = 64;
+    desc->dtype = dtype;
+    desc->page_size = 0;
+    desc->scale = 0.f;
+    desc->n_retrieval = n_retrieval;
+    desc->io_order = DUO_ORDER_MODEL;
+    if (n_kv_heads < 1 || n_kv_heads > DUO_MAX_KV_HEADS)
+        return fail(DUO_ERR_INVALID_ARG, "n_kv_heads must be in 1..%d (got %d)", DUO_MAX_KV_HEADS, n_kv_heads);
+    for (int i = 0; i < n_kv_heads; ++i) desc->kv_perm[i] = kv_perm[i];
+    const duo_status s = check_desc(desc);
+    return s == DUO_OK ? ok() : s;
+}
+
+duo_status duo_desc_validate(const duo_layer_desc* desc) {
+    const duo_status s = check_desc(desc);
+    return s == DUO_OK ? ok() : s;
+}
+
+size_t duo_workspace_bytes(const duo_layer_desc* desc, int32_t op, int32_t max_tokens) {
+    if (check_desc(desc) != DUO_OK) return 0;
+    if (op == DUO_OP_DECODE) {
+        duo::LayerArgs a;
+        fill_args(desc, a);
+        a.capacity = max_tokens > 0 ? max_tokens : 1;
+        return duo::decode_plan(a).bytes;
+    }
+    if (op == DUO_OP_PREFILL) return 256;
+    return 0;
+}
+
+duo_status duo_permute_heads(const duo_layer_desc* desc, const void* x, void* y, int64_t rows,
+                             int32_t heads_per_kv, int64_t head_elems, int32_t elem_bytes, int32_t direction,
+                             duo_stream_t stream) {
+    duo_status s = check_desc(desc);
+    if (s != DUO_OK) return s;
+    if (!x || !y) return fail(DUO_ERR_INVALID_ARG, "duo_permute_heads: NULL tensor");
+    if (rows < 0 || heads_per_kv < 1 || head_elems < 1)
+        return fail(DUO_ERR_SHAPE, "duo_permute_heads: need rows >= 0, heads_per_kv >= 1, head_elems >= 1");
+    if (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4 && elem_bytes != 8)
+        return fail(DUO_ERR_INVALID_ARG, "elem_bytes must be 1, 2, 4 or 8 (got %d)", elem_bytes);
+    if (direction != DUO_MODEL_TO_BLOCK && direction != DUO_BLOCK_TO_MODEL)
+        return fail(DUO_ERR_INVALID_ARG, "unknown direction %d", direction);
+    const int64_t total = rows * (int64_t)desc->n_kv_heads * heads_per_kv * head_elems * elem_bytes;
+    const char* xa = static_cast<const char*>(x);
+    const char* ya = static_cast<const char*>(y);
+    if (xa < ya + total && ya < xa + total) return fail(DUO_ERR_INVALID_ARG, "x and y overlap");
+    if (rows == 0) return ok();
+    const cudaError_t e = duo::launch_permute(x, y, rows, desc->n_kv_heads, desc->kv_perm, heads_per_kv,
+                                              head_elems, elem_bytes, direction, (cudaStream_t)stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "duo_permute_heads");
+}
+
+duo_status duo_append_kv(const duo_layer_desc* desc, const duo_kv_state* st, const void* k_new, const void* v_new,
+                         int32_t T, duo_stream_t stream) {
+    duo_status s = check_desc(desc);
+    if (s != DUO_OK) return s;
+    duo::LayerArgs a;
+    duo::CacheArgs c;
+    fill_args(desc, a);
+    if ((s = check_state(desc, st, a, c)) != DUO_OK) return s;
+    if (T < 0) return fail(DUO_ERR_SHAPE, "T must be >= 0 (got %d)", T);
+    if (T == 0) return ok();
+    if (!k_new || !v_new) return fail(DUO_ERR_INVALID_ARG, "k_new / v_new is NULL");
+    if (!aligned16(k_new) || !aligned16(v_new)) return fail(DUO_ERR_INVALID_ARG, "k_new / v_new not 16-byte aligned");
+    const cudaError_t e = duo::launch_append(a, c, k_new, v_new, T, (cudaStream_t)stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "duo_append_kv");
+}
+
+duo_status duo_decode_attn(const duo_layer_desc* desc, const duo_kv_state* st, const void* q, void* out,
+                           void* workspace, size_t ws_bytes, duo_stream_t stream) {
+    duo_status s = check_desc(desc);
+    if (s != DUO_OK) return s;
+    duo::LayerArgs a;
+    duo::CacheArgs c;
+    fill_args(desc, a);
+    if ((s = check_state(desc, st, a, c)) != DUO_OK) return s;
+    if (!q || !out) return fail(DUO_ERR_INVALID_ARG, "q / out is NULL");
+    if (!aligned16(q) || !aligned16(out)) return fail(DUO_ERR_INVALID_ARG, "q / out not 16-byte aligned");
+    const duo::DecodePlan plan = duo::decode_plan(a);
+    if (!workspace) return fail(DUO_ERR_INVALID_ARG, "workspace is NULL");
+    if (!aligned16(workspace)) return fail(DUO_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+    if (ws_bytes < plan.bytes)
+        return fail(DUO_ERR_CAPACITY, "workspace holds %zu bytes, decode needs %zu", ws_bytes, plan.bytes);
+    const cudaError_t e = duo::launch_decode(a, c, plan, q, out, workspace, (cudaStream_t)stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "duo_decode_attn");
+}
+
+duo_status duo_prefill_chunk(const duo_layer_desc* desc, const duo_kv_state* st, const void* q, const void* k_chunk,
+                             const void* v_chunk, int32_t C, void* out, void* workspace, size_t ws_bytes,
+                             duo_stream_t stream) {
+    (void)workspace;
+    (void)ws_bytes;
+    duo_status s = check_desc(desc);
+    if (s != DUO_OK) return s;
+    duo::LayerArgs a;
+    duo::CacheArgs c;
+    fill_args(desc, a);
+    if ((s = check_state(desc, st, a, c)) != DUO_OK) return s;
+    if (C < 1) return fail(DUO_ERR_SHAPE, "chunk length must be >= 1 (got %d)", C);
+    if (!q || !k_chunk || !v_chunk || !out) return fail(DUO_ERR_INVALID_ARG, "q / k_chunk / v_chunk / out is NULL");
+    if (!aligned16(q) || !aligned16(k_chunk) || !aligned16(v_chunk) || !aligned16(out))
+        return fail(DUO_ERR_INVALID_ARG, "pre-fill tensors must be 16-byte aligned");
+    if (desc->page_size != 0)
+        return fail(DUO_ERR_UNSUPPORTED, "duo_prefill_chunk takes a contiguous full cache (page_size 0)");
+    cudaError_t e;
+    if (a.dtype == DUO_BF16 && a.D == 128) {
+        if (!duo::prefill_tc_supported(a))
+            return fail(DUO_ERR_UNSUPPORTED, "tensor-core pre-fill cannot take this layer");
+        e = duo::launch_prefill_tc(a, c, q, k_chunk, v_chunk, C, out, (cudaStream_t)stream);
+    } else {
+        e = duo::launch_simt_attention(a, &c, nullptr, q, k_chunk, v_chunk, C, out, 0, (cudaStream_t)stream);
+    }
+    return e == cudaSuccess ? ok() : cuda_fail(e, "duo_prefill_chunk");
+}
+
+duo_status duo_gated_mix(const duo_layer_desc* desc, const float* alpha, const void* q, const void* k, const void* v,
+                         int32_t N, void* out, duo_stream_t stream) {
+    duo_status s = check_desc(desc);
+    if (s != DUO_OK) return s;
+    if (!alpha || !q || !k || !v || !out) return fail(DUO_ERR_INVALID_ARG, "duo_gated_mix: NULL argument");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return fail(DUO_ERR_INVALID_ARG, "duo_gated_mix tensors must be 16-byte aligned");
+    if (N < 0) return fail(DUO_ERR_SHAPE, "N must be >= 0 (got %d)", N);
+    if (N == 0) return ok();
+    duo::LayerArgs a;
+    fill_args(desc, a);
+    // the mix runs in model head order over whole sequences
+    for (int i = 0; i < a.Hkv; ++i) {
+        a.kv_head[i] = i;
+        a.q_head0[i] = i * a.G;
+        a.slot_of[i] = i;
+    }
+    const cudaError_t e = duo::launch_simt_attention(a, nullptr, alpha, q, k, v, N, out, 1, (cudaStream_t)stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "duo_gated_mix");
+}
+
+duo_status duo_check_status(const duo_kv_state* st, int32_t* host_status, duo_stream_t stream) {
+    if (!st || !st->status || !host_status) return fail(DUO_ERR_INVALID_ARG, "duo_check_status: NULL argument");
+    int32_t v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, st->status, sizeof v, cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "duo_check_status");
+    *host_status = v;
+    if (v) return fail(DUO_ERR_DEVICE, "device status bits 0x%x", v);
+    return ok();
+}
+
+}  // extern "C"

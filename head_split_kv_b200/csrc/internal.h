@@ -1,0 +1,65 @@
+// internal.h -- launch parameters shared between the C-ABI layer (duo_abi.cu)
+// and the kernels.  Not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "duo.h"
+
+namespace duo {
+
+// Flattened, validated view of a layer descriptor plus state, passed by
+// value to every kernel.
+struct LayerArgs {
+    int B, Hq, Hkv, G, D, R, S, sink, recent, W;
+    int dtype, page_size, capacity, max_pages, n_pages;
+    float scale;       // softmax scale
+    // For block slot i (0..Hkv-1): index of its first query head and of its
+    // KV head in the caller's q / k / v / out tensors (model or block order).
+    int q_head0[DUO_MAX_KV_HEADS];
+    int kv_head[DUO_MAX_KV_HEADS];
+    // Inverse of kv_head: block slot of the caller's KV head h.
+    int slot_of[DUO_MAX_KV_HEADS];
+};
+
+struct CacheArgs {
+    void* k_full;
+    void* v_full;
+    const int32_t* page_table;
+    void* k_ring;
+    void* v_ring;
+    int32_t* ring_pos;
+    int32_t* seq_len;
+    uint32_t* counters;
+    int32_t* status;
+};
+
+// Split-K plan of a decode call: number of splits per (sequence, retrieval
+// head) and the workspace carve-up.
+struct DecodePlan {
+    int nsplit;
+    size_t partial_floats;  // B * R * nsplit * G * (D + 2)
+    size_t ticket_offset;   // bytes from workspace start to the ticket words
+    size_t bytes;           // total workspace bytes
+};
+
+DecodePlan decode_plan(const LayerArgs& a);
+
+cudaError_t launch_append(const LayerArgs& a, const CacheArgs& c, const void* k_new, const void* v_new, int T,
+                          cudaStream_t s);
+cudaError_t launch_decode(const LayerArgs& a, const CacheArgs& c, const DecodePlan& plan, const void* q, void* out,
+                          void* workspace, cudaStream_t s);
+// CUDA-core attention: chunked pre-fill (mode 0) or gated mix (mode 1).
+cudaError_t launch_simt_attention(const LayerArgs& a, const CacheArgs* c, const float* alpha, const void* q,
+                                  const void* k, const void* v, int n_tokens, void* out, int mode, cudaStream_t s);
+// tcgen05 pre-fill for bf16, d = 128; returns cudaErrorNotSupported when it
+// cannot take the call.
+cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void* q, const void* k_chunk,
+                              const void* v_chunk, int C, void* out, cudaStream_t s);
+bool prefill_tc_supported(const LayerArgs& a);
+cudaError_t launch_permute(const void* x, void* y, int64_t rows, int hkv, const int* perm, int heads_per_kv,
+                           int64_t head_elems, int elem_bytes, int direction, cudaStream_t s);
+
+}  // namespace duo

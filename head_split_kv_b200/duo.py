@@ -1,0 +1,260 @@
+"""Thin ctypes binding over libduo.so (include/duo.h).
+
+Argument marshalling only: every step of the attention path runs in the
+library's CUDA kernels.  Tensor arguments are raw device pointers (ints) or
+objects with ``data_ptr()`` (torch tensors); streams are raw ``cudaStream_t``
+values, torch streams, or None for torch's current stream.
+
+Importing this module fails with ImportError when libduo.so has not been
+built; there is no other implementation to fall back to.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libduo.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is not built; run `python -m head_split_kv_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+# --------------------------------------------------------------- constants
+OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_DTYPE, ERR_CAPACITY, ERR_UNSUPPORTED, ERR_CUDA, ERR_DEVICE = range(8)
+BF16, FP32 = 0, 1
+ORDER_MODEL, ORDER_BLOCK = 0, 1
+MODEL_TO_BLOCK, BLOCK_TO_MODEL = 0, 1
+OP_DECODE, OP_PREFILL = 0, 1
+DEV_FULL_CACHE_OVERFLOW, DEV_BAD_PAGE, DEV_WAIT_TIMEOUT, DEV_BAD_LENGTH = 1, 2, 4, 8
+MAX_KV_HEADS = 64
+STATE_COUNTER_WORDS = 4
+
+
+class LayerDesc(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32), ("sink", ctypes.c_int32), ("recent", ctypes.c_int32),
+        ("dtype", ctypes.c_int32), ("page_size", ctypes.c_int32), ("scale", ctypes.c_float),
+        ("n_retrieval", ctypes.c_int32), ("io_order", ctypes.c_int32),
+        ("kv_perm", ctypes.c_int32 * MAX_KV_HEADS),
+    ]
+
+
+class KVState(ctypes.Structure):
+    _fields_ = [
+        ("k_full", ctypes.c_void_p), ("v_full", ctypes.c_void_p), ("page_table", ctypes.c_void_p),
+        ("capacity", ctypes.c_int32), ("max_pages", ctypes.c_int32), ("n_pages", ctypes.c_int32),
+        ("reserved0", ctypes.c_int32),
+        ("k_ring", ctypes.c_void_p), ("v_ring", ctypes.c_void_p), ("ring_pos", ctypes.c_void_p),
+        ("seq_len", ctypes.c_void_p), ("counters", ctypes.c_void_p), ("status", ctypes.c_void_p),
+    ]
+
+
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_DESC = ctypes.POINTER(LayerDesc)
+_STATE = ctypes.POINTER(KVState)
+
+
+def _fn(name, restype, *argtypes):
+    f = getattr(_lib, name)
+    f.restype = restype
+    f.argtypes = list(argtypes)
+    return f
+
+
+_lib_last_error = _fn("duo_last_error", ctypes.c_char_p)
+_lib_status_string = _fn("duo_status_string", ctypes.c_char_p, ctypes.c_int)
+_lib_abi_version = _fn("duo_abi_version", _I32)
+_lib_partition = _fn("duo_partition_heads", ctypes.c_int, ctypes.POINTER(ctypes.c_float), _I32, ctypes.c_float,
+                     _I32, ctypes.POINTER(ctypes.c_uint8), ctypes.POINTER(_I32), ctypes.POINTER(_I32),
+                     ctypes.POINTER(_I32))
+_lib_desc_init = _fn("duo_desc_init", ctypes.c_int, _DESC, _I32, _I32, _I32, _I32, _I32, ctypes.POINTER(_I32), _I32)
+_lib_desc_validate = _fn("duo_desc_validate", ctypes.c_int, _DESC)
+_lib_ws_bytes = _fn("duo_workspace_bytes", ctypes.c_size_t, _DESC, _I32, _I32)
+_lib_permute = _fn("duo_permute_heads", ctypes.c_int, _DESC, _P, _P, ctypes.c_int64, _I32, ctypes.c_int64, _I32,
+                   _I32, _P)
+_lib_append = _fn("duo_append_kv", ctypes.c_int, _DESC, _STATE, _P, _P, _I32, _P)
+_lib_decode = _fn("duo_decode_attn", ctypes.c_int, _DESC, _STATE, _P, _P, _P, ctypes.c_size_t, _P)
+_lib_prefill = _fn("duo_prefill_chunk", ctypes.c_int, _DESC, _STATE, _P, _P, _P, _I32, _P, _P, ctypes.c_size_t, _P)
+_lib_mix = _fn("duo_gated_mix", ctypes.c_int, _DESC, _P, _P, _P, _P, _I32, _P, _P)
+_lib_check = _fn("duo_check_status", ctypes.c_int, _STATE, ctypes.POINTER(_I32), _P)
+
+
+class DuoError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib_last_error().decode()
+        super().__init__(f"{where}: {_lib_status_string(status).decode()}: {msg}")
+
+
+def _check(st: int, where: str) -> None:
+    if st != OK:
+        raise DuoError(st, where)
+
+
+def _ptr(x) -> int:
+    if x is None:
+        return 0
+    if isinstance(x, int):
+        return x
+    return int(x.data_ptr())
+
+
+def _stream(s) -> int:
+    if s is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream)
+    if isinstance(s, int):
+        return s
+    return int(s.cuda_stream)
+
+
+def last_error() -> str:
+    return _lib_last_error().decode()
+
+
+def status_string(s: int) -> str:
+    return _lib_status_string(s).decode()
+
+
+def abi_version() -> int:
+    return int(_lib_abi_version())
+
+
+# ------------------------------------------------------------------- set-up
+
+def partition_heads(alpha, tau: float, target_n_retrieval: int = -1):
+    """Host call: (gate list[int], kv_perm list[int], kv_inv_perm list[int], n_retrieval)."""
+    alpha = [float(a) for a in alpha]
+    n = len(alpha)
+    a = (ctypes.c_float * max(n, 1))(*alpha)
+    gate = (ctypes.c_uint8 * max(n, 1))()
+    perm = (_I32 * max(n, 1))()
+    inv = (_I32 * max(n, 1))()
+    nret = _I32()
+    _check(_lib_partition(a, n, tau, target_n_retrieval, gate, perm, inv, ctypes.byref(nret)),
+           "duo_partition_heads")
+    return list(gate[:n]), list(perm[:n]), list(inv[:n]), int(nret.value)
+
+
+def desc_init(batch, n_q_heads, n_kv_heads, head_dim, dtype, kv_perm, n_retrieval, *, sink=None, recent=None,
+              page_size=0, io_order=ORDER_MODEL, scale=0.0) -> LayerDesc:
+    d = LayerDesc()
+    perm = (_I32 * max(len(kv_perm), 1))(*[int(p) for p in kv_perm])
+    _check(_lib_desc_init(ctypes.byref(d), batch, n_q_heads, n_kv_heads, head_dim, dtype, perm, n_retrieval),
+           "duo_desc_init")
+    if sink is not None:
+        d.sink = sink
+    if recent is not None:
+        d.recent = recent
+    d.page_size = page_size
+    d.io_order = io_order
+    d.scale = scale
+    _check(_lib_desc_validate(ctypes.byref(d)), "duo_desc_validate")
+    return d
+
+
+def desc_validate(desc: LayerDesc) -> int:
+    return int(_lib_desc_validate(ctypes.byref(desc)))
+
+
+def workspace_bytes(desc: LayerDesc, op: int, max_tokens: int) -> int:
+    return int(_lib_ws_bytes(ctypes.byref(desc), op, max_tokens))
+
+
+# ------------------------------------------------------------ device calls
+
+def permute_heads(desc, x, y, rows, heads_per_kv, head_elems, elem_bytes, direction, stream=None) -> None:
+    _check(_lib_permute(ctypes.byref(desc), _ptr(x), _ptr(y), rows, heads_per_kv, head_elems, elem_bytes,
+                        direction, _stream(stream)), "duo_permute_heads")
+
+
+def append_kv(desc, state: KVState, k_new, v_new, T: int, stream=None) -> None:
+    _check(_lib_append(ctypes.byref(desc), ctypes.byref(state), _ptr(k_new), _ptr(v_new), T, _stream(stream)),
+           "duo_append_kv")
+
+
+def decode_attn(desc, state: KVState, q, out, workspace, ws_bytes: int, stream=None) -> None:
+    _check(_lib_decode(ctypes.byref(desc), ctypes.byref(state), _ptr(q), _ptr(out), _ptr(workspace), ws_bytes,
+                       _stream(stream)), "duo_decode_attn")
+
+
+def prefill_chunk(desc, state: KVState, q, k_chunk, v_chunk, C: int, out, workspace=None, ws_bytes: int = 0,
+                  stream=None) -> None:
+    _check(_lib_prefill(ctypes.byref(desc), ctypes.byref(state), _ptr(q), _ptr(k_chunk), _ptr(v_chunk), C,
+                        _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)), "duo_prefill_chunk")
+
+
+def gated_mix(desc, alpha, q, k, v, N: int, out, stream=None) -> None:
+    _check(_lib_mix(ctypes.byref(desc), _ptr(alpha), _ptr(q), _ptr(k), _ptr(v), N, _ptr(out), _stream(stream)),
+           "duo_gated_mix")
+
+
+def check_status(state: KVState, stream=None, raise_on_error: bool = False) -> int:
+    v = _I32()
+    st = _lib_check(ctypes.byref(state), ctypes.byref(v), _stream(stream))
+    if st not in (OK, ERR_DEVICE) or (raise_on_error and st != OK):
+        raise DuoError(st, "duo_check_status")
+    return int(v.value)
+
+
+# ----------------------------------------------------- torch-owned buffers
+
+class LayerCaches:
+    """Device buffers of one layer's two caches, allocated through torch in
+    the layout include/duo.h documents, plus the KVState that points at them.
+
+    Contiguous full cache: k_full/v_full [B, R, capacity, d].
+    Paged full cache: k_full/v_full [n_pages, R, page_size, d] and page_table
+    [B, max_pages] int32 (copied from the given host table).
+    Rings: k_ring/v_ring [B, S, sink + recent, d]; ring_pos [B, W] (-1);
+    seq_len [B] (0); counters [4] (0); status [1] (0).
+    """
+
+    def __init__(self, desc: LayerDesc, capacity: int = 0, page_table=None, n_pages: int = 0, device="cuda"):
+        import torch
+        dt = torch.bfloat16 if desc.dtype == BF16 else torch.float32
+        B, R, S = desc.batch, desc.n_retrieval, desc.n_kv_heads - desc.n_retrieval
+        d, W = desc.head_dim, desc.sink + desc.recent
+        self.desc = desc
+        if desc.page_size:
+            pt = torch.as_tensor(page_table, dtype=torch.int32)
+            max_pages = pt.shape[1]
+            self.page_table = pt.to(device).contiguous()
+            self.k_full = torch.zeros((n_pages, R, desc.page_size, d), dtype=dt, device=device)
+            self.v_full = torch.zeros_like(self.k_full)
+            capacity = max_pages * desc.page_size
+        else:
+            max_pages = 0
+            self.page_table = None
+            self.k_full = torch.zeros((B, R, max(capacity, 0), d), dtype=dt, device=device)
+            self.v_full = torch.zeros_like(self.k_full)
+        self.capacity = capacity
+        self.k_ring = torch.zeros((B, S, W, d), dtype=dt, device=device)
+        self.v_ring = torch.zeros_like(self.k_ring)
+        self.ring_pos = torch.full((B, W), -1, dtype=torch.int32, device=device)
+        self.seq_len = torch.zeros((B,), dtype=torch.int32, device=device)
+        self.counters = torch.zeros((STATE_COUNTER_WORDS,), dtype=torch.int32, device=device)
+        self.status = torch.zeros((1,), dtype=torch.int32, device=device)
+        self.state = KVState(
+            k_full=_ptr(self.k_full), v_full=_ptr(self.v_full), page_table=_ptr(self.page_table),
+            capacity=capacity, max_pages=max_pages, n_pages=n_pages, reserved0=0,
+            k_ring=_ptr(self.k_ring), v_ring=_ptr(self.v_ring), ring_pos=_ptr(self.ring_pos),
+            seq_len=_ptr(self.seq_len), counters=_ptr(self.counters), status=_ptr(self.status))
+
+
+class Workspace:
+    """A zero-filled device workspace of the size the library asks for."""
+
+    def __init__(self, desc: LayerDesc, op: int, max_tokens: int, device="cuda"):
+        import torch
+        self.nbytes = workspace_bytes(desc, op, max_tokens)
+        self.buf = torch.zeros((max(self.nbytes, 16),), dtype=torch.uint8, device=device)
+
+    @property
+    def ptr(self) -> int:
+        return _ptr(self.buf)

@@ -1,0 +1,311 @@
+/*
+ * duo.h -- C ABI of libduo.so: head-split (retrieval / streaming) attention
+ * for DuoAttention on NVIDIA B200 (sm_100a).
+ *
+ * The method (sources cited by page title and section):
+ *   [Review]  "DuoAttention: Efficient Long-Context LLM Inference with
+ *             Retrieval and Streaming Heads", paper review, xllm-io.github.io,
+ *             S3 "Core formula", "Retrieval-head identification",
+ *             "Inference flow", "Deployment optimisation"; S5 "Ablations".
+ *   [Summary] paperlayer.ai summary of arXiv:2410.10819v1, S2 bullets
+ *             "Optimization-based Identification", "Binarizing Attention
+ *             Implementations", "Chunked Pre-filling".
+ *
+ * Retrieval heads attend causally over a full KV cache that grows with the
+ * context; streaming heads keep only the first `sink` tokens and the last
+ * `recent` tokens (the Lambda-shaped mask) in a constant-size cache.
+ *
+ * Conventions shared by every entry point
+ *   - Every tensor argument is a device pointer owned by the caller, except
+ *     where a comment says "host".  Except for duo_check_status, the library
+ *     never allocates, frees or synchronises; work is queued on `stream`
+ *     (a cudaStream_t; NULL = the legacy default stream).
+ *   - Layouts are dense row-major with the head dimension innermost
+ *     (contiguous).  Pointers must be 16-byte aligned.
+ *   - Element type is bf16 (bit patterns, 2 bytes) or fp32, as
+ *     duo_layer_desc.dtype says; every tensor of a call has that type.
+ *     Accumulation is always fp32; bf16 results are rounded to nearest even
+ *     once, at the final store.
+ *   - Head order: with io_order = DUO_ORDER_MODEL, q / k / v / out use the
+ *     model's head order and the kernels gather and scatter through kv_perm
+ *     (the concatenation back into model order [Review S3 "Inference flow"]
+ *     is the address of the final store).  With DUO_ORDER_BLOCK they are
+ *     already in [retrieval | streaming] block order, as after reordering
+ *     the projection weights [Review S3 "Deployment optimisation"].
+ *     Query head h of the model belongs to KV head h / G, G = n_q_heads /
+ *     n_kv_heads [Summary S2 "Optimization-based Identification"].
+ *   - Return value: DUO_OK, or an error code with a message available from
+ *     duo_last_error() (thread-local).  Argument checks run on the host
+ *     before anything is queued; on an error nothing is queued.  Conditions
+ *     only the device can see (a full cache, a bad page id, a wait that ran
+ *     out) set bits in the state's device status word and skip the access;
+ *     they never trap.  duo_check_status() reads that word back.
+ */
+#ifndef DUO_H
+#define DUO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* duo_stream_t; /* = cudaStream_t */
+
+typedef enum {
+    DUO_OK = 0,
+    DUO_ERR_INVALID_ARG = 1, /* null pointer, bad enum, bad permutation     */
+    DUO_ERR_SHAPE = 2,       /* inconsistent sizes                          */
+    DUO_ERR_DTYPE = 3,       /* unknown element type                        */
+    DUO_ERR_CAPACITY = 4,    /* workspace or cache too small                */
+    DUO_ERR_UNSUPPORTED = 5, /* valid, but not built (e.g. head_dim 96)     */
+    DUO_ERR_CUDA = 6,        /* a CUDA runtime call failed                  */
+    DUO_ERR_DEVICE = 7       /* duo_check_status found device status bits  */
+} duo_status;
+
+/* element types */
+enum { DUO_BF16 = 0, DUO_FP32 = 1 };
+/* head order of q / k / v / out */
+enum { DUO_ORDER_MODEL = 0, DUO_ORDER_BLOCK = 1 };
+/* duo_permute_heads directions */
+enum { DUO_MODEL_TO_BLOCK = 0, DUO_BLOCK_TO_MODEL = 1 };
+/* workspace queries */
+enum { DUO_OP_DECODE = 0, DUO_OP_PREFILL = 1 };
+/* device status bits (OR-ed into duo_kv_state.status) */
+enum {
+    DUO_DEV_FULL_CACHE_OVERFLOW = 1, /* append past capacity: row not written */
+    DUO_DEV_BAD_PAGE = 2,            /* page table entry missing / out of pool */
+    DUO_DEV_WAIT_TIMEOUT = 4,        /* a bounded device wait ran out          */
+    DUO_DEV_BAD_LENGTH = 8           /* a sequence length outside [0, capacity] */
+};
+
+#define DUO_MAX_KV_HEADS 64
+#define DUO_STATE_COUNTER_WORDS 4
+
+/* One attention layer.  Fill it with duo_desc_init(). */
+typedef struct {
+    int32_t batch;        /* B: sequences                                     */
+    int32_t n_q_heads;    /* Hq                                               */
+    int32_t n_kv_heads;   /* Hkv (Hq % Hkv == 0)                              */
+    int32_t head_dim;     /* d: 64 or 128                                     */
+    int32_t sink;         /* attention-sink tokens of streaming heads (16)    */
+    int32_t recent;       /* recent tokens of streaming heads (64)            */
+    int32_t dtype;        /* DUO_BF16 or DUO_FP32                             */
+    int32_t page_size;    /* 0: contiguous full cache; 64: paged full cache   */
+    float scale;          /* softmax scale; 1/sqrt(d) when <= 0               */
+    int32_t n_retrieval;  /* R: retrieval KV heads (block slots 0..R-1)       */
+    int32_t io_order;     /* DUO_ORDER_MODEL or DUO_ORDER_BLOCK               */
+    int32_t kv_perm[DUO_MAX_KV_HEADS]; /* block slot i holds model KV head kv_perm[i] */
+} duo_layer_desc;
+
+/*
+ * The two caches of one layer, all caller-owned device memory.
+ *   R = n_retrieval, S = n_kv_heads - R, W = sink + recent.
+ *
+ * Full cache (retrieval heads) [Review S3 "Inference flow"]:
+ *   contiguous (page_size 0): k_full, v_full = [B][R][capacity][d];
+ *     token p of sequence b, retrieval slot r is row (b*R + r)*capacity + p.
+ *   paged (page_size 64): k_full, v_full = [n_pages][R][64][d]; token p of
+ *     sequence b lives in page page_table[b*max_pages + p/64], row p%64.
+ *     capacity = max_pages * 64.
+ * Streaming ring (streaming heads) [Review S3 "Inference flow"]:
+ *   k_ring, v_ring = [B][S][W][d]; position p lives in slot p if p < sink,
+ *   else in slot sink + (p - sink) % recent, evicting the token `recent`
+ *   positions older.  ring_pos = [B][W] int32, the position held by each
+ *   slot (-1 = empty); all streaming heads of a sequence share it.
+ * seq_len = [B] int32: tokens appended so far per sequence.
+ * counters = DUO_STATE_COUNTER_WORDS uint32 words that must be zero before
+ *   the first call; every call leaves them zero.
+ * status = one int32 word of DUO_DEV_* bits; the library only ORs into it.
+ * Initial values: ring_pos all -1, seq_len 0, status 0 (or a state built by
+ *   the caller that keeps these invariants).
+ */
+typedef struct {
+    void* k_full;
+    void* v_full;
+    int32_t* page_table; /* paged only, else NULL                    */
+    int32_t capacity;    /* tokens per sequence in the full cache    */
+    int32_t max_pages;   /* paged: columns of page_table             */
+    int32_t n_pages;     /* paged: pages in the pool                 */
+    int32_t reserved0;
+    void* k_ring;
+    void* v_ring;
+    int32_t* ring_pos;
+    int32_t* seq_len;
+    uint32_t* counters;
+    int32_t* status;
+} duo_kv_state;
+
+/* ------------------------------------------------------------------------ */
+/* Library information                                                      */
+/* ------------------------------------------------------------------------ */
+
+/* Message of the last error on this thread ("" after success). */
+const char* duo_last_error(void);
+/* Name of a status code. */
+const char* duo_status_string(duo_status s);
+/* ABI version: 1. */
+int32_t duo_abi_version(void);
+
+/* ------------------------------------------------------------------------ */
+/* Set-up (host only)                                                       */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * duo_partition_heads -- gate binarisation and head partition.
+ * [Review S3 "Retrieval-head identification": alpha = 1[alpha >= tau];
+ *  Summary S2 "Binarizing Attention Implementations": tau is a sparsity
+ *  quantile; Review S3 "Deployment optimisation": heads are regrouped into a
+ *  contiguous retrieval block and a streaming block.]
+ *
+ * alpha        host float[n_kv_heads], the optimised gate of each KV head.
+ * tau          threshold, used when target_n_retrieval < 0: gate = alpha >= tau.
+ * target_n_retrieval  >= 0: keep exactly that many heads, those with the
+ *              largest alpha, ties going to the lower head index (the
+ *              quantile threshold).
+ * gate         host uint8[n_kv_heads] out: 1 = retrieval head.
+ * kv_perm      host int32[n_kv_heads] out: block slot i holds model head
+ *              kv_perm[i]; retrieval heads first, each block ascending.
+ * kv_inv_perm  host int32[n_kv_heads] out: kv_inv_perm[kv_perm[i]] = i.
+ * n_retrieval  host int32 out.
+ * Errors: DUO_ERR_INVALID_ARG (null, n_kv_heads outside 1..DUO_MAX_KV_HEADS,
+ * NaN alpha), DUO_ERR_SHAPE (target above n_kv_heads).
+ */
+duo_status duo_partition_heads(const float* alpha, int32_t n_kv_heads, float tau,
+                               int32_t target_n_retrieval, uint8_t* gate, int32_t* kv_perm,
+                               int32_t* kv_inv_perm, int32_t* n_retrieval);
+
+/*
+ * duo_desc_init -- fill a layer descriptor with the deployment defaults
+ * (sink 16, recent 64 [Review S5 "Ablations" item 3], scale 1/sqrt(d),
+ * contiguous full cache, model head order) and the given partition.
+ * kv_perm: host int32[n_kv_heads] from duo_partition_heads.
+ * Errors: DUO_ERR_INVALID_ARG / DUO_ERR_SHAPE / DUO_ERR_DTYPE /
+ * DUO_ERR_UNSUPPORTED for values the kernels do not take.
+ */
+duo_status duo_desc_init(duo_layer_desc* desc, int32_t batch, int32_t n_q_heads,
+                         int32_t n_kv_heads, int32_t head_dim, int32_t dtype,
+                         const int32_t* kv_perm, int32_t n_retrieval);
+
+/* Checks a filled descriptor the way every entry point does. */
+duo_status duo_desc_validate(const duo_layer_desc* desc);
+
+/*
+ * duo_workspace_bytes -- device workspace needed by duo_decode_attn
+ * (op DUO_OP_DECODE) or duo_prefill_chunk (op DUO_OP_PREFILL, max_tokens =
+ * largest chunk).  The workspace holds split-K partial results and ticket
+ * words; it must be zero-filled once before its first use, and every call
+ * leaves the ticket words zero again.  Returns 0 for an invalid descriptor.
+ */
+size_t duo_workspace_bytes(const duo_layer_desc* desc, int32_t op, int32_t max_tokens);
+
+/* ------------------------------------------------------------------------ */
+/* Device entry points                                                      */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * duo_permute_heads -- physical reorder of head blocks between model order
+ * and [retrieval | streaming] block order [Review S3 "Deployment
+ * optimisation"].  Works for activations and for projection weights alike.
+ *
+ * x, y        [rows][n_kv_heads * heads_per_kv][head_elems] of elem_bytes
+ *             each (1, 2, 4 or 8); x and y must not overlap.
+ * direction   DUO_MODEL_TO_BLOCK: y[.., i*hpk + g, ..] = x[.., kv_perm[i]*hpk + g, ..]
+ *             DUO_BLOCK_TO_MODEL: the inverse.
+ * Errors: DUO_ERR_INVALID_ARG, DUO_ERR_SHAPE, DUO_ERR_CUDA.
+ */
+duo_status duo_permute_heads(const duo_layer_desc* desc, const void* x, void* y, int64_t rows,
+                             int32_t heads_per_kv, int64_t head_elems, int32_t elem_bytes,
+                             int32_t direction, duo_stream_t stream);
+
+/*
+ * duo_append_kv -- add T tokens per sequence to the two caches.
+ * [Review S3 "Inference flow": each layer keeps a full cache for retrieval
+ *  heads and a sink + recent cache for streaming heads; Summary S2
+ *  "Chunked Pre-filling": pre-fill fills both caches.]
+ *
+ * k_new, v_new [B][T][Hkv][d], head order per desc->io_order.  Token t of
+ * sequence b gets position p = seq_len[b] + t.  Retrieval heads: written to
+ * the full cache at p.  Streaming heads: written to the ring only if
+ * p < sink or p >= seq_len[b] + T - recent (the tokens that survive), and
+ * ring_pos is updated.  seq_len[b] += T once every row is written.
+ * T == 0 is a no-op.  A row past capacity (or with no page) is not written
+ * and sets DUO_DEV_FULL_CACHE_OVERFLOW (DUO_DEV_BAD_PAGE).
+ * Errors: DUO_ERR_INVALID_ARG, DUO_ERR_SHAPE, DUO_ERR_CUDA.
+ */
+duo_status duo_append_kv(const duo_layer_desc* desc, const duo_kv_state* st, const void* k_new,
+                         const void* v_new, int32_t T, duo_stream_t stream);
+
+/*
+ * duo_decode_attn -- attention of one new token per sequence, both head
+ * types in one launch [Review S3 "Inference flow", decode: Q/K/V are split
+ * along the head dimension, each part attends against its own cache, and the
+ * results are concatenated before the output projection].
+ *
+ * Call after duo_append_kv of the token (the token attends to itself).
+ * q   [B][Hq][d]; out [B][Hq][d]; head order per desc->io_order.
+ * Retrieval heads: out = softmax(scale q K^T) V over cache rows
+ * 0..seq_len[b]-1, split-K across CTAs with a last-CTA combine.  Streaming
+ * heads: the same over the min(seq_len[b], W) ring slots.  The G query heads
+ * of a KV head share every K/V tile.
+ * workspace: >= duo_workspace_bytes(desc, DUO_OP_DECODE, 0) bytes, zeroed once.
+ * Concurrent calls must not share a workspace.
+ * Errors: DUO_ERR_INVALID_ARG, DUO_ERR_SHAPE, DUO_ERR_CAPACITY (workspace),
+ * DUO_ERR_UNSUPPORTED, DUO_ERR_CUDA.
+ */
+duo_status duo_decode_attn(const duo_layer_desc* desc, const duo_kv_state* st, const void* q,
+                           void* out, void* workspace, size_t ws_bytes, duo_stream_t stream);
+
+/*
+ * duo_prefill_chunk -- attention of a chunk of C prompt tokens per sequence
+ * [Summary S2 "Chunked Pre-filling"; Review S3 "Inference flow", pre-fill:
+ *  retrieval heads use full causal attention, streaming heads need linear
+ *  time and constant memory].
+ *
+ * Call BEFORE duo_append_kv of the same chunk: the caches hold tokens
+ * 0..seq_len[b]-1 and the chunk's own keys come from k_chunk / v_chunk.
+ * q [B][C][Hq][d]; k_chunk, v_chunk [B][C][Hkv][d]; out [B][C][Hq][d].
+ * Query c of the chunk has position P = seq_len[b] + c.
+ *   Retrieval head: keys 0..P (causal), prior ones from the full cache.
+ *   Streaming head: keys j <= P with j < sink or P - j < recent (Lambda),
+ *     prior ones from the ring.
+ * bf16 with d = 128 runs on the tcgen05 tensor cores (TMA-fed tiles, TMEM
+ * accumulators); fp32 and d = 64 run on the CUDA cores.
+ * workspace: >= duo_workspace_bytes(desc, DUO_OP_PREFILL, C) bytes (may be 0).
+ * The full cache must be contiguous (page_size 0) here.
+ * Errors: DUO_ERR_INVALID_ARG, DUO_ERR_SHAPE, DUO_ERR_CAPACITY,
+ * DUO_ERR_UNSUPPORTED, DUO_ERR_CUDA.
+ */
+duo_status duo_prefill_chunk(const duo_layer_desc* desc, const duo_kv_state* st, const void* q,
+                             const void* k_chunk, const void* v_chunk, int32_t C, void* out,
+                             void* workspace, size_t ws_bytes, duo_stream_t stream);
+
+/*
+ * duo_gated_mix -- the head-identification forward over whole sequences, no
+ * cache: attn = alpha * full_attn + (1 - alpha) * streaming_attn per head,
+ * with full_attn = softmax(Q K^T (.) M_causal) V and streaming_attn the same
+ * under the Lambda mask [Review S3 "Core formula"], one continuous alpha per
+ * KV head shared by its query heads [Summary S2 "Optimization-based
+ * Identification"].
+ *
+ * alpha [Hkv] fp32 device, in model KV head order.
+ * q [B][N][Hq][d]; k, v [B][N][Hkv][d]; out [B][N][Hq][d]; model head order
+ * (kv_perm and io_order are not used).  One pass over QK^T feeds both
+ * softmax states.
+ * Errors: DUO_ERR_INVALID_ARG, DUO_ERR_SHAPE, DUO_ERR_UNSUPPORTED, DUO_ERR_CUDA.
+ */
+duo_status duo_gated_mix(const duo_layer_desc* desc, const float* alpha, const void* q,
+                         const void* k, const void* v, int32_t N, void* out, duo_stream_t stream);
+
+/*
+ * duo_check_status -- synchronise `stream`, copy the state's device status
+ * word to *host_status and return DUO_ERR_DEVICE if any bit is set.
+ * The only entry point that blocks.
+ */
+duo_status duo_check_status(const duo_kv_state* st, int32_t* host_status, duo_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DUO_H */

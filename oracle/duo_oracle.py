@@ -400,8 +400,10 @@ class HeadSplitCache:
         out = np.empty((bsz, hq, d), dtype=np.float64)
         for b in range(bsz):
             p = self.length[b] - 1
-            for h in range(hq):
-                out[b, h] = self._head_attention(b, h // g, q[b, h][None], np.array([p]), scale=sc)[0]
+            for kv in range(self.n_kv_heads):
+                # the G query heads of this KV head as G independent query rows at position p
+                rows = q[b, kv * g:(kv + 1) * g]
+                out[b, kv * g:(kv + 1) * g] = self._head_attention(b, kv, rows, np.full(g, p), scale=sc)
         return out
 
     def prefill_chunk(self, q, k_chunk, v_chunk, scale=None) -> np.ndarray:

@@ -35,3 +35,12 @@ def read_golden(name):
 @pytest.fixture(scope="session")
 def golden():
     return read_golden
+
+
+@pytest.fixture(scope="session")
+def duo():
+    """The ctypes binding; builds libduo.so first when it is missing or stale."""
+    from head_split_kv_b200 import build as B
+    B.build()
+    from head_split_kv_b200 import duo as D
+    return D

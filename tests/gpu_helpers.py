@@ -1,0 +1,185 @@
+"""Shared plumbing for the GPU parity tests: moving seeded inputs to the device
+in the layouts include/duo.h documents, reading results back, and the
+tolerances (bf16 inputs with fp32 accumulation: max-abs 2e-2 and mean-abs
+2e-3; fp32 inputs: max-abs 1e-4)."""
+
+from __future__ import annotations
+
+import numpy as np
+
+import oracle as O
+from head_split_kv_b200 import synthetic as S
+
+BF16_MAX_ABS, BF16_MEAN_ABS, FP32_MAX_ABS = 2e-2, 2e-3, 1e-4
+
+
+def torch():
+    import torch as t
+    return t
+
+
+def to_dev(a: np.ndarray):
+    """uint16 bf16 bits -> torch.bfloat16; float32 -> torch.float32; on cuda."""
+    t = torch()
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return t.from_numpy(a.view(np.int16)).view(t.bfloat16).cuda()
+    return t.from_numpy(a).cuda()
+
+
+def bits(x) -> np.ndarray:
+    """Device tensor -> numpy with the exact bytes (bf16 as uint16 bits)."""
+    t = torch()
+    x = x.detach().contiguous().cpu()
+    if x.dtype == t.bfloat16:
+        return x.view(t.int16).numpy().view(np.uint16)
+    return x.numpy()
+
+
+def f64(x) -> np.ndarray:
+    return O.as_f64(bits(x))
+
+
+def assert_close(got: np.ndarray, want: np.ndarray, dtype: str, what: str = "") -> dict:
+    err = np.abs(np.asarray(got, dtype=np.float64) - np.asarray(want, dtype=np.float64))
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    mx, mean = float(err.max()) if err.size else 0.0, float(err.mean()) if err.size else 0.0
+    if dtype == "bf16":
+        assert mx <= BF16_MAX_ABS and mean <= BF16_MEAN_ABS, f"{what}: max {mx:.3e} mean {mean:.3e}"
+    else:
+        assert mx <= FP32_MAX_ABS, f"{what}: max {mx:.3e}"
+    return dict(max_abs=mx, mean_abs=mean)
+
+
+class Layer:
+    """One attention layer on the device plus its oracle twin."""
+
+    def __init__(self, duo, shape: S.LayerShape, retrieval, batch: int, capacity: int = 0, page_size: int = 0,
+                 page_table=None, n_pages: int = 0, io_order=None):
+        self.duo = duo
+        self.shape = shape
+        self.B = batch
+        hkv = shape.n_kv_heads
+        alpha = S.binary_alpha(hkv, retrieval)
+        self.gate, self.perm, self.inv, self.R = duo.partition_heads(alpha, 0.5)
+        og, op, oi, on = O.partition_heads(alpha.astype(np.float64), 0.5)
+        assert self.gate == list(og) and self.perm == list(op) and self.R == on
+        self.io_order = duo.ORDER_MODEL if io_order is None else io_order
+        self.desc = duo.desc_init(batch, shape.n_q_heads, hkv, shape.head_dim,
+                                  duo.BF16 if shape.dtype == "bf16" else duo.FP32, self.perm, self.R,
+                                  sink=shape.sink, recent=shape.recent, page_size=page_size,
+                                  io_order=self.io_order)
+        self.page_table = None if page_table is None else np.asarray(page_table, dtype=np.int32)
+        self.caches = duo.LayerCaches(self.desc, capacity, self.page_table, n_pages)
+        self.oracle = O.HeadSplitCache(batch, hkv, shape.head_dim, gate=self.gate, sink=shape.sink,
+                                       recent=shape.recent)
+        self.ws = duo.Workspace(self.desc, duo.OP_DECODE, self.caches.capacity)
+
+    # -- head order ----------------------------------------------------------
+    def to_io(self, x: np.ndarray, axis: int, per_kv: int) -> np.ndarray:
+        """Model head order -> the layer's io order along `axis` (blocks of per_kv heads)."""
+        if self.io_order == self.duo.ORDER_MODEL:
+            return x
+        idx = np.concatenate([np.arange(h * per_kv, (h + 1) * per_kv) for h in self.perm])
+        return np.take(x, idx, axis=axis)
+
+    def from_io(self, x: np.ndarray, axis: int, per_kv: int) -> np.ndarray:
+        if self.io_order == self.duo.ORDER_MODEL:
+            return x
+        idx = np.concatenate([np.arange(self.inv[h] * per_kv, (self.inv[h] + 1) * per_kv)
+                              for h in range(self.shape.n_kv_heads)])
+        return np.take(x, idx, axis=axis)
+
+    # -- state ----------------------------------------------------------------
+    def load_state(self, st: dict) -> None:
+        """Install a synthetic.decode_state() on the device and in the oracle."""
+        t = torch()
+        c = self.caches
+        sh = self.shape
+        ring_pos = np.full((self.B, sh.sink + sh.recent), -1, dtype=np.int32)
+        for (b, h), (k, v) in st["full"].items():
+            r = self.inv[h]
+            L = k.shape[0]
+            if self.page_table is None:
+                c.k_full[b, r, :L] = to_dev(k)
+                c.v_full[b, r, :L] = to_dev(v)
+            else:
+                pos = np.arange(L)
+                pages = t.from_numpy(self.page_table[b, pos // 64].astype(np.int64)).cuda()
+                rows = t.from_numpy(pos % 64).cuda()
+                c.k_full[pages, r, rows] = to_dev(k)
+                c.v_full[pages, r, rows] = to_dev(v)
+            self.oracle.load_state(b, h, np.arange(L), k, v)
+        for (b, h), (pos, k, v) in st["stream"].items():
+            s = self.inv[h] - self.R
+            slots = np.array([O.ring_slot(int(p), sh.sink, sh.recent) for p in pos], dtype=np.int64)
+            if len(slots):
+                idx = t.from_numpy(slots).cuda()
+                c.k_ring[b, s, idx] = to_dev(k)
+                c.v_ring[b, s, idx] = to_dev(v)
+                ring_pos[b, slots] = pos
+            self.oracle.load_state(b, h, pos, k, v)
+        c.ring_pos.copy_(t.from_numpy(ring_pos))
+        c.seq_len.copy_(t.from_numpy(st["lengths"].astype(np.int32)))
+        for b, L in enumerate(st["lengths"]):
+            self.oracle.set_length(b, int(L))
+
+    # -- calls ------------------------------------------------------------------
+    def append(self, k: np.ndarray, v: np.ndarray) -> None:
+        """k, v [B, T, Hkv, d] in model order."""
+        T = k.shape[1]
+        kd = to_dev(self.to_io(k, 2, 1))
+        vd = to_dev(self.to_io(v, 2, 1))
+        self.duo.append_kv(self.desc, self.caches.state, kd, vd, T)
+        self.oracle.append(k, v)
+
+    def decode(self, q: np.ndarray, k: np.ndarray, v: np.ndarray, check_oracle: bool = True):
+        """One step: q [B, Hq, d], k/v [B, Hkv, d] (model order).  Returns (gpu, oracle)."""
+        t = torch()
+        g = self.shape.group
+        kd = to_dev(self.to_io(k[:, None], 2, 1))
+        vd = to_dev(self.to_io(v[:, None], 2, 1))
+        qd = to_dev(self.to_io(q, 1, g))
+        out = t.empty_like(qd)
+        self.duo.append_kv(self.desc, self.caches.state, kd, vd, 1)
+        self.duo.decode_attn(self.desc, self.caches.state, qd, out, self.ws.ptr, self.ws.nbytes)
+        got = self.from_io(f64(out), 1, g)
+        if check_oracle:
+            want = self.oracle.decode(q, k, v)
+        else:
+            self.oracle.append(k[:, None], v[:, None])
+            want = None
+        return got, want
+
+    def status(self) -> int:
+        return self.duo.check_status(self.caches.state)
+
+    # -- bit-exact cache comparison --------------------------------------------
+    def assert_caches_match(self, upto=None) -> None:
+        sh = self.shape
+        dt = np.uint16 if sh.dtype == "bf16" else np.float32
+        c = self.caches
+        seq = bits(c.seq_len)
+        assert list(seq) == list(self.oracle.length), (list(seq), self.oracle.length)
+        kf, vf = (bits(c.k_full), bits(c.v_full)) if self.R else (None, None)
+        kr, vr, rp = bits(c.k_ring), bits(c.v_ring), bits(c.ring_pos)
+        for b in range(self.B):
+            L = self.oracle.length[b]
+            for h in range(sh.n_kv_heads):
+                slot = self.inv[h]
+                if self.gate[h]:
+                    pos, ko, vo = self.oracle.rows(b, h)
+                    if self.page_table is None:
+                        gk, gv = kf[b, slot, pos], vf[b, slot, pos]
+                    else:
+                        pages = self.page_table[b, pos // 64]
+                        gk, gv = kf[pages, slot, pos % 64], vf[pages, slot, pos % 64]
+                    assert np.array_equal(gk, ko) and np.array_equal(gv, vo), f"full cache b={b} h={h}"
+                    assert np.array_equal(pos, np.arange(L))
+                else:
+                    ko, vo, po = self.oracle.ring_layout(b, h, dt)
+                    s = slot - self.R
+                    assert np.array_equal(rp[b], po), f"ring_pos b={b}: {rp[b]} vs {po}"
+                    valid = po >= 0
+                    assert np.array_equal(kr[b, s][valid], ko[valid]), f"ring K b={b} h={h}"
+                    assert np.array_equal(vr[b, s][valid], vo[valid]), f"ring V b={b} h={h}"

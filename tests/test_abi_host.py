@@ -1,0 +1,221 @@
+"""The C-ABI library on the host: it loads, exports every symbol include/duo.h
+declares, its struct layouts match the C compiler's, and its host-side logic
+(gate binarisation, head partition, argument checks) behaves -- all without a
+GPU: every call here returns before anything is queued on a device."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "duo.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(duo_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for want in ["duo_partition_heads", "duo_permute_heads", "duo_append_kv", "duo_decode_attn",
+                 "duo_prefill_chunk", "duo_gated_mix", "duo_workspace_bytes", "duo_last_error"]:
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(duo):
+    out = subprocess.run(["nm", "-D", "--defined-only", duo.LIB_PATH], capture_output=True, text=True, check=True)
+    exported = set(re.findall(r"\s[TW]\s(duo_\w+)", out.stdout))
+    missing = [n for n in _declared_functions() if n not in exported]
+    assert not missing, f"declared in duo.h but not exported: {missing}"
+    lib = ctypes.CDLL(duo.LIB_PATH)
+    for n in _declared_functions():
+        assert hasattr(lib, n)
+
+
+def test_struct_layouts_match_the_c_compiler(duo, tmp_path):
+    src = tmp_path / "layout.c"
+    src.write_text("""
+#include <stdio.h>
+#include <stddef.h>
+#include "duo.h"
+int main(void) {
+  printf("%zu %zu %zu %zu %zu\\n", sizeof(duo_layer_desc), offsetof(duo_layer_desc, scale),
+         offsetof(duo_layer_desc, kv_perm), sizeof(duo_kv_state), offsetof(duo_kv_state, k_ring));
+  printf("%zu %zu %zu\\n", offsetof(duo_kv_state, seq_len), offsetof(duo_kv_state, counters),
+         offsetof(duo_kv_state, status));
+  return 0;
+}
+""")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    a, b = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")[:2]
+    L, K = duo.LayerDesc, duo.KVState
+    assert [int(x) for x in a.split()] == [ctypes.sizeof(L), L.scale.offset, L.kv_perm.offset,
+                                           ctypes.sizeof(K), K.k_ring.offset]
+    assert [int(x) for x in b.split()] == [K.seq_len.offset, K.counters.offset, K.status.offset]
+
+
+def test_abi_version_and_status_strings(duo):
+    assert duo.abi_version() == 1
+    assert duo.status_string(duo.OK) == "DUO_OK"
+    assert duo.status_string(duo.ERR_CAPACITY) == "DUO_ERR_CAPACITY"
+
+
+# ---------------------------------------------------------------------------
+# Gate binarisation + partition: bit-exact against the oracle
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("seed", range(20))
+def test_partition_matches_oracle(duo, seed):
+    rng = np.random.default_rng(seed)
+    hkv = int(rng.integers(1, 65))
+    alpha = rng.uniform(0, 1, hkv).astype(np.float32)
+    if seed % 3 == 0:  # ties and values exactly at tau
+        alpha = rng.choice(np.array([0.0, 0.25, 0.5, 0.75, 1.0], dtype=np.float32), hkv)
+    tau = float(np.float32(0.5))
+    for target in (-1, 0, hkv // 4, hkv // 2, hkv):
+        g, p, ip, n = duo.partition_heads(alpha, tau, target)
+        og, op, oip, on = O.partition_heads(alpha.astype(np.float64), tau, target)
+        assert g == list(og) and p == list(op) and ip == list(oip) and n == on
+
+
+def test_partition_rejects_bad_arguments(duo):
+    with pytest.raises(duo.DuoError) as e:
+        duo.partition_heads([0.1] * 65, 0.5)
+    assert e.value.status == duo.ERR_INVALID_ARG
+    with pytest.raises(duo.DuoError) as e:
+        duo.partition_heads([0.1, float("nan")], 0.5)
+    assert e.value.status == duo.ERR_INVALID_ARG
+    with pytest.raises(duo.DuoError) as e:
+        duo.partition_heads([0.1, 0.2], 0.5, target_n_retrieval=3)
+    assert e.value.status == duo.ERR_SHAPE
+
+
+# ---------------------------------------------------------------------------
+# Descriptor checks
+# ---------------------------------------------------------------------------
+
+def _desc(duo, **kw):
+    args = dict(batch=1, n_q_heads=32, n_kv_heads=8, head_dim=128, dtype=duo.BF16,
+                kv_perm=list(range(8)), n_retrieval=4)
+    args.update(kw)
+    return duo.desc_init(**args)
+
+
+def test_desc_defaults(duo):
+    d = _desc(duo)
+    assert (d.sink, d.recent, d.page_size, d.io_order) == (16, 64, 0, duo.ORDER_MODEL)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(batch=0), "ERR_SHAPE"),
+    (dict(n_q_heads=30), "ERR_SHAPE"),
+    (dict(n_q_heads=24), "ERR_UNSUPPORTED"),         # group of 3
+    (dict(head_dim=96), "ERR_UNSUPPORTED"),
+    (dict(head_dim=0), "ERR_SHAPE"),
+    (dict(dtype=7), "ERR_DTYPE"),
+    (dict(n_retrieval=9), "ERR_SHAPE"),
+    (dict(kv_perm=[0, 1, 2, 3, 4, 5, 6, 6]), "ERR_INVALID_ARG"),
+    (dict(kv_perm=[0, 1, 2, 3, 4, 5, 6, 8]), "ERR_INVALID_ARG"),
+    (dict(page_size=32), "ERR_UNSUPPORTED"),
+    (dict(sink=-1), "ERR_SHAPE"),
+    (dict(recent=0), "ERR_SHAPE"),
+])
+def test_desc_rejections(duo, kw, status):
+    with pytest.raises(duo.DuoError) as e:
+        _desc(duo, **kw)
+    assert e.value.status == getattr(duo, status)
+    assert duo.last_error()
+
+
+def test_workspace_bytes(duo):
+    d = _desc(duo)
+    n = duo.workspace_bytes(d, duo.OP_DECODE, 131072 + 64)
+    assert n >= 4 * 4 * 130 * 4 and n % 256 == 0
+    assert duo.workspace_bytes(d, 99, 0) == 0
+
+
+# ---------------------------------------------------------------------------
+# Device entry points reject bad arguments on the host, before any launch
+# ---------------------------------------------------------------------------
+
+def _state(duo, **kw):
+    st = duo.KVState()
+    for k, v in dict(k_full=16, v_full=32, capacity=1024, k_ring=48, v_ring=64, ring_pos=80,
+                     seq_len=96, counters=112, status=128).items():
+        setattr(st, k, v)
+    for k, v in kw.items():
+        setattr(st, k, v)
+    return st
+
+
+def test_append_rejects(duo):
+    d = _desc(duo)
+    with pytest.raises(duo.DuoError) as e:
+        duo.append_kv(d, _state(duo, seq_len=None), 256, 512, 1, stream=0)
+    assert e.value.status == duo.ERR_INVALID_ARG
+    with pytest.raises(duo.DuoError) as e:
+        duo.append_kv(d, _state(duo), 256, 512, -1, stream=0)
+    assert e.value.status == duo.ERR_SHAPE
+    with pytest.raises(duo.DuoError) as e:
+        duo.append_kv(d, _state(duo), 255, 512, 1, stream=0)     # misaligned
+    assert e.value.status == duo.ERR_INVALID_ARG
+    with pytest.raises(duo.DuoError) as e:
+        duo.append_kv(d, _state(duo, capacity=0), 256, 512, 1, stream=0)
+    assert e.value.status == duo.ERR_SHAPE
+    duo.append_kv(d, _state(duo), 256, 512, 0, stream=0)         # T = 0: nothing to do
+
+
+def test_decode_rejects_small_workspace(duo):
+    d = _desc(duo)
+    need = duo.workspace_bytes(d, duo.OP_DECODE, 1024)
+    with pytest.raises(duo.DuoError) as e:
+        duo.decode_attn(d, _state(duo), 256, 512, 1024, need - 16, stream=0)
+    assert e.value.status == duo.ERR_CAPACITY
+    with pytest.raises(duo.DuoError) as e:
+        duo.decode_attn(d, _state(duo), 256, 512, None, need, stream=0)
+    assert e.value.status == duo.ERR_INVALID_ARG
+
+
+def test_paged_state_checks(duo):
+    d = _desc(duo, page_size=64)
+    with pytest.raises(duo.DuoError) as e:
+        duo.append_kv(d, _state(duo), 256, 512, 1, stream=0)      # no page table
+    assert e.value.status == duo.ERR_INVALID_ARG
+    with pytest.raises(duo.DuoError) as e:
+        duo.append_kv(d, _state(duo, page_table=144, max_pages=4, n_pages=8, capacity=300), 256, 512, 1, stream=0)
+    assert e.value.status == duo.ERR_SHAPE
+
+
+def test_prefill_rejects(duo):
+    d = _desc(duo)
+    with pytest.raises(duo.DuoError) as e:
+        duo.prefill_chunk(d, _state(duo), 256, 512, 768, 0, 1024, stream=0)
+    assert e.value.status == duo.ERR_SHAPE
+    with pytest.raises(duo.DuoError) as e:
+        duo.prefill_chunk(_desc(duo, page_size=64), _state(duo, page_table=144, max_pages=16, n_pages=16),
+                          256, 512, 768, 64, 1024, stream=0)
+    assert e.value.status == duo.ERR_UNSUPPORTED
+
+
+def test_gated_mix_rejects(duo):
+    d = _desc(duo)
+    with pytest.raises(duo.DuoError) as e:
+        duo.gated_mix(d, None, 256, 512, 768, 10, 1024, stream=0)
+    assert e.value.status == duo.ERR_INVALID_ARG
+    duo.gated_mix(d, 16, 256, 512, 768, 0, 1024, stream=0)       # N = 0: nothing to do
+
+
+def test_permute_rejects_overlap(duo):
+    d = _desc(duo)
+    with pytest.raises(duo.DuoError) as e:
+        duo.permute_heads(d, 4096, 4096 + 64, 4, 4, 128, 2, duo.MODEL_TO_BLOCK, stream=0)
+    assert e.value.status == duo.ERR_INVALID_ARG
