@@ -16,6 +16,10 @@ Other workloads: gqa_decode_128k, gqa_decode_1m (Llama-3-8B-shaped GQA, 4 of
 32768], 64-token pages), gqa_prefill_128k (one 131,072-token prompt in 32
 chunks of 4,096; a step is one chunk's duo_prefill_chunk + duo_append_kv).
 
+A decode run also measures the pre-fill workload (unless --no-prefill) and
+reports it under "prefill" in the same line; its TFLOP/s count 4*d FLOPs per
+visible (query, key) pair and query head.
+
 Prints one JSON line (rank 0).  Under torchrun each rank runs an independent
 replica of the workload on its own GPU (the path has no exchange step); the
 time is the max over ranks.
@@ -245,7 +249,7 @@ def run_decode(args, wl, world, rank):
     kd = [_to_dev(env["ks"][i][:, None]) for i in range(total)]
     vd = [_to_dev(env["vs"][i][:, None]) for i in range(total)]
     out = torch.empty_like(qd[0])
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush = torch.empty(1 << 30, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
     sp = int(stream.cuda_stream)
 
@@ -299,7 +303,7 @@ def run_decode(args, wl, world, rank):
                    "head_dim": sh.head_dim, "n_retrieval": R, "sink": sh.sink, "recent": sh.recent,
                    "context": [int(env["lengths"].min()), int(env["lengths"].max())],
                    "paged": bool(wl.get("paged", False)), "parallelism": f"replicas{world}",
-                   "l2": "flushed (256 MiB write) before every timed step, outside the timed interval"},
+                   "l2": "flushed (1 GiB write) before every timed step, outside the timed interval"},
         "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": round(achieved, 1), "peak": hbm,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / hbm, 4),
                      "traffic": None, "algorithmic_bytes_per_launch": int(bytes_per_launch),
@@ -331,7 +335,7 @@ def _decode_e2e(duo, env, args, world):
     dout = torch.empty_like(dq)
     stream = torch.cuda.current_stream()
     sp = int(stream.cuda_stream)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush = torch.empty(1 << 30, dtype=torch.uint8, device="cuda")
     times = []
     _barrier(world)
     for i in range(n):
@@ -388,8 +392,104 @@ def _blas_threads():
     return os.cpu_count()
 
 
-def run_prefill(args, wl, world, rank):
-    raise NotImplementedError("pre-fill workload not wired yet")
+def _lambda_pairs(p0: int, n: int, sink: int, recent: int) -> int:
+    """Visible (query, key) pairs of the Lambda mask for queries p0 .. p0+n-1."""
+    P = np.arange(p0, p0 + n, dtype=np.int64)
+    sinks = np.minimum(P + 1, sink)
+    band = np.minimum(P + 1, recent)
+    both = np.clip(np.minimum(sink, P + 1) - np.maximum(0, P - recent + 1), 0, None)
+    return int((sinks + band - both).sum())
+
+
+def _prefill_flops(n_ret_q, n_str_q, d, c0, C, sink, recent):
+    """Algorithmic FLOPs of one chunk: 4*d per visible (query, key) pair and
+    query head (2*d for Q K^T, 2*d for P V); masked pairs are not counted."""
+    causal = C * c0 + C * (C + 1) // 2
+    return 4 * d * (n_ret_q * causal + n_str_q * _lambda_pairs(c0, C, sink, recent))
+
+
+def run_prefill(args, wl, world, rank, steps=None, warmup=None):
+    """Chunked pre-fill of one prompt: a step is one chunk (duo_prefill_chunk
+    then duo_append_kv).  The timed steps are the prompt's chunks in order from
+    an empty cache; warm-up chunks run first on the same buffers, which are then
+    reset (seq_len 0, ring positions -1) outside the timed region."""
+    import torch
+    from head_split_kv_b200 import duo
+    sh = S.LayerShape(wl["hq"], wl["hkv"], wl["d"], "bf16")
+    n, C = wl["n"], wl["chunk"]
+    n_chunks = n // C
+    steps = n_chunks if steps is None else min(steps, n_chunks)
+    warmup = 3 if warmup is None else warmup
+    retrieval = S.retrieval_heads_by_seed(wl["hkv"], wl["n_ret"], seed=1)
+    gate, perm, inv, R = duo.partition_heads(S.binary_alpha(wl["hkv"], retrieval), 0.5)
+    desc = duo.desc_init(1, sh.n_q_heads, sh.n_kv_heads, sh.head_dim, duo.BF16, perm, R)
+    caches = duo.LayerCaches(desc, n)
+    q, k, v = S.prompt(sh, n, seed=0)
+    qd, kd, vd = _to_dev(q), _to_dev(k), _to_dev(v)
+    del q, k, v
+    out = torch.empty((1, C, sh.n_q_heads, sh.head_dim), dtype=torch.bfloat16, device="cuda")
+    flush = torch.empty(1 << 30, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    sp = int(stream.cuda_stream)
+    G = sh.group
+
+    def chunk(i):
+        sl = slice(i * C, (i + 1) * C)
+        qc, kc, vc = qd[:, sl].contiguous(), kd[:, sl].contiguous(), vd[:, sl].contiguous()
+        return qc, kc, vc
+
+    chunks = [chunk(i) for i in range(n_chunks)]
+    for i in range(min(warmup, n_chunks)):
+        qc, kc, vc = chunks[i]
+        duo.prefill_chunk(desc, caches.state, qc, kc, vc, C, out, None, 0, sp)
+        duo.append_kv(desc, caches.state, kc, vc, C, sp)
+    torch.cuda.synchronize()
+    caches.seq_len.zero_()
+    caches.ring_pos.fill_(-1)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    _barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(int(os.environ.get("LOCAL_RANK", "0"))) as clk:
+        for i in range(steps):
+            flush.zero_()
+            qc, kc, vc = chunks[i]
+            e0, e1, e2 = ev[i]
+            e0.record(stream)
+            duo.prefill_chunk(desc, caches.state, qc, kc, vc, C, out, None, 0, sp)
+            e1.record(stream)
+            duo.append_kv(desc, caches.state, kc, vc, C, sp)
+            e2.record(stream)
+        torch.cuda.synchronize()
+    _barrier(world)
+    st_code = duo.check_status(caches.state)
+    if st_code:
+        raise RuntimeError(f"device status 0x{st_code:x} after the timed chunks")
+    pre_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    step_ms = [a.elapsed_time(c) for a, _, c in ev]
+    flops = [_prefill_flops(R * G, (sh.n_kv_heads - R) * G, sh.head_dim, i * C, C, sh.sink, sh.recent)
+             for i in range(steps)]
+    total_ms = _max_over_ranks(sum(step_ms), world)
+    _, tf_peak, peak_kind = _peaks()
+    achieved = sum(flops) / (sum(pre_ms) * 1e-3) / 1e12
+    value = sum(flops) * world / (total_ms * 1e-3) / 1e12
+    return {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": steps,
+        "warmup": warmup, "ms_per_step": round(total_ms / steps, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "gqa_prefill_128k", "prompt": n, "chunk": C, "n_q_heads": sh.n_q_heads,
+                   "n_kv_heads": sh.n_kv_heads, "head_dim": sh.head_dim, "n_retrieval": R, "sink": sh.sink,
+                   "recent": sh.recent, "parallelism": f"replicas{world}",
+                   "l2": "flushed (1 GiB write) before every timed chunk, outside the timed interval"},
+        "roofline": {"bound": "tensor", "kernel": "prefill_tc_kernel", "achieved": round(achieved, 1),
+                     "peak": tf_peak, "peak_kind": peak_kind + " (burst; sustained 1381.5)", "unit": "TFLOP/s",
+                     "frac": round(achieved / tf_peak, 4), "traffic": None,
+                     "algorithmic_tflop_total": round(sum(flops) / 1e12, 3),
+                     "prefill_ms_total": round(sum(pre_ms), 3), "append_ms_total": round(sum(step_ms) - sum(pre_ms), 3),
+                     "per_chunk_ms": [round(x, 3) for x in pre_ms]},
+        "gpu_launches": 2 * steps,
+        "clocks": clk.summary(),
+    }
 
 
 # ---------------------------------------------------------------------------
@@ -441,12 +541,13 @@ def run_reference(args, wl):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--steps", type=int, default=256)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="mha_decode_32k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the pre-fill measurement of a decode run")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -466,8 +567,12 @@ def main(argv=None):
     try:
         if wl["kind"] == "decode":
             res = run_decode(args, wl, world, rank)
+            if not args.no_prefill:
+                pre = run_prefill(args, WORKLOADS["gqa_prefill_128k"], world, rank)
+                res["prefill"] = {k: pre[k] for k in ("value", "unit", "steps", "ms_per_step", "config",
+                                                      "roofline", "gpu_launches", "clocks")}
         else:
-            res = run_prefill(args, wl, world, rank)
+            res = run_prefill(args, wl, world, rank, steps=args.steps, warmup=args.warmup)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

@@ -16,12 +16,14 @@
 // Per CTA: warp 4 is the producer -- one lane issues cp.async.bulk copies
 // (the TMA engine, no tensor map needed: K/V rows of one head are contiguous,
 // or one 64-token page) into a STAGES-deep ring of 64-key shared-memory tiles,
-// signalled through mbarriers.  Warps 0-3 consume: warp w takes keys
-// [16w, 16w+16) of each tile, half-warp h keys 16w + 8h + (0..7); each lane
-// holds D/16 elements of q (pre-scaled by scale*log2 e) and of the output
-// accumulator for every query head of the group.  Dot products are reduced
-// across the 16 lanes by a transposed butterfly (8 keys in 8 shuffles instead
-// of 32), each warp keeps its own online-softmax state, and the four states
+// signalled through mbarriers.  NW consumer warps (8 for query groups of 1
+// or 2, 4 for larger groups, whose accumulators need more registers) split
+// each tile: warp w takes keys [KW*w, KW*w + KW) with KW = 64 / NW, half-warp
+// h the KH = KW / 2 keys after KW*w + KH*h; each lane holds D/16 elements of
+// q (pre-scaled by scale*log2 e) and of the output accumulator for every
+// query head of the group.  Dot products are reduced across the 16 lanes by a
+// transposed butterfly (KH keys in KH + log2(16/KH) - 1 shuffles instead of
+// 4*KH), each warp keeps its own online-softmax state, and the warp states
 // are merged at the end.  With several splits, each CTA stores (m, l, o) to
 // the workspace and the last CTA of the (b, r) pair -- found with an atomic
 // ticket, never a wait -- combines them and writes the output.
@@ -32,13 +34,14 @@ namespace duo {
 namespace {
 
 constexpr int kTile = 64;            // keys per pipeline stage
-constexpr int kConsumerWarps = 4;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
+
+// consumer warps per CTA for a query group of G heads
+__host__ __device__ constexpr int consumer_warps(int G) { return G <= 2 ? 8 : 4; }
 
 struct DecodeArgs {
     const void* q;
     void* out;
-    float* partial;      // [B*R][nsplit][G][D + 2]: m, l, o[D]
+    float* partial;      // [B*R][nsplit][G][D + 4]: m, l, -, -, o[D]
     uint32_t* ticket;    // [B*R]
     int nsplit;
     int n_ret_units;     // B * R * nsplit
@@ -57,50 +60,60 @@ template <typename T, int D, int G>
 constexpr size_t decode_smem_bytes() {
     using C = Cfg<T, D>;
     size_t s = 2 * (size_t)C::kStages * C::kTileBytes;     // K and V stages
-    s += (size_t)kConsumerWarps * 16 * G * sizeof(float);   // probabilities
+    s += (size_t)kTile * G * sizeof(float);                  // probabilities of one tile
     s += 2 * C::kStages * sizeof(uint64_t) + 64;            // barriers, flag, rows per stage
     return s + 1024;                                        // alignment slack
 }
 
 // Transposed butterfly over the 16 lanes of a half-warp: on entry v[j] is this
-// lane's partial dot for key j (j < 8); on exit v[0] is the full dot of key
-// ((lane & 15) >> 1), held by lanes 2k and 2k+1.
-__device__ __forceinline__ float reduce8_transposed(float (&v)[8], int lane) {
+// lane's partial dot for key j (j < K, K = 8 or 4); on exit the return value
+// is the full dot of key ((lane & 15) >> (4 - log2 K)), held by the 16/K
+// lanes that share those high bits.
+template <int K>
+__device__ __forceinline__ float reduce_transposed(float (&v)[K], int lane) {
+    static_assert(K == 8 || K == 4, "4 or 8 keys per half-warp");
     const bool b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float send = b3 ? v[i] : v[i + 4];
-        const float keep = b3 ? v[i + 4] : v[i];
+    for (int i = 0; i < K / 2; ++i) {
+        const float send = b3 ? v[i] : v[i + K / 2];
+        const float keep = b3 ? v[i + K / 2] : v[i];
         v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
     }
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const float send = b2 ? v[i] : v[i + 2];
-        const float keep = b2 ? v[i + 2] : v[i];
+    for (int i = 0; i < K / 4; ++i) {
+        const float send = b2 ? v[i] : v[i + K / 4];
+        const float keep = b2 ? v[i + K / 4] : v[i];
         v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
     }
-    {
+    if (K == 8) {
         const float send = b1 ? v[0] : v[1];
         const float keep = b1 ? v[1] : v[0];
         v[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    } else {
+        v[0] += __shfl_xor_sync(0xffffffffu, v[0], 2);
     }
     v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
     return v[0];
 }
 
 template <typename T, int D, int G, bool PAGED>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__((consumer_warps(G) + 1) * 32, 2)
     decode_kernel(const LayerArgs a, const CacheArgs c, const DecodeArgs d) {
     using C = Cfg<T, D>;
     constexpr int EPL = C::kEPL;
     constexpr int STAGES = C::kStages;
+    constexpr int NW = consumer_warps(G);     // consumer warps
+    constexpr int kThreads = (NW + 1) * 32;
+    constexpr int KW = kTile / NW;            // keys per warp and tile
+    constexpr int KH = KW / 2;                // keys per half-warp
+    constexpr int DUP = 16 / KH;              // lanes holding the same key after the butterfly
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     T* sK = reinterpret_cast<T*>(smem);
     T* sV = reinterpret_cast<T*>(smem + (size_t)STAGES * C::kTileBytes);
-    float* sP = reinterpret_cast<float*>(smem + 2 * (size_t)STAGES * C::kTileBytes);  // [warp][16 keys][G]
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sP + kConsumerWarps * 16 * G);
+    float* sP = reinterpret_cast<float*>(smem + 2 * (size_t)STAGES * C::kTileBytes);  // [warp][KW keys][G]
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sP + kTile * G);
     uint64_t* empty_bar = full_bar + STAGES;
     int* s_flag = reinterpret_cast<int*>(empty_bar + STAGES);
     int* s_tile_n = s_flag + 1;  // valid rows of each stage, written by the producer before its arrive
@@ -152,13 +165,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full_bar[s], 1);
-            mbar_init(&empty_bar[s], kConsumerWarps);
+            mbar_init(&empty_bar[s], NW);
         }
         fence_barrier_init();
     }
     __syncthreads();
 
-    if (warp == kConsumerWarps) {
+    if (warp == NW) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
             for (int t = 0; t < n_tiles; ++t) {
@@ -201,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     float m_run[G], l_run[G];
     const int hw = lane >> 4;        // half-warp
     const int dl = lane & 15;        // lane within the half-warp: owns d-slice [dl*EPL, dl*EPL+EPL)
-    if (warp < kConsumerWarps) {
+    if (warp < NW) {
         float q[G][EPL];
         const T* qp = static_cast<const T*>(d.q) + ((size_t)b * a.Hq + a.q_head0[slot]) * D + dl * EPL;
         const float qs = a.scale * kLog2e;
@@ -215,8 +228,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
             for (int e = 0; e < EPL; ++e) o[g][e] = 0.f;
         }
-        float* myP = sP + warp * 16 * G;
-        const int kidx = (lane & 15) >> 1;  // key this lane scores after the butterfly
+        float* myP = sP + warp * KW * G;
+        const int kidx = (lane & 15) / DUP;  // key this lane scores after the butterfly
 
         for (int t = 0; t < n_tiles; ++t) {
             const int st = t % STAGES, round = t / STAGES;
@@ -224,16 +237,16 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int n = s_tile_n[st];
             const T* tK = sK + (size_t)st * kTile * D;
             const T* tV = sV + (size_t)st * kTile * D;
-            const int key0 = warp * 16 + hw * 8;    // first key of this half-warp in the tile
+            const int key0 = warp * KW + hw * KH;   // first key of this half-warp in the tile
 
             // scores: s[g] of key key0 + kidx
             float s[G];
 #pragma unroll
             for (int g = 0; g < G; ++g) s[g] = 0.f;
             {
-                float part[G][8];
+                float part[G][KH];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
+                for (int j = 0; j < KH; ++j) {
                     float kf[EPL];
                     load_row_f32<T, EPL>(tK + (size_t)(key0 + j) * D + dl * EPL, kf);
 #pragma unroll
@@ -245,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                     }
                 }
 #pragma unroll
-                for (int g = 0; g < G; ++g) s[g] = reduce8_transposed(part[g], lane);
+                for (int g = 0; g < G; ++g) s[g] = reduce_transposed<KH>(part[g], lane);
             }
             const bool valid = key0 + kidx < n;
             float m_new[G], corr[G], p[G];
@@ -253,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int g = 0; g < G; ++g) {
                 float sv = valid ? s[g] : kNegBig;
                 float mt = sv;
-                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+                if (DUP == 2) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
                 mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 4));
                 mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
                 mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
@@ -261,23 +274,23 @@ __global__ void __launch_bounds__(kThreads, 2)
                 corr[g] = exp2f(m_run[g] - m_new[g]);
                 p[g] = valid ? exp2f(sv - m_new[g]) : 0.f;
                 m_run[g] = m_new[g];
-                l_run[g] = l_run[g] * corr[g] + ((lane & 1) ? 0.f : p[g]);
+                l_run[g] = l_run[g] * corr[g] + ((lane & (DUP - 1)) ? 0.f : p[g]);
 #pragma unroll
                 for (int e = 0; e < EPL; ++e) o[g][e] *= corr[g];
             }
-            if ((lane & 1) == 0) {
+            if ((lane & (DUP - 1)) == 0) {
 #pragma unroll
-                for (int g = 0; g < G; ++g) myP[(hw * 8 + kidx) * G + g] = p[g];
+                for (int g = 0; g < G; ++g) myP[(hw * KH + kidx) * G + g] = p[g];
             }
             __syncwarp();
             // o += p v over this half-warp's keys
-            const int nh = min(8, n - key0);
+            const int nh = min(KH, n - key0);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < KH; ++j) {
                 if (j < nh) {
                     float vf[EPL];
                     load_row_f32<T, EPL>(tV + (size_t)(key0 + j) * D + dl * EPL, vf);
-                    const float* pj = myP + (hw * 8 + j) * G;
+                    const float* pj = myP + (hw * KH + j) * G;
 #pragma unroll
                     for (int g = 0; g < G; ++g) {
                         const float pg = pj[g];
@@ -305,17 +318,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     __syncthreads();  // all tiles consumed: the stage buffers are free
 
-    // ---------------------------------------------- merge the 4 warp states
-    // layout in the (now free) K stages: [warp][G][D + 2]
+    // ---------------------------------------------- merge the warp states
+    // layout in the (now free) K stages: [warp][G][STRIDE] with m, l, -, -, o[D]
     float* sM = reinterpret_cast<float*>(sK);
-    constexpr int STRIDE = D + 2;
-    if (warp < kConsumerWarps) {
+    constexpr int STRIDE = D + 4;
+    if (warp < NW) {
         float* dst = sM + (size_t)warp * G * STRIDE;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
             if (lane < 16) {
 #pragma unroll
-                for (int e = 0; e < EPL; ++e) dst[g * STRIDE + 2 + dl * EPL + e] = o[g][e];
+                for (int e = 0; e < EPL; ++e) dst[g * STRIDE + 4 + dl * EPL + e] = o[g][e];
             }
             if (lane == 0) {
                 dst[g * STRIDE + 0] = m_run[g];
@@ -324,22 +337,21 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
     }
     __syncthreads();
-    // the CTA's combined state, one (g, element) per thread step; stored in
-    // slot [kConsumerWarps] of sM
-    float* cta = sM + (size_t)kConsumerWarps * G * STRIDE;
+    // the CTA's combined state, in slot [NW] of sM
+    float* cta = sM + (size_t)NW * G * STRIDE;
     for (int i = threadIdx.x; i < G * D; i += kThreads) {
         const int g = i / D, e = i % D;
         float M = kNegBig;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sM[(w * G + g) * STRIDE]);
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, sM[(w * G + g) * STRIDE]);
         float L = 0.f, O = 0.f;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
+        for (int w = 0; w < NW; ++w) {
             const float sc = exp2f(sM[(w * G + g) * STRIDE] - M);
             L += sc * sM[(w * G + g) * STRIDE + 1];
-            O += sc * sM[(w * G + g) * STRIDE + 2 + e];
+            O += sc * sM[(w * G + g) * STRIDE + 4 + e];
         }
-        cta[g * STRIDE + 2 + e] = O;
+        cta[g * STRIDE + 4 + e] = O;
         if (e == 0) {
             cta[g * STRIDE + 0] = M;
             cta[g * STRIDE + 1] = L;
@@ -352,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int i = threadIdx.x; i < G * D; i += kThreads) {
             const int g = i / D, e = i % D;
             const float L = cta[g * STRIDE + 1];
-            const float v = L > 0.f ? cta[g * STRIDE + 2 + e] / L : 0.f;
+            const float v = L > 0.f ? cta[g * STRIDE + 4 + e] / L : 0.f;
             outp[(size_t)g * D + e] = Elem<T>::from_f32(v);
         }
         return;
@@ -371,19 +383,64 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
     if (!*s_flag) return;
     __threadfence();
+    // This CTA is the last of its (b, r) pair: every split's record is in
+    // global memory.  (1) m and l of all splits into shared memory, (2) the
+    // per-head maximum and each split's weight, (3) warp w sums splits
+    // w, w + 5, ... with 16-byte loads all in flight, (4) the warps' sums are
+    // added and normalised.
     const float* all = d.partial + pair * d.nsplit * (size_t)G * STRIDE;
-    for (int i = threadIdx.x; i < G * D; i += kThreads) {
-        const int g = i / D, e = i % D;
+    const int ns = d.nsplit;
+    float* s_w = cta + G * STRIDE;            // [ns][G] weights
+    float* s_l = s_w + ns * G;                // [ns][G]
+    float* s_inv = s_l + ns * G;              // [G] 1 / L
+    // [kThreads / 32][G * D], written with float4 stores: 16-byte aligned
+    float* s_acc = s_inv + ((G + 3) & ~3) + ((4 - (((NW + 1) * G * STRIDE + 2 * ns * G) & 3)) & 3);
+    for (int i = threadIdx.x; i < ns * G; i += kThreads) {
+        const int sp = i / G, g = i % G;
+        const float* rec = all + ((size_t)sp * G + g) * STRIDE;
+        s_w[i] = __ldcg(rec);
+        s_l[i] = __ldcg(rec + 1);
+    }
+    __syncthreads();
+    if (threadIdx.x < G) {
+        const int g = threadIdx.x;
         float M = kNegBig;
-        for (int sp = 0; sp < d.nsplit; ++sp) M = fmaxf(M, __ldcg(all + ((size_t)sp * G + g) * STRIDE));
-        float L = 0.f, O = 0.f;
-        for (int sp = 0; sp < d.nsplit; ++sp) {
-            const float* ps = all + ((size_t)sp * G + g) * STRIDE;
-            const float sc = exp2f(__ldcg(ps) - M);
-            L += sc * __ldcg(ps + 1);
-            O += sc * __ldcg(ps + 2 + e);
+        for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, s_w[sp * G + g]);
+        float L = 0.f;
+        for (int sp = 0; sp < ns; ++sp) {
+            const float w = exp2f(s_w[sp * G + g] - M);
+            s_w[sp * G + g] = w;
+            L += w * s_l[sp * G + g];
         }
-        outp[(size_t)g * D + e] = Elem<T>::from_f32(L > 0.f ? O / L : 0.f);
+        s_inv[g] = L > 0.f ? 1.f / L : 0.f;
+    }
+    __syncthreads();
+    constexpr int kWarps = kThreads / 32;
+    constexpr int NV = G * D / 4;             // float4 pieces of one split's outputs
+    // everything above lives in the (free) K and V stage buffers
+    static_assert(((NW + 1) * G * (D + 4) + 2 * 128 * G + G + 8 + kWarps * G * D) * sizeof(float) <=
+                      2 * (size_t)STAGES * C::kTileBytes,
+                  "combine scratch exceeds the stage buffers");
+    for (int c = lane; c < NV; c += 32) {
+        const int g = (c * 4) / D, e = (c * 4) % D;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+        for (int sp = warp; sp < ns; sp += kWarps) {
+            const float w = s_w[sp * G + g];
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(all + ((size_t)sp * G + g) * STRIDE + 4 + e));
+            acc.x = fmaf(w, v.x, acc.x);
+            acc.y = fmaf(w, v.y, acc.y);
+            acc.z = fmaf(w, v.z, acc.z);
+            acc.w = fmaf(w, v.w, acc.w);
+        }
+        reinterpret_cast<float4*>(s_acc + (size_t)warp * G * D)[c] = acc;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < G * D; i += kThreads) {
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) v += s_acc[(size_t)w * G * D + i];
+        outp[i] = Elem<T>::from_f32(v * s_inv[i / D]);
     }
     if (threadIdx.x == 0) d.ticket[pair] = 0u;  // leave the workspace ready for the next call
 }
@@ -392,8 +449,13 @@ template <typename T, int D, int G, bool PAGED>
 cudaError_t launch_t(const LayerArgs& a, const CacheArgs& c, const DecodeArgs& d, int grid, cudaStream_t s) {
     constexpr size_t smem = decode_smem_bytes<T, D, G>();
     auto kern = decode_kernel<T, D, G, PAGED>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    constexpr int kThreads = (consumer_warps(G) + 1) * 32;
+    static bool configured = false;  // function attributes are per process, set once
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
     kern<<<grid, kThreads, smem, s>>>(a, c, d);
     return cudaGetLastError();
 }

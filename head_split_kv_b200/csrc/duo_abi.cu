@@ -152,15 +152,18 @@ DecodePlan decode_plan(const LayerArgs& a) {
     const long pairs = (long)a.B * a.R;
     int ns = 1;
     if (pairs > 0) {
-        const long target_ctas = 296;  // 148 SMs x 2 resident CTAs
-        ns = (int)((target_ctas + pairs - 1) / pairs);
+        // 148 SMs x 2 resident CTAs; the streaming CTAs share the same wave
+        const long slots = 296, streaming = (long)a.B * a.S;
+        const long target_ctas = slots - streaming >= pairs ? slots - streaming : slots;
+        ns = (int)(target_ctas / pairs);
+        if (ns < 1) ns = 1;
         const int by_len = (a.capacity + 16383) / 16384;
         if (by_len > ns) ns = by_len;
-        if (ns > 256) ns = 256;
+        if (ns > 128) ns = 128;
         if (ns < 1) ns = 1;
     }
     p.nsplit = ns;
-    p.partial_floats = (size_t)pairs * ns * a.G * (a.D + 2);
+    p.partial_floats = (size_t)pairs * ns * a.G * (a.D + 4);
     p.ticket_offset = ((p.partial_floats * sizeof(float)) + 255) / 256 * 256;
     p.bytes = p.ticket_offset + ((size_t)pairs * sizeof(uint32_t) + 255) / 256 * 256;
     if (pairs == 0) p.bytes = 256;

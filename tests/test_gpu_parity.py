@@ -42,8 +42,8 @@ def test_append_bit_exact(duo, dtype, io_order):
 
 def test_append_paged_bit_exact(duo):
     sh = S.LayerShape(32, 32, 128, "bf16")
-    lengths = np.array([0, 0, 0], dtype=np.int64)
-    table, n_pages = S.page_assignment([1000, 700, 64], 0, 64, seed=5)
+    # 493 tokens are appended per sequence: give each 10 pages (640 tokens)
+    table, n_pages = S.page_assignment([600, 600, 600], 0, 64, seed=5)
     lay = Layer(duo, sh, retrieval=S.retrieval_heads_by_seed(32, 8), batch=3, page_size=64, page_table=table,
                 n_pages=n_pages)
     rng = S.rng_for(4, 99)
@@ -53,7 +53,6 @@ def test_append_paged_bit_exact(duo):
         lay.append(k, v)
     lay.assert_caches_match()
     assert lay.status() == 0
-    del lengths
 
 
 def test_append_overflow_sets_status_and_skips(duo):
