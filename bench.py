@@ -53,7 +53,11 @@ WORKLOADS = {
     "batch64_paged_decode": dict(kind="decode", hq=32, hkv=32, d=128, n_ret=8, batch=64, lo=4096, hi=32768,
                                  steps=32, sigma=False, paged=True),
     "gqa_prefill_128k": dict(kind="prefill", hq=32, hkv=8, d=128, n_ret=4, n=131072, chunk=4096, sigma=False),
+    # the same pre-fill on a 32K prompt: a small case for profiler captures
+    "gqa_prefill_32k": dict(kind="prefill", hq=32, hkv=8, d=128, n_ret=4, n=32768, chunk=4096, sigma=False),
 }
+for _name, _wl in WORKLOADS.items():
+    _wl["name"] = _name
 
 
 def _peaks():
@@ -477,7 +481,7 @@ def run_prefill(args, wl, world, rank, steps=None, warmup=None):
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": steps,
         "warmup": warmup, "ms_per_step": round(total_ms / steps, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "gqa_prefill_128k", "prompt": n, "chunk": C, "n_q_heads": sh.n_q_heads,
+        "config": {"workload": wl["name"], "prompt": n, "chunk": C, "n_q_heads": sh.n_q_heads,
                    "n_kv_heads": sh.n_kv_heads, "head_dim": sh.head_dim, "n_retrieval": R, "sink": sh.sink,
                    "recent": sh.recent, "parallelism": f"replicas{world}",
                    "l2": "flushed (1 GiB write) before every timed chunk, outside the timed interval"},
