@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -384,3 +385,61 @@ duo_status duo_check_status(const duo_kv_state* st, int32_t* host_status, duo_st
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// duo_decode_attn_noalloc: decode with library-owned scratch for callers that
+// cannot allocate device memory themselves (see include/duo.h).
+// ===========================================================================
+namespace {
+
+// Split-K partials and ticket words of duo_decode_attn_noalloc.  In host code
+// this name is only a stand-in for the symbol: the device address comes from
+// cudaGetSymbolAddress, looked up once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[DUO_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+}  // namespace
+
+extern "C" duo_status duo_decode_attn_noalloc(const duo_layer_desc* desc, const duo_kv_state* st, const void* q,
+                                              void* out, duo_stream_t stream) {
+    duo_status s = check_desc(desc);
+    if (s != DUO_OK) return s;
+    duo::LayerArgs a;
+    duo::CacheArgs c;
+    fill_args(desc, a);
+    if ((s = check_state(desc, st, a, c)) != DUO_OK) return s;
+    if (!q || !out) return fail(DUO_ERR_INVALID_ARG, "q / out is NULL");
+    if (!aligned16(q) || !aligned16(out)) return fail(DUO_ERR_INVALID_ARG, "q / out not 16-byte aligned");
+    const duo::DecodePlan plan = duo::decode_plan(a);
+    if (plan.bytes > DUO_NOALLOC_SCRATCH_BYTES)
+        return fail(DUO_ERR_CAPACITY,
+                    "duo_decode_attn_noalloc: this layer needs %zu bytes of split-K scratch, the built-in array "
+                    "holds %u; call duo_decode_attn with a workspace instead",
+                    plan.bytes, (unsigned)DUO_NOALLOC_SCRATCH_BYTES);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "duo_decode_attn_noalloc: cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(DUO_ERR_UNSUPPORTED, "device ordinal %d above %d", dev, kMaxDevices);
+    void* scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        if (!g_noalloc_ptr[dev]) {
+            // once per device, with that device current
+            void* p = nullptr;
+            e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+            if (e != cudaSuccess) return cuda_fail(e, "duo_decode_attn_noalloc: cudaGetSymbolAddress");
+            g_noalloc_ptr[dev] = p;
+        }
+        scratch = g_noalloc_ptr[dev];
+    }
+    // the ticket words must start at zero; the array keeps the previous call's contents
+    const size_t ticket_bytes = plan.bytes - plan.ticket_offset;
+    e = cudaMemsetAsync(static_cast<unsigned char*>(scratch) + plan.ticket_offset, 0, ticket_bytes,
+                        (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "duo_decode_attn_noalloc: clearing the ticket words");
+    e = duo::launch_decode(a, c, plan, q, out, scratch, (cudaStream_t)stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "duo_decode_attn_noalloc");
+}

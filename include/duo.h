@@ -299,6 +299,39 @@ duo_status duo_gated_mix(const duo_layer_desc* desc, const float* alpha, const v
                          const void* k, const void* v, int32_t N, void* out, duo_stream_t stream);
 
 /*
+ * duo_decode_attn_noalloc -- duo_decode_attn without a caller workspace.
+ * (No counterpart on the pages: this is a deployment convenience.)
+ *
+ * Some callers cannot hand the library device memory for scratch: a plugin
+ * running inside a host engine whose allocator owns every byte of HBM, a
+ * thin C binding with no device-memory management of its own, or a decode
+ * loop that must never call cudaMalloc / cudaFree because those calls can
+ * synchronise the whole device.  This entry point computes exactly what
+ * duo_decode_attn computes (same kernel, same split plan), but keeps the
+ * split-K partial results and ticket words in a statically sized array that
+ * is part of the library image; it calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ *
+ * q, out, desc and st are as for duo_decode_attn; there is no workspace.
+ * Scratch limit: DUO_NOALLOC_SCRATCH_BYTES (2 MiB), i.e. duo_workspace_bytes(
+ * desc, DUO_OP_DECODE, st->capacity) must not exceed it; larger layers get
+ * DUO_ERR_CAPACITY with the two sizes in the message (use duo_decode_attn).
+ * Every GPU that loads the library holds the array until the process exits.
+ * The first call on each device looks up the array's device address with
+ * that device current (cudaGetSymbolAddress); make that first call before
+ * any stream capture begins.
+ * All calls on a device share the one array and it keeps the previous call's
+ * contents: each call clears the ticket words it needs on `stream` before the
+ * kernel runs.  Calls that can overlap on the GPU (other streams, other host
+ * threads) race on the array and must be serialised by the caller.
+ * Errors: as duo_decode_attn, plus DUO_ERR_CAPACITY for a layer too large
+ * for the array.
+ */
+#define DUO_NOALLOC_SCRATCH_BYTES (2u << 20)
+duo_status duo_decode_attn_noalloc(const duo_layer_desc* desc, const duo_kv_state* st, const void* q,
+                                   void* out, duo_stream_t stream);
+
+/*
  * duo_check_status -- synchronise `stream`, copy the state's device status
  * word to *host_status and return DUO_ERR_DEVICE if any bit is set.
  * The only entry point that blocks.
