@@ -6,10 +6,12 @@
 Default workload ``mha_decode_32k``: a Llama-2-7B-shaped MHA attention layer
 (32 heads, head_dim 128, bf16, batch 1), 8 of 32 heads retrieval (chosen by
 seed), sink 16 / recent 64, context 32,768 tokens, one token appended and
-attended per decode step.  A step is one pass of the path: duo_append_kv then
-duo_decode_attn (both caches, both head types, output concatenated in model
-head order).  Inputs are resident in HBM before timing starts; L2 is flushed
-(a 256 MiB write) before every timed step, outside the timed interval.
+attended per decode step.  A step is one pass of the path: duo_decode_step,
+the one-launch form of duo_append_kv + duo_decode_attn (both caches, both
+head types, output concatenated in model head order), for each of 4 layers
+with their own caches, back to back as in a forward pass; the value is per
+layer.  Inputs are resident in HBM before timing starts; the 4 layers'
+caches (540 MB) exceed the 126 MB L2, so nothing is flushed between steps.
 
 Other workloads: gqa_decode_128k, gqa_decode_1m (Llama-3-8B-shaped GQA, 4 of
 8 KV heads retrieval), batch64_paged_decode (64 sequences, lengths U[4096,
@@ -67,6 +69,29 @@ def _peaks():
         return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
     except (OSError, KeyError, ValueError):
         return 6650.0, 1590.0, "fallback"
+
+
+def _traffic(kernel: str, workload: str):
+    """DRAM bytes (read + write) per launch of `kernel` on `workload` from the
+    committed ncu record profiles/traffic.json -- only while every source file
+    the record lists still has the recorded SHA-256 (a changed kernel has no
+    measured traffic until it is captured again)."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f).get(kernel)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("workload") != workload:
+        return None
+    for rel, digest in rec.get("source_sha256", {}).items():
+        try:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest() != digest:
+                    return None
+        except OSError:
+            return None
+    return int(rec["dram_bytes_read"] + rec["dram_bytes_write"])
 
 
 # ---------------------------------------------------------------------------
@@ -189,7 +214,8 @@ def _decode_setup(duo, wl, total_steps, seed=0):
     qs, ks, vs = S.decode_steps(sh, B, total_steps, seed=seed, sigma=sigma)
     torch.cuda.synchronize()
     return dict(sh=sh, desc=desc, caches=caches, ws=ws, qs=qs, ks=ks, vs=vs, lengths=lengths, B=B, R=R,
-                retrieval=retrieval, gate=gate, state=st, sigma=sigma)
+                retrieval=retrieval, gate=gate, state=st, sigma=sigma, table=table,
+                n_pages=n_pages if paged else 0)
 
 
 def _to_dev(a):
@@ -229,76 +255,94 @@ def _load_decode_state(caches, st, inv, R, sh, table):
 
 
 def _decode_bytes(sh, R, lengths_after):
-    """Algorithmic HBM bytes of one decode launch: every cached K/V row of
-    every retrieval head once, the ring rows of the streaming heads, q and out."""
+    """Algorithmic HBM bytes of one fused decode step: every cached K/V row of
+    every retrieval head once, the ring rows of the streaming heads, q and out,
+    and the new token's K/V rows read once and written once into the caches."""
     S_ = sh.n_kv_heads - R
     row = sh.head_dim * 2
     total = 0
     for L in lengths_after:
-        total += R * L * row * 2
-        total += S_ * min(L, sh.sink + sh.recent) * row * 2
+        total += R * (L - 1) * row * 2
+        total += S_ * (min(L, sh.sink + sh.recent) - 1) * row * 2
+        total += sh.n_kv_heads * row * 2 * 2
     total += len(lengths_after) * sh.n_q_heads * sh.head_dim * 2 * 2
     return total
 
 
+def _replicate_layers(duo, env, n_layers):
+    """n_layers independent caches of the same shape, each a device copy of the
+    seeded state (the layers of one model), each with its own workspace."""
+    import torch
+    first = env["caches"]
+    layers = [(first, env["ws"])]
+    for _ in range(n_layers - 1):
+        c = duo.LayerCaches(env["desc"], first.capacity, env.get("table"), env.get("n_pages", 0))
+        for name in ("k_full", "v_full", "k_ring", "v_ring", "ring_pos", "seq_len"):
+            getattr(c, name).copy_(getattr(first, name))
+        layers.append((c, duo.Workspace(env["desc"], duo.OP_DECODE, c.capacity)))
+    torch.cuda.synchronize()
+    return layers
+
+
 def run_decode(args, wl, world, rank):
+    """Decode steps over `layers` layers: per step, every layer's
+    duo_decode_step (append + attend, one launch) runs back to back as in a
+    model's forward pass.  Each layer has its own caches, so a step streams
+    layers x (retrieval cache) bytes -- more than the 126 MB L2 -- and no
+    flush is needed between steps."""
     import torch
     from head_split_kv_b200 import duo
-    steps, warm = args.steps, args.warmup
+    steps, warm, nl = args.steps, args.warmup, args.layers
     total = warm + steps
     # capacity for the warm-up, the timed steps and the end-to-end steps
     env = _decode_setup(duo, wl, max(total + 32, wl["steps"]) + 1)
-    sh, desc, caches, ws, B, R = env["sh"], env["desc"], env["caches"], env["ws"], env["B"], env["R"]
+    sh, desc, B, R = env["sh"], env["desc"], env["B"], env["R"]
+    layers = _replicate_layers(duo, env, nl)
     qd = [_to_dev(env["qs"][i]) for i in range(total)]
     kd = [_to_dev(env["ks"][i][:, None]) for i in range(total)]
     vd = [_to_dev(env["vs"][i][:, None]) for i in range(total)]
     out = torch.empty_like(qd[0])
-    flush = torch.empty(1 << 30, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
     sp = int(stream.cuda_stream)
 
     def step(i):
-        duo.append_kv(desc, caches.state, kd[i], vd[i], 1, sp)
-        duo.decode_attn(desc, caches.state, qd[i], out, ws.ptr, ws.nbytes, sp)
+        for caches, ws in layers:
+            duo.decode_step(desc, caches.state, qd[i], kd[i], vd[i], out, ws.ptr, ws.nbytes, sp)
 
     for i in range(warm):
-        flush.zero_()
         step(i)
     torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     lengths_seen = []
     base = env["lengths"] + warm
     _barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(int(os.environ.get("LOCAL_RANK", "0"))) as clk:
         for j in range(steps):
-            flush.zero_()
-            e0, e1, e2 = ev[j]
+            e0, e1 = ev[j]
             e0.record(stream)
-            duo.append_kv(desc, caches.state, kd[warm + j], vd[warm + j], 1, sp)
+            step(warm + j)
             e1.record(stream)
-            duo.decode_attn(desc, caches.state, qd[warm + j], out, ws.ptr, ws.nbytes, sp)
-            e2.record(stream)
             lengths_seen.append(base + j + 1)
         torch.cuda.synchronize()
     _barrier(world)
-    step_ms = [e0.elapsed_time(e2) for e0, _, e2 in ev]
-    dec_ms = [e1.elapsed_time(e2) for _, e1, e2 in ev]
-    app_ms = [e0.elapsed_time(e1) for e0, e1, _ in ev]
+    # one launch per layer and step (append fused into the decode kernel)
+    step_ms = [e0.elapsed_time(e1) for e0, e1 in ev]
+    dec_ms = [t / nl for t in step_ms]
     total_ms = _max_over_ranks(sum(step_ms), world)
-    st_code = duo.check_status(caches.state)
-    if st_code:
-        raise RuntimeError(f"device status 0x{st_code:x} after the timed steps")
+    for caches, _ in layers:
+        st_code = duo.check_status(caches.state)
+        if st_code:
+            raise RuntimeError(f"device status 0x{st_code:x} after the timed steps")
 
     # end to end through the public API with host buffers
-    e2e = _decode_e2e(duo, env, args, world)
+    e2e = _decode_e2e(duo, env, layers, args, world)
 
     hbm, _, peak_kind = _peaks()
     bytes_per_launch = statistics.mean(_decode_bytes(sh, R, L) for L in lengths_seen)
     dec_avg_s = statistics.mean(dec_ms) * 1e-3
     achieved = bytes_per_launch / dec_avg_s / 1e9
-    us_step = total_ms * 1e3 / (steps * world)
+    us_step = total_ms * 1e3 / (steps * nl * world)
     res = {
         "metric": METRIC, "value": round(us_step, 3), "unit": "us/step/layer", "n_gpus": world, "steps": steps,
         "warmup": warm, "ms_per_step": round(total_ms / steps, 6), "higher_is_better": False, "scaling": "weak",
@@ -306,15 +350,17 @@ def run_decode(args, wl, world, rank):
         "config": {"workload": args.workload, "batch": B, "n_q_heads": sh.n_q_heads, "n_kv_heads": sh.n_kv_heads,
                    "head_dim": sh.head_dim, "n_retrieval": R, "sink": sh.sink, "recent": sh.recent,
                    "context": [int(env["lengths"].min()), int(env["lengths"].max())],
-                   "paged": bool(wl.get("paged", False)), "parallelism": f"replicas{world}",
-                   "l2": "flushed (1 GiB write) before every timed step, outside the timed interval"},
+                   "paged": bool(wl.get("paged", False)), "layers_per_step": nl,
+                   "parallelism": f"replicas{world}",
+                   "l2": f"not flushed: inputs larger than L2 (each step streams {nl} layers' caches, "
+                         f"{nl * bytes_per_launch / 1e6:.0f} MB > 126 MB)"},
         "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": round(achieved, 1), "peak": hbm,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / hbm, 4),
-                     "traffic": None, "algorithmic_bytes_per_launch": int(bytes_per_launch),
-                     "decode_us": round(statistics.mean(dec_ms) * 1e3, 3),
-                     "append_us": round(statistics.mean(app_ms) * 1e3, 3)},
+                     "traffic": _traffic("decode_kernel", args.workload),
+                     "algorithmic_bytes_per_launch": int(bytes_per_launch),
+                     "kernel_us": round(statistics.mean(dec_ms) * 1e3, 3)},
         "e2e": e2e,
-        "gpu_launches": 2 * steps,
+        "gpu_launches": steps * nl,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -322,44 +368,48 @@ def run_decode(args, wl, world, rank):
     return res
 
 
-def _decode_e2e(duo, env, args, world):
-    """Same steps through the binding with pinned host buffers: per step the
-    new token's q/k/v go host->device and the output comes back."""
+def _decode_e2e(duo, env, layers, args, world):
+    """The same steps through the binding with pinned host buffers: per step
+    and layer the new token's q/k/v go host->device and the output comes back
+    device->host, all inside the timed interval."""
     import torch
-    sh, desc, caches, ws, B = env["sh"], env["desc"], env["caches"], env["ws"], env["B"]
+    desc = env["desc"]
+    nl = len(layers)
     n = min(args.steps, 32)
-    h_q = [torch.from_numpy(env["qs"][i].view(np.int16)).view(torch.bfloat16).pin_memory() for i in range(n)]
-    h_k = [torch.from_numpy(env["ks"][i][:, None].copy().view(np.int16)).view(torch.bfloat16).pin_memory()
-           for i in range(n)]
-    h_v = [torch.from_numpy(env["vs"][i][:, None].copy().view(np.int16)).view(torch.bfloat16).pin_memory()
-           for i in range(n)]
-    h_out = torch.empty_like(h_q[0]).pin_memory()
-    dq, dk, dv = torch.empty_like(h_q[0], device="cuda"), torch.empty_like(h_k[0], device="cuda"), \
-        torch.empty_like(h_v[0], device="cuda")
-    dout = torch.empty_like(dq)
+
+    def pinned(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
+
+    h_q = [pinned(env["qs"][i]) for i in range(n)]
+    h_k = [pinned(env["ks"][i][:, None]) for i in range(n)]
+    h_v = [pinned(env["vs"][i][:, None]) for i in range(n)]
+    h_out = [torch.empty_like(h_q[0]).pin_memory() for _ in range(nl)]
+    dq = [torch.empty_like(h_q[0], device="cuda") for _ in range(nl)]
+    dk = [torch.empty_like(h_k[0], device="cuda") for _ in range(nl)]
+    dv = [torch.empty_like(h_v[0], device="cuda") for _ in range(nl)]
+    dout = [torch.empty_like(dq[0]) for _ in range(nl)]
     stream = torch.cuda.current_stream()
     sp = int(stream.cuda_stream)
-    flush = torch.empty(1 << 30, dtype=torch.uint8, device="cuda")
     times = []
     _barrier(world)
+    torch.cuda.synchronize()
     for i in range(n):
-        flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        dq.copy_(h_q[i], non_blocking=True)
-        dk.copy_(h_k[i], non_blocking=True)
-        dv.copy_(h_v[i], non_blocking=True)
-        duo.append_kv(desc, caches.state, dk, dv, 1, sp)
-        duo.decode_attn(desc, caches.state, dq, dout, ws.ptr, ws.nbytes, sp)
-        h_out.copy_(dout, non_blocking=True)
+        for l, (caches, ws) in enumerate(layers):
+            dq[l].copy_(h_q[i], non_blocking=True)
+            dk[l].copy_(h_k[i], non_blocking=True)
+            dv[l].copy_(h_v[i], non_blocking=True)
+            duo.decode_step(desc, caches.state, dq[l], dk[l], dv[l], dout[l], ws.ptr, ws.nbytes, sp)
+            h_out[l].copy_(dout[l], non_blocking=True)
         e1.record(stream)
         times.append((e0, e1))
     torch.cuda.synchronize()
     _barrier(world)
     tot = _max_over_ranks(sum(a.elapsed_time(b) for a, b in times), world)
     h2d = (h_q[0].numel() + h_k[0].numel() + h_v[0].numel()) * 2
-    return {"value": round(tot * 1e3 / (n * world), 3), "unit": "us/step/layer", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": h_out.numel() * 2, "steps": n}
+    return {"value": round(tot * 1e3 / (n * nl * world), 3), "unit": "us/step/layer", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": h_out[0].numel() * 2, "steps": n, "note": "bytes per layer and step"}
 
 
 def _decode_cpu_baseline(env, budget_s=15.0):
@@ -487,7 +537,7 @@ def run_prefill(args, wl, world, rank, steps=None, warmup=None):
                    "l2": "flushed (1 GiB write) before every timed chunk, outside the timed interval"},
         "roofline": {"bound": "tensor", "kernel": "prefill_tc_kernel", "achieved": round(achieved, 1),
                      "peak": tf_peak, "peak_kind": peak_kind + " (burst; sustained 1381.5)", "unit": "TFLOP/s",
-                     "frac": round(achieved / tf_peak, 4), "traffic": None,
+                     "frac": round(achieved / tf_peak, 4), "traffic": _traffic("prefill_tc_kernel", wl["name"]),
                      "algorithmic_tflop_total": round(sum(flops) / 1e12, 3),
                      "prefill_ms_total": round(sum(pre_ms), 3), "append_ms_total": round(sum(step_ms) - sum(pre_ms), 3),
                      "per_chunk_ms": [round(x, 3) for x in pre_ms]},
@@ -552,6 +602,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the pre-fill measurement of a decode run")
+    ap.add_argument("--layers", type=int, default=4,
+                    help="decode: layers per step, each with its own caches (their total exceeds L2)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
