@@ -27,6 +27,12 @@
 // are merged at the end.  With several splits, each CTA stores (m, l, o) to
 // the workspace and the last CTA of the (b, r) pair -- found with an atomic
 // ticket, never a wait -- combines them and writes the output.
+//
+// duo_decode_step runs the same kernel with the append fused in: the CTA
+// whose rows include the new token's position splices the token into its
+// shared-memory tile straight from the call's k/v inputs and stores it into
+// the cache (full-cache row or ring slot), and the last CTA of the grid
+// advances seq_len, so one launch does duo_append_kv(T = 1) + decode.
 #include "common.cuh"
 #include "internal.h"
 
@@ -45,6 +51,11 @@ struct DecodeArgs {
     uint32_t* ticket;    // [B*R]
     int nsplit;
     int n_ret_units;     // B * R * nsplit
+    // Fused append (duo_decode_step): the new token's K/V rows [B][Hkv][D];
+    // NULL for plain decode.
+    const void* k_new;
+    const void* v_new;
+    uint32_t* grid_ticket;  // one state counter word: the last CTA advances seq_len
 };
 
 template <typename T, int D>
@@ -133,7 +144,28 @@ __global__ void __launch_bounds__((consumer_warps(G) + 1) * 32, 2)
         slot = a.R + u % a.S;
         b = u / a.S;
     }
-    int len = c.seq_len[b];
+    // With a fused append the new token (position L0 = seq_len[b]) goes to
+    // full-cache row L0 or ring slot ring_slot(L0) -- `new_row` -- and is read
+    // from k_new / v_new; every other row comes from the caches.
+    const bool fused = d.k_new != nullptr;
+    const int L0 = c.seq_len[b];
+    int len = L0;
+    int new_row = -1;
+    const T* kn = nullptr;
+    const T* vn = nullptr;
+    if (fused) {
+        kn = static_cast<const T*>(d.k_new) + ((size_t)b * a.Hkv + a.kv_head[slot]) * D;
+        vn = static_cast<const T*>(d.v_new) + ((size_t)b * a.Hkv + a.kv_head[slot]) * D;
+        if (L0 < 0) {
+            if (threadIdx.x == 0) atomicOr(c.status, DUO_DEV_BAD_LENGTH);
+            len = 0;
+        } else if (retrieval && L0 >= a.capacity) {
+            if (threadIdx.x == 0 && split == 0) atomicOr(c.status, DUO_DEV_FULL_CACHE_OVERFLOW);
+        } else {
+            new_row = retrieval ? L0 : ring_slot(L0, a.sink, a.recent);
+            len = L0 + 1;
+        }
+    }
     int row_begin = 0, row_end = 0;
     const T* k_base;
     const T* v_base;
@@ -171,6 +203,41 @@ __global__ void __launch_bounds__((consumer_warps(G) + 1) * 32, 2)
     }
     __syncthreads();
 
+    // the CTA that covers the new token's row stores it into its cache
+    const bool owns_new = new_row >= 0 && (!retrieval || (new_row >= row_begin && new_row < row_end));
+    if (warp == NW && owns_new) {
+        T* dk = nullptr;
+        T* dv = nullptr;
+        if (!retrieval) {
+            const size_t off = (((size_t)b * a.S + (slot - a.R)) * a.W + new_row) * D;
+            dk = static_cast<T*>(c.k_ring) + off;
+            dv = static_cast<T*>(c.v_ring) + off;
+            if (slot == a.R && lane == 0) c.ring_pos[(size_t)b * a.W + new_row] = L0;
+        } else if (!PAGED) {
+            const size_t off = (((size_t)b * a.R + slot) * a.capacity + new_row) * D;
+            dk = static_cast<T*>(c.k_full) + off;
+            dv = static_cast<T*>(c.v_full) + off;
+        } else {
+            const int pg = c.page_table[(size_t)b * a.max_pages + new_row / kTile];
+            if (pg >= 0 && pg < a.n_pages) {
+                const size_t off = (((size_t)pg * a.R + slot) * kTile + new_row % kTile) * D;
+                dk = static_cast<T*>(c.k_full) + off;
+                dv = static_cast<T*>(c.v_full) + off;
+            } else if (lane == 0) {
+                atomicOr(c.status, DUO_DEV_BAD_PAGE);
+            }
+        }
+        if (dk) {
+            constexpr int kPieces = C::kRowBytes / 16;
+            for (int i = lane; i < 2 * kPieces; i += 32) {
+                if (i < kPieces)
+                    reinterpret_cast<uint4*>(dk)[i] = reinterpret_cast<const uint4*>(kn)[i];
+                else
+                    reinterpret_cast<uint4*>(dv)[i - kPieces] = reinterpret_cast<const uint4*>(vn)[i - kPieces];
+            }
+        }
+    }
+
     if (warp == NW) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
@@ -197,10 +264,28 @@ __global__ void __launch_bounds__((consumer_warps(G) + 1) * 32, 2)
                     vs = v_base + (size_t)r0 * D;
                 }
                 s_tile_n[st] = ok ? n : 0;
-                if (ok) {
+                T* dK = sK + (size_t)st * kTile * D;
+                T* dV = sV + (size_t)st * kTile * D;
+                if (ok && new_row >= r0 && new_row < r0 + n) {
+                    // splice: cached rows before, the new row from k_new / v_new, cached rows after
+                    const int nb = new_row - r0, na = n - nb - 1;
                     mbar_arrive_expect_tx(&full_bar[st], 2 * bytes);
-                    bulk_g2s(sK + (size_t)st * kTile * D, ks, bytes, &full_bar[st]);
-                    bulk_g2s(sV + (size_t)st * kTile * D, vs, bytes, &full_bar[st]);
+                    if (nb > 0) {
+                        bulk_g2s(dK, ks, (uint32_t)nb * C::kRowBytes, &full_bar[st]);
+                        bulk_g2s(dV, vs, (uint32_t)nb * C::kRowBytes, &full_bar[st]);
+                    }
+                    bulk_g2s(dK + (size_t)nb * D, kn, C::kRowBytes, &full_bar[st]);
+                    bulk_g2s(dV + (size_t)nb * D, vn, C::kRowBytes, &full_bar[st]);
+                    if (na > 0) {
+                        bulk_g2s(dK + (size_t)(nb + 1) * D, ks + (size_t)(nb + 1) * D, (uint32_t)na * C::kRowBytes,
+                                 &full_bar[st]);
+                        bulk_g2s(dV + (size_t)(nb + 1) * D, vs + (size_t)(nb + 1) * D, (uint32_t)na * C::kRowBytes,
+                                 &full_bar[st]);
+                    }
+                } else if (ok) {
+                    mbar_arrive_expect_tx(&full_bar[st], 2 * bytes);
+                    bulk_g2s(dK, ks, bytes, &full_bar[st]);
+                    bulk_g2s(dV, vs, bytes, &full_bar[st]);
                 } else {
                     mbar_arrive(&full_bar[st]);  // an empty tile: every key of it is masked
                 }
@@ -359,6 +444,21 @@ __global__ void __launch_bounds__((consumer_warps(G) + 1) * 32, 2)
     }
     __syncthreads();
 
+    // With a fused append, the last CTA of the grid to finish advances every
+    // sequence's length; each CTA read seq_len before taking its ticket.
+    auto grid_done = [&]() {
+        if (fused && threadIdx.x == 0) {
+            __threadfence();
+            const unsigned tk = atomicAdd(d.grid_ticket, 1u);
+            if (tk == gridDim.x - 1) {
+                __threadfence();
+                for (int bb = 0; bb < a.B; ++bb) c.seq_len[bb] += 1;
+                *d.grid_ticket = 0u;
+                __threadfence();
+            }
+        }
+    };
+
     T* outp = static_cast<T*>(d.out) + ((size_t)b * a.Hq + a.q_head0[slot]) * D;
     if (!retrieval || d.nsplit == 1) {
         for (int i = threadIdx.x; i < G * D; i += kThreads) {
@@ -367,6 +467,7 @@ __global__ void __launch_bounds__((consumer_warps(G) + 1) * 32, 2)
             const float v = L > 0.f ? cta[g * STRIDE + 4 + e] / L : 0.f;
             outp[(size_t)g * D + e] = Elem<T>::from_f32(v);
         }
+        grid_done();
         return;
     }
 
@@ -381,7 +482,10 @@ __global__ void __launch_bounds__((consumer_warps(G) + 1) * 32, 2)
         *s_flag = (tk == (unsigned)d.nsplit - 1);
     }
     __syncthreads();
-    if (!*s_flag) return;
+    if (!*s_flag) {
+        grid_done();
+        return;
+    }
     __threadfence();
     // This CTA is the last of its (b, r) pair: every split's record is in
     // global memory.  (1) m and l of all splits into shared memory, (2) the
@@ -443,6 +547,7 @@ __global__ void __launch_bounds__((consumer_warps(G) + 1) * 32, 2)
         outp[i] = Elem<T>::from_f32(v * s_inv[i / D]);
     }
     if (threadIdx.x == 0) d.ticket[pair] = 0u;  // leave the workspace ready for the next call
+    grid_done();
 }
 
 template <typename T, int D, int G, bool PAGED>
@@ -480,8 +585,11 @@ cudaError_t launch_d(const LayerArgs& a, const CacheArgs& c, const DecodeArgs& d
 }  // namespace
 
 cudaError_t launch_decode(const LayerArgs& a, const CacheArgs& c, const DecodePlan& plan, const void* q, void* out,
-                          void* workspace, cudaStream_t s) {
+                          void* workspace, cudaStream_t s, const void* k_new, const void* v_new) {
     DecodeArgs d;
+    d.k_new = k_new;
+    d.v_new = v_new;
+    d.grid_ticket = c.counters + 1;
     d.q = q;
     d.out = out;
     d.partial = static_cast<float*>(workspace);

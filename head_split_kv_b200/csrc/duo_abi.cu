@@ -324,6 +324,26 @@ duo_status duo_decode_attn(const duo_layer_desc* desc, const duo_kv_state* st, c
     return e == cudaSuccess ? ok() : cuda_fail(e, "duo_decode_attn");
 }
 
+duo_status duo_decode_step(const duo_layer_desc* desc, const duo_kv_state* st, const void* q, const void* k_new,
+                           const void* v_new, void* out, void* workspace, size_t ws_bytes, duo_stream_t stream) {
+    duo_status s = check_desc(desc);
+    if (s != DUO_OK) return s;
+    duo::LayerArgs a;
+    duo::CacheArgs c;
+    fill_args(desc, a);
+    if ((s = check_state(desc, st, a, c)) != DUO_OK) return s;
+    if (!q || !out || !k_new || !v_new) return fail(DUO_ERR_INVALID_ARG, "q / k_new / v_new / out is NULL");
+    if (!aligned16(q) || !aligned16(out) || !aligned16(k_new) || !aligned16(v_new))
+        return fail(DUO_ERR_INVALID_ARG, "q / k_new / v_new / out not 16-byte aligned");
+    const duo::DecodePlan plan = duo::decode_plan(a);
+    if (!workspace) return fail(DUO_ERR_INVALID_ARG, "workspace is NULL");
+    if (!aligned16(workspace)) return fail(DUO_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+    if (ws_bytes < plan.bytes)
+        return fail(DUO_ERR_CAPACITY, "workspace holds %zu bytes, decode needs %zu", ws_bytes, plan.bytes);
+    const cudaError_t e = duo::launch_decode(a, c, plan, q, out, workspace, (cudaStream_t)stream, k_new, v_new);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "duo_decode_step");
+}
+
 duo_status duo_prefill_chunk(const duo_layer_desc* desc, const duo_kv_state* st, const void* q, const void* k_chunk,
                              const void* v_chunk, int32_t C, void* out, void* workspace, size_t ws_bytes,
                              duo_stream_t stream) {

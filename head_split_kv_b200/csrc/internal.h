@@ -49,8 +49,10 @@ DecodePlan decode_plan(const LayerArgs& a);
 
 cudaError_t launch_append(const LayerArgs& a, const CacheArgs& c, const void* k_new, const void* v_new, int T,
                           cudaStream_t s);
+// k_new / v_new non-NULL: append the new token first (duo_decode_step).
 cudaError_t launch_decode(const LayerArgs& a, const CacheArgs& c, const DecodePlan& plan, const void* q, void* out,
-                          void* workspace, cudaStream_t s);
+                          void* workspace, cudaStream_t s, const void* k_new = nullptr,
+                          const void* v_new = nullptr);
 // CUDA-core attention: chunked pre-fill (mode 0) or gated mix (mode 1).
 cudaError_t launch_simt_attention(const LayerArgs& a, const CacheArgs* c, const float* alpha, const void* q,
                                   const void* k, const void* v, int n_tokens, void* out, int mode, cudaStream_t s);

@@ -141,6 +141,13 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
         : "memory");
 }
 
+// 2^x on the SFU (PTX ex2.approx, flush-to-zero; 2^-inf = +0)
+__device__ __forceinline__ float exp2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout: start,
@@ -301,9 +308,9 @@ __global__ void __launch_bounds__(kThreadsTC, 2)
             mbar_init(&v_full[i], 1);
             mbar_init(&v_empty[i], 1);
             mbar_init(&s_full[i], 1);
-            mbar_init(&s_empty[i], 128);
+            mbar_init(&s_empty[i], 4);
         }
-        mbar_init(p_full, 128);
+        mbar_init(p_full, 4);
         mbar_init(o_done, 1);
         fence_barrier_init();
     }
@@ -411,38 +418,52 @@ __global__ void __launch_bounds__(kThreadsTC, 2)
                 }
             }
             tc_fence_before();
-            mbar_arrive(&s_empty[st]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[st]);       // one arrival per warp
             const Tile t = tile_at(sc, j);
-            float mx = -INFINITY;
             if (t.mask) {
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
                     const int kp = t.src == SRC_RING ? (t.row + c < a.W ? sPos[t.row + c] : -1) : t.pos0 + c;
                     bool vis = kp >= 0 && kp <= P;
                     if (!sc.retrieval) vis = vis && (kp < a.sink || P - kp < a.recent);
-                    s[c] = vis ? s[c] * sl : -INFINITY;
-                    mx = fmaxf(mx, s[c]);
+                    if (!vis) s[c] = -INFINITY;
                 }
-            } else {
+            }
+            // row maximum of the raw scores (8 independent chains), then into
+            // the log2 domain: the scale is positive, so it commutes with max
+            float mx;
+            {
+                float m8[8];
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    s[c] *= sl;
-                    mx = fmaxf(mx, s[c]);
-                }
+                for (int i = 0; i < 8; ++i) m8[i] = s[i];
+#pragma unroll
+                for (int c = 8; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+                mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                           fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+                mx *= sl;
             }
             const float m_new = fmaxf(m_ref, mx);
             const bool need = m_new > m_ref + 8.f;            // lazy rescale threshold: 2^8
             const float m_use = need ? m_new : m_ref;
             const float m_safe = m_use == -INFINITY ? 0.f : m_use;
-            const float corr = need ? exp2f(m_ref - m_use) : 1.f;
-            // P is rounded to bf16 for the PV MMA; the row sum uses the same
-            // rounded values, so each output is a convex combination of V rows
-            float rs = 0.f;
+            const float corr = need ? exp2_approx(m_ref - m_use) : 1.f;
+            // p = 2^(s*scale*log2e - m), rounded once to bf16 for the PV MMA;
+            // the row sum uses the same rounded values, so each output is a
+            // convex combination of V rows
+            uint32_t pk[32];
+            float rs8[8];
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                s[c] = __bfloat162float(__float2bfloat16_rn(exp2f(s[c] - m_safe)));
-                rs += s[c];
+            for (int i = 0; i < 8; ++i) rs8[i] = 0.f;
+#pragma unroll
+            for (int c2 = 0; c2 < 32; ++c2) {
+                const float p0 = exp2_approx(fmaf(s[2 * c2], sl, -m_safe));
+                const float p1 = exp2_approx(fmaf(s[2 * c2 + 1], sl, -m_safe));
+                __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+                pk[c2] = *reinterpret_cast<uint32_t*>(&h);
+                rs8[c2 & 7] += bf16_lo(pk[c2]) + bf16_hi(pk[c2]);
             }
+            const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
             l_sum = l_sum * corr + rs;
             m_ref = m_use;
             if (j >= 1) {
@@ -464,18 +485,13 @@ __global__ void __launch_bounds__(kThreadsTC, 2)
             // P row -> shared memory, K-major with the 128-byte swizzle
             uint8_t* prow = smem + kOffP + row * 128;
 #pragma unroll
-            for (int c16 = 0; c16 < 8; ++c16) {
-                uint4 w;
-                __nv_bfloat162 h;
-                h = __floats2bfloat162_rn(s[8 * c16 + 0], s[8 * c16 + 1]); w.x = *reinterpret_cast<uint32_t*>(&h);
-                h = __floats2bfloat162_rn(s[8 * c16 + 2], s[8 * c16 + 3]); w.y = *reinterpret_cast<uint32_t*>(&h);
-                h = __floats2bfloat162_rn(s[8 * c16 + 4], s[8 * c16 + 5]); w.z = *reinterpret_cast<uint32_t*>(&h);
-                h = __floats2bfloat162_rn(s[8 * c16 + 6], s[8 * c16 + 7]); w.w = *reinterpret_cast<uint32_t*>(&h);
-                *reinterpret_cast<uint4*>(prow + ((c16 ^ (row & 7)) * 16)) = w;
-            }
+            for (int c16 = 0; c16 < 8; ++c16)
+                *reinterpret_cast<uint4*>(prow + ((c16 ^ (row & 7)) * 16)) =
+                    make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(p_full);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);               // one arrival per warp
         }
         // epilogue: O / l -> bf16
         if (ok && n >= 1) ok = __all_sync(0xffffffffu, mbar_wait(o_done, (n - 1) & 1, p.status));

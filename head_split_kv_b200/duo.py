@@ -82,6 +82,7 @@ _lib_decode = _fn("duo_decode_attn", ctypes.c_int, _DESC, _STATE, _P, _P, _P, ct
 _lib_prefill = _fn("duo_prefill_chunk", ctypes.c_int, _DESC, _STATE, _P, _P, _P, _I32, _P, _P, ctypes.c_size_t, _P)
 _lib_mix = _fn("duo_gated_mix", ctypes.c_int, _DESC, _P, _P, _P, _P, _I32, _P, _P)
 _lib_check = _fn("duo_check_status", ctypes.c_int, _STATE, ctypes.POINTER(_I32), _P)
+_lib_decode_step = _fn("duo_decode_step", ctypes.c_int, _DESC, _STATE, _P, _P, _P, _P, _P, ctypes.c_size_t, _P)
 _lib_decode_noalloc = _fn("duo_decode_attn_noalloc", ctypes.c_int, _DESC, _STATE, _P, _P, _P)
 NOALLOC_SCRATCH_BYTES = 2 << 20
 
@@ -183,6 +184,12 @@ def append_kv(desc, state: KVState, k_new, v_new, T: int, stream=None) -> None:
 def decode_attn(desc, state: KVState, q, out, workspace, ws_bytes: int, stream=None) -> None:
     _check(_lib_decode(ctypes.byref(desc), ctypes.byref(state), _ptr(q), _ptr(out), _ptr(workspace), ws_bytes,
                        _stream(stream)), "duo_decode_attn")
+
+
+def decode_step(desc, state: KVState, q, k_new, v_new, out, workspace, ws_bytes: int, stream=None) -> None:
+    """Append one token per sequence and attend, in one launch."""
+    _check(_lib_decode_step(ctypes.byref(desc), ctypes.byref(state), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out),
+                            _ptr(workspace), ws_bytes, _stream(stream)), "duo_decode_step")
 
 
 def decode_attn_noalloc(desc, state: KVState, q, out, stream=None) -> None:

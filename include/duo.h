@@ -258,6 +258,22 @@ duo_status duo_decode_attn(const duo_layer_desc* desc, const duo_kv_state* st, c
                            void* out, void* workspace, size_t ws_bytes, duo_stream_t stream);
 
 /*
+ * duo_decode_step -- duo_append_kv (T = 1) followed by duo_decode_attn, in one
+ * launch [Review S3 "Inference flow", decode: both caches take the new token,
+ * then each part of the head split attends against its own cache].
+ *
+ * k_new, v_new [B][Hkv][d] (the new token's K/V, head order per io_order);
+ * q, out, workspace as for duo_decode_attn.  Results, caches, ring_pos and
+ * seq_len end exactly as after the two separate calls: the CTA whose rows
+ * include the new position reads the token from k_new / v_new and stores it
+ * into the full cache or the ring, and the last CTA of the launch advances
+ * seq_len.  Uses state counter word 1.
+ * Errors: as duo_decode_attn.
+ */
+duo_status duo_decode_step(const duo_layer_desc* desc, const duo_kv_state* st, const void* q, const void* k_new,
+                           const void* v_new, void* out, void* workspace, size_t ws_bytes, duo_stream_t stream);
+
+/*
  * duo_prefill_chunk -- attention of a chunk of C prompt tokens per sequence
  * [Summary S2 "Chunked Pre-filling"; Review S3 "Inference flow", pre-fill:
  *  retrieval heads use full causal attention, streaming heads need linear

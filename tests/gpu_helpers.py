@@ -133,16 +133,20 @@ class Layer:
         self.duo.append_kv(self.desc, self.caches.state, kd, vd, T)
         self.oracle.append(k, v)
 
-    def decode(self, q: np.ndarray, k: np.ndarray, v: np.ndarray, check_oracle: bool = True):
-        """One step: q [B, Hq, d], k/v [B, Hkv, d] (model order).  Returns (gpu, oracle)."""
+    def decode(self, q: np.ndarray, k: np.ndarray, v: np.ndarray, check_oracle: bool = True, fused: bool = False):
+        """One step: q [B, Hq, d], k/v [B, Hkv, d] (model order).  Returns (gpu, oracle).
+        fused: duo_decode_step instead of duo_append_kv + duo_decode_attn."""
         t = torch()
         g = self.shape.group
         kd = to_dev(self.to_io(k[:, None], 2, 1))
         vd = to_dev(self.to_io(v[:, None], 2, 1))
         qd = to_dev(self.to_io(q, 1, g))
         out = t.empty_like(qd)
-        self.duo.append_kv(self.desc, self.caches.state, kd, vd, 1)
-        self.duo.decode_attn(self.desc, self.caches.state, qd, out, self.ws.ptr, self.ws.nbytes)
+        if fused:
+            self.duo.decode_step(self.desc, self.caches.state, qd, kd, vd, out, self.ws.ptr, self.ws.nbytes)
+        else:
+            self.duo.append_kv(self.desc, self.caches.state, kd, vd, 1)
+            self.duo.decode_attn(self.desc, self.caches.state, qd, out, self.ws.ptr, self.ws.nbytes)
         got = self.from_io(f64(out), 1, g)
         if check_oracle:
             want = self.oracle.decode(q, k, v)

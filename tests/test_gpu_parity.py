@@ -72,7 +72,7 @@ def test_append_overflow_sets_status_and_skips(duo):
 # ---------------------------------------------------------------------------
 
 def _decode_run(duo, sh, retrieval, lengths, steps, check_steps, capacity=None, paged=False, io_order=None,
-                sigma=None, seed=0):
+                sigma=None, seed=0, fused=False):
     lengths = np.asarray(lengths, dtype=np.int64)
     B = len(lengths)
     cap = int(lengths.max()) + steps if capacity is None else capacity
@@ -86,7 +86,7 @@ def _decode_run(duo, sh, retrieval, lengths, steps, check_steps, capacity=None, 
     errs = []
     for i in range(steps):
         check = i in check_steps
-        got, want = lay.decode(qs[i], ks[i], vs[i], check_oracle=check)
+        got, want = lay.decode(qs[i], ks[i], vs[i], check_oracle=check, fused=fused)
         if check:
             errs.append(assert_close(got, want, sh.dtype, f"step {i}"))
     assert lay.status() == 0
@@ -145,13 +145,74 @@ def test_decode_workspace_reuse_leaves_tickets_zero(duo):
 
 
 # ---------------------------------------------------------------------------
+# duo_decode_step: append + decode in one launch
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("L0", [0, 1, 15, 16, 17, 63, 64, 79, 80, 81, 4097])
+def test_decode_step_boundaries(duo, L0):
+    sh = S.LayerShape(8, 4, 128, "bf16")
+    lay, _ = _decode_run(duo, sh, [0, 3], [L0], 4, {0, 1, 2, 3}, fused=True)
+    lay.assert_caches_match()
+
+
+@pytest.mark.parametrize("io_order", [0, 1])
+def test_decode_step_mha(duo, io_order):
+    sh = S.LayerShape(32, 32, 128, "bf16")
+    lay, _ = _decode_run(duo, sh, S.retrieval_heads_by_seed(32, 8), [5000], 6, {0, 5}, io_order=io_order,
+                         fused=True)
+    lay.assert_caches_match()
+
+
+def test_decode_step_gqa_and_fp32(duo):
+    sh = S.LayerShape(32, 8, 128, "bf16")
+    lay, _ = _decode_run(duo, sh, S.retrieval_heads_by_seed(8, 4), [20011], 3, {2}, sigma=S.head_sigma(8),
+                         fused=True)
+    lay.assert_caches_match()
+    sh = S.LayerShape(8, 8, 64, "fp32")
+    lay, _ = _decode_run(duo, sh, [1, 5], [512], 16, set(range(16)), fused=True)
+    lay.assert_caches_match()
+
+
+def test_decode_step_paged_batch(duo):
+    sh = S.LayerShape(32, 32, 128, "bf16")
+    lengths = S.context_lengths(6, 1, 3000, seed=3)
+    lengths[0] = 0
+    lengths[1] = 63
+    lay, _ = _decode_run(duo, sh, S.retrieval_heads_by_seed(32, 8), lengths, 3, {0, 2}, paged=True, fused=True)
+    lay.assert_caches_match()
+
+
+def test_decode_step_mixed_with_separate_calls(duo):
+    sh = S.LayerShape(16, 4, 128, "bf16")
+    retrieval = [1, 2]
+    lay = Layer(duo, sh, retrieval, 2, capacity=700)
+    lay.load_state(S.decode_state(sh, retrieval, [300, 555], seed=4))
+    qs, ks, vs = S.decode_steps(sh, 2, 6, seed=4)
+    for i in range(6):
+        got, want = lay.decode(qs[i], ks[i], vs[i], fused=(i % 2 == 0))
+        assert_close(got, want, "bf16", f"step {i}")
+    lay.assert_caches_match()
+    assert lay.status() == 0
+
+
+def test_decode_step_full_cache_overflow(duo):
+    sh = S.LayerShape(4, 4, 64, "bf16")
+    lay = Layer(duo, sh, [0], 1, capacity=40)
+    lay.load_state(S.decode_state(sh, [0], [40], seed=6))
+    qs, ks, vs = S.decode_steps(sh, 1, 1, seed=6)
+    lay.decode(qs[0], ks[0], vs[0], check_oracle=False, fused=True)
+    assert lay.status() & duo.DEV_FULL_CACHE_OVERFLOW
+
+
+# ---------------------------------------------------------------------------
 # Full-size decode workloads in the launch configuration the bench times
 # ---------------------------------------------------------------------------
 
 @pytest.mark.slow
-def test_decode_mha_32k_full(duo):
+@pytest.mark.parametrize("fused", [False, True])
+def test_decode_mha_32k_full(duo, fused):
     sh = S.LayerShape(32, 32, 128, "bf16")
-    lay, errs = _decode_run(duo, sh, S.retrieval_heads_by_seed(32, 8), [32768], 256, {0, 1, 127, 255})
+    lay, errs = _decode_run(duo, sh, S.retrieval_heads_by_seed(32, 8), [32768], 256, {0, 1, 127, 255}, fused=fused)
     lay.assert_caches_match()
 
 
@@ -159,14 +220,14 @@ def test_decode_mha_32k_full(duo):
 @pytest.mark.parametrize("L0", [131072, 1048576])
 def test_decode_gqa_long_full(duo, L0):
     sh = S.LayerShape(32, 8, 128, "bf16")
-    _decode_run(duo, sh, S.retrieval_heads_by_seed(8, 4), [L0], 64, {0, 31, 63}, sigma=S.head_sigma(8))
+    _decode_run(duo, sh, S.retrieval_heads_by_seed(8, 4), [L0], 64, {0, 31, 63}, sigma=S.head_sigma(8), fused=True)
 
 
 @pytest.mark.slow
 def test_decode_batch64_paged_full(duo):
     sh = S.LayerShape(32, 32, 128, "bf16")
     lengths = S.context_lengths(64, 4096, 32768, seed=0)
-    _decode_run(duo, sh, S.retrieval_heads_by_seed(32, 8), lengths, 32, {0, 31}, paged=True)
+    _decode_run(duo, sh, S.retrieval_heads_by_seed(32, 8), lengths, 32, {0, 31}, paged=True, fused=True)
 
 
 # ---------------------------------------------------------------------------
