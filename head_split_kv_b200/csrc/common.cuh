@@ -98,6 +98,26 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, u
         : "memory");
 }
 
+// ------------------------------------------------- packed fp32 arithmetic
+
+// Two fp32 fused multiply-adds in one instruction (sm_100 f32x2 forms).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(*reinterpret_cast<unsigned long long*>(&d))
+        : "l"(*reinterpret_cast<unsigned long long*>(&a)), "l"(*reinterpret_cast<unsigned long long*>(&b)),
+          "l"(*reinterpret_cast<unsigned long long*>(&c)));
+    return d;
+}
+
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+    float2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;"
+        : "=l"(*reinterpret_cast<unsigned long long*>(&d))
+        : "l"(*reinterpret_cast<unsigned long long*>(&a)), "l"(*reinterpret_cast<unsigned long long*>(&b)));
+    return d;
+}
+
 // ------------------------------------------------------------ conversions
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -148,6 +168,40 @@ template <>
 __device__ __forceinline__ void load_row_f32<float, 4>(const float* p, float (&o)[4]) {
     const float4 a = *reinterpret_cast<const float4*>(p);
     o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+}
+
+// Loads 2*N consecutive elements as N fp32 pairs.
+template <typename T, int N>
+__device__ __forceinline__ void load_pairs_f32(const T* p, float2 (&out)[N]);
+
+template <>
+__device__ __forceinline__ void load_pairs_f32<__nv_bfloat16, 4>(const __nv_bfloat16* p, float2 (&o)[4]) {
+    const uint4 w = *reinterpret_cast<const uint4*>(p);
+    o[0] = make_float2(bf16_lo(w.x), bf16_hi(w.x));
+    o[1] = make_float2(bf16_lo(w.y), bf16_hi(w.y));
+    o[2] = make_float2(bf16_lo(w.z), bf16_hi(w.z));
+    o[3] = make_float2(bf16_lo(w.w), bf16_hi(w.w));
+}
+template <>
+__device__ __forceinline__ void load_pairs_f32<__nv_bfloat16, 2>(const __nv_bfloat16* p, float2 (&o)[2]) {
+    const uint2 w = *reinterpret_cast<const uint2*>(p);
+    o[0] = make_float2(bf16_lo(w.x), bf16_hi(w.x));
+    o[1] = make_float2(bf16_lo(w.y), bf16_hi(w.y));
+}
+template <>
+__device__ __forceinline__ void load_pairs_f32<float, 4>(const float* p, float2 (&o)[4]) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    const float4 b = *reinterpret_cast<const float4*>(p + 4);
+    o[0] = make_float2(a.x, a.y);
+    o[1] = make_float2(a.z, a.w);
+    o[2] = make_float2(b.x, b.y);
+    o[3] = make_float2(b.z, b.w);
+}
+template <>
+__device__ __forceinline__ void load_pairs_f32<float, 2>(const float* p, float2 (&o)[2]) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    o[0] = make_float2(a.x, a.y);
+    o[1] = make_float2(a.z, a.w);
 }
 
 // Stores N fp32 values as N consecutive elements (rounded once for bf16).

@@ -72,7 +72,7 @@ constexpr size_t decode_smem_bytes() {
     using C = Cfg<T, D>;
     size_t s = 2 * (size_t)C::kStages * C::kTileBytes;     // K and V stages
     s += (size_t)kTile * G * sizeof(float);                  // probabilities of one tile
-    s += 2 * C::kStages * sizeof(uint64_t) + 64;            // barriers, flag, rows per stage
+    s += (2 * C::kStages + 1) * sizeof(uint64_t) + 64;      // barriers, flag, rows per stage
     return s + 1024;                                        // alignment slack
 }
 
@@ -107,8 +107,14 @@ __device__ __forceinline__ float reduce_transposed(float (&v)[K], int lane) {
     return v[0];
 }
 
+// Registers per thread that let two CTAs share an SM: 65536 / (2 * threads),
+// rounded down to the allocation granularity of 8.
+__host__ __device__ constexpr int decode_max_regs(int G) {
+    return (65536 / (2 * (consumer_warps(G) + 1) * 32)) / 8 * 8;
+}
+
 template <typename T, int D, int G, bool PAGED>
-__global__ void __launch_bounds__((consumer_warps(G) + 1) * 32, 2)
+__global__ void __maxnreg__(decode_max_regs(G))
     decode_kernel(const LayerArgs a, const CacheArgs c, const DecodeArgs d) {
     using C = Cfg<T, D>;
     constexpr int EPL = C::kEPL;
@@ -126,7 +132,8 @@ __global__ void __launch_bounds__((consumer_warps(G) + 1) * 32, 2)
     float* sP = reinterpret_cast<float*>(smem + 2 * (size_t)STAGES * C::kTileBytes);  // [warp][KW keys][G]
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(sP + kTile * G);
     uint64_t* empty_bar = full_bar + STAGES;
-    int* s_flag = reinterpret_cast<int*>(empty_bar + STAGES);
+    uint64_t* comb_bar = empty_bar + STAGES;     // bulk loads of the split-K records
+    int* s_flag = reinterpret_cast<int*>(comb_bar + 1);
     int* s_tile_n = s_flag + 1;  // valid rows of each stage, written by the producer before its arrive
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -199,6 +206,7 @@ __global__ void __launch_bounds__((consumer_warps(G) + 1) * 32, 2)
             mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], NW);
         }
+        mbar_init(comb_bar, 1);
         fence_barrier_init();
     }
     __syncthreads();
@@ -488,20 +496,24 @@ __global__ void __launch_bounds__((consumer_warps(G) + 1) * 32, 2)
     }
     __threadfence();
     // This CTA is the last of its (b, r) pair: every split's record is in
-    // global memory.  (1) m and l of all splits into shared memory, (2) the
-    // per-head maximum and each split's weight, (3) warp w sums splits
-    // w, w + 5, ... with 16-byte loads all in flight, (4) the warps' sums are
-    // added and normalised.
+    // global memory (L2).  (1) m and l of all splits into shared memory,
+    // (2) the per-head maximum, each split's weight and 1 / L, (3) the
+    // records themselves stream into the free stage buffers with bulk copies
+    // (the TMA engine moves them at L2 bandwidth), a batch at a time, and each
+    // thread accumulates its outputs from shared memory.
     const float* all = d.partial + pair * d.nsplit * (size_t)G * STRIDE;
     const int ns = d.nsplit;
-    float* s_w = cta + G * STRIDE;            // [ns][G] weights
-    float* s_l = s_w + ns * G;                // [ns][G]
-    float* s_inv = s_l + ns * G;              // [G] 1 / L
-    // [kThreads / 32][G * D], written with float4 stores: 16-byte aligned
-    float* s_acc = s_inv + ((G + 3) & ~3) + ((4 - (((NW + 1) * G * STRIDE + 2 * ns * G) & 3)) & 3);
+    float* s_w = reinterpret_cast<float*>(sK);  // [ns][G] weights (the stage buffers are free)
+    float* s_l = s_w + ns * G;                  // [ns][G]
+    float* s_inv = s_l + ns * G;                // [G] 1 / L
+    constexpr int kRecFloats = G * STRIDE;      // one split's record
+    constexpr size_t kStageBytes = 2 * (size_t)STAGES * C::kTileBytes;
+    constexpr size_t kHead = ((2 * 128 * G + G) * sizeof(float) + 1023) / 1024 * 1024;
+    constexpr int kBatch = (int)((kStageBytes - kHead) / (kRecFloats * sizeof(float)));
+    static_assert(kBatch >= 1, "a split-K record must fit in the stage buffers");
+    float* stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sK) + kHead);
     for (int i = threadIdx.x; i < ns * G; i += kThreads) {
-        const int sp = i / G, g = i % G;
-        const float* rec = all + ((size_t)sp * G + g) * STRIDE;
+        const float* rec = all + (size_t)i * STRIDE;  // records of one split are [G][STRIDE]
         s_w[i] = __ldcg(rec);
         s_l[i] = __ldcg(rec + 1);
     }
@@ -519,32 +531,38 @@ __global__ void __launch_bounds__((consumer_warps(G) + 1) * 32, 2)
         s_inv[g] = L > 0.f ? 1.f / L : 0.f;
     }
     __syncthreads();
-    constexpr int kWarps = kThreads / 32;
-    constexpr int NV = G * D / 4;             // float4 pieces of one split's outputs
-    // everything above lives in the (free) K and V stage buffers
-    static_assert(((NW + 1) * G * (D + 4) + 2 * 128 * G + G + 8 + kWarps * G * D) * sizeof(float) <=
-                      2 * (size_t)STAGES * C::kTileBytes,
-                  "combine scratch exceeds the stage buffers");
-    for (int c = lane; c < NV; c += 32) {
-        const int g = (c * 4) / D, e = (c * 4) % D;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-        for (int sp = warp; sp < ns; sp += kWarps) {
-            const float w = s_w[sp * G + g];
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(all + ((size_t)sp * G + g) * STRIDE + 4 + e));
-            acc.x = fmaf(w, v.x, acc.x);
-            acc.y = fmaf(w, v.y, acc.y);
-            acc.z = fmaf(w, v.z, acc.z);
-            acc.w = fmaf(w, v.w, acc.w);
-        }
-        reinterpret_cast<float4*>(s_acc + (size_t)warp * G * D)[c] = acc;
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < G * D; i += kThreads) {
-        float v = 0.f;
+    constexpr int kOut = (G * D + kThreads - 1) / kThreads;  // outputs per thread
+    float acc[kOut];
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) v += s_acc[(size_t)w * G * D + i];
-        outp[i] = Elem<T>::from_f32(v * s_inv[i / D]);
+    for (int k = 0; k < kOut; ++k) acc[k] = 0.f;
+    uint32_t phase = 0;
+    for (int b0 = 0; b0 < ns; b0 += kBatch) {
+        const int nb = min(kBatch, ns - b0);
+        if (threadIdx.x == 0) {
+            const uint32_t bytes = (uint32_t)(nb * kRecFloats * sizeof(float));
+            fence_proxy_async_smem();  // earlier thread accesses of this space before the async-proxy writes
+            mbar_arrive_expect_tx(comb_bar, bytes);
+            bulk_g2s(stage, all + (size_t)b0 * kRecFloats, bytes, comb_bar);
+        }
+        if (!mbar_wait(comb_bar, phase, c.status)) break;
+        phase ^= 1;
+#pragma unroll
+        for (int k = 0; k < kOut; ++k) {
+            const int i = threadIdx.x + k * kThreads;
+            if (i < G * D) {
+                const int g = i / D, e = i % D;
+                float v = acc[k];
+                for (int sp = 0; sp < nb; ++sp)
+                    v = fmaf(s_w[(b0 + sp) * G + g], stage[sp * kRecFloats + g * STRIDE + 4 + e], v);
+                acc[k] = v;
+            }
+        }
+        __syncthreads();  // the next batch overwrites the staging area
+    }
+#pragma unroll
+    for (int k = 0; k < kOut; ++k) {
+        const int i = threadIdx.x + k * kThreads;
+        if (i < G * D) outp[i] = Elem<T>::from_f32(acc[k] * s_inv[i / D]);
     }
     if (threadIdx.x == 0) d.ticket[pair] = 0u;  // leave the workspace ready for the next call
     grid_done();
