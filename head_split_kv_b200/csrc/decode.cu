@@ -33,6 +33,8 @@
 // shared-memory tile straight from the call's k/v inputs and stores it into
 // the cache (full-cache row or ring slot), and the last CTA of the grid
 // advances seq_len, so one launch does duo_append_kv(T = 1) + decode.
+#include <utility>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -113,6 +115,172 @@ __host__ __device__ constexpr int decode_max_regs(int G) {
     return (65536 / (2 * (consumer_warps(G) + 1) * 32)) / 8 * 8;
 }
 
+// With a fused append every CTA reads its sequence's length once (thread 0,
+// broadcast through shared memory) and then takes a grid-wide ticket; the
+// CTA that takes the last ticket knows every CTA has read the old lengths and
+// advances them.  Taken at the start, this stays off the kernel's tail.
+__device__ __forceinline__ void length_ticket(const LayerArgs& a, const CacheArgs& c, const DecodeArgs& d) {
+    __threadfence();
+    const unsigned tk = atomicAdd(d.grid_ticket, 1u);
+    if (tk == gridDim.x - 1) {
+        __threadfence();
+        for (int bb = 0; bb < a.B; ++bb) c.seq_len[bb] += 1;
+        *d.grid_ticket = 0u;
+        __threadfence();
+    }
+}
+
+// The end of a decode CTA, shared by both decode kernels.  On entry every
+// consumer warp w has stored its online-softmax state for each query head g
+// of the group into sM[w][g][D + 4] (m, l, -, -, o[D]) and the CTA has
+// synchronised; the K/V stage buffers (kStageBytes from sM) are free.  Merges
+// the warp states, then writes the output (streaming heads, single split) or
+// stores the split-K record and, in the last CTA of the (sequence, head)
+// pair, combines all splits.
+template <typename T, int D, int G, int NW, int kThreads, size_t kStageBytes>
+__device__ __forceinline__ void decode_finish(float* sM, uint64_t* comb_bar, int* s_flag, const LayerArgs& a,
+                                              const CacheArgs& c, const DecodeArgs& d, int b, int slot, int split,
+                                              bool retrieval, bool fused) {
+    constexpr int STRIDE = D + 4;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // the CTA's combined state, in slot [NW] of sM
+    float* cta = sM + (size_t)NW * G * STRIDE;
+    for (int i = threadIdx.x; i < G * D; i += kThreads) {
+        const int g = i / D, e = i % D;
+        float M = kNegBig;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, sM[(w * G + g) * STRIDE]);
+        float L = 0.f, O = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            const float sc = exp2f(sM[(w * G + g) * STRIDE] - M);
+            L += sc * sM[(w * G + g) * STRIDE + 1];
+            O += sc * sM[(w * G + g) * STRIDE + 4 + e];
+        }
+        cta[g * STRIDE + 4 + e] = O;
+        if (e == 0) {
+            cta[g * STRIDE + 0] = M;
+            cta[g * STRIDE + 1] = L;
+        }
+    }
+    __syncthreads();
+
+    T* outp = static_cast<T*>(d.out) + ((size_t)b * a.Hq + a.q_head0[slot]) * D;
+    if (!retrieval || d.nsplit == 1) {
+        for (int i = threadIdx.x; i < G * D; i += kThreads) {
+            const int g = i / D, e = i % D;
+            const float L = cta[g * STRIDE + 1];
+            const float v = L > 0.f ? cta[g * STRIDE + 4 + e] / L : 0.f;
+            outp[(size_t)g * D + e] = Elem<T>::from_f32(v);
+        }
+        return;
+    }
+
+    // ------------------------------------------------ split-K combine
+    const size_t pair = (size_t)b * a.R + slot;
+    float* mine = d.partial + (pair * d.nsplit + split) * (size_t)G * STRIDE;
+    for (int i = threadIdx.x; i < G * STRIDE; i += kThreads) mine[i] = cta[i];
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const unsigned tk = atomicAdd(&d.ticket[pair], 1u);
+        *s_flag = (tk == (unsigned)d.nsplit - 1);
+    }
+    __syncthreads();
+    if (!*s_flag) {
+        return;
+    }
+    __threadfence();
+    // This CTA is the last of its (b, r) pair: every split's record is in
+    // global memory (L2).  (1) m and l of all splits into shared memory,
+    // (2) the per-head maximum, each split's weight and 1 / L, (3) the
+    // records themselves stream into the free stage buffers with bulk copies
+    // (the TMA engine moves them at L2 bandwidth), a batch at a time, and each
+    // thread accumulates its outputs from shared memory.
+    const float* all = d.partial + pair * d.nsplit * (size_t)G * STRIDE;
+    const int ns = d.nsplit;
+    float* s_w = sM;                            // [ns][G] weights (the stage buffers are free)
+    float* s_l = s_w + ns * G;                  // [ns][G]
+    float* s_inv = s_l + ns * G;                // [G] 1 / L
+    constexpr int kRecFloats = G * STRIDE;      // one split's record
+    constexpr size_t kHead = ((2 * 128 * G + G) * sizeof(float) + 1023) / 1024 * 1024;
+    constexpr int kBatch = (int)((kStageBytes - kHead) / (kRecFloats * sizeof(float)));
+    static_assert(kBatch >= 1, "a split-K record must fit in the stage buffers");
+    float* stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sM) + kHead);
+    uint32_t phase = 0;
+    const bool one_batch = ns <= kBatch;
+    if (one_batch) {
+        // every record fits: one bulk copy brings m, l and o of all splits
+        if (threadIdx.x == 0) {
+            const uint32_t bytes = (uint32_t)(ns * kRecFloats * sizeof(float));
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(comb_bar, bytes);
+            bulk_g2s(stage, all, bytes, comb_bar);
+        }
+        if (!mbar_wait(comb_bar, phase, c.status)) return;
+        phase ^= 1;
+        for (int i = threadIdx.x; i < ns * G; i += kThreads) {
+            s_w[i] = stage[(size_t)i * STRIDE];
+            s_l[i] = stage[(size_t)i * STRIDE + 1];
+        }
+    } else {
+        for (int i = threadIdx.x; i < ns * G; i += kThreads) {
+            const float* rec = all + (size_t)i * STRIDE;  // records of one split are [G][STRIDE]
+            s_w[i] = __ldcg(rec);
+            s_l[i] = __ldcg(rec + 1);
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < G) {
+        const int g = threadIdx.x;
+        float M = kNegBig;
+        for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, s_w[sp * G + g]);
+        float L = 0.f;
+        for (int sp = 0; sp < ns; ++sp) {
+            const float w = exp2f(s_w[sp * G + g] - M);
+            s_w[sp * G + g] = w;
+            L += w * s_l[sp * G + g];
+        }
+        s_inv[g] = L > 0.f ? 1.f / L : 0.f;
+    }
+    __syncthreads();
+    constexpr int kOut = (G * D + kThreads - 1) / kThreads;  // outputs per thread
+    float acc[kOut];
+#pragma unroll
+    for (int k = 0; k < kOut; ++k) acc[k] = 0.f;
+    for (int b0 = 0; b0 < ns; b0 += kBatch) {
+        const int nb = min(kBatch, ns - b0);
+        if (!one_batch && threadIdx.x == 0) {
+            const uint32_t bytes = (uint32_t)(nb * kRecFloats * sizeof(float));
+            fence_proxy_async_smem();  // earlier thread accesses of this space before the async-proxy writes
+            mbar_arrive_expect_tx(comb_bar, bytes);
+            bulk_g2s(stage, all + (size_t)b0 * kRecFloats, bytes, comb_bar);
+        }
+        if (!one_batch) {
+            if (!mbar_wait(comb_bar, phase, c.status)) break;
+            phase ^= 1;
+        }
+#pragma unroll
+        for (int k = 0; k < kOut; ++k) {
+            const int i = threadIdx.x + k * kThreads;
+            if (i < G * D) {
+                const int g = i / D, e = i % D;
+                float v = acc[k];
+                for (int sp = 0; sp < nb; ++sp)
+                    v = fmaf(s_w[(b0 + sp) * G + g], stage[sp * kRecFloats + g * STRIDE + 4 + e], v);
+                acc[k] = v;
+            }
+        }
+        __syncthreads();  // the next batch overwrites the staging area
+    }
+#pragma unroll
+    for (int k = 0; k < kOut; ++k) {
+        const int i = threadIdx.x + k * kThreads;
+        if (i < G * D) outp[i] = Elem<T>::from_f32(acc[k] * s_inv[i / D]);
+    }
+    if (threadIdx.x == 0) d.ticket[pair] = 0u;  // leave the workspace ready for the next call
+}
+
 template <typename T, int D, int G, bool PAGED>
 __global__ void __maxnreg__(decode_max_regs(G))
     decode_kernel(const LayerArgs a, const CacheArgs c, const DecodeArgs d) {
@@ -155,7 +323,15 @@ __global__ void __maxnreg__(decode_max_regs(G))
     // full-cache row L0 or ring slot ring_slot(L0) -- `new_row` -- and is read
     // from k_new / v_new; every other row comes from the caches.
     const bool fused = d.k_new != nullptr;
-    const int L0 = c.seq_len[b];
+    // launched with programmatic stream serialization: let the next launch's
+    // CTAs take SM slots as ours free, and wait for the previous grid before
+    // the first read of anything it may have written
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (threadIdx.x == 0) *s_flag = c.seq_len[b];
+    __syncthreads();
+    const int L0 = *s_flag;
+    if (fused && threadIdx.x == 0) length_ticket(a, c, d);
     int len = L0;
     int new_row = -1;
     const T* kn = nullptr;
@@ -430,142 +606,413 @@ __global__ void __maxnreg__(decode_max_regs(G))
         }
     }
     __syncthreads();
-    // the CTA's combined state, in slot [NW] of sM
-    float* cta = sM + (size_t)NW * G * STRIDE;
-    for (int i = threadIdx.x; i < G * D; i += kThreads) {
-        const int g = i / D, e = i % D;
-        float M = kNegBig;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) M = fmaxf(M, sM[(w * G + g) * STRIDE]);
-        float L = 0.f, O = 0.f;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) {
-            const float sc = exp2f(sM[(w * G + g) * STRIDE] - M);
-            L += sc * sM[(w * G + g) * STRIDE + 1];
-            O += sc * sM[(w * G + g) * STRIDE + 4 + e];
-        }
-        cta[g * STRIDE + 4 + e] = O;
-        if (e == 0) {
-            cta[g * STRIDE + 0] = M;
-            cta[g * STRIDE + 1] = L;
-        }
-    }
-    __syncthreads();
+    decode_finish<T, D, G, NW, kThreads, 2 * (size_t)STAGES * C::kTileBytes>(sM, comb_bar, s_flag, a, c, d, b, slot,
+                                                                         split, retrieval, fused);
+}
 
-    // With a fused append, the last CTA of the grid to finish advances every
-    // sequence's length; each CTA read seq_len before taking its ticket.
-    auto grid_done = [&]() {
-        if (fused && threadIdx.x == 0) {
-            __threadfence();
-            const unsigned tk = atomicAdd(d.grid_ticket, 1u);
-            if (tk == gridDim.x - 1) {
-                __threadfence();
-                for (int bb = 0; bb < a.B; ++bb) c.seq_len[bb] += 1;
-                *d.grid_ticket = 0u;
-                __threadfence();
-            }
-        }
-    };
+// ===========================================================================
+// Tensor-core decode consumer (bf16, head_dim 128).
+//
+// The same work units, pipeline and epilogue as decode_kernel, but the K/V
+// tiles arrive through TMA tensor copies with the 128-byte swizzle (two
+// 64-column boxes per tile), so warps read them conflict-free with ldmatrix,
+// and the contraction runs on mma.sync m16n8k16 (bf16 in, fp32 accumulate):
+// the G query heads of the group are the rows of the A operand, padded to 16.
+// Four consumer warps each take 16 keys of a 64-key tile:
+//   S (16 x 16) = Q K^T  -- 8 k-steps x 2 key blocks, K fragments by ldmatrix
+//   softmax on the lane's 4 scores (2 shuffles per row for the maximum)
+//   O (16 x 128) += P V  -- P reused in registers as the A fragment, V
+//                           fragments by ldmatrix.trans
+// For a group of 4 heads this is about a tenth of the instructions of the
+// CUDA-core loop, which makes the kernel bound by HBM instead of by issue.
+// With a fused append the new token's row is stored into its cache first and
+// the tile that holds it is then loaded from there (after a proxy fence).
+// ===========================================================================
 
-    T* outp = static_cast<T*>(d.out) + ((size_t)b * a.Hq + a.q_head0[slot]) * D;
-    if (!retrieval || d.nsplit == 1) {
-        for (int i = threadIdx.x; i < G * D; i += kThreads) {
-            const int g = i / D, e = i % D;
-            const float L = cta[g * STRIDE + 1];
-            const float v = L > 0.f ? cta[g * STRIDE + 4 + e] / L : 0.f;
-            outp[(size_t)g * D + e] = Elem<T>::from_f32(v);
-        }
-        grid_done();
+constexpr int kMmaWarps = 4;
+constexpr int kMmaThreads = (kMmaWarps + 1) * 32;
+constexpr int kMmaStages = 3;
+constexpr uint32_t kMmaTileBytes = kTile * 128 * 2;   // one K or V tile: two 8 KB swizzled halves
+
+constexpr size_t decode_mma_smem_bytes() {
+    return 2 * (size_t)kMmaStages * kMmaTileBytes + (2 * kMmaStages + 1) * sizeof(uint64_t) + 64;
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr)
+                 : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr)
+                 : "memory");
+}
+
+// D = A (16 x 16, rows 8..15 zero) * B (16 x 8) + C with C rows 8..15 zero;
+// returns the two accumulators of rows 0..7 this lane holds.
+__device__ __forceinline__ void mma_rows8(float& c0, float& c1, uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+    float d2, d3;
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%10, %11, %12, %13};"
+        : "=f"(c0), "=f"(c1), "=f"(d2), "=f"(d3)
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(0.f), "f"(0.f));
+}
+
+// byte offset of (row, 16-byte chunk c16 of the 256-byte row) in a tile made
+// of two [64 rows][128 B] boxes written by TMA with the 128-byte swizzle
+__device__ __forceinline__ uint32_t sw_off(int row, int c16) {
+    return (uint32_t)((c16 >> 3) * (kMmaTileBytes / 2) + row * 128 + (((c16 & 7) ^ (row & 7)) << 4));
+}
+
+template <int G, bool PAGED>
+__global__ void __maxnreg__(200)
+    decode_mma_kernel(const __grid_constant__ CUtensorMap tmKf, const __grid_constant__ CUtensorMap tmVf,
+                      const __grid_constant__ CUtensorMap tmKr, const __grid_constant__ CUtensorMap tmVr,
+                      const LayerArgs a, const CacheArgs c, const DecodeArgs d) {
+    using T = __nv_bfloat16;
+    constexpr int D = 128;
+    constexpr int STAGES = kMmaStages;
+    constexpr int NW = kMmaWarps;
+    constexpr int kThreads = kMmaThreads;
+    static_assert(G <= 8, "the group must fit the 8 live rows of an m16 tile");
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t* sKb = smem;
+    uint8_t* sVb = smem + (size_t)STAGES * kMmaTileBytes;
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + 2 * (size_t)STAGES * kMmaTileBytes);
+    uint64_t* empty_bar = full_bar + STAGES;
+    uint64_t* comb_bar = empty_bar + STAGES;
+    int* s_flag = reinterpret_cast<int*>(comb_bar + 1);
+    int* s_tile_n = s_flag + 1;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if ((smem_u32(smem) & 1023u) != 0) {  // the swizzled tiles need 1024-byte alignment
+        if (threadIdx.x == 0) atomicOr(c.status, DUO_DEV_BAD_LENGTH);
         return;
     }
 
-    // ------------------------------------------------ split-K combine
-    const size_t pair = (size_t)b * a.R + slot;
-    float* mine = d.partial + (pair * d.nsplit + split) * (size_t)G * STRIDE;
-    for (int i = threadIdx.x; i < G * STRIDE; i += kThreads) mine[i] = cta[i];
-    __threadfence();
+    // ---------------------------------------------------------- work unit
+    const bool retrieval = (int)blockIdx.x < d.n_ret_units;
+    int b, slot, split = 0;
+    if (retrieval) {
+        split = blockIdx.x % d.nsplit;
+        const int pair = blockIdx.x / d.nsplit;
+        slot = pair % a.R;
+        b = pair / a.R;
+    } else {
+        const int u = blockIdx.x - d.n_ret_units;
+        slot = a.R + u % a.S;
+        b = u / a.S;
+    }
+    const bool fused = d.k_new != nullptr;
+    // launched with programmatic stream serialization: let the next launch's
+    // CTAs take SM slots as ours free, and wait for the previous grid before
+    // the first read of anything it may have written
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (threadIdx.x == 0) *s_flag = c.seq_len[b];
     __syncthreads();
+    const int L0 = *s_flag;
+    if (fused && threadIdx.x == 0) length_ticket(a, c, d);
+    int len = L0;
+    int new_row = -1;
+    if (fused) {
+        if (L0 < 0) {
+            if (threadIdx.x == 0) atomicOr(c.status, DUO_DEV_BAD_LENGTH);
+            len = 0;
+        } else if (retrieval && L0 >= a.capacity) {
+            if (threadIdx.x == 0 && split == 0) atomicOr(c.status, DUO_DEV_FULL_CACHE_OVERFLOW);
+        } else {
+            new_row = retrieval ? L0 : ring_slot(L0, a.sink, a.recent);
+            len = L0 + 1;
+        }
+    }
+    int row_begin = 0, row_end = 0;
+    if (retrieval) {
+        if (len > a.capacity || len < 0) {
+            if (threadIdx.x == 0 && split == 0) atomicOr(c.status, DUO_DEV_BAD_LENGTH);
+            len = len < 0 ? 0 : a.capacity;
+        }
+        const int per = (len + d.nsplit - 1) / d.nsplit;
+        const int chunk = (per + kTile - 1) / kTile * kTile;
+        row_begin = min(len, split * chunk);
+        row_end = min(len, row_begin + chunk);
+    } else {
+        row_end = len < 0 ? 0 : min(len, a.W);
+    }
+    const int n_tiles = (row_end - row_begin + kTile - 1) / kTile;
+
     if (threadIdx.x == 0) {
-        const unsigned tk = atomicAdd(&d.ticket[pair], 1u);
-        *s_flag = (tk == (unsigned)d.nsplit - 1);
-    }
-    __syncthreads();
-    if (!*s_flag) {
-        grid_done();
-        return;
-    }
-    __threadfence();
-    // This CTA is the last of its (b, r) pair: every split's record is in
-    // global memory (L2).  (1) m and l of all splits into shared memory,
-    // (2) the per-head maximum, each split's weight and 1 / L, (3) the
-    // records themselves stream into the free stage buffers with bulk copies
-    // (the TMA engine moves them at L2 bandwidth), a batch at a time, and each
-    // thread accumulates its outputs from shared memory.
-    const float* all = d.partial + pair * d.nsplit * (size_t)G * STRIDE;
-    const int ns = d.nsplit;
-    float* s_w = reinterpret_cast<float*>(sK);  // [ns][G] weights (the stage buffers are free)
-    float* s_l = s_w + ns * G;                  // [ns][G]
-    float* s_inv = s_l + ns * G;                // [G] 1 / L
-    constexpr int kRecFloats = G * STRIDE;      // one split's record
-    constexpr size_t kStageBytes = 2 * (size_t)STAGES * C::kTileBytes;
-    constexpr size_t kHead = ((2 * 128 * G + G) * sizeof(float) + 1023) / 1024 * 1024;
-    constexpr int kBatch = (int)((kStageBytes - kHead) / (kRecFloats * sizeof(float)));
-    static_assert(kBatch >= 1, "a split-K record must fit in the stage buffers");
-    float* stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sK) + kHead);
-    for (int i = threadIdx.x; i < ns * G; i += kThreads) {
-        const float* rec = all + (size_t)i * STRIDE;  // records of one split are [G][STRIDE]
-        s_w[i] = __ldcg(rec);
-        s_l[i] = __ldcg(rec + 1);
-    }
-    __syncthreads();
-    if (threadIdx.x < G) {
-        const int g = threadIdx.x;
-        float M = kNegBig;
-        for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, s_w[sp * G + g]);
-        float L = 0.f;
-        for (int sp = 0; sp < ns; ++sp) {
-            const float w = exp2f(s_w[sp * G + g] - M);
-            s_w[sp * G + g] = w;
-            L += w * s_l[sp * G + g];
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], NW);
         }
-        s_inv[g] = L > 0.f ? 1.f / L : 0.f;
+        mbar_init(comb_bar, 1);
+        fence_barrier_init();
     }
     __syncthreads();
-    constexpr int kOut = (G * D + kThreads - 1) / kThreads;  // outputs per thread
-    float acc[kOut];
-#pragma unroll
-    for (int k = 0; k < kOut; ++k) acc[k] = 0.f;
-    uint32_t phase = 0;
-    for (int b0 = 0; b0 < ns; b0 += kBatch) {
-        const int nb = min(kBatch, ns - b0);
-        if (threadIdx.x == 0) {
-            const uint32_t bytes = (uint32_t)(nb * kRecFloats * sizeof(float));
-            fence_proxy_async_smem();  // earlier thread accesses of this space before the async-proxy writes
-            mbar_arrive_expect_tx(comb_bar, bytes);
-            bulk_g2s(stage, all + (size_t)b0 * kRecFloats, bytes, comb_bar);
+
+    if (warp == NW) {
+        // ------------------------------------------------------ producer
+        const bool owns_new = new_row >= 0 && (!retrieval || (new_row >= row_begin && new_row < row_end));
+        if (owns_new) {
+            // the new token goes into its cache first; the tile that holds it
+            // is then read back through TMA
+            const T* kn = static_cast<const T*>(d.k_new) + ((size_t)b * a.Hkv + a.kv_head[slot]) * D;
+            const T* vn = static_cast<const T*>(d.v_new) + ((size_t)b * a.Hkv + a.kv_head[slot]) * D;
+            T* dk = nullptr;
+            T* dv = nullptr;
+            if (!retrieval) {
+                const size_t off = (((size_t)b * a.S + (slot - a.R)) * a.W + new_row) * D;
+                dk = static_cast<T*>(c.k_ring) + off;
+                dv = static_cast<T*>(c.v_ring) + off;
+                if (slot == a.R && lane == 0) c.ring_pos[(size_t)b * a.W + new_row] = L0;
+            } else if (!PAGED) {
+                const size_t off = (((size_t)b * a.R + slot) * a.capacity + new_row) * D;
+                dk = static_cast<T*>(c.k_full) + off;
+                dv = static_cast<T*>(c.v_full) + off;
+            } else {
+                const int pg = c.page_table[(size_t)b * a.max_pages + new_row / kTile];
+                if (pg >= 0 && pg < a.n_pages) {
+                    const size_t off = (((size_t)pg * a.R + slot) * kTile + new_row % kTile) * D;
+                    dk = static_cast<T*>(c.k_full) + off;
+                    dv = static_cast<T*>(c.v_full) + off;
+                } else if (lane == 0) {
+                    atomicOr(c.status, DUO_DEV_BAD_PAGE);
+                }
+            }
+            if (dk) {
+                if (lane < 16)
+                    reinterpret_cast<uint4*>(dk)[lane] = reinterpret_cast<const uint4*>(kn)[lane];
+                else
+                    reinterpret_cast<uint4*>(dv)[lane - 16] = reinterpret_cast<const uint4*>(vn)[lane - 16];
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+            }
+            __syncwarp();
         }
-        if (!mbar_wait(comb_bar, phase, c.status)) break;
-        phase ^= 1;
-#pragma unroll
-        for (int k = 0; k < kOut; ++k) {
-            const int i = threadIdx.x + k * kThreads;
-            if (i < G * D) {
-                const int g = i / D, e = i % D;
-                float v = acc[k];
-                for (int sp = 0; sp < nb; ++sp)
-                    v = fmaf(s_w[(b0 + sp) * G + g], stage[sp * kRecFloats + g * STRIDE + 4 + e], v);
-                acc[k] = v;
+        if (lane == 0) {
+            const CUtensorMap* mk = retrieval ? &tmKf : &tmKr;
+            const CUtensorMap* mv = retrieval ? &tmVf : &tmVr;
+            prefetch_map(mk);
+            prefetch_map(mv);
+            const int z = retrieval ? b * a.R + slot : b * a.S + (slot - a.R);
+            for (int t = 0; t < n_tiles; ++t) {
+                const int st = t % STAGES, round = t / STAGES;
+                if (round > 0 && !mbar_wait(&empty_bar[st], (round - 1) & 1, c.status)) break;
+                const int r0 = row_begin + t * kTile;
+                const int n = min(kTile, row_end - r0);
+                int pg = 0;
+                bool ok = true;
+                if (PAGED && retrieval) {
+                    pg = c.page_table[(size_t)b * a.max_pages + r0 / kTile];
+                    if (pg < 0 || pg >= a.n_pages) {
+                        atomicOr(c.status, DUO_DEV_BAD_PAGE);
+                        ok = false;
+                    }
+                }
+                s_tile_n[st] = ok ? n : 0;
+                if (!ok) {
+                    mbar_arrive(&full_bar[st]);  // an empty tile: every key of it is masked
+                    continue;
+                }
+                mbar_arrive_expect_tx(&full_bar[st], 2 * kMmaTileBytes);
+                const uint32_t dk = smem_u32(sKb + (size_t)st * kMmaTileBytes);
+                const uint32_t dv = smem_u32(sVb + (size_t)st * kMmaTileBytes);
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t off = h * (kMmaTileBytes / 2);
+                    if (PAGED && retrieval) {
+                        tma_load_4d(dk + off, mk, 64 * h, 0, slot, pg, &full_bar[st]);
+                        tma_load_4d(dv + off, mv, 64 * h, 0, slot, pg, &full_bar[st]);
+                    } else {
+                        tma_load_3d(dk + off, mk, 64 * h, r0, z, &full_bar[st]);
+                        tma_load_3d(dv + off, mv, 64 * h, r0, z, &full_bar[st]);
+                    }
+                }
             }
         }
-        __syncthreads();  // the next batch overwrites the staging area
     }
+
+    // ------------------------------------------------------ consumers
+    const int row = lane >> 2;   // query head of the group for this lane (rows >= G are padding)
+    const int quad = lane & 3;
+    float o[16][2];
+    float m_run = kNegBig, l_run = 0.f;
+    if (warp < NW) {
+        uint32_t qa[8][2];
+        {
+            const bool row_ok = row < G;
+            const T* qp = static_cast<const T*>(d.q) + ((size_t)b * a.Hq + a.q_head0[slot] + (row_ok ? row : 0)) * D;
 #pragma unroll
-    for (int k = 0; k < kOut; ++k) {
-        const int i = threadIdx.x + k * kThreads;
-        if (i < G * D) outp[i] = Elem<T>::from_f32(acc[k] * s_inv[i / D]);
+            for (int ks = 0; ks < 8; ++ks) {
+                const int d0 = 16 * ks + 2 * quad;
+                qa[ks][0] = row_ok ? *reinterpret_cast<const uint32_t*>(qp + d0) : 0u;
+                qa[ks][1] = row_ok ? *reinterpret_cast<const uint32_t*>(qp + d0 + 8) : 0u;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = 0.f;
+        const float sl = a.scale * kLog2e;
+        const int key_base = warp * 16;
+        for (int t = 0; t < n_tiles; ++t) {
+            const int st = t % STAGES, round = t / STAGES;
+            if (!mbar_wait(&full_bar[st], round & 1, c.status)) break;
+            const int n = s_tile_n[st];
+            const uint32_t tK = smem_u32(sKb + (size_t)st * kMmaTileBytes);
+            uint8_t* tVp = sVb + (size_t)st * kMmaTileBytes;
+            const uint32_t tV = smem_u32(tVp);
+            const bool partial = n < key_base + 16;
+            if (partial) {
+                // V rows past the valid keys may hold anything: zero this warp's
+                // rows so that P = 0 meets finite V in the MMA
+                for (int i = lane; i < 16 * 16; i += 32) {
+                    const int key = key_base + (i >> 4), piece = i & 15;
+                    if (key >= n)
+                        *reinterpret_cast<uint4*>(tVp + (piece >> 3) * (kMmaTileBytes / 2) + key * 128 +
+                                                  (piece & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
+                }
+                __syncwarp();
+            }
+            // S = Q K^T for keys key_base .. key_base + 15
+            float s0[2] = {0.f, 0.f}, s1[2] = {0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const int key = key_base + (lane & 7) + ((lane >> 4) & 1) * 8;
+                const int c16 = 2 * ks + ((lane >> 3) & 1);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(tK + sw_off(key, c16), b0, b1, b2, b3);
+                mma_rows8(s0[0], s0[1], qa[ks][0], qa[ks][1], b0, b1);
+                mma_rows8(s1[0], s1[1], qa[ks][0], qa[ks][1], b2, b3);
+            }
+            // this lane's keys: key_base + 2 quad + {0, 1} and + 8
+            const int k0 = key_base + 2 * quad;
+            float sv[4] = {s0[0] * sl, s0[1] * sl, s1[0] * sl, s1[1] * sl};
+            const bool vk[4] = {k0 < n, k0 + 1 < n, k0 + 8 < n, k0 + 9 < n};
+            float mx = kNegBig;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) mx = vk[i] ? fmaxf(mx, sv[i]) : mx;
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float m_new = fmaxf(m_run, mx);
+            const float corr = exp2f(m_run - m_new);
+            // P rounded to bf16 for the PV MMA; the row sum uses the rounded values
+            __nv_bfloat162 p01 = __floats2bfloat162_rn(vk[0] ? exp2f(sv[0] - m_new) : 0.f,
+                                                       vk[1] ? exp2f(sv[1] - m_new) : 0.f);
+            __nv_bfloat162 p23 = __floats2bfloat162_rn(vk[2] ? exp2f(sv[2] - m_new) : 0.f,
+                                                       vk[3] ? exp2f(sv[3] - m_new) : 0.f);
+            const uint32_t pa0 = *reinterpret_cast<uint32_t*>(&p01);
+            const uint32_t pa1 = *reinterpret_cast<uint32_t*>(&p23);
+            l_run = l_run * corr + (bf16_lo(pa0) + bf16_hi(pa0)) + (bf16_lo(pa1) + bf16_hi(pa1));
+            m_run = m_new;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                o[j][0] *= corr;
+                o[j][1] *= corr;
+            }
+            // O += P V over the 16 keys, 8 pairs of 8-column blocks of d
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+                const int key = key_base + (lane & 7) + ((lane >> 3) & 1) * 8;
+                const int c16 = 2 * jj + (lane >> 4);
+                uint32_t r0, r1, r2, r3;
+                ldsm_x4_t(tV + sw_off(key, c16), r0, r1, r2, r3);
+                mma_rows8(o[2 * jj][0], o[2 * jj][1], pa0, pa1, r0, r1);
+                mma_rows8(o[2 * jj + 1][0], o[2 * jj + 1][1], pa0, pa1, r2, r3);
+            }
+            __syncwarp();
+            if (partial) fence_proxy_async_smem();  // the zero stores before the next TMA write
+            if (lane == 0) mbar_arrive(&empty_bar[st]);
+        }
+        l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+        l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
     }
-    if (threadIdx.x == 0) d.ticket[pair] = 0u;  // leave the workspace ready for the next call
-    grid_done();
+    __syncthreads();  // all tiles consumed: the stage buffers are free
+
+    // warp states -> sM[warp][g][STRIDE]: m, l, -, -, o[D]
+    constexpr int STRIDE = D + 4;
+    float* sM = reinterpret_cast<float*>(sKb);
+    if (warp < NW && row < G) {
+        float* dst = sM + ((size_t)warp * G + row) * STRIDE;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            dst[4 + 8 * j + 2 * quad] = o[j][0];
+            dst[4 + 8 * j + 2 * quad + 1] = o[j][1];
+        }
+        if (quad == 0) {
+            dst[0] = m_run;
+            dst[1] = l_run;
+        }
+    }
+    __syncthreads();
+    decode_finish<T, D, G, NW, kThreads, 2 * (size_t)STAGES * kMmaTileBytes>(sM, comb_bar, s_flag, a, c, d, b, slot,
+                                                                         split, retrieval, fused);
+}
+
+template <int G, bool PAGED>
+cudaError_t launch_mma_t(const LayerArgs& a, const CacheArgs& c, const DecodeArgs& d, int grid, cudaStream_t s) {
+    const uint64_t row = 128 * 2;
+    const uint32_t box3[3] = {64, (uint32_t)kTile, 1};
+    CUtensorMap mKf{}, mVf{}, mKr{}, mVr{};
+    bool have_f = false, have_r = false;
+    if (a.R > 0) {
+        if (PAGED) {
+            const uint64_t dims[4] = {128, (uint64_t)kTile, (uint64_t)a.R, (uint64_t)a.n_pages};
+            const uint64_t st[3] = {row, row * kTile, row * kTile * a.R};
+            const uint32_t box[4] = {64, (uint32_t)kTile, 1, 1};
+            if (!encode_tmap_bf16(&mKf, c.k_full, 4, dims, st, box) || !encode_tmap_bf16(&mVf, c.v_full, 4, dims, st, box))
+                return cudaErrorInvalidValue;
+        } else {
+            const uint64_t dims[3] = {128, (uint64_t)a.capacity, (uint64_t)a.B * a.R};
+            const uint64_t st[2] = {row, row * a.capacity};
+            if (!encode_tmap_bf16(&mKf, c.k_full, 3, dims, st, box3) || !encode_tmap_bf16(&mVf, c.v_full, 3, dims, st, box3))
+                return cudaErrorInvalidValue;
+        }
+        have_f = true;
+    }
+    if (a.S > 0) {
+        const uint64_t dims[3] = {128, (uint64_t)a.W, (uint64_t)a.B * a.S};
+        const uint64_t st[2] = {row, row * a.W};
+        if (!encode_tmap_bf16(&mKr, c.k_ring, 3, dims, st, box3) || !encode_tmap_bf16(&mVr, c.v_ring, 3, dims, st, box3))
+            return cudaErrorInvalidValue;
+        have_r = true;
+    }
+    if (!have_f) { mKf = mKr; mVf = mVr; }  // never read: there are no retrieval heads
+    if (!have_r) { mKr = mKf; mVr = mVf; }  // never read: there are no streaming heads
+    constexpr size_t smem = decode_mma_smem_bytes();
+    auto kern = decode_mma_kernel<G, PAGED>;
+    static bool configured = false;  // function attributes are per process, set once
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    return launch_pdl(kern, grid, kMmaThreads, smem, s, mKf, mVf, mKr, mVr, a, c, d);
+}
+
+template <int G>
+cudaError_t launch_mma_g(const LayerArgs& a, const CacheArgs& c, const DecodeArgs& d, int grid, cudaStream_t s) {
+    if (a.page_size) return launch_mma_t<G, true>(a, c, d, grid, s);
+    return launch_mma_t<G, false>(a, c, d, grid, s);
+}
+
+// Launch with programmatic stream serialization (PDL): the kernel may start
+// while the previous grid on the stream finishes; its griddepcontrol.wait
+// orders every dependent read after that grid.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int threads, size_t smem, cudaStream_t s, Args&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 template <typename T, int D, int G, bool PAGED>
@@ -579,8 +1026,7 @@ cudaError_t launch_t(const LayerArgs& a, const CacheArgs& c, const DecodeArgs& d
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    kern<<<grid, kThreads, smem, s>>>(a, c, d);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, kThreads, smem, s, a, c, d);
 }
 
 template <typename T, int D, int G>
@@ -618,7 +1064,16 @@ cudaError_t launch_decode(const LayerArgs& a, const CacheArgs& c, const DecodePl
     if (grid == 0) return cudaSuccess;
     if (grid > 0x7fffffffL) return cudaErrorInvalidConfiguration;
     if (a.dtype == DUO_BF16) {
-        if (a.D == 128) return launch_d<__nv_bfloat16, 128>(a, c, d, (int)grid, s);
+        if (a.D == 128) {
+            // bf16, head_dim 128: the tensor-core consumer
+            switch (a.G) {
+                case 1: return launch_mma_g<1>(a, c, d, (int)grid, s);
+                case 2: return launch_mma_g<2>(a, c, d, (int)grid, s);
+                case 4: return launch_mma_g<4>(a, c, d, (int)grid, s);
+                case 8: return launch_mma_g<8>(a, c, d, (int)grid, s);
+            }
+            return cudaErrorInvalidValue;
+        }
         return launch_d<__nv_bfloat16, 64>(a, c, d, (int)grid, s);
     }
     if (a.D == 128) return launch_d<float, 128>(a, c, d, (int)grid, s);

@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "duo.h"
@@ -61,6 +62,12 @@ cudaError_t launch_simt_attention(const LayerArgs& a, const CacheArgs* c, const 
 cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void* q, const void* k_chunk,
                               const void* v_chunk, int C, void* out, cudaStream_t s);
 bool prefill_tc_supported(const LayerArgs& a);
+// bf16 tensor map of `rank` dims (innermost first), 64-element-wide boxes with
+// the 128-byte swizzle, out-of-range elements read as zero; encodings are
+// cached per (base, dims, strides, box).  False if the driver refuses.
+bool encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                      const uint64_t* strides_bytes, const uint32_t* box);
+
 cudaError_t launch_permute(const void* x, void* y, int64_t rows, int hkv, const int* perm, int heads_per_kv,
                            int64_t head_elems, int elem_bytes, int direction, cudaStream_t s);
 

@@ -73,27 +73,6 @@ struct TcArgs {
 
 // ------------------------------------------------------------ PTX wrappers
 
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
-        "[%5];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, int w,
-                                            uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
-        "%5}], [%6];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -524,44 +503,6 @@ __global__ void __launch_bounds__(kThreadsTC, 2)
     }
 }
 
-// ------------------------------------------------------- host: tensor maps
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
-// bf16 tensor of `rank` dims (innermost first), 64-element-wide boxes with the
-// 128-byte swizzle; out-of-range elements read as zero.
-bool encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
-                 const uint32_t* box) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t gd[5], gs[4];
-    cuuint32_t bx[5], es[5];
-    for (int i = 0; i < rank; ++i) {
-        gd[i] = dims[i];
-        bx[i] = box[i];
-        es[i] = 1;
-    }
-    for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
-    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bx,
-                          es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 bool prefill_tc_supported(const LayerArgs& a) {
@@ -578,20 +519,20 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
         const uint64_t d[4] = {HD, (uint64_t)a.Hq, (uint64_t)C, (uint64_t)a.B};
         const uint64_t st[3] = {row, row * a.Hq, row * a.Hq * C};
         const uint32_t bx[4] = {64, 1, BM, 1};
-        if (!encode_bf16(&mQ, q, 4, d, st, bx)) return cudaErrorInvalidValue;
+        if (!encode_tmap_bf16(&mQ, q, 4, d, st, bx)) return cudaErrorInvalidValue;
     }
     {
         const uint64_t d[4] = {HD, (uint64_t)a.Hkv, (uint64_t)C, (uint64_t)a.B};
         const uint64_t st[3] = {row, row * a.Hkv, row * a.Hkv * C};
         const uint32_t bx[4] = {64, 1, BN, 1};
-        if (!encode_bf16(&mKx, k_chunk, 4, d, st, bx) || !encode_bf16(&mVx, v_chunk, 4, d, st, bx))
+        if (!encode_tmap_bf16(&mKx, k_chunk, 4, d, st, bx) || !encode_tmap_bf16(&mVx, v_chunk, 4, d, st, bx))
             return cudaErrorInvalidValue;
     }
     const uint32_t bx3[3] = {64, BN, 1};
     if (a.R > 0) {
         const uint64_t d[3] = {HD, (uint64_t)a.capacity, (uint64_t)a.B * a.R};
         const uint64_t st[2] = {row, row * a.capacity};
-        if (!encode_bf16(&mKc, c.k_full, 3, d, st, bx3) || !encode_bf16(&mVc, c.v_full, 3, d, st, bx3))
+        if (!encode_tmap_bf16(&mKc, c.k_full, 3, d, st, bx3) || !encode_tmap_bf16(&mVc, c.v_full, 3, d, st, bx3))
             return cudaErrorInvalidValue;
     } else {
         mKc = mKx;  // never read: there are no retrieval heads
@@ -600,7 +541,7 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
     if (a.S > 0) {
         const uint64_t d[3] = {HD, (uint64_t)a.W, (uint64_t)a.B * a.S};
         const uint64_t st[2] = {row, row * a.W};
-        if (!encode_bf16(&mKr, c.k_ring, 3, d, st, bx3) || !encode_bf16(&mVr, c.v_ring, 3, d, st, bx3))
+        if (!encode_tmap_bf16(&mKr, c.k_ring, 3, d, st, bx3) || !encode_tmap_bf16(&mVr, c.v_ring, 3, d, st, bx3))
             return cudaErrorInvalidValue;
     } else {
         mKr = mKx;  // never read: there are no streaming heads
