@@ -354,9 +354,9 @@ def run_decode(args, wl, world, rank):
                    "parallelism": f"replicas{world}",
                    "l2": f"not flushed: inputs larger than L2 (each step streams {nl} layers' caches, "
                          f"{nl * bytes_per_launch / 1e6:.0f} MB > 126 MB)"},
-        "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": round(achieved, 1), "peak": hbm,
+        "roofline": {"bound": "hbm", "kernel": "decode_mma_kernel", "achieved": round(achieved, 1), "peak": hbm,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / hbm, 4),
-                     "traffic": _traffic("decode_kernel", args.workload),
+                     "traffic": _traffic("decode_mma_kernel", args.workload),
                      "algorithmic_bytes_per_launch": int(bytes_per_launch),
                      "kernel_us": round(statistics.mean(dec_ms) * 1e3, 3)},
         "e2e": e2e,
