@@ -170,17 +170,28 @@ def _barrier(world):
     if world > 1:
         import torch
         import torch.distributed as dist
-        dist.barrier(device_ids=[torch.cuda.current_device()])
+        if dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[torch.cuda.current_device()])
+        else:
+            dist.barrier()
 
 
 def _max_over_ranks(x: float, world: int) -> float:
+    """The largest of the ranks' values (the job's time is its slowest rank's)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_us_per_unit(local_total_ms: float, units_per_rank: int, world: int) -> float:
+    """Whole-job time per unit for replicas: the slowest rank's time over
+    every rank's units (each rank runs the same number of units)."""
+    return _max_over_ranks(local_total_ms, world) * 1e3 / (units_per_rank * world)
 
 
 # ---------------------------------------------------------------------------
@@ -330,6 +341,7 @@ def run_decode(args, wl, world, rank):
     step_ms = [e0.elapsed_time(e1) for e0, e1 in ev]
     dec_ms = [t / nl for t in step_ms]
     total_ms = _max_over_ranks(sum(step_ms), world)
+    us_step = total_ms * 1e3 / (steps * nl * world)
     for caches, _ in layers:
         st_code = duo.check_status(caches.state)
         if st_code:
@@ -342,7 +354,6 @@ def run_decode(args, wl, world, rank):
     bytes_per_launch = statistics.mean(_decode_bytes(sh, R, L) for L in lengths_seen)
     dec_avg_s = statistics.mean(dec_ms) * 1e-3
     achieved = bytes_per_launch / dec_avg_s / 1e9
-    us_step = total_ms * 1e3 / (steps * nl * world)
     res = {
         "metric": METRIC, "value": round(us_step, 3), "unit": "us/step/layer", "n_gpus": world, "steps": steps,
         "warmup": warm, "ms_per_step": round(total_ms / steps, 6), "higher_is_better": False, "scaling": "weak",
@@ -550,7 +561,12 @@ def run_prefill(args, wl, world, rank, steps=None, warmup=None):
 # reference arm: the oracle, timed on the host cores
 # ---------------------------------------------------------------------------
 
-def run_reference(args, wl):
+def run_reference(args, wl, budget_s: float = 120.0):
+    """The oracle, as it stands, timed on this host's cores on the same
+    workload.  When K + W full steps would exceed `budget_s`, each step is a
+    bounded sample -- sequence 0, one retrieval and one streaming KV head with
+    their query heads -- and its time is scaled to the whole step by the ratio
+    of algorithmic bytes; the line says which."""
     import oracle as O
     sh = S.LayerShape(wl["hq"], wl["hkv"], wl["d"], "bf16")
     if wl["kind"] != "decode":
@@ -562,21 +578,57 @@ def run_reference(args, wl):
     sigma = S.head_sigma(wl["hkv"]) if wl.get("sigma") else None
     gate, _, _, R = O.partition_heads(S.binary_alpha(wl["hkv"], retrieval).astype(np.float64), 0.5)
     st = S.decode_state(sh, retrieval, lengths, sigma=sigma)
-    cache = O.HeadSplitCache(B, sh.n_kv_heads, sh.head_dim, gate=gate, sink=sh.sink, recent=sh.recent)
-    for (b, h), (k, v) in st["full"].items():
-        cache.load_state(b, h, np.arange(k.shape[0]), k, v)
-    for (b, h), (pos, k, v) in st["stream"].items():
-        cache.load_state(b, h, pos, k, v)
-    for b, L in enumerate(lengths):
-        cache.set_length(b, int(L))
     total = args.warmup + args.steps
     qs, ks, vs = S.decode_steps(sh, B, total, sigma=sigma)
-    for i in range(args.warmup):
-        cache.decode(qs[i], ks[i], vs[i])
+
+    def build(b_list, heads):
+        g = np.array([gate[h] for h in heads], dtype=np.uint8)
+        cache = O.HeadSplitCache(len(b_list), len(heads), sh.head_dim, gate=g, sink=sh.sink, recent=sh.recent)
+        for bi, b in enumerate(b_list):
+            for hi, h in enumerate(heads):
+                if gate[h]:
+                    k, v = st["full"][(b, h)]
+                    cache.load_state(bi, hi, np.arange(k.shape[0]), k, v)
+                else:
+                    pos, k, v = st["stream"][(b, h)]
+                    cache.load_state(bi, hi, pos, k, v)
+            cache.set_length(bi, int(lengths[b]))
+        return cache
+
+    def sl(i, b_list, heads):
+        G = sh.group
+        qh = [h * G + g for h in heads for g in range(G)]
+        return qs[i][b_list][:, qh], ks[i][b_list][:, heads], vs[i][b_list][:, heads]
+
+    full_heads = list(range(sh.n_kv_heads))
+    full_b = list(range(B))
+    cache = build(full_b, full_heads)
+    t0 = time.perf_counter()
+    cache.decode(*sl(0, full_b, full_heads))
+    t_full = time.perf_counter() - t0
+    bytes_full = _decode_bytes(sh, R, lengths + 1)
+    if total * t_full <= budget_s:
+        b_list, heads, scale, sample = full_b, full_heads, 1.0, "full decode steps"
+        first = 1
+    else:
+        ret0 = int(np.flatnonzero(gate)[0]) if R else None
+        str0 = int(np.flatnonzero(gate == 0)[0]) if R < sh.n_kv_heads else None
+        heads = [h for h in (ret0, str0) if h is not None]
+        b_list = [0]
+        sub = S.LayerShape(sh.group * len(heads), len(heads), sh.head_dim, "bf16", sh.sink, sh.recent)
+        n_ret = 1 if ret0 is not None else 0
+        bytes_sample = _decode_bytes(sub, n_ret, lengths[:1] + 1)
+        scale = bytes_full / bytes_sample
+        sample = (f"sequence 0, KV heads {heads} (one retrieval, one streaming) with their query heads; "
+                  f"time scaled x{scale:.1f} to the whole step by algorithmic bytes")
+        cache = build(b_list, heads)
+        first = 0
+    for i in range(first, args.warmup):
+        cache.decode(*sl(i, b_list, heads))
     t0 = time.perf_counter()
     for i in range(args.warmup, total):
-        cache.decode(qs[i], ks[i], vs[i])
-    dt = time.perf_counter() - t0
+        cache.decode(*sl(i, b_list, heads))
+    dt = (time.perf_counter() - t0) * scale
     v = round(dt * 1e6 / args.steps, 1)
     cores = _blas_threads()
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "us/step/layer", "n_gpus": 1,
@@ -586,7 +638,7 @@ def run_reference(args, wl):
                        "n_kv_heads": sh.n_kv_heads, "head_dim": sh.head_dim, "n_retrieval": R,
                        "context": [int(lengths.min()), int(lengths.max())]},
             "cpu_baseline": {"value": v, "unit": "us/step/layer", "cores": cores, "kind": "oracle",
-                             "sample": f"{args.steps} timed decode steps after {args.warmup} warm-up steps"},
+                             "sample": f"{args.steps} timed steps after {args.warmup} warm-up steps: {sample}"},
             "e2e": {"value": v, "unit": "us/step/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
