@@ -140,6 +140,21 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
+// Asks the bulk-copy engine to bring a contiguous global range into L2 (a
+// hint: nothing is written to shared memory, nothing to wait for).  The
+// address is 16-byte aligned and `bytes` a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// A relaxed, device-scope load: well defined even while another grid
+// updates the word with atomics (it returns the old or the new value).
+__device__ __forceinline__ int ld_relaxed_gpu(const int32_t* p) {
+    int v;
+    asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -124,7 +124,7 @@ __device__ __forceinline__ void length_ticket(const LayerArgs& a, const CacheArg
     const unsigned tk = atomicAdd(d.grid_ticket, 1u);
     if (tk == gridDim.x - 1) {
         __threadfence();
-        for (int bb = 0; bb < a.B; ++bb) c.seq_len[bb] += 1;
+        for (int bb = 0; bb < a.B; ++bb) atomicAdd(&c.seq_len[bb], 1);
         *d.grid_ticket = 0u;
         __threadfence();
     }
@@ -668,6 +668,42 @@ __device__ __forceinline__ uint32_t sw_off(int row, int c16) {
     return (uint32_t)((c16 >> 3) * (kMmaTileBytes / 2) + row * 128 + (((c16 & 7) ^ (row & 7)) << 4));
 }
 
+constexpr int kWarmTiles = 2;  // K and V tiles per split brought into L2 before the dependency wait
+
+// Runs before griddepcontrol.wait, while the previous grid on the stream may
+// still be streaming its own caches: asks L2 for the first kWarmTiles K and V
+// tiles of this CTA's split, so the first TMA loads after the wait hit L2.
+// The rows come from a relaxed read of seq_len and (paged) of the page table
+// and are clamped to the cache, so a stale value only wastes a prefetch.
+template <bool PAGED>
+__device__ __forceinline__ void warm_l2_split(const LayerArgs& a, const CacheArgs& c, const DecodeArgs& d, int b,
+                                              int slot, int split) {
+    constexpr int kRowBytes = 128 * 2;
+    int len = ld_relaxed_gpu(&c.seq_len[b]) + (d.k_new != nullptr ? 1 : 0);
+    len = max(0, min(len, a.capacity));
+    const int per = (len + d.nsplit - 1) / d.nsplit;
+    const int chunk = (per + kTile - 1) / kTile * kTile;
+    const int row_begin = min(len, split * chunk);
+    const int row_end = min(len, row_begin + chunk);
+    const int n_tiles = min(kWarmTiles, (row_end - row_begin + kTile - 1) / kTile);
+    const uint8_t* kf = static_cast<const uint8_t*>(c.k_full);
+    const uint8_t* vf = static_cast<const uint8_t*>(c.v_full);
+    for (int t = 0; t < n_tiles; ++t) {
+        const int r0 = row_begin + t * kTile;
+        const uint32_t bytes = (uint32_t)min(kTile, row_end - r0) * kRowBytes;
+        size_t off;
+        if (PAGED) {
+            const int pg = ld_relaxed_gpu(&c.page_table[(size_t)b * a.max_pages + r0 / kTile]);
+            if (pg < 0 || pg >= a.n_pages) continue;
+            off = ((size_t)pg * a.R + slot) * kTile * kRowBytes;
+        } else {
+            off = (((size_t)b * a.R + slot) * a.capacity + r0) * kRowBytes;
+        }
+        bulk_prefetch_l2(kf + off, bytes);
+        bulk_prefetch_l2(vf + off, bytes);
+    }
+}
+
 template <int G, bool PAGED>
 __global__ void __maxnreg__(200)
     decode_mma_kernel(const __grid_constant__ CUtensorMap tmKf, const __grid_constant__ CUtensorMap tmVf,
@@ -708,6 +744,21 @@ __global__ void __maxnreg__(200)
         b = u / a.S;
     }
     const bool fused = d.k_new != nullptr;
+    // Work that reads nothing the previous grid writes: barriers, the tensor
+    // maps (kernel parameters) and the L2 warm-up of this split's first tiles.
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], NW);
+        }
+        mbar_init(comb_bar, 1);
+        fence_barrier_init();
+    }
+    if (warp == NW && lane == 0) {
+        prefetch_map(retrieval ? &tmKf : &tmKr);
+        prefetch_map(retrieval ? &tmVf : &tmVr);
+        if (retrieval) warm_l2_split<PAGED>(a, c, d, b, slot, split);
+    }
     // launched with programmatic stream serialization: let the next launch's
     // CTAs take SM slots as ours free, and wait for the previous grid before
     // the first read of anything it may have written
@@ -744,16 +795,6 @@ __global__ void __maxnreg__(200)
         row_end = len < 0 ? 0 : min(len, a.W);
     }
     const int n_tiles = (row_end - row_begin + kTile - 1) / kTile;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full_bar[s], 1);
-            mbar_init(&empty_bar[s], NW);
-        }
-        mbar_init(comb_bar, 1);
-        fence_barrier_init();
-    }
-    __syncthreads();
 
     if (warp == NW) {
         // ------------------------------------------------------ producer
@@ -796,8 +837,6 @@ __global__ void __maxnreg__(200)
         if (lane == 0) {
             const CUtensorMap* mk = retrieval ? &tmKf : &tmKr;
             const CUtensorMap* mv = retrieval ? &tmVf : &tmVr;
-            prefetch_map(mk);
-            prefetch_map(mv);
             const int z = retrieval ? b * a.R + slot : b * a.S + (slot - a.R);
             for (int t = 0; t < n_tiles; ++t) {
                 const int st = t % STAGES, round = t / STAGES;
