@@ -98,25 +98,74 @@ def _traffic(kernel: str, workload: str):
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 
+_NVML_POLL = r"""
+import sys, time
+import pynvml as nv
+nv.nvmlInit()
+h = nv.nvmlDeviceGetHandleByPciBusId(sys.argv[1])
+period = float(sys.argv[2])
+print("ready", nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM), flush=True)
+while True:
+    print(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), nv.nvmlDeviceGetCurrentClocksEventReasons(h), flush=True)
+    time.sleep(period)
+"""
+
+
 class ClockSampler:
+    """SM clock and clock-event (throttle) reasons of this process's GPU,
+    sampled while the timed region runs, from a separate process so that the
+    launching thread's hold on the interpreter cannot starve the sampling.
+    Through NVML every 10 ms when the bindings load (the CUDA device is
+    matched to its NVML handle by PCI bus id, so CUDA_VISIBLE_DEVICES cannot
+    point it at another GPU), else through `nvidia-smi -lms 200`.  Only
+    reads; nothing about the GPU is changed."""
+
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    # NVML clock-event reason bits
+    BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40}
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, period_s: float = 0.01):
         self.gpu = gpu_index
+        self.period = period_s
         self.proc = None
         self.lines = []
+        self.mode = None
+        self.max_mhz = None
+
+    def _start_nvml(self) -> bool:
+        import torch
+        props = torch.cuda.get_device_properties(self.gpu)
+        bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+        self.proc = subprocess.Popen([sys.executable, "-c", _NVML_POLL, bus, str(self.period)],
+                                     stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        first = self.proc.stdout.readline().split()
+        if len(first) != 2 or first[0] != "ready":
+            self.proc.kill()
+            self.proc = None
+            return False
+        self.max_mhz = float(first[1])
+        return True
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            if self._start_nvml():
+                self.mode = "nvml 10 ms"
+        except Exception:
+            self.proc = None
+        if self.proc is None:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                     "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.mode = "nvidia-smi 200 ms"
+            except OSError:
+                self.proc = None
+        if self.proc is not None:
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
-        except OSError:
-            self.proc = None
         return self
 
     def _read(self):
@@ -125,7 +174,8 @@ class ClockSampler:
 
     def __exit__(self, *exc):
         if self.proc:
-            time.sleep(0.25)
+            if self.mode != "nvml 10 ms":
+                time.sleep(0.25)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -133,22 +183,32 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        mhz, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                mhz.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
+        mhz, mx, reasons = [], self.max_mhz, set()
+        for ln in list(self.lines):
+            if self.mode == "nvml 10 ms":
+                parts = ln.split()
+                if len(parts) != 2:
+                    continue
+                try:
+                    mhz.append(float(parts[0]))
+                    bits = int(parts[1])
+                except ValueError:
+                    continue
+                reasons |= {n for n, bit in self.BITS.items() if bits & bit}
+            else:
+                parts = [p.strip() for p in ln.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    mhz.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(self.NAMES, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
         return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(mhz)}
+                "reasons": sorted(reasons), "samples": len(mhz), "sampler": self.mode}
 
 
 # ---------------------------------------------------------------------------
