@@ -62,10 +62,6 @@ cudaError_t launch_simt_attention(const LayerArgs& a, const CacheArgs* c, const 
 cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void* q, const void* k_chunk,
                               const void* v_chunk, int C, void* out, cudaStream_t s);
 bool prefill_tc_supported(const LayerArgs& a);
-// The earlier one-query-tile-per-CTA tcgen05 pre-fill (same contract).
-cudaError_t launch_prefill_tc_v1(const LayerArgs& a, const CacheArgs& c, const void* q, const void* k_chunk,
-                                 const void* v_chunk, int C, void* out, cudaStream_t s);
-bool prefill_tc_v1_supported(const LayerArgs& a);
 // bf16 tensor map of `rank` dims (innermost first), 64-element-wide boxes with
 // the 128-byte swizzle, out-of-range elements read as zero; encodings are
 // cached per (base, dims, strides, box).  False if the driver refuses.
