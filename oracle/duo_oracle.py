@@ -46,6 +46,12 @@ repository's design notes):
   p < sink, else in slot ``sink + (p - sink) % recent``; ``pos[slot]`` holds the
   position, -1 when the slot is empty.
 * Top-k selection of retrieval heads breaks ties by the lower head index.
+* 8-bit retrieval cache (the pages pair the method with a quantized KV cache
+  but give no scheme): each cached K or V row of a head is stored as int8
+  codes with one float32 scale, symmetric, amax = max |x|,
+  code = rint(x * (127 / amax)) (round half to even), scale = amax / 127,
+  all in float32 as written; a zero row has scale 0 and codes 0.  Attention
+  reads code * scale.
 """
 
 from __future__ import annotations
@@ -71,6 +77,8 @@ __all__ = [
     "HeadSplitCache",
     "prefill_direct",
     "decode_direct",
+    "quantize_int8_rows",
+    "dequantize_int8_rows",
 ]
 
 
@@ -250,6 +258,36 @@ def ring_slot(p: int, sink: int, recent: int) -> int:
     return p if p < sink else sink + (p - sink) % recent
 
 
+# ---------------------------------------------------------------------------
+# 8-bit retrieval cache [Review S5 "Decoding performance": combined with a
+# quantized KV cache; Summary S3 results] -- scheme: see the module notes
+# ---------------------------------------------------------------------------
+
+def quantize_int8_rows(x) -> tuple:
+    """Per-row symmetric int8 codes of x [n, d] (bf16 bits, float32 or
+    float64 holding float32 values): returns (codes int8 [n, d], scales
+    float32 [n]).  Every step is one float32 operation as written, so the
+    codes are those any IEEE float32 implementation of the same steps gets."""
+    x32 = as_f64(x).astype(np.float32)
+    codes = np.zeros(x32.shape, dtype=np.int8)
+    scales = np.zeros(x32.shape[:-1], dtype=np.float32)
+    for i in range(x32.shape[0]):
+        row = x32[i]
+        amax = np.float32(np.max(np.abs(row))) if row.size else np.float32(0)
+        if amax == 0:
+            continue
+        inv = np.float32(127.0) / amax
+        q = np.rint(row * inv)                      # float32 product, round half to even
+        codes[i] = np.clip(q, -127, 127).astype(np.int8)
+        scales[i] = amax / np.float32(127.0)
+    return codes, scales
+
+
+def dequantize_int8_rows(codes, scales) -> np.ndarray:
+    """code * scale, exactly, in float64 [n, d]."""
+    return np.asarray(codes, dtype=np.float64) * np.asarray(scales, dtype=np.float64)[:, None]
+
+
 @dataclass
 class HeadSplitCache:
     """Per-layer caches for a batch: full lists for retrieval heads, a
@@ -266,8 +304,10 @@ class HeadSplitCache:
     gate: np.ndarray
     sink: int = 16
     recent: int = 64
+    kv_int8: bool = False                # retrieval heads keep int8 codes + a scale per row
     length: list = field(default=None)
-    full: list = field(default=None)     # full[b][h] -> list of (pos int64[n], k[n, d], v[n, d])
+    full: list = field(default=None)     # full[b][h] -> list of (pos int64[n], k[n, d], v[n, d]
+                                         #   [, k codes, k scales, v codes, v scales] when kv_int8)
     stream: list = field(default=None)   # stream[b][h] -> list of (pos, k[d], v[d]) per token
 
     def __post_init__(self):
@@ -291,7 +331,7 @@ class HeadSplitCache:
             for h in range(hkv):
                 if self.gate[h]:
                     if t:
-                        self.full[b][h].append((pos, k_new[b, :, h].copy(), v_new[b, :, h].copy()))
+                        self.full[b][h].append(self._full_entry(pos, k_new[b, :, h], v_new[b, :, h]))
                 else:
                     lst = self.stream[b][h]
                     for i in range(t):
@@ -311,13 +351,31 @@ class HeadSplitCache:
         context without replaying the prompt token by token."""
         pos = np.asarray(pos, dtype=np.int64)
         if self.gate[h]:
-            self.full[b][h] = [(pos.copy(), np.asarray(k).copy(), np.asarray(v).copy())]
+            self.full[b][h] = [self._full_entry(pos, np.asarray(k), np.asarray(v))] if len(pos) else []
         else:
             self.stream[b][h] = [(int(p), np.asarray(k)[i].copy(), np.asarray(v)[i].copy())
                                  for i, p in enumerate(pos)]
 
     def set_length(self, b: int, n: int) -> None:
         self.length[b] = int(n)
+
+    def _full_entry(self, pos, k, v):
+        """A retrieval-head list entry: the rows as given, or (kv_int8) their
+        dequantized values followed by the codes and scales."""
+        if not self.kv_int8:
+            return (pos.copy(), k.copy(), v.copy())
+        kc, ks = quantize_int8_rows(k)
+        vc, vs = quantize_int8_rows(v)
+        return (pos.copy(), dequantize_int8_rows(kc, ks), dequantize_int8_rows(vc, vs), kc, ks, vc, vs)
+
+    def quantized(self, b: int, h: int):
+        """A kv_int8 retrieval head's (positions, K codes, K scales, V codes, V scales)."""
+        assert self.kv_int8 and self.gate[h]
+        ent = self.full[b][h]
+        if not ent:
+            z8, z32 = np.zeros((0, self.head_dim), np.int8), np.zeros(0, np.float32)
+            return np.zeros(0, dtype=np.int64), z8, z32, z8, z32
+        return tuple(np.concatenate([e[i] for e in ent]) for i in (0, 3, 4, 5, 6))
 
     # -- views ------------------------------------------------------------
 

@@ -50,6 +50,9 @@ def _pins():
         P.test_partition_by_threshold,
         P.test_partition_top_k_ties_go_to_lower_index,
         P.test_binarize_uses_greater_or_equal,
+        lambda: P.test_int8_codes_match_hand_worked_rows(g),
+        lambda: P.test_int8_round_trip_is_within_half_a_step(0),
+        P.test_int8_cache_decode_equals_direct_on_reconstructed_rows,
     ]
 
 
@@ -159,3 +162,30 @@ def test_planted_gqa_mapping_mistake_is_caught(monkeypatch):
         return out
     _patch(monkeypatch, "gated_mix", mix_mod_mapping)
     assert _fails(*_pins())
+
+
+def _q8(x, factor_num=127.0, scale_den=127.0, rnd=np.rint, per_tensor=False):
+    x32 = D.as_f64(x).astype(np.float32)
+    codes = np.zeros(x32.shape, dtype=np.int8)
+    scales = np.zeros(x32.shape[:-1], dtype=np.float32)
+    amax_all = np.float32(np.abs(x32).max()) if x32.size else np.float32(0)
+    for i in range(x32.shape[0]):
+        amax = amax_all if per_tensor else np.float32(np.abs(x32[i]).max())
+        if amax == 0:
+            continue
+        codes[i] = np.clip(rnd(x32[i] * (np.float32(factor_num) / amax)), -128, 127).astype(np.int8)
+        scales[i] = amax / np.float32(scale_den)
+    return codes, scales
+
+
+@pytest.mark.parametrize("mistake", [
+    dict(rnd=np.floor),                     # rounds down instead of to nearest
+    dict(rnd=np.trunc),                     # rounds toward zero
+    dict(rnd=lambda v: np.floor(v + np.float32(0.5))),   # ties away from even
+    dict(factor_num=128.0, scale_den=128.0),             # 128 steps: the extreme code overflows
+    dict(scale_den=128.0),                  # scale from a different step than the codes
+    dict(per_tensor=True),                  # one scale for all rows
+])
+def test_planted_int8_mistake_is_caught(monkeypatch, mistake):
+    _patch(monkeypatch, "quantize_int8_rows", lambda x: _q8(x, **mistake))
+    assert _fails(*_pins()), f"no pin caught the planted quantizer mistake {mistake}"

@@ -391,3 +391,67 @@ def test_bf16_widening_is_exact():
     x = np.array([1.0, -2.5, 3.140625, 2.0 ** -100, 65280.0], dtype=np.float32)
     bits = S.to_bf16_bits(x)
     np.testing.assert_array_equal(O.bf16_bits_to_f64(bits), x.astype(np.float64))
+
+
+# ---------------------------------------------------------------------------
+# 8-bit retrieval cache (the build's reading of the pages' quantized KV cache)
+# ---------------------------------------------------------------------------
+
+def test_int8_codes_match_hand_worked_rows(golden):
+    params, _ = golden("int8_rows.txt")
+    for i in range(3):
+        x = np.array([params[f"x{i}"]], dtype=np.float32)
+        codes, scales = O.quantize_int8_rows(x)
+        assert codes.dtype == np.int8 and scales.dtype == np.float32
+        assert codes[0].tolist() == [int(c) for c in params[f"codes{i}"]], i
+        assert scales[0] == np.float32(float(params[f"scale{i}"])), i
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_int8_round_trip_is_within_half_a_step(seed):
+    rng = np.random.default_rng([seed, 91])
+    d = 128
+    # bf16-representable rows of very different magnitudes, some with a zero
+    x = (rng.standard_normal((64, d)) * np.exp(rng.uniform(-8, 8, (64, 1)))).astype(np.float32)
+    x = (x.view(np.uint32) & np.uint32(0xFFFF0000)).view(np.float32)
+    x[5] = 0.0
+    x[7, :10] = 0.0
+    codes, scales = O.quantize_int8_rows(x)
+    assert np.all(np.abs(codes.astype(np.int32)) <= 127)
+    amax = np.abs(x).max(axis=1)
+    nz = amax > 0
+    # the largest element of every nonzero row gets code +-127
+    assert np.all(np.abs(codes[nz]).max(axis=1) == 127)
+    assert np.all(scales[~nz] == 0) and np.all(codes[~nz] == 0)
+    # each value is within half a step of its code
+    err = np.abs(x.astype(np.float64) - O.dequantize_int8_rows(codes, scales))
+    assert np.all(err <= scales.astype(np.float64)[:, None] * (0.5 + 1e-5))
+    # signs are kept, and zeros stay zero
+    assert np.all((codes == 0) | (np.sign(codes) == np.sign(x)))
+    assert np.all(codes[x == 0] == 0)
+    # codes of the reconstructed rows are the codes again
+    again, _ = O.quantize_int8_rows(O.dequantize_int8_rows(codes, scales).astype(np.float32))
+    assert np.array_equal(again, codes)
+
+
+def test_int8_cache_decode_equals_direct_on_reconstructed_rows():
+    """The 8-bit cache only changes what the retrieval heads' lists hold: a
+    decode from it equals the direct mask definition over the history whose
+    retrieval rows are replaced by code * scale."""
+    sh = S.LayerShape(8, 4, 16, "bf16")
+    gate = np.array([1, 0, 1, 0], dtype=np.uint8)
+    n = 150
+    q, k, v = S.prompt(sh, n, seed=4)
+    c = O.HeadSplitCache(1, 4, 16, gate=gate, kv_int8=True)
+    c.append(k[:, :n - 1], v[:, :n - 1])
+    got = c.decode(q[:, n - 1], k[:, n - 1], v[:, n - 1])[0]
+    k_hat, v_hat = O.as_f64(k[0]), O.as_f64(v[0])
+    for h in (0, 2):
+        kc, ks = O.quantize_int8_rows(k[0, :, h])
+        vc, vs = O.quantize_int8_rows(v[0, :, h])
+        k_hat[:, h] = O.dequantize_int8_rows(kc, ks)
+        v_hat[:, h] = O.dequantize_int8_rows(vc, vs)
+    want = O.decode_direct(q[0, n - 1], k_hat, v_hat, gate, 16, 64)
+    assert np.max(np.abs(got - want)) < 1e-12
+    pos, kc, ks, vc, vs = c.quantized(0, 2)
+    assert np.array_equal(pos, np.arange(n)) and kc.shape == (n, 16) and ks.shape == (n,)
