@@ -408,7 +408,7 @@ def run_decode(args, wl, world, rank):
             raise RuntimeError(f"device status 0x{st_code:x} after the timed steps")
 
     # end to end through the public API with host buffers
-    e2e = _decode_e2e(duo, env, layers, args, world)
+    e2e = None if getattr(args, "no_e2e", False) else _decode_e2e(duo, env, layers, args, world)
 
     hbm, _, peak_kind = _peaks()
     bytes_per_launch = statistics.mean(_decode_bytes(sh, R, L) for L in lengths_seen)
@@ -704,6 +704,49 @@ def run_reference(args, wl, budget_s: float = 120.0):
 
 # ---------------------------------------------------------------------------
 
+def _linear_fit(xs, ys):
+    """Least-squares line y = a + b x and its coefficient of determination."""
+    x = np.asarray(xs, dtype=np.float64)
+    y = np.asarray(ys, dtype=np.float64)
+    b, a = np.polyfit(x, y, 1)
+    resid = y - (a + b * x)
+    ss = float(((y - y.mean()) ** 2).sum())
+    return {"intercept": round(float(a), 4), "slope": round(float(b), 4),
+            "r2": round(1.0 - float((resid ** 2).sum()) / ss, 5) if ss > 0 else 1.0}
+
+
+def run_ratio_sweep(args, world, rank):
+    """Decode and pre-fill time against the share of retrieval heads (the
+    pages report both as linear in it).  Decode: the 32K MHA layer with 0, 4,
+    ..., 32 of its 32 heads retrieval; pre-fill: the 32K-token GQA prompt in
+    4,096-token chunks with 0 .. 8 of its 8 KV heads retrieval.  Heads chosen
+    by the same seeded draw as the workloads."""
+    import copy
+    dec, pre = [], []
+    a2 = copy.copy(args)
+    a2.steps, a2.warmup, a2.no_e2e, a2.no_cpu_baseline = 64, 3, True, True
+    for r in range(0, 33, 4):
+        wl = dict(WORKLOADS["mha_decode_32k"], n_ret=r, name="mha_decode_32k")
+        res = run_decode(a2, wl, world, rank)
+        dec.append({"n_retrieval": r, "ratio": r / 32, "us_per_step_layer": res["value"],
+                    "achieved_gbs": res["roofline"]["achieved"],
+                    "bytes_per_launch": res["roofline"]["algorithmic_bytes_per_launch"]})
+    for r in range(0, 9):
+        wl = dict(WORKLOADS["gqa_prefill_32k"], n_ret=r, name="gqa_prefill_32k")
+        res = run_prefill(a2, wl, world, rank, steps=8, warmup=3)
+        pre.append({"n_retrieval": r, "ratio": r / 8, "ms_total": res["roofline"]["prefill_ms_total"],
+                    "tflops": res["roofline"]["achieved"]})
+    return {"metric": "decode us/step/layer and pre-fill ms vs retrieval-head ratio", "n_gpus": world,
+            "data": "synthetic",
+            "decode": {"workload": "mha_decode_32k (32 heads, context 32,768, 4 layers/step, 64 steps)",
+                       "points": dec,
+                       "fit_us_vs_ratio": _linear_fit([d["ratio"] for d in dec],
+                                                      [d["us_per_step_layer"] for d in dec])},
+            "prefill": {"workload": "gqa_prefill_32k (8 KV heads, 32,768 tokens in 8 chunks of 4,096)",
+                        "points": pre,
+                        "fit_ms_vs_ratio": _linear_fit([d["ratio"] for d in pre], [d["ms_total"] for d in pre])}}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -716,6 +759,8 @@ def main(argv=None):
     ap.add_argument("--no-prefill", action="store_true", help="skip the pre-fill measurement of a decode run")
     ap.add_argument("--layers", type=int, default=4,
                     help="decode: layers per step, each with its own caches (their total exceeds L2)")
+    ap.add_argument("--retrieval-ratio-sweep", action="store_true",
+                    help="time decode and pre-fill against the share of retrieval heads (one JSON line)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -733,7 +778,9 @@ def main(argv=None):
     torch.cuda.set_device(local)
     from head_split_kv_b200 import duo  # noqa: F401  (fails loudly without libduo.so)
     try:
-        if wl["kind"] == "decode":
+        if args.retrieval_ratio_sweep:
+            res = run_ratio_sweep(args, world, rank)
+        elif wl["kind"] == "decode":
             res = run_decode(args, wl, world, rank)
             if not args.no_prefill:
                 pre = run_prefill(args, WORKLOADS["gqa_prefill_128k"], world, rank)

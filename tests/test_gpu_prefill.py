@@ -62,6 +62,50 @@ def test_prefill_tc_gqa_chunkings(duo, chunks):
     _run(duo, sh, [1, 2], sum(chunks), chunks)
 
 
+def _history(sh, st, b, L, k_new, v_new):
+    """Token history [L + C, Hkv, d] of sequence b: the decode state's rows
+    (zeros where a streaming head kept nothing -- the Lambda mask never reads
+    those positions from a later query) followed by the chunk's rows."""
+    C = k_new.shape[0]
+    k_all = np.zeros((L + C, sh.n_kv_heads, sh.head_dim), dtype=np.float64)
+    v_all = np.zeros_like(k_all)
+    for h in range(sh.n_kv_heads):
+        if (b, h) in st["full"]:
+            k, v = st["full"][(b, h)]
+            k_all[:L, h], v_all[:L, h] = O.as_f64(k), O.as_f64(v)
+        else:
+            pos, k, v = st["stream"][(b, h)]
+            k_all[pos, h], v_all[pos, h] = O.as_f64(k), O.as_f64(v)
+    k_all[L:], v_all[L:] = O.as_f64(k_new), O.as_f64(v_new)
+    return k_all, v_all
+
+
+@pytest.mark.parametrize("chunk", [1000, 256])
+def test_prefill_tc_uneven_batch(duo, chunk):
+    """Sequences of one batch at different lengths (0, 1100, 2300 tokens
+    cached) take one chunk together: each sequence's query tiles see their
+    own prior tiles, the first of them partly before position 0 when the
+    length is not a multiple of the tile."""
+    t = torch()
+    sh = S.LayerShape(16, 4, 128, "bf16")
+    retrieval = [0, 3]
+    lengths = [0, 1100, 2300]
+    B = len(lengths)
+    lay = Layer(duo, sh, retrieval, B, capacity=max(lengths) + chunk + 16)
+    st = S.decode_state(sh, retrieval, lengths, seed=5)
+    lay.load_state(st)
+    q, k, v = S.prompt(sh, chunk, seed=6, batch=B)
+    rows = np.unique(np.concatenate([[0, chunk - 1], S.rng_for(6, 78).choice(chunk, 96, replace=False)]))
+    want = [O.prefill_direct(q[b], *_history(sh, st, b, L, k[b], v[b]), L, np.array(lay.gate), sh.sink, sh.recent,
+                             rows=rows) for b, L in enumerate(lengths)]
+    out = t.empty((B, chunk, sh.n_q_heads, sh.head_dim), dtype=t.bfloat16, device="cuda")
+    duo.prefill_chunk(lay.desc, lay.caches.state, to_dev(q), to_dev(k), to_dev(v), chunk, out)
+    got = f64(out)
+    for b, L in enumerate(lengths):
+        assert_close(got[b, rows], want[b], "bf16", f"b={b} (cached {L})")
+    assert lay.status() == 0
+
+
 def test_prefill_tc_mha_25pct(duo):
     sh = S.LayerShape(32, 32, 128, "bf16")
     _run(duo, sh, S.retrieval_heads_by_seed(32, 8), 2048, [512] * 4, sample_rows=64)
