@@ -46,6 +46,13 @@ repository's design notes):
   p < sink, else in slot ``sink + (p - sink) % recent``; ``pos[slot]`` holds the
   position, -1 when the slot is empty.
 * Top-k selection of retrieval heads breaks ties by the lower head index.
+* Whole-chunk streaming pre-fill (a second pre-fill mode; the pages note
+  that pre-fill gains grow as the chunk shrinks, which is what happens when a
+  streaming head attends to its whole chunk): a streaming query at position
+  i of the chunk starting at c0 sees the streaming cache as it stood before
+  the chunk -- its sinks and the last ``recent`` tokens before c0 -- and every
+  chunk token up to itself: ``j <= i and (j < sink or j >= c0 - recent)``.
+  Decode is unchanged.
 * 8-bit retrieval cache (the pages pair the method with a quantized KV cache
   but give no scheme): each cached K or V row of a head is stored as int8
   codes with one float32 scale, symmetric, amax = max |x|,
@@ -66,6 +73,7 @@ __all__ = [
     "bf16_bits_to_f64",
     "causal_mask",
     "streaming_mask",
+    "chunk_streaming_mask",
     "masked_softmax",
     "masked_attention",
     "full_attn",
@@ -129,6 +137,18 @@ def streaming_mask(q_pos: np.ndarray, k_pos: np.ndarray, sink: int, recent: int)
     qi = q_pos[:, None]
     kj = k_pos[None, :]
     return (kj <= qi) & ((kj < sink) | (qi - kj < recent))
+
+
+def chunk_streaming_mask(q_pos: np.ndarray, k_pos: np.ndarray, c0: int, sink: int, recent: int) -> np.ndarray:
+    """A streaming head's mask in whole-chunk pre-fill: queries of the chunk
+    that starts at ``c0`` see the sinks, the ``recent`` tokens before the
+    chunk, and every chunk token up to themselves [Summary S2 "Chunked
+    Pre-filling"; Review S5 "Pre-filling performance"]."""
+    q_pos = np.asarray(q_pos, dtype=np.int64)
+    k_pos = np.asarray(k_pos, dtype=np.int64)
+    qi = q_pos[:, None]
+    kj = k_pos[None, :]
+    return (kj <= qi) & ((kj < sink) | (kj >= c0 - recent))
 
 
 # ---------------------------------------------------------------------------
@@ -424,10 +444,12 @@ class HeadSplitCache:
 
     # -- attention ----------------------------------------------------------
 
-    def _head_attention(self, b, h_kv, q_rows, q_pos, extra=None, scale=1.0):
+    def _head_attention(self, b, h_kv, q_rows, q_pos, extra=None, scale=1.0, whole_chunk=False):
         """Attention of query rows (positions q_pos) against what head h_kv of
         sequence b holds, plus optional extra (pos, k, v) rows, under the head's
-        mask (causal for retrieval heads, Lambda for streaming heads)."""
+        mask (causal for retrieval heads, Lambda for streaming heads).  With
+        ``whole_chunk`` a streaming head sees all it holds and the extra rows
+        causally: its list is the cache as it stood before the chunk."""
         pos, k, v = self.rows(b, h_kv)
         k = as_f64(k) if len(pos) else np.zeros((0, self.head_dim))
         v = as_f64(v) if len(pos) else np.zeros((0, self.head_dim))
@@ -435,7 +457,7 @@ class HeadSplitCache:
             pos = np.concatenate([pos, extra[0]])
             k = np.concatenate([k, as_f64(extra[1])])
             v = np.concatenate([v, as_f64(extra[2])])
-        if self.gate[h_kv]:
+        if self.gate[h_kv] or whole_chunk:
             mask = causal_mask(q_pos, pos)
         else:
             mask = streaming_mask(q_pos, pos, self.sink, self.recent)
@@ -464,13 +486,14 @@ class HeadSplitCache:
                 out[b, kv * g:(kv + 1) * g] = self._head_attention(b, kv, rows, np.full(g, p), scale=sc)
         return out
 
-    def prefill_chunk(self, q, k_chunk, v_chunk, scale=None) -> np.ndarray:
+    def prefill_chunk(self, q, k_chunk, v_chunk, scale=None, stream_mode: str = "lambda") -> np.ndarray:
         """Chunked pre-fill from the caches [Summary S2 "Chunked Pre-filling"].
 
         Each query of the chunk attends to what its head's cache held before the
         chunk plus the chunk's own tokens, under the head's mask; afterwards the
         chunk is appended to both caches.  q: [B, C, Hq, d]; k_chunk, v_chunk:
-        [B, C, Hkv, d].  Returns float64 [B, C, Hq, d].
+        [B, C, Hkv, d].  Returns float64 [B, C, Hq, d].  ``stream_mode="chunk"``:
+        a streaming head attends to its whole list and the chunk causally.
         """
         q = np.asarray(q)
         k_chunk = np.asarray(k_chunk)
@@ -485,7 +508,8 @@ class HeadSplitCache:
             for h in range(hq):
                 kv = h // g
                 extra = (qpos, k_chunk[b, :, kv], v_chunk[b, :, kv])
-                out[b, :, h] = self._head_attention(b, kv, q[b, :, h], qpos, extra, sc)
+                out[b, :, h] = self._head_attention(b, kv, q[b, :, h], qpos, extra, sc,
+                                                    whole_chunk=stream_mode == "chunk")
         self.append(k_chunk, v_chunk)
         return out
 
@@ -495,12 +519,13 @@ class HeadSplitCache:
 # ---------------------------------------------------------------------------
 
 def prefill_direct(q_chunk, k_all, v_all, c0: int, gate, sink: int, recent: int,
-                   scale=None, rows=None, row_block: int = 64) -> np.ndarray:
+                   scale=None, rows=None, row_block: int = 64, stream_mode: str = "lambda") -> np.ndarray:
     """Chunk queries at positions c0 .. c0+C-1 attend to the whole token history
     k_all/v_all [N, Hkv, d] (N >= c0 + C) through the head's mask: causal for a
     retrieval head, Lambda for a streaming head.
 
     q_chunk: [C, Hq, d].  ``rows`` optionally selects chunk rows (sampling).
+    ``stream_mode="chunk"`` gives streaming heads the whole-chunk mask.
     Rows are independent, so they are processed ``row_block`` at a time to bound
     memory; each row's arithmetic is the plain masked softmax above.
     Returns float64 [len(rows), Hq, d].
@@ -521,6 +546,8 @@ def prefill_direct(q_chunk, k_all, v_all, c0: int, gate, sink: int, recent: int,
         for kv in range(hkv):
             if gate[kv]:
                 mask = causal_mask(qpos, kpos)
+            elif stream_mode == "chunk":
+                mask = chunk_streaming_mask(qpos, kpos, c0, sink, recent)
             else:
                 mask = streaming_mask(qpos, kpos, sink, recent)
             kk = as_f64(k_all[:last, kv])

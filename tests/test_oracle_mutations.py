@@ -53,6 +53,9 @@ def _pins():
         lambda: P.test_int8_codes_match_hand_worked_rows(g),
         lambda: P.test_int8_round_trip_is_within_half_a_step(0),
         P.test_int8_cache_decode_equals_direct_on_reconstructed_rows,
+        lambda: P.test_chunk_streaming_mask_matches_hand_drawn(g),
+        P.test_whole_chunk_streaming_first_chunk_is_causal,
+        lambda: P.test_whole_chunk_streaming_from_caches_equals_direct(7),
     ]
 
 
@@ -189,3 +192,23 @@ def _q8(x, factor_num=127.0, scale_den=127.0, rnd=np.rint, per_tensor=False):
 def test_planted_int8_mistake_is_caught(monkeypatch, mistake):
     _patch(monkeypatch, "quantize_int8_rows", lambda x: _q8(x, **mistake))
     assert _fails(*_pins()), f"no pin caught the planted quantizer mistake {mistake}"
+
+
+def _chunk_mask_window_short(q_pos, k_pos, c0, sink, recent):
+    qi, kj = np.asarray(q_pos)[:, None], np.asarray(k_pos)[None, :]
+    return (kj <= qi) & ((kj < sink) | (kj >= c0 - recent + 1))   # one recent token too few
+
+
+def _chunk_mask_is_lambda(q_pos, k_pos, c0, sink, recent):
+    return D.streaming_mask(q_pos, k_pos, sink, recent)
+
+
+def _chunk_mask_no_sink(q_pos, k_pos, c0, sink, recent):
+    qi, kj = np.asarray(q_pos)[:, None], np.asarray(k_pos)[None, :]
+    return (kj <= qi) & (kj >= c0 - recent)
+
+
+@pytest.mark.parametrize("fn", [_chunk_mask_window_short, _chunk_mask_is_lambda, _chunk_mask_no_sink])
+def test_planted_chunk_mask_mistake_is_caught(monkeypatch, fn):
+    _patch(monkeypatch, "chunk_streaming_mask", fn)
+    assert _fails(*_pins()), f"no pin caught {fn.__name__}"

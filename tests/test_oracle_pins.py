@@ -455,3 +455,51 @@ def test_int8_cache_decode_equals_direct_on_reconstructed_rows():
     assert np.max(np.abs(got - want)) < 1e-12
     pos, kc, ks, vc, vs = c.quantized(0, 2)
     assert np.array_equal(pos, np.arange(n)) and kc.shape == (n, 16) and ks.shape == (n,)
+
+
+# ---------------------------------------------------------------------------
+# Whole-chunk streaming pre-fill (the second pre-fill mode)
+# ---------------------------------------------------------------------------
+
+def test_chunk_streaming_mask_matches_hand_drawn(golden):
+    params, lines = golden("chunk_stream_mask_n10_c5_s1_r2.txt")
+    want = _mask_from_lines(lines)
+    c0 = int(params["c0"])
+    got = O.chunk_streaming_mask(np.arange(c0, c0 + want.shape[0]), np.arange(want.shape[1]), c0,
+                                 int(params["sink"]), int(params["recent"]))
+    assert np.array_equal(got, want)
+    # and it differs from the Lambda rows of the same queries
+    lam = O.streaming_mask(np.arange(c0, c0 + want.shape[0]), np.arange(want.shape[1]), 1, 2)
+    assert not np.array_equal(got, lam)
+
+
+def test_whole_chunk_streaming_first_chunk_is_causal():
+    """The first chunk has nothing cached before it, so a streaming head sees
+    its whole causal prefix: the chunk-mode pre-fill of a prompt in one chunk
+    is full causal attention for every head."""
+    rng = np.random.default_rng(21)
+    n, hq, hkv, d = 90, 4, 2, 8
+    q, k, v = _rand_qkv(rng, n, hq, hkv, d)
+    gate = np.array([0, 0], dtype=np.uint8)
+    got = O.prefill_direct(q, k, v, 0, gate, 4, 8, stream_mode="chunk")
+    want = O.prefill_direct(q, k, v, 0, np.array([1, 1], dtype=np.uint8), 4, 8)
+    np.testing.assert_allclose(got, want, atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("chunk", [1, 7, 64, 200])
+def test_whole_chunk_streaming_from_caches_equals_direct(chunk):
+    """Cache lists (sinks + recent tokens before the chunk, then the chunk
+    causally) against the direct mask over the whole history, chunk by chunk."""
+    rng = np.random.default_rng(22)
+    n, hq, hkv, d, s, r = 200, 4, 2, 8, 4, 16
+    q, k, v = _rand_qkv(rng, n, hq, hkv, d)
+    gate = np.array([1, 0], dtype=np.uint8)
+    c = O.HeadSplitCache(1, hkv, d, gate=gate, sink=s, recent=r)
+    for c0 in range(0, n, chunk):
+        c1 = min(n, c0 + chunk)
+        got = c.prefill_chunk(q[None, c0:c1], k[None, c0:c1], v[None, c0:c1], stream_mode="chunk")[0]
+        want = O.prefill_direct(q[c0:c1], k[:c1], v[:c1], c0, gate, s, r, stream_mode="chunk")
+        np.testing.assert_allclose(got, want, atol=1e-12, rtol=0)
+    # the retrieval head's rows are those of the Lambda-mode pre-fill
+    lam = O.prefill_direct(q[n - chunk:], k, v, n - chunk, gate, s, r)
+    np.testing.assert_allclose(got[:, :2], lam[-got.shape[0]:, :2], atol=1e-12, rtol=0)
