@@ -79,6 +79,7 @@ __all__ = [
     "full_attn",
     "streaming_attn",
     "gated_mix",
+    "gated_mix_grad_alpha",
     "binarize_gates",
     "partition_heads",
     "ring_slot",
@@ -225,6 +226,33 @@ def gated_mix(q, k, v, alpha, sink: int, recent: int, scale=None) -> np.ndarray:
         sa = streaming_attn(q[:, h], k[:, kv], v[:, kv], sink, recent, scale)
         out[:, h] = a * fa + (1.0 - a) * sa
     return out
+
+
+def gated_mix_grad_alpha(q, k, v, dout, sink: int, recent: int, scale=None) -> np.ndarray:
+    """Gradient of a loss with respect to the gates, given the gradient dout
+    [N, Hq, d] of the gated-mix output.  The mix is linear in alpha, with
+    d attn / d alpha = full_attn - streaming_attn for every query head of the
+    gate's KV head [Review S3 "Core formula"; S3 "Retrieval-head
+    identification": the gates are the only trained parameters], so
+
+        dalpha[kv] = sum over the group's query heads h, rows i and features
+                     of dout[i, h] * (full_attn[i, h] - streaming_attn[i, h]).
+
+    Returns float64 [Hkv]."""
+    q = np.asarray(q)
+    k = np.asarray(k)
+    v = np.asarray(v)
+    dout = as_f64(dout)
+    n, hq, d = q.shape
+    hkv = k.shape[1]
+    g = hq // hkv
+    grad = np.zeros(hkv, dtype=np.float64)
+    for h in range(hq):
+        kv = h // g
+        fa = full_attn(q[:, h], k[:, kv], v[:, kv], scale)
+        sa = streaming_attn(q[:, h], k[:, kv], v[:, kv], sink, recent, scale)
+        grad[kv] += float(np.sum(dout[:, h] * (fa - sa)))
+    return grad
 
 
 # ---------------------------------------------------------------------------

@@ -56,6 +56,9 @@ def _pins():
         lambda: P.test_chunk_streaming_mask_matches_hand_drawn(g),
         P.test_whole_chunk_streaming_first_chunk_is_causal,
         lambda: P.test_whole_chunk_streaming_from_caches_equals_direct(7),
+        lambda: P.test_grad_alpha_worked_example_d1(g),
+        P.test_grad_alpha_equals_central_difference,
+        P.test_grad_alpha_vanishes_when_the_window_covers_the_sequence,
     ]
 
 
@@ -212,3 +215,27 @@ def _chunk_mask_no_sink(q_pos, k_pos, c0, sink, recent):
 def test_planted_chunk_mask_mistake_is_caught(monkeypatch, fn):
     _patch(monkeypatch, "chunk_streaming_mask", fn)
     assert _fails(*_pins()), f"no pin caught {fn.__name__}"
+
+
+def _grad(q, k, v, dout, sink, recent, scale=None, sign=1.0, mapping="group", first_only=False, mean=False):
+    q, k, v, dout = np.asarray(q), np.asarray(k), np.asarray(v), D.as_f64(dout)
+    n, hq, _ = q.shape
+    hkv = k.shape[1]
+    g = hq // hkv
+    grad = np.zeros(hkv)
+    for h in range(hq):
+        kv = h // g if mapping == "group" else h % hkv
+        if first_only and h % g:
+            continue
+        fa = D.full_attn(q[:, h], k[:, kv], v[:, kv], scale)
+        sa = D.streaming_attn(q[:, h], k[:, kv], v[:, kv], sink, recent, scale)
+        t = float(np.sum(dout[:, h] * (fa - sa))) * sign
+        grad[kv] += t / n if mean else t
+    return grad
+
+
+@pytest.mark.parametrize("mistake", [dict(sign=-1.0), dict(mapping="interleaved"), dict(first_only=True),
+                                     dict(mean=True)])
+def test_planted_grad_alpha_mistake_is_caught(monkeypatch, mistake):
+    _patch(monkeypatch, "gated_mix_grad_alpha", lambda *a, **kw: _grad(*a, **kw, **mistake))
+    assert _fails(*_pins()), f"no pin caught {mistake}"

@@ -503,3 +503,49 @@ def test_whole_chunk_streaming_from_caches_equals_direct(chunk):
     # the retrieval head's rows are those of the Lambda-mode pre-fill
     lam = O.prefill_direct(q[n - chunk:], k, v, n - chunk, gate, s, r)
     np.testing.assert_allclose(got[:, :2], lam[-got.shape[0]:, :2], atol=1e-12, rtol=0)
+
+
+# ---------------------------------------------------------------------------
+# Gate gradient of the gated mix [Review S3 "Core formula",
+# "Retrieval-head identification"]
+# ---------------------------------------------------------------------------
+
+def test_grad_alpha_worked_example_d1(golden):
+    """d = 1 example: full = (6, 2, 7), streaming = (6, 2, 10.5); with
+    dout = (1, 1, 1) the gate gradient is 0 + 0 + (7 - 10.5) = -3.5, and with
+    dout = (0, 0, 2) it is -7."""
+    params, _ = golden("tiny_attention_d1.txt")
+    q = np.ones((3, 1, 1))
+    k = np.array([0.0, math.log(2), math.log(3)]).reshape(3, 1, 1)
+    v = np.array([6.0, 0.0, 12.0]).reshape(3, 1, 1)
+    fa, sa = np.array(params["full"]), np.array(params["streaming"])
+    for dout, want in ((np.ones(3), -3.5), (np.array([0.0, 0.0, 2.0]), -7.0)):
+        got = O.gated_mix_grad_alpha(q, k, v, dout.reshape(3, 1, 1), 1, 1, scale=1.0)
+        assert abs(got[0] - want) < 1e-12
+        assert abs(got[0] - float(np.dot(dout, fa - sa))) < 1e-12
+
+
+def test_grad_alpha_equals_central_difference():
+    """The mix is linear in alpha, so a central difference of <dout, mix>
+    equals the gradient up to rounding."""
+    rng = np.random.default_rng(31)
+    n, hq, hkv, d, s, r = 60, 8, 4, 8, 2, 9
+    q, k, v = _rand_qkv(rng, n, hq, hkv, d)
+    dout = rng.standard_normal((n, hq, d))
+    alpha = rng.uniform(0, 1, hkv)
+    got = O.gated_mix_grad_alpha(q, k, v, dout, s, r)
+    for kv in range(hkv):
+        e = np.zeros(hkv)
+        e[kv] = 1e-3
+        fd = (np.sum(dout * O.gated_mix(q, k, v, alpha + e, s, r)) -
+              np.sum(dout * O.gated_mix(q, k, v, alpha - e, s, r))) / 2e-3
+        assert abs(fd - got[kv]) < 1e-8 * max(1.0, abs(got[kv]))
+
+
+def test_grad_alpha_vanishes_when_the_window_covers_the_sequence():
+    rng = np.random.default_rng(32)
+    n, hq, hkv, d = 40, 4, 2, 8
+    q, k, v = _rand_qkv(rng, n, hq, hkv, d)
+    dout = rng.standard_normal((n, hq, d))
+    assert np.all(np.abs(O.gated_mix_grad_alpha(q, k, v, dout, 8, 32)) < 1e-12)
+    assert np.any(np.abs(O.gated_mix_grad_alpha(q, k, v, dout, 2, 5)) > 1e-3)
