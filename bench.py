@@ -526,11 +526,14 @@ def _lambda_pairs(p0: int, n: int, sink: int, recent: int) -> int:
     return int((sinks + band - both).sum())
 
 
-def _prefill_flops(n_ret_q, n_str_q, d, c0, C, sink, recent):
+def _prefill_flops(n_ret_q, n_str_q, d, c0, C, sink, recent, stream_chunk=False):
     """Algorithmic FLOPs of one chunk: 4*d per visible (query, key) pair and
-    query head (2*d for Q K^T, 2*d for P V); masked pairs are not counted."""
+    query head (2*d for Q K^T, 2*d for P V); masked pairs are not counted.
+    Whole-chunk streaming: every query sees the min(c0, sink + recent) cached
+    tokens and the chunk up to itself."""
     causal = C * c0 + C * (C + 1) // 2
-    return 4 * d * (n_ret_q * causal + n_str_q * _lambda_pairs(c0, C, sink, recent))
+    stream = (C * min(c0, sink + recent) + C * (C + 1) // 2) if stream_chunk else _lambda_pairs(c0, C, sink, recent)
+    return 4 * d * (n_ret_q * causal + n_str_q * stream)
 
 
 def run_prefill(args, wl, world, rank, steps=None, warmup=None):
@@ -547,7 +550,9 @@ def run_prefill(args, wl, world, rank, steps=None, warmup=None):
     warmup = 3 if warmup is None else warmup
     retrieval = S.retrieval_heads_by_seed(wl["hkv"], wl["n_ret"], seed=1)
     gate, perm, inv, R = duo.partition_heads(S.binary_alpha(wl["hkv"], retrieval), 0.5)
-    desc = duo.desc_init(1, sh.n_q_heads, sh.n_kv_heads, sh.head_dim, duo.BF16, perm, R)
+    stream_chunk = wl.get("stream") == "chunk"
+    desc = duo.desc_init(1, sh.n_q_heads, sh.n_kv_heads, sh.head_dim, duo.BF16, perm, R,
+                         stream_prefill=duo.STREAM_CHUNK if stream_chunk else duo.STREAM_LAMBDA)
     caches = duo.LayerCaches(desc, n)
     q, k, v = S.prompt(sh, n, seed=0)
     qd, kd, vd = _to_dev(q), _to_dev(k), _to_dev(v)
@@ -592,7 +597,7 @@ def run_prefill(args, wl, world, rank, steps=None, warmup=None):
         raise RuntimeError(f"device status 0x{st_code:x} after the timed chunks")
     pre_ms = [a.elapsed_time(b) for a, b, _ in ev]
     step_ms = [a.elapsed_time(c) for a, _, c in ev]
-    flops = [_prefill_flops(R * G, (sh.n_kv_heads - R) * G, sh.head_dim, i * C, C, sh.sink, sh.recent)
+    flops = [_prefill_flops(R * G, (sh.n_kv_heads - R) * G, sh.head_dim, i * C, C, sh.sink, sh.recent, stream_chunk)
              for i in range(steps)]
     total_ms = _max_over_ranks(sum(step_ms), world)
     _, tf_peak, peak_kind = _peaks()
@@ -747,6 +752,33 @@ def run_ratio_sweep(args, world, rank):
                         "fit_ms_vs_ratio": _linear_fit([d["ratio"] for d in pre], [d["ms_total"] for d in pre])}}
 
 
+def run_chunk_sweep(args, world, rank):
+    """Pre-fill time of the 32K-token GQA prompt against the chunk length,
+    with streaming heads in Lambda mode and in whole-chunk mode, next to the
+    same prompt with every KV head retrieval (full attention).  The pages
+    report the pre-fill speed-up over full attention growing as the chunk
+    shrinks ([Review] S5 "Pre-filling performance")."""
+    import copy
+    a2 = copy.copy(args)
+    a2.no_cpu_baseline = True
+    base = WORKLOADS["gqa_prefill_32k"]
+    rows = []
+    for C in (512, 1024, 2048, 4096, 8192):
+        point = {"chunk": C}
+        for tag, extra in (("full", dict(n_ret=base["hkv"])), ("lambda", {}), ("chunk", dict(stream="chunk"))):
+            wl = dict(base, chunk=C, name="gqa_prefill_32k", **extra)
+            res = run_prefill(a2, wl, world, rank, warmup=3)
+            point[tag + "_ms"] = res["roofline"]["prefill_ms_total"]
+            point[tag + "_tflops"] = res["roofline"]["achieved"]
+        point["speedup_lambda"] = round(point["full_ms"] / point["lambda_ms"], 3)
+        point["speedup_chunk"] = round(point["full_ms"] / point["chunk_ms"], 3)
+        rows.append(point)
+    return {"metric": "pre-fill ms vs chunk length; speed-up over full attention", "n_gpus": world,
+            "data": "synthetic",
+            "workload": "gqa_prefill_32k (32 query / 8 KV heads, 4 retrieval, 32,768 tokens); full = 8 retrieval",
+            "points": rows}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -761,10 +793,20 @@ def main(argv=None):
                     help="decode: layers per step, each with its own caches (their total exceeds L2)")
     ap.add_argument("--retrieval-ratio-sweep", action="store_true",
                     help="time decode and pre-fill against the share of retrieval heads (one JSON line)")
+    ap.add_argument("--chunk-sweep", action="store_true",
+                    help="time the pre-fill against the chunk length, both streaming modes (one JSON line)")
+    ap.add_argument("--n-retrieval", type=int, default=None,
+                    help="override the workload's number of retrieval KV heads (profiling)")
+    ap.add_argument("--stream-prefill", choices=["lambda", "chunk"], default="lambda",
+                    help="pre-fill workloads: what streaming heads see inside a chunk")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    wl = WORKLOADS[args.workload]
+    wl = dict(WORKLOADS[args.workload])
+    if args.n_retrieval is not None:
+        wl["n_ret"] = args.n_retrieval
+    if args.stream_prefill == "chunk":
+        wl["stream"] = "chunk"
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
@@ -780,6 +822,8 @@ def main(argv=None):
     try:
         if args.retrieval_ratio_sweep:
             res = run_ratio_sweep(args, world, rank)
+        elif args.chunk_sweep:
+            res = run_chunk_sweep(args, world, rank)
         elif wl["kind"] == "decode":
             res = run_decode(args, wl, world, rank)
             if not args.no_prefill:

@@ -61,6 +61,8 @@ duo_status check_desc(const duo_layer_desc* d) {
         return fail(DUO_ERR_SHAPE, "n_retrieval %d outside 0..%d", d->n_retrieval, d->n_kv_heads);
     if (d->io_order != DUO_ORDER_MODEL && d->io_order != DUO_ORDER_BLOCK)
         return fail(DUO_ERR_INVALID_ARG, "unknown io_order %d", d->io_order);
+    if (d->stream_prefill != DUO_STREAM_LAMBDA && d->stream_prefill != DUO_STREAM_CHUNK)
+        return fail(DUO_ERR_INVALID_ARG, "unknown stream_prefill %d", d->stream_prefill);
     if (!std::isfinite(d->scale)) return fail(DUO_ERR_INVALID_ARG, "scale is not finite");
     bool seen[DUO_MAX_KV_HEADS] = {};
     for (int i = 0; i < d->n_kv_heads; ++i) {
@@ -85,6 +87,7 @@ void fill_args(const duo_layer_desc* d, duo::LayerArgs& a) {
     a.recent = d->recent;
     a.W = d->sink + d->recent;
     a.dtype = d->dtype;
+    a.stream_chunk = d->stream_prefill == DUO_STREAM_CHUNK ? 1 : 0;
     a.page_size = d->page_size;
     a.capacity = a.max_pages = a.n_pages = 0;
     a.scale = d->scale > 0.f ? d->scale : 1.0f / std::sqrt(static_cast<float>(d->head_dim));
@@ -193,7 +196,7 @@ const char* duo_status_string(duo_status s) {
     return "DUO_ERR_UNKNOWN";
 }
 
-int32_t duo_abi_version(void) { return 1; }
+int32_t duo_abi_version(void) { return 2; }
 
 duo_status duo_partition_heads(const float* alpha, int32_t n_kv_heads, float tau, int32_t target_n_retrieval,
                                uint8_t* gate, int32_t* kv_perm, int32_t* kv_inv_perm, int32_t* n_retrieval) {
@@ -243,6 +246,7 @@ duo_status duo_desc_init(duo_layer_desc* desc, int32_t batch, int32_t n_q_heads,
     desc->scale = 0.f;
     desc->n_retrieval = n_retrieval;
     desc->io_order = DUO_ORDER_MODEL;
+    desc->stream_prefill = DUO_STREAM_LAMBDA;
     if (n_kv_heads < 1 || n_kv_heads > DUO_MAX_KV_HEADS)
         return fail(DUO_ERR_INVALID_ARG, "n_kv_heads must be in 1..%d (got %d)", DUO_MAX_KV_HEADS, n_kv_heads);
     for (int i = 0; i < n_kv_heads; ++i) desc->kv_perm[i] = kv_perm[i];
@@ -391,6 +395,29 @@ duo_status duo_gated_mix(const duo_layer_desc* desc, const float* alpha, const v
     }
     const cudaError_t e = duo::launch_simt_attention(a, nullptr, alpha, q, k, v, N, out, 1, (cudaStream_t)stream);
     return e == cudaSuccess ? ok() : cuda_fail(e, "duo_gated_mix");
+}
+
+duo_status duo_gated_mix_grad_alpha(const duo_layer_desc* desc, const void* q, const void* k, const void* v,
+                                    int32_t N, const void* dout, float* dalpha, duo_stream_t stream) {
+    duo_status s = check_desc(desc);
+    if (s != DUO_OK) return s;
+    if (!q || !k || !v || !dout || !dalpha)
+        return fail(DUO_ERR_INVALID_ARG, "duo_gated_mix_grad_alpha: NULL argument");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout))
+        return fail(DUO_ERR_INVALID_ARG, "duo_gated_mix_grad_alpha tensors must be 16-byte aligned");
+    if (N < 0) return fail(DUO_ERR_SHAPE, "N must be >= 0 (got %d)", N);
+    cudaError_t e = cudaMemsetAsync(dalpha, 0, sizeof(float) * desc->n_kv_heads, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "duo_gated_mix_grad_alpha");
+    if (N == 0) return ok();
+    duo::LayerArgs a;
+    fill_args(desc, a);
+    for (int i = 0; i < a.Hkv; ++i) {   // model head order, as for duo_gated_mix
+        a.kv_head[i] = i;
+        a.q_head0[i] = i * a.G;
+        a.slot_of[i] = i;
+    }
+    e = duo::launch_simt_attention(a, nullptr, nullptr, q, k, v, N, nullptr, 2, (cudaStream_t)stream, dout, dalpha);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "duo_gated_mix_grad_alpha");
 }
 
 duo_status duo_check_status(const duo_kv_state* st, int32_t* host_status, duo_stream_t stream) {

@@ -16,6 +16,7 @@ namespace duo {
 struct LayerArgs {
     int B, Hq, Hkv, G, D, R, S, sink, recent, W;
     int dtype, page_size, capacity, max_pages, n_pages;
+    int stream_chunk;  // pre-fill: streaming heads see the whole chunk (DUO_STREAM_CHUNK)
     float scale;       // softmax scale
     // For block slot i (0..Hkv-1): index of its first query head and of its
     // KV head in the caller's q / k / v / out tensors (model or block order).
@@ -54,9 +55,11 @@ cudaError_t launch_append(const LayerArgs& a, const CacheArgs& c, const void* k_
 cudaError_t launch_decode(const LayerArgs& a, const CacheArgs& c, const DecodePlan& plan, const void* q, void* out,
                           void* workspace, cudaStream_t s, const void* k_new = nullptr,
                           const void* v_new = nullptr);
-// CUDA-core attention: chunked pre-fill (mode 0) or gated mix (mode 1).
+// CUDA-core attention: chunked pre-fill (mode 0), gated mix (mode 1) or the
+// gated mix's gate gradient (mode 2: dout in, dalpha accumulated).
 cudaError_t launch_simt_attention(const LayerArgs& a, const CacheArgs* c, const float* alpha, const void* q,
-                                  const void* k, const void* v, int n_tokens, void* out, int mode, cudaStream_t s);
+                                  const void* k, const void* v, int n_tokens, void* out, int mode, cudaStream_t s,
+                                  const void* dout = nullptr, float* dalpha = nullptr);
 // tcgen05 pre-fill for bf16, d = 128; returns cudaErrorNotSupported when it
 // cannot take the call.
 cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void* q, const void* k_chunk,

@@ -14,7 +14,9 @@
 //     stops one tile earlier when the last tile lies wholly above its diagonal;
 //   streaming head: the ring (sinks + recent tokens before c0, positions from
 //     ring_pos), the chunk's sink tile when c0 < sink, and the chunk tiles of
-//     the two tiles' recent bands -- a handful of tiles at any context length.
+//     the two tiles' recent bands -- a handful of tiles at any context length;
+//     in whole-chunk mode (DUO_STREAM_CHUNK) the ring, then the chunk's keys up
+//     to Q1's diagonal, masked like a retrieval head's chunk tiles.
 // TMEM: S0 | S1 | O0 | O1, 128 columns each.  After softmax warpgroup i has
 // read S_i it writes P_i as packed bf16 over the last 64 columns of S_i, and
 // the PV product reads P_i from TMEM (the A operand), so P never touches
@@ -84,6 +86,7 @@ struct TcArgs {
 // Tiles are listed in visiting order; tile j is described by tile_at(j).
 struct Sched {
     bool retrieval;
+    bool chunk;      // streaming head in whole-chunk mode: ring, then the chunk causally
     int c0;          // chunk start position (cached tokens before the chunk)
     int m;           // query-tile pair: chunk rows 256m .. 256m+255
     int n;           // tiles visited by Q1
@@ -106,12 +109,19 @@ __device__ __forceinline__ Sched make_sched(const TcArgs& p, bool retrieval, int
     s.m = m;
     const int n_ct = (p.C + BN - 1) / BN;                 // chunk tiles that hold keys
     const int hi = min(2 * m + 1, n_ct - 1);              // last chunk tile (Q1's diagonal)
+    s.chunk = !retrieval && a.stream_chunk;
     if (retrieval) {
         s.n_prior = (c0 + BN - 1) / BN;
         s.n_ring = 0;
         s.sink_tile = 0;
         s.lo = 0;
         s.n = s.n_prior + hi + 1;
+    } else if (s.chunk) {
+        s.n_prior = 0;
+        s.n_ring = min(c0, a.W) > 0 ? 1 : 0;
+        s.sink_tile = 0;
+        s.lo = 0;
+        s.n = s.n_ring + hi + 1;
     } else {
         s.n_prior = 0;
         s.n_ring = min(c0, a.W) > 0 ? 1 : 0;
@@ -152,11 +162,12 @@ __device__ __forceinline__ Tile tile_at(const Sched& s, int j) {
     return t;
 }
 
-// Whether query tile `qi` needs the mask on tile j: every streaming tile, the
-// retrieval tile that starts before position 0, and the chunk tiles that
-// reach past the tile's first row.
+// Whether query tile `qi` needs the mask on tile j: every Lambda-mode
+// streaming tile and ring tile, the retrieval tile that starts before
+// position 0, and the chunk tiles that reach past the query tile's first row.
 __device__ __forceinline__ bool needs_mask(const Sched& s, const Tile& t, int qi) {
-    if (!s.retrieval) return true;
+    if (!s.retrieval && !s.chunk) return true;
+    if (t.src == SRC_RING) return true;
     if (t.src == SRC_CACHE) return t.row < 0;
     return t.row + BN - 1 > BM * (2 * s.m + qi);
 }
@@ -353,7 +364,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < 64; ++c) {
                     const int kp = t.src == SRC_RING ? sPos[c_base + c] : t.pos0 + c_base + c;
                     bool vis = kp >= 0 && kp <= P;
-                    if (!sc.retrieval) vis = vis && (kp < a.sink || P - kp < a.recent);
+                    if (!sc.retrieval)
+                        vis = vis && (kp < a.sink || (sc.chunk ? kp >= sc.c0 - a.recent : P - kp < a.recent));
                     if (!vis) v[c] = -INFINITY;
                 }
             };

@@ -5,10 +5,15 @@
 //   mode 0, chunked pre-fill [Summary S2 "Chunked Pre-filling"]: the queries
 //     of a chunk attend to the caches as they stand plus the chunk's own keys;
 //     retrieval heads causally over the full cache, streaming heads under the
-//     Lambda mask over the ring (positions from ring_pos) and the chunk.
+//     Lambda mask over the ring (positions from ring_pos) and the chunk, or in
+//     whole-chunk mode over the ring and the chunk causally.
 //   mode 1, gated mix [Review S3 "Core formula"]: every head over the whole
 //     sequence, alpha * causal + (1 - alpha) * Lambda; one score per (query,
 //     key) feeds both online-softmax states.
+//   mode 2, gate gradient of the gated mix [Review S3 "Core formula",
+//     "Retrieval-head identification": the gates are what training updates]:
+//     the same two attentions per row, then dout . (causal - Lambda) summed
+//     over the CTA's rows and added atomically into dalpha[kv].
 //
 // A CTA holds 32 query rows of one query head; four threads share a row, each
 // with a quarter of the head dimension, and reduce the dot product with two
@@ -29,8 +34,10 @@ struct SimtArgs {
     const void* v;
     void* out;
     const float* alpha;   // mode 1
-    int n_tokens;         // C (mode 0) or N (mode 1)
+    int n_tokens;         // C (mode 0) or N (modes 1, 2)
     int mode;
+    const void* dout;     // mode 2: [B][N][Hq][D]
+    float* dalpha;        // mode 2: [Hkv], accumulated
 };
 
 template <typename T, int D>
@@ -50,7 +57,7 @@ __global__ void __launch_bounds__(kThreadsSimt) simt_attention_kernel(const Laye
     const int row = r0 + (threadIdx.x >> 2);
     const int quarter = threadIdx.x & 3;
     const int N = s.n_tokens;
-    const bool mix = s.mode == 1;
+    const bool mix = s.mode >= 1;       // modes 1 and 2 run both attentions over the whole sequence
     const bool retrieval = slot < a.R;
 
     int c0 = 0;
@@ -85,6 +92,10 @@ __global__ void __launch_bounds__(kThreadsSimt) simt_attention_kernel(const Laye
     } else if (retrieval) {
         seg_begin[0] = 0; seg_end[0] = c0;
         seg_begin[1] = 0; seg_end[1] = last_row;
+        seg_begin[2] = seg_end[2] = 0;
+    } else if (a.stream_chunk) {
+        seg_begin[0] = 0; seg_end[0] = a.W;                                    // ring slots
+        seg_begin[1] = 0; seg_end[1] = last_row;                               // the whole chunk
         seg_begin[2] = seg_end[2] = 0;
     } else {
         seg_begin[0] = 0; seg_end[0] = a.W;                                    // ring slots
@@ -141,7 +152,8 @@ __global__ void __launch_bounds__(kThreadsSimt) simt_attention_kernel(const Laye
                 part += __shfl_xor_sync(0xffffffffu, part, 2);
                 const int kp = sPos[j];
                 const bool causal = kp >= 0 && kp <= qpos;
-                const bool lam = causal && (kp < a.sink || qpos - kp < a.recent);
+                const bool lam = causal && (kp < a.sink || (a.stream_chunk && !mix ? kp >= c0 - a.recent
+                                                                                   : qpos - kp < a.recent));
                 const bool vis0 = mix ? causal : (retrieval ? causal : lam);
                 if (vis0) {
                     const float mn = fmaxf(m0, part);
@@ -161,6 +173,28 @@ __global__ void __launch_bounds__(kThreadsSimt) simt_attention_kernel(const Laye
                 }
             }
         }
+    }
+    if (s.mode == 2) {
+        // this row's dout . (causal - Lambda), then the CTA's sum, once per CTA
+        __shared__ float sPart[kThreadsSimt / 32];
+        float part = 0.f;
+        if (row_ok) {
+            const T* dp = static_cast<const T*>(s.dout) + (((size_t)b * N + row) * a.Hq + q_idx) * D + quarter * QD;
+#pragma unroll
+            for (int e = 0; e < QD; ++e)
+                part = fmaf(Elem<T>::to_f32(dp[e]), (l0 > 0.f ? o0[e] / l0 : 0.f) - (l1 > 0.f ? o1[e] / l1 : 0.f), part);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if ((threadIdx.x & 31) == 0) sPart[threadIdx.x >> 5] = part;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float sum = 0.f;
+#pragma unroll
+            for (int w = 0; w < kThreadsSimt / 32; ++w) sum += sPart[w];
+            atomicAdd(&s.dalpha[kv_idx], sum);
+        }
+        return;
     }
     if (!row_ok) return;
     float res[QD];
@@ -188,8 +222,9 @@ cudaError_t launch_simt_t(const LayerArgs& a, const CacheArgs& c, const SimtArgs
 }  // namespace
 
 cudaError_t launch_simt_attention(const LayerArgs& a, const CacheArgs* c, const float* alpha, const void* q,
-                                  const void* k, const void* v, int n_tokens, void* out, int mode, cudaStream_t st) {
-    SimtArgs s{q, k, v, out, alpha, n_tokens, mode};
+                                  const void* k, const void* v, int n_tokens, void* out, int mode, cudaStream_t st,
+                                  const void* dout, float* dalpha) {
+    SimtArgs s{q, k, v, out, alpha, n_tokens, mode, dout, dalpha};
     CacheArgs cc{};
     if (c) cc = *c;
     if (a.B > 65535 || a.Hq > 65535) return cudaErrorInvalidConfiguration;

@@ -26,6 +26,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_DTYPE, ERR_CAPACITY, ERR_UNSUPPORTED, ERR_CUDA, ERR_DEVICE = range(8)
 BF16, FP32 = 0, 1
 ORDER_MODEL, ORDER_BLOCK = 0, 1
+STREAM_LAMBDA, STREAM_CHUNK = 0, 1
 MODEL_TO_BLOCK, BLOCK_TO_MODEL = 0, 1
 OP_DECODE, OP_PREFILL = 0, 1
 DEV_FULL_CACHE_OVERFLOW, DEV_BAD_PAGE, DEV_WAIT_TIMEOUT, DEV_BAD_LENGTH = 1, 2, 4, 8
@@ -38,7 +39,7 @@ class LayerDesc(ctypes.Structure):
         ("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
         ("head_dim", ctypes.c_int32), ("sink", ctypes.c_int32), ("recent", ctypes.c_int32),
         ("dtype", ctypes.c_int32), ("page_size", ctypes.c_int32), ("scale", ctypes.c_float),
-        ("n_retrieval", ctypes.c_int32), ("io_order", ctypes.c_int32),
+        ("n_retrieval", ctypes.c_int32), ("io_order", ctypes.c_int32), ("stream_prefill", ctypes.c_int32),
         ("kv_perm", ctypes.c_int32 * MAX_KV_HEADS),
     ]
 
@@ -69,6 +70,9 @@ def _fn(name, restype, *argtypes):
 _lib_last_error = _fn("duo_last_error", ctypes.c_char_p)
 _lib_status_string = _fn("duo_status_string", ctypes.c_char_p, ctypes.c_int)
 _lib_abi_version = _fn("duo_abi_version", _I32)
+ABI_VERSION = 2           # the layout of LayerDesc / KVState below
+if _lib_abi_version() != ABI_VERSION:
+    raise ImportError(f"{LIB_PATH} has ABI version {_lib_abi_version()}, this binding needs {ABI_VERSION}; rebuild it")
 _lib_partition = _fn("duo_partition_heads", ctypes.c_int, ctypes.POINTER(ctypes.c_float), _I32, ctypes.c_float,
                      _I32, ctypes.POINTER(ctypes.c_uint8), ctypes.POINTER(_I32), ctypes.POINTER(_I32),
                      ctypes.POINTER(_I32))
@@ -81,6 +85,7 @@ _lib_append = _fn("duo_append_kv", ctypes.c_int, _DESC, _STATE, _P, _P, _I32, _P
 _lib_decode = _fn("duo_decode_attn", ctypes.c_int, _DESC, _STATE, _P, _P, _P, ctypes.c_size_t, _P)
 _lib_prefill = _fn("duo_prefill_chunk", ctypes.c_int, _DESC, _STATE, _P, _P, _P, _I32, _P, _P, ctypes.c_size_t, _P)
 _lib_mix = _fn("duo_gated_mix", ctypes.c_int, _DESC, _P, _P, _P, _P, _I32, _P, _P)
+_lib_mix_grad = _fn("duo_gated_mix_grad_alpha", ctypes.c_int, _DESC, _P, _P, _P, _I32, _P, _P, _P)
 _lib_check = _fn("duo_check_status", ctypes.c_int, _STATE, ctypes.POINTER(_I32), _P)
 _lib_decode_step = _fn("duo_decode_step", ctypes.c_int, _DESC, _STATE, _P, _P, _P, _P, _P, ctypes.c_size_t, _P)
 _lib_decode_noalloc = _fn("duo_decode_attn_noalloc", ctypes.c_int, _DESC, _STATE, _P, _P, _P)
@@ -145,7 +150,7 @@ def partition_heads(alpha, tau: float, target_n_retrieval: int = -1):
 
 
 def desc_init(batch, n_q_heads, n_kv_heads, head_dim, dtype, kv_perm, n_retrieval, *, sink=None, recent=None,
-              page_size=0, io_order=ORDER_MODEL, scale=0.0) -> LayerDesc:
+              page_size=0, io_order=ORDER_MODEL, scale=0.0, stream_prefill=STREAM_LAMBDA) -> LayerDesc:
     d = LayerDesc()
     perm = (_I32 * max(len(kv_perm), 1))(*[int(p) for p in kv_perm])
     _check(_lib_desc_init(ctypes.byref(d), batch, n_q_heads, n_kv_heads, head_dim, dtype, perm, n_retrieval),
@@ -157,6 +162,7 @@ def desc_init(batch, n_q_heads, n_kv_heads, head_dim, dtype, kv_perm, n_retrieva
     d.page_size = page_size
     d.io_order = io_order
     d.scale = scale
+    d.stream_prefill = stream_prefill
     _check(_lib_desc_validate(ctypes.byref(d)), "duo_desc_validate")
     return d
 
@@ -210,6 +216,11 @@ def prefill_chunk(desc, state: KVState, q, k_chunk, v_chunk, C: int, out, worksp
 def gated_mix(desc, alpha, q, k, v, N: int, out, stream=None) -> None:
     _check(_lib_mix(ctypes.byref(desc), _ptr(alpha), _ptr(q), _ptr(k), _ptr(v), N, _ptr(out), _stream(stream)),
            "duo_gated_mix")
+
+
+def gated_mix_grad_alpha(desc, q, k, v, N: int, dout, dalpha, stream=None) -> None:
+    _check(_lib_mix_grad(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), N, _ptr(dout), _ptr(dalpha),
+                         _stream(stream)), "duo_gated_mix_grad_alpha")
 
 
 def check_status(state: KVState, stream=None, raise_on_error: bool = False) -> int:

@@ -68,6 +68,11 @@ typedef enum {
 enum { DUO_BF16 = 0, DUO_FP32 = 1 };
 /* head order of q / k / v / out */
 enum { DUO_ORDER_MODEL = 0, DUO_ORDER_BLOCK = 1 };
+/* what a streaming head sees in duo_prefill_chunk (decode is the same for both) */
+enum {
+    DUO_STREAM_LAMBDA = 0, /* the Lambda mask per query: sinks + its last `recent` tokens */
+    DUO_STREAM_CHUNK = 1   /* sinks + the `recent` tokens before the chunk + the whole chunk up to itself */
+};
 /* duo_permute_heads directions */
 enum { DUO_MODEL_TO_BLOCK = 0, DUO_BLOCK_TO_MODEL = 1 };
 /* workspace queries */
@@ -96,6 +101,7 @@ typedef struct {
     float scale;          /* softmax scale; 1/sqrt(d) when <= 0               */
     int32_t n_retrieval;  /* R: retrieval KV heads (block slots 0..R-1)       */
     int32_t io_order;     /* DUO_ORDER_MODEL or DUO_ORDER_BLOCK               */
+    int32_t stream_prefill; /* DUO_STREAM_LAMBDA (default) or DUO_STREAM_CHUNK */
     int32_t kv_perm[DUO_MAX_KV_HEADS]; /* block slot i holds model KV head kv_perm[i] */
 } duo_layer_desc;
 
@@ -145,7 +151,7 @@ typedef struct {
 const char* duo_last_error(void);
 /* Name of a status code. */
 const char* duo_status_string(duo_status s);
-/* ABI version: 1. */
+/* ABI version: 2 (duo_layer_desc gained stream_prefill). */
 int32_t duo_abi_version(void);
 
 /* ------------------------------------------------------------------------ */
@@ -282,10 +288,15 @@ duo_status duo_decode_step(const duo_layer_desc* desc, const duo_kv_state* st, c
  * Call BEFORE duo_append_kv of the same chunk: the caches hold tokens
  * 0..seq_len[b]-1 and the chunk's own keys come from k_chunk / v_chunk.
  * q [B][C][Hq][d]; k_chunk, v_chunk [B][C][Hkv][d]; out [B][C][Hq][d].
- * Query c of the chunk has position P = seq_len[b] + c.
+ * Query c of the chunk has position P = seq_len[b] + c; c0 = seq_len[b].
  *   Retrieval head: keys 0..P (causal), prior ones from the full cache.
- *   Streaming head: keys j <= P with j < sink or P - j < recent (Lambda),
- *     prior ones from the ring.
+ *   Streaming head, desc->stream_prefill = DUO_STREAM_LAMBDA: keys j <= P
+ *     with j < sink or P - j < recent (Lambda), prior ones from the ring.
+ *   Streaming head, DUO_STREAM_CHUNK: keys j <= P with j < sink or
+ *     j >= c0 - recent -- the ring as it stood before the chunk and the whole
+ *     chunk up to the query (the reading under which pre-fill gains grow as
+ *     the chunk shrinks [Review S5 "Pre-filling performance"]); the first
+ *     chunk of a prompt is then causal for every head.
  * bf16 with d = 128 runs on the tcgen05 tensor cores (TMA-fed tiles, TMEM
  * accumulators); fp32 and d = 64 run on the CUDA cores.
  * workspace: >= duo_workspace_bytes(desc, DUO_OP_PREFILL, C) bytes (may be 0).
@@ -346,6 +357,24 @@ duo_status duo_gated_mix(const duo_layer_desc* desc, const float* alpha, const v
 #define DUO_NOALLOC_SCRATCH_BYTES (2u << 20)
 duo_status duo_decode_attn_noalloc(const duo_layer_desc* desc, const duo_kv_state* st, const void* q,
                                    void* out, duo_stream_t stream);
+
+/*
+ * duo_gated_mix_grad_alpha -- gradient of a loss with respect to the gates of
+ * duo_gated_mix, given the gradient dout of its output.  The mix is linear
+ * in alpha, d attn / d alpha = full_attn - streaming_attn [Review S3 "Core
+ * formula"], and the gates are the only parameters head identification
+ * trains [Review S3 "Retrieval-head identification"], so
+ *   dalpha[kv] = sum over the query heads h of KV head kv, the sequences,
+ *                rows i and features of dout[i][h] * (full - streaming)[i][h].
+ *
+ * q [B][N][Hq][d]; k, v [B][N][Hkv][d]; dout [B][N][Hq][d] (same dtype);
+ * model head order as for duo_gated_mix.  dalpha [Hkv] fp32 device: zeroed
+ * by the call, then accumulated with atomics (one add per 32 rows), so the
+ * last bits vary with the order the CTAs finish in.
+ * Errors: DUO_ERR_INVALID_ARG, DUO_ERR_SHAPE, DUO_ERR_UNSUPPORTED, DUO_ERR_CUDA.
+ */
+duo_status duo_gated_mix_grad_alpha(const duo_layer_desc* desc, const void* q, const void* k, const void* v,
+                                    int32_t N, const void* dout, float* dalpha, duo_stream_t stream);
 
 /*
  * duo_check_status -- synchronise `stream`, copy the state's device status

@@ -55,7 +55,7 @@ class Layer:
     """One attention layer on the device plus its oracle twin."""
 
     def __init__(self, duo, shape: S.LayerShape, retrieval, batch: int, capacity: int = 0, page_size: int = 0,
-                 page_table=None, n_pages: int = 0, io_order=None):
+                 page_table=None, n_pages: int = 0, io_order=None, stream_prefill: int = 0):
         self.duo = duo
         self.shape = shape
         self.B = batch
@@ -68,7 +68,7 @@ class Layer:
         self.desc = duo.desc_init(batch, shape.n_q_heads, hkv, shape.head_dim,
                                   duo.BF16 if shape.dtype == "bf16" else duo.FP32, self.perm, self.R,
                                   sink=shape.sink, recent=shape.recent, page_size=page_size,
-                                  io_order=self.io_order)
+                                  io_order=self.io_order, stream_prefill=stream_prefill)
         self.page_table = None if page_table is None else np.asarray(page_table, dtype=np.int32)
         self.caches = duo.LayerCaches(self.desc, capacity, self.page_table, n_pages)
         self.oracle = O.HeadSplitCache(batch, hkv, shape.head_dim, gate=self.gate, sink=shape.sink,

@@ -64,7 +64,7 @@ int main(void) {
 
 
 def test_abi_version_and_status_strings(duo):
-    assert duo.abi_version() == 1
+    assert duo.abi_version() == duo.ABI_VERSION == 2
     assert duo.status_string(duo.OK) == "DUO_OK"
     assert duo.status_string(duo.ERR_CAPACITY) == "DUO_ERR_CAPACITY"
 
@@ -219,3 +219,11 @@ def test_permute_rejects_overlap(duo):
     with pytest.raises(duo.DuoError) as e:
         duo.permute_heads(d, 4096, 4096 + 64, 4, 4, 128, 2, duo.MODEL_TO_BLOCK, stream=0)
     assert e.value.status == duo.ERR_INVALID_ARG
+
+
+def test_stream_prefill_mode_is_validated(duo):
+    d = duo.desc_init(1, 8, 4, 128, duo.BF16, [0, 1, 2, 3], 2, stream_prefill=duo.STREAM_CHUNK)
+    assert d.stream_prefill == duo.STREAM_CHUNK and duo.desc_validate(d) == duo.OK
+    assert duo.desc_init(1, 8, 4, 128, duo.BF16, [0, 1, 2, 3], 2).stream_prefill == duo.STREAM_LAMBDA
+    d.stream_prefill = 2
+    assert duo.desc_validate(d) == duo.ERR_INVALID_ARG

@@ -234,8 +234,9 @@ def test_decode_batch64_paged_full(duo):
 # duo_prefill_chunk on the CUDA cores (fp32, d = 64) and duo_gated_mix
 # ---------------------------------------------------------------------------
 
-def _prefill_run(duo, sh, retrieval, n, chunk, B=1, seed=0, check_cache=True):
-    lay = Layer(duo, sh, retrieval, B, capacity=n + 8)
+def _prefill_run(duo, sh, retrieval, n, chunk, B=1, seed=0, check_cache=True, stream_mode="lambda"):
+    lay = Layer(duo, sh, retrieval, B, capacity=n + 8,
+                stream_prefill=duo.STREAM_CHUNK if stream_mode == "chunk" else duo.STREAM_LAMBDA)
     q, k, v = S.prompt(sh, n, seed=seed, batch=B)
     t = torch()
     outs = []
@@ -254,7 +255,12 @@ def _prefill_run(duo, sh, retrieval, n, chunk, B=1, seed=0, check_cache=True):
             lay.assert_caches_match()
     got = np.concatenate(outs, axis=1)
     for b in range(B):
-        want = O.prefill_direct(q[b], k[b], v[b], 0, np.array(lay.gate), sh.sink, sh.recent)
+        if stream_mode == "chunk":      # the direct definition depends on where each chunk starts
+            want = np.concatenate([O.prefill_direct(q[b, c0:c0 + chunk], k[b, :c0 + chunk], v[b, :c0 + chunk], c0,
+                                                    np.array(lay.gate), sh.sink, sh.recent, stream_mode="chunk")
+                                   for c0 in range(0, n, chunk)])
+        else:
+            want = O.prefill_direct(q[b], k[b], v[b], 0, np.array(lay.gate), sh.sink, sh.recent)
         assert_close(got[b], want, sh.dtype, f"prefill b={b}")
     assert lay.status() == 0
     return lay
@@ -263,6 +269,13 @@ def _prefill_run(duo, sh, retrieval, n, chunk, B=1, seed=0, check_cache=True):
 def test_prefill_tiny_fp32(duo):
     sh = S.LayerShape(8, 8, 64, "fp32")
     _prefill_run(duo, sh, [1, 5], 512, 128)
+
+
+@pytest.mark.parametrize("chunk", [1, 7, 64, 128])
+def test_prefill_whole_chunk_streaming_fp32(duo, chunk):
+    """The tiny fp32 layer with streaming heads in whole-chunk mode (CUDA-core path)."""
+    sh = S.LayerShape(8, 8, 64, "fp32")
+    _prefill_run(duo, sh, [1, 5], 512, chunk, check_cache=(chunk >= 64), stream_mode="chunk")
 
 
 @pytest.mark.parametrize("chunk", [1, 7, 64, 300])
@@ -303,6 +316,56 @@ def test_gated_mix_bf16_gqa(duo, alpha_kind):
     for b in range(2):
         want = O.gated_mix(q[b], k[b], v[b], alpha.astype(np.float64), sh.sink, sh.recent)
         assert_close(got[b], want, "bf16", f"mix b={b}")
+
+
+# duo_gated_mix_grad_alpha: each dalpha[kv] sums dout * (full - streaming)
+# over its heads, rows and features, so its error is at most the attention
+# error bound times sum |dout| of those terms: 1e-4 for fp32; for bf16 the
+# mean-abs bound 2e-3 (dout is drawn independently of the rounding errors).
+
+def _grad_check(got, want, dout64, g, tol):
+    hkv = got.shape[0]
+    w = np.abs(dout64).reshape(-1, hkv, g, dout64.shape[-1]).sum(axis=(0, 2, 3))
+    err = np.abs(got - want)
+    assert np.all(err <= tol * w), f"dalpha error {err} vs bound {tol * w}"
+
+
+def test_gated_mix_grad_alpha_tiny_fp32(duo):
+    t = torch()
+    w = S.tiny_prompt()
+    sh = w["shape"]
+    desc = duo.desc_init(1, 8, 8, 64, duo.FP32, list(range(8)), 0)
+    q, k, v = (to_dev(w[x][None]) for x in ("q", "k", "v"))
+    dout = S.rng_for(9, 60).standard_normal((1, 512, 8, 64)).astype(np.float32)
+    dalpha = t.full((8,), 7.0, dtype=t.float32, device="cuda")      # overwritten by the call
+    duo.gated_mix_grad_alpha(desc, q, k, v, 512, to_dev(dout), dalpha)
+    want = O.gated_mix_grad_alpha(w["q"], w["k"], w["v"], dout[0], sh.sink, sh.recent)
+    _grad_check(dalpha.cpu().numpy().astype(np.float64), want, dout.astype(np.float64), 1, 1e-4)
+
+
+def test_gated_mix_grad_alpha_bf16_gqa_batch(duo):
+    t = torch()
+    sh = S.LayerShape(16, 4, 128, "bf16")
+    q, k, v = S.prompt(sh, 333, seed=4, batch=2)
+    dout = S.normal(S.rng_for(4, 61), (2, 333, 16, 128), "bf16")
+    desc = duo.desc_init(2, 16, 4, 128, duo.BF16, [0, 1, 2, 3], 0)
+    dalpha = t.empty((4,), dtype=t.float32, device="cuda")
+    duo.gated_mix_grad_alpha(desc, to_dev(q), to_dev(k), to_dev(v), 333, to_dev(dout), dalpha)
+    want = sum(O.gated_mix_grad_alpha(q[b], k[b], v[b], dout[b], sh.sink, sh.recent) for b in range(2))
+    _grad_check(dalpha.cpu().numpy().astype(np.float64), want, O.as_f64(dout), 4, 2e-3)
+
+
+def test_gated_mix_grad_alpha_zero_when_window_covers_sequence(duo):
+    """Both attentions see every key, in the same order: the difference, and
+    with it the gradient, is exactly zero."""
+    t = torch()
+    sh = S.LayerShape(8, 4, 64, "bf16", sink=16, recent=64)
+    q, k, v = S.prompt(sh, 80, seed=5)
+    dout = S.normal(S.rng_for(5, 62), (1, 80, 8, 64), "bf16")
+    desc = duo.desc_init(1, 8, 4, 64, duo.BF16, [0, 1, 2, 3], 0)
+    dalpha = t.empty((4,), dtype=t.float32, device="cuda")
+    duo.gated_mix_grad_alpha(desc, to_dev(q), to_dev(k), to_dev(v), 80, to_dev(dout), dalpha)
+    assert t.count_nonzero(dalpha).item() == 0
 
 
 # ---------------------------------------------------------------------------

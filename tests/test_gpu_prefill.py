@@ -22,11 +22,13 @@ def _cuda():
     t.cuda.synchronize()
 
 
-def _run(duo, sh, retrieval, n, chunks, B=1, seed=0, sample_rows=None, check_cache=True, sigma=None):
+def _run(duo, sh, retrieval, n, chunks, B=1, seed=0, sample_rows=None, check_cache=True, sigma=None,
+         stream_mode="lambda"):
     """Pre-fill n tokens in the given chunk lengths; compare every output row
     (or `sample_rows` seeded rows per chunk) with the oracle."""
     t = torch()
-    lay = Layer(duo, sh, retrieval, B, capacity=n + 16)
+    lay = Layer(duo, sh, retrieval, B, capacity=n + 16,
+                stream_prefill=duo.STREAM_CHUNK if stream_mode == "chunk" else duo.STREAM_LAMBDA)
     q, k, v = S.prompt(sh, n, seed=seed, batch=B, sigma=sigma)
     c0 = 0
     rng = S.rng_for(seed, 77)
@@ -47,7 +49,7 @@ def _run(duo, sh, retrieval, n, chunks, B=1, seed=0, sample_rows=None, check_cac
             rows = np.unique(np.concatenate([[0, C - 1], rng.choice(C, sample_rows, replace=False)]))
         for b in range(B):
             want = O.prefill_direct(q[b, c0:c1], k[b, :c1], v[b, :c1], c0, np.array(lay.gate), sh.sink, sh.recent,
-                                    rows=rows)
+                                    rows=rows, stream_mode=stream_mode)
             errs.append(assert_close(got[b, rows], want, "bf16", f"chunk {ci} (c0={c0}) b={b}"))
         c0 = c1
     if check_cache:
@@ -104,6 +106,20 @@ def test_prefill_tc_uneven_batch(duo, chunk):
     for b, L in enumerate(lengths):
         assert_close(got[b, rows], want[b], "bf16", f"b={b} (cached {L})")
     assert lay.status() == 0
+
+
+@pytest.mark.parametrize("chunks", [[700], [128] * 5 + [60], [300, 300, 100], [7, 9, 64, 1, 200, 419]])
+def test_prefill_tc_whole_chunk_streaming(duo, chunks):
+    """Streaming heads in whole-chunk mode on the tensor cores: the ring as it
+    stood before the chunk, then the chunk causally."""
+    sh = S.LayerShape(16, 4, 128, "bf16")
+    _run(duo, sh, [1, 2], sum(chunks), chunks, stream_mode="chunk")
+
+
+def test_prefill_tc_whole_chunk_streaming_long_prefix(duo):
+    sh = S.LayerShape(32, 8, 128, "bf16")
+    _run(duo, sh, S.retrieval_heads_by_seed(8, 4), 12288, [8192, 4096], sample_rows=96, check_cache=False,
+         stream_mode="chunk")
 
 
 def test_prefill_tc_mha_25pct(duo):
