@@ -64,8 +64,7 @@ constexpr uint32_t kOffK = kOffQ + 2 * kQBytes;
 constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;
 constexpr uint32_t kOffBar = kOffV + 2 * kTileBytes;
 constexpr uint32_t kOffHolder = kOffBar + 16 * 8;
-constexpr uint32_t kOffPos = kOffHolder + 16;
-constexpr uint32_t kSmemBytes = kOffPos + kMaxRing * 4;
+constexpr uint32_t kSmemBytes = kOffHolder + 16;
 static_assert(kSmemBytes + 1024 <= 232448, "one CTA per SM");
 
 enum { SRC_CACHE = 0, SRC_CHUNK = 1, SRC_RING = 2 };
@@ -76,7 +75,6 @@ struct TcArgs {
     int n_mpairs;          // ceil(C / 256)
     int n_ret_ctas;        // B * R * G * n_mpairs
     const int32_t* seq_len;
-    const int32_t* ring_pos;
     int32_t* status;
     void* out;
 };
@@ -172,6 +170,143 @@ __device__ __forceinline__ bool needs_mask(const Sched& s, const Tile& t, int qi
     return t.row + BN - 1 > BM * (2 * s.m + qi);
 }
 
+// ------------------------------------------------------------------ masks
+//
+// A row's visible keys in one 128-key tile, set as bits (column c = bit c % 32
+// of word c / 32), so that masking costs a bit test per score.  The ranges
+// follow from the key positions of the tile:
+//   cache / chunk tile, keys pos0 + c: causal (retrieval head, whole-chunk
+//     streaming head) c <= P - pos0 and pos0 + c >= 0; Lambda streaming head
+//     additionally pos0 + c < sink or pos0 + c > P - recent;
+//   ring tile, the streaming cache as it stood at the chunk start c0: slot s
+//     < min(c0, sink) holds sink s; the recent slots hold positions
+//     max(sink, c0 - recent) .. c0 - 1, position p in slot
+//     sink + (p - sink) % recent.  Whole-chunk mode sees all of them, Lambda
+//     mode the positions above P - recent.
+
+// columns lo .. hi (inclusive, clipped to the tile)
+__device__ __forceinline__ void set_columns(uint32_t (&m)[4], int lo, int hi) {
+    lo = max(lo, 0);
+    hi = min(hi, BN - 1);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const int a = max(lo - 32 * w, 0), b = min(hi - 32 * w, 31);
+        if (a <= b) m[w] |= (0xffffffffu >> (31 - b)) & (0xffffffffu << a);
+    }
+}
+
+__device__ __forceinline__ void visible_columns(const LayerArgs& a, const Sched& sc, const Tile& t, int P,
+                                                uint32_t (&m)[4]) {
+    if (t.src != SRC_RING) {
+        const int last = P - t.pos0;                      // causal: columns 0 .. last
+        if (sc.retrieval || sc.chunk) {
+            set_columns(m, -t.pos0, last);
+        } else {
+            set_columns(m, 0, min(last, a.sink - 1 - t.pos0));
+            set_columns(m, P - a.recent + 1 - t.pos0, last);
+        }
+        return;
+    }
+    const int c0 = sc.c0;
+    set_columns(m, 0, min(c0, a.sink) - 1);               // the sinks
+    int lo = max(a.sink, c0 - a.recent);                  // oldest recent position held
+    if (!sc.chunk) lo = max(lo, P - a.recent + 1);
+    const int len = c0 - lo;                              // positions lo .. c0 - 1
+    if (len <= 0) return;
+    const int start = (lo - a.sink) % a.recent;           // slot of lo, relative to the recent block
+    set_columns(m, a.sink + start, a.sink + min(start + len, a.recent) - 1);
+    if (start + len > a.recent) set_columns(m, a.sink, a.sink + start + len - a.recent - 1);
+}
+
+// ------------------------------------------------------------------ softmax
+
+// One row's share of one tile: S (128 columns at s_addr) from TMEM, the
+// running maximum m_ref (log2 domain, lazy: raised only when the tile's
+// maximum exceeds it by more than 2^8) and row sum l_sum updated, and
+// p = 2^(s * scale * log2e - m) written back as packed bf16 over the second
+// half of S for the PV MMA.  Returns the factor by which O must be rescaled
+// (1 unless `need`).
+//
+// S is read in two 64-column halves (a whole row would need more registers
+// than three warps per SM sub-partition leave): keys 0..63 for the maximum
+// only, then keys 64..127, which stay in registers; p of keys 64..127 goes to
+// columns 96..127, then keys 0..63 (loaded again) to columns 64..95.  The row
+// sum adds the rounded p, so each output is a convex combination of V rows.
+__device__ __forceinline__ float softmax_tile(uint32_t s_addr, float sl, float& m_ref, float& l_sum, bool& need) {
+    // maximum of 64 raw scores: three-input max, 4 chains
+    auto max_half = [](const float (&v)[64]) {
+        float m4[4] = {v[0], v[1], v[2], v[3]};
+#pragma unroll
+        for (int c = 4; c < 60; c += 8) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) m4[i] = fmax3(m4[i], v[c + i], v[c + 4 + i]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m4[i] = fmaxf(m4[i], v[60 + i]);
+        return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+    };
+    float s[64];
+    tmem_ld64(s_addr, s);
+    float mx = max_half(s);
+    tmem_ld64(s_addr + 64, s);
+    // into the log2 domain: the scale is positive, so it commutes with max
+    mx = fmaxf(mx, max_half(s)) * sl;
+    const float m_new = fmaxf(m_ref, mx);
+    need = m_new > m_ref + 8.f;                           // lazy rescale threshold: 2^8
+    const float m_use = need ? m_new : m_ref;
+    const float m_safe = m_use == -INFINITY ? 0.f : m_use;
+    const float corr = need ? exp2_approx(m_ref - m_use) : 1.f;
+    const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(-m_safe, -m_safe);
+    float2 rs2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    auto exp_half = [&](const float (&v)[64], uint32_t taddr) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c2 = 0; c2 < 32; ++c2) {
+            const float2 x = ffma2(make_float2(v[2 * c2], v[2 * c2 + 1]), sl2, nm2);
+            const float2 e = make_float2(exp2_approx(x.x), exp2_approx(x.y));
+            __nv_bfloat162 hb = __floats2bfloat162_rn(e.x, e.y);
+            pk[c2] = *reinterpret_cast<uint32_t*>(&hb);
+            rs2[c2 & 3] = fadd2(rs2[c2 & 3], make_float2(bf16_lo(pk[c2]), bf16_hi(pk[c2])));
+        }
+        tmem_st32(taddr, pk);
+    };
+    exp_half(s, s_addr + 96);
+    tmem_ld64(s_addr, s);
+    exp_half(s, s_addr + 64);
+    const float rs = ((rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y)) + ((rs2[2].x + rs2[2].y) + (rs2[3].x + rs2[3].y));
+    l_sum = l_sum * corr + rs;
+    m_ref = m_use;
+    return corr;
+}
+
+// A masked tile (diagonal, first prior tile, streaming tiles): this row's
+// invisible scores are overwritten with -inf in TMEM, so the softmax itself
+// never tests a mask and keeps no mask state across its loop.  Costs one more
+// TMEM round trip on the few masked tiles of a query tile; a streaming tile
+// is 6x cheaper than with a per-score position test.
+__device__ __forceinline__ void mask_tile_in_tmem(const LayerArgs& a, const Sched& sc, const Tile& t, int P,
+                                               uint32_t s_addr) {
+    uint32_t vis[4] = {0u, 0u, 0u, 0u};   // the tile's keys this row sees, a bit per column
+    visible_columns(a, sc, t, P, vis);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        float v[64];
+        tmem_ld64(s_addr + 64 * h, v);
+        uint32_t r[32];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                const int col = 64 * h + 32 * half + c;
+                r[c] = ((vis[col >> 5] >> (col & 31)) & 1u) ? __float_as_uint(v[32 * half + c])
+                                                            : __float_as_uint(-INFINITY);
+            }
+            tmem_st32(s_addr + 64 * h + 32 * half, r);
+        }
+    }
+    tmem_wait_st();
+}
+
 // ------------------------------------------------------------------ kernel
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -197,7 +332,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* p_full = bars + 11;   // [2]: per query tile
     uint64_t* o_done = bars + 13;   // [2]: per query tile, once
     uint32_t* holder = reinterpret_cast<uint32_t*>(smem + kOffHolder);
-    int* sPos = reinterpret_cast<int*>(smem + kOffPos);
 
     // ------------------------------------------------------- work item
     const int per_m_ret = a.B * a.R * a.G, per_m_str = a.B * a.S * a.G;
@@ -235,9 +369,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_barrier_init();
     }
-    if (!retrieval)
-        for (int i = tid; i < kMaxRing; i += kThreads)
-            sPos[i] = (i < a.W && c0 > 0) ? p.ring_pos[(size_t)b * a.W + i] : -1;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -353,75 +484,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = __all_sync(0xffffffffu, mbar_wait(&s_full[qi], j & 1, p.status));
             if (!ok) break;
             tc_fence_after();
-            // S is read in two 64-column halves (a whole row would need more
-            // registers than three warps per SM sub-partition leave): keys
-            // 0..63 for the maximum only, then keys 64..127, which stay in
-            // registers
             const Tile t = tile_at(sc, j);
-            const bool msk = needs_mask(sc, t, qi);
-            auto mask_half = [&](float (&v)[64], int c_base) {
-#pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    const int kp = t.src == SRC_RING ? sPos[c_base + c] : t.pos0 + c_base + c;
-                    bool vis = kp >= 0 && kp <= P;
-                    if (!sc.retrieval)
-                        vis = vis && (kp < a.sink || (sc.chunk ? kp >= sc.c0 - a.recent : P - kp < a.recent));
-                    if (!vis) v[c] = -INFINITY;
-                }
-            };
-            // maximum of 64 raw scores: three-input max, 4 chains
-            auto max_half = [](const float (&v)[64]) {
-                float m4[4] = {v[0], v[1], v[2], v[3]};
-#pragma unroll
-                for (int c = 4; c < 60; c += 8) {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) m4[i] = fmax3(m4[i], v[c + i], v[c + 4 + i]);
-                }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) m4[i] = fmaxf(m4[i], v[60 + i]);
-                return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-            };
-            float s[64];
-            tmem_ld64(lane_base + col_s(qi), s);
-            if (msk) mask_half(s, 0);
-            float mx = max_half(s);
-            tmem_ld64(lane_base + col_s(qi) + 64, s);
-            if (msk) mask_half(s, 64);
-            // into the log2 domain: the scale is positive, so it commutes with max
-            mx = fmaxf(mx, max_half(s)) * sl;
-            const float m_new = fmaxf(m_ref, mx);
-            const bool need = m_new > m_ref + 8.f;            // lazy rescale threshold: 2^8
-            const float m_use = need ? m_new : m_ref;
-            const float m_safe = m_use == -INFINITY ? 0.f : m_use;
-            const float corr = need ? exp2_approx(m_ref - m_use) : 1.f;
-            // p = 2^(s*scale*log2e - m), rounded once to bf16 for the PV MMA,
-            // packed in pairs and written over the second half of S: keys
-            // 64..127 (in registers) to columns 96..127, then keys 0..63
-            // (loaded again) to columns 64..95.  The row sum adds the rounded
-            // values, so each output is a convex combination of V rows.
-            const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(-m_safe, -m_safe);
-            float2 rs2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                             make_float2(0.f, 0.f)};
-            auto exp_half = [&](const float (&v)[64], uint32_t taddr) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int c2 = 0; c2 < 32; ++c2) {
-                    const float2 x = ffma2(make_float2(v[2 * c2], v[2 * c2 + 1]), sl2, nm2);
-                    const float2 e = make_float2(exp2_approx(x.x), exp2_approx(x.y));
-                    __nv_bfloat162 hb = __floats2bfloat162_rn(e.x, e.y);
-                    pk[c2] = *reinterpret_cast<uint32_t*>(&hb);
-                    rs2[c2 & 3] = fadd2(rs2[c2 & 3], make_float2(bf16_lo(pk[c2]), bf16_hi(pk[c2])));
-                }
-                tmem_st32(taddr, pk);
-            };
-            exp_half(s, lane_base + col_s(qi) + 96);
-            tmem_ld64(lane_base + col_s(qi), s);
-            if (msk) mask_half(s, 0);
-            exp_half(s, lane_base + col_s(qi) + 64);
-            const float rs = ((rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y)) +
-                             ((rs2[2].x + rs2[2].y) + (rs2[3].x + rs2[3].y));
-            l_sum = l_sum * corr + rs;
-            m_ref = m_use;
+            if (needs_mask(sc, t, qi)) mask_tile_in_tmem(a, sc, t, P, lane_base + col_s(qi));
+            bool need;
+            const float corr = softmax_tile(lane_base + col_s(qi), sl, m_ref, l_sum, need);
             // O_qi holds every PV up to tile j - 1 (the commit behind s_full
             // covered them); rescale it before PV_qi(j) is issued
             if (j >= 1 && __any_sync(0xffffffffu, need)) {
@@ -518,7 +584,6 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
     p.n_mpairs = (C + 2 * BM - 1) / (2 * BM);
     p.n_ret_ctas = a.B * a.R * a.G * p.n_mpairs;
     p.seq_len = c.seq_len;
-    p.ring_pos = c.ring_pos;
     p.status = c.status;
     p.out = out;
     const long grid = (long)a.B * a.Hkv * a.G * p.n_mpairs;
