@@ -54,6 +54,13 @@ WORKLOADS = {
     "gqa_decode_1m": dict(kind="decode", hq=32, hkv=8, d=128, n_ret=4, lengths=[1048576], steps=64, sigma=True),
     "batch64_paged_decode": dict(kind="decode", hq=32, hkv=32, d=128, n_ret=8, batch=64, lo=4096, hi=32768,
                                  steps=32, sigma=False, paged=True),
+    # the same decode workloads over the 8-bit retrieval cache (codes + a scale per row)
+    "mha_decode_32k_int8": dict(kind="decode", hq=32, hkv=32, d=128, n_ret=8, lengths=[32768], steps=256,
+                                sigma=False, kv_int8=True),
+    "gqa_decode_128k_int8": dict(kind="decode", hq=32, hkv=8, d=128, n_ret=4, lengths=[131072], steps=64,
+                                 sigma=True, kv_int8=True),
+    "gqa_decode_1m_int8": dict(kind="decode", hq=32, hkv=8, d=128, n_ret=4, lengths=[1048576], steps=64,
+                               sigma=True, kv_int8=True),
     "gqa_prefill_128k": dict(kind="prefill", hq=32, hkv=8, d=128, n_ret=4, n=131072, chunk=4096, sigma=False),
     # the same pre-fill on a 32K prompt: a small case for profiler captures
     "gqa_prefill_32k": dict(kind="prefill", hq=32, hkv=8, d=128, n_ret=4, n=32768, chunk=4096, sigma=False),
@@ -277,14 +284,19 @@ def _decode_setup(duo, wl, total_steps, seed=0):
         caches = duo.LayerCaches(desc, 0, table, n_pages)
     else:
         table = None
-        desc = duo.desc_init(B, sh.n_q_heads, sh.n_kv_heads, sh.head_dim, duo.BF16, perm, R)
+        desc = duo.desc_init(B, sh.n_q_heads, sh.n_kv_heads, sh.head_dim, duo.BF16, perm, R,
+                             kv_quant=duo.KV_INT8 if wl.get("kv_int8") else duo.KV_PLAIN)
         caches = duo.LayerCaches(desc, int(lengths.max()) + total_steps)
     st = S.decode_state(sh, retrieval, lengths, seed=seed, sigma=sigma)
-    _load_decode_state(caches, st, inv, R, sh, table)
+    if wl.get("kv_int8"):
+        _append_decode_state(duo, desc, caches, st, retrieval, sh)
+    else:
+        _load_decode_state(caches, st, inv, R, sh, table)
     ws = duo.Workspace(desc, duo.OP_DECODE, caches.capacity)
     qs, ks, vs = S.decode_steps(sh, B, total_steps, seed=seed, sigma=sigma)
     torch.cuda.synchronize()
     return dict(sh=sh, desc=desc, caches=caches, ws=ws, qs=qs, ks=ks, vs=vs, lengths=lengths, B=B, R=R,
+                kv_int8=bool(wl.get("kv_int8")),
                 retrieval=retrieval, gate=gate, state=st, sigma=sigma, table=table,
                 n_pages=n_pages if paged else 0)
 
@@ -325,15 +337,49 @@ def _load_decode_state(caches, st, inv, R, sh, table):
     caches.seq_len.copy_(torch.from_numpy(st["lengths"].astype(np.int32)))
 
 
-def _decode_bytes(sh, R, lengths_after):
+def _append_decode_state(duo, desc, caches, st, retrieval, sh, chunk=32768):
+    """Fill an 8-bit layer with a seeded state through duo_append_kv, which
+    quantizes the retrieval rows on the device (the streaming heads' rows are
+    zeros there), then install the streaming rings as _load_decode_state does."""
+    import torch
+    lengths = st["lengths"]
+    B, L = len(lengths), int(lengths.max())
+    assert np.all(lengths == L), "8-bit states are built for equal lengths"
+    for c0 in range(0, L, chunk):
+        T = min(chunk, L - c0)
+        kc = torch.zeros((B, T, sh.n_kv_heads, sh.head_dim), dtype=torch.bfloat16, device="cuda")
+        vc = torch.zeros_like(kc)
+        for (b, h), (k, v) in st["full"].items():
+            kc[b, :, h] = _to_dev(k[c0:c0 + T])
+            vc[b, :, h] = _to_dev(v[c0:c0 + T])
+        duo.append_kv(desc, caches.state, kc, vc, T)
+    inv = {int(h): i for i, h in enumerate(list(desc.kv_perm)[:sh.n_kv_heads])}
+    R = desc.n_retrieval
+    ring_pos = np.full((B, sh.sink + sh.recent), -1, dtype=np.int32)
+    for (b, h), (pos, k, v) in st["stream"].items():
+        s_ = inv[h] - R
+        slots = np.array([p if p < sh.sink else sh.sink + (p - sh.sink) % sh.recent for p in pos], dtype=np.int64)
+        if len(slots):
+            idx = torch.from_numpy(slots).cuda()
+            caches.k_ring[b, s_, idx] = _to_dev(k)
+            caches.v_ring[b, s_, idx] = _to_dev(v)
+            ring_pos[b, slots] = pos
+    caches.ring_pos.copy_(torch.from_numpy(ring_pos))
+    torch.cuda.synchronize()
+    assert duo.check_status(caches.state) == 0
+
+
+def _decode_bytes(sh, R, lengths_after, kv_int8=False):
     """Algorithmic HBM bytes of one fused decode step: every cached K/V row of
-    every retrieval head once, the ring rows of the streaming heads, q and out,
-    and the new token's K/V rows read once and written once into the caches."""
+    every retrieval head once (8-bit: d codes + a 4-byte scale per row), the
+    ring rows of the streaming heads, q and out, and the new token's K/V rows
+    read once and written once into the caches."""
     S_ = sh.n_kv_heads - R
     row = sh.head_dim * 2
+    full_row = sh.head_dim + 4 if kv_int8 else row
     total = 0
     for L in lengths_after:
-        total += R * (L - 1) * row * 2
+        total += R * (L - 1) * full_row * 2
         total += S_ * (min(L, sh.sink + sh.recent) - 1) * row * 2
         total += sh.n_kv_heads * row * 2 * 2
     total += len(lengths_after) * sh.n_q_heads * sh.head_dim * 2 * 2
@@ -348,8 +394,9 @@ def _replicate_layers(duo, env, n_layers):
     layers = [(first, env["ws"])]
     for _ in range(n_layers - 1):
         c = duo.LayerCaches(env["desc"], first.capacity, env.get("table"), env.get("n_pages", 0))
-        for name in ("k_full", "v_full", "k_ring", "v_ring", "ring_pos", "seq_len"):
-            getattr(c, name).copy_(getattr(first, name))
+        for name in ("k_full", "v_full", "k_ring", "v_ring", "ring_pos", "seq_len", "k_scale", "v_scale"):
+            if getattr(first, name, None) is not None:
+                getattr(c, name).copy_(getattr(first, name))
         layers.append((c, duo.Workspace(env["desc"], duo.OP_DECODE, c.capacity)))
     torch.cuda.synchronize()
     return layers
@@ -411,7 +458,7 @@ def run_decode(args, wl, world, rank):
     e2e = None if getattr(args, "no_e2e", False) else _decode_e2e(duo, env, layers, args, world)
 
     hbm, _, peak_kind = _peaks()
-    bytes_per_launch = statistics.mean(_decode_bytes(sh, R, L) for L in lengths_seen)
+    bytes_per_launch = statistics.mean(_decode_bytes(sh, R, L, bool(wl.get("kv_int8"))) for L in lengths_seen)
     dec_avg_s = statistics.mean(dec_ms) * 1e-3
     achieved = bytes_per_launch / dec_avg_s / 1e9
     res = {
@@ -422,6 +469,7 @@ def run_decode(args, wl, world, rank):
                    "head_dim": sh.head_dim, "n_retrieval": R, "sink": sh.sink, "recent": sh.recent,
                    "context": [int(env["lengths"].min()), int(env["lengths"].max())],
                    "paged": bool(wl.get("paged", False)), "layers_per_step": nl,
+                   "full_cache": "int8 codes + fp32 scale per row" if wl.get("kv_int8") else "bf16",
                    "parallelism": f"replicas{world}",
                    "l2": f"not flushed: inputs larger than L2 (each step streams {nl} layers' caches, "
                          f"{nl * bytes_per_launch / 1e6:.0f} MB > 126 MB)"},
@@ -488,7 +536,8 @@ def _decode_cpu_baseline(env, budget_s=15.0):
     same seeded state until the time budget is used."""
     import oracle as O
     sh, B = env["sh"], env["B"]
-    cache = O.HeadSplitCache(B, sh.n_kv_heads, sh.head_dim, gate=env["gate"], sink=sh.sink, recent=sh.recent)
+    cache = O.HeadSplitCache(B, sh.n_kv_heads, sh.head_dim, gate=env["gate"], sink=sh.sink, recent=sh.recent,
+                             kv_int8=env.get("kv_int8", False))
     st = env["state"]
     for (b, h), (k, v) in st["full"].items():
         cache.load_state(b, h, np.arange(k.shape[0]), k, v)
@@ -648,7 +697,8 @@ def run_reference(args, wl, budget_s: float = 120.0):
 
     def build(b_list, heads):
         g = np.array([gate[h] for h in heads], dtype=np.uint8)
-        cache = O.HeadSplitCache(len(b_list), len(heads), sh.head_dim, gate=g, sink=sh.sink, recent=sh.recent)
+        cache = O.HeadSplitCache(len(b_list), len(heads), sh.head_dim, gate=g, sink=sh.sink, recent=sh.recent,
+                                 kv_int8=bool(wl.get("kv_int8")))
         for bi, b in enumerate(b_list):
             for hi, h in enumerate(heads):
                 if gate[h]:
@@ -671,7 +721,7 @@ def run_reference(args, wl, budget_s: float = 120.0):
     t0 = time.perf_counter()
     cache.decode(*sl(0, full_b, full_heads))
     t_full = time.perf_counter() - t0
-    bytes_full = _decode_bytes(sh, R, lengths + 1)
+    bytes_full = _decode_bytes(sh, R, lengths + 1, bool(wl.get("kv_int8")))
     if total * t_full <= budget_s:
         b_list, heads, scale, sample = full_b, full_heads, 1.0, "full decode steps"
         first = 1
@@ -682,7 +732,7 @@ def run_reference(args, wl, budget_s: float = 120.0):
         b_list = [0]
         sub = S.LayerShape(sh.group * len(heads), len(heads), sh.head_dim, "bf16", sh.sink, sh.recent)
         n_ret = 1 if ret0 is not None else 0
-        bytes_sample = _decode_bytes(sub, n_ret, lengths[:1] + 1)
+        bytes_sample = _decode_bytes(sub, n_ret, lengths[:1] + 1, bool(wl.get("kv_int8")))
         scale = bytes_full / bytes_sample
         sample = (f"sequence 0, KV heads {heads} (one retrieval, one streaming) with their query heads; "
                   f"time scaled x{scale:.1f} to the whole step by algorithmic bytes")

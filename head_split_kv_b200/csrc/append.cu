@@ -11,6 +11,7 @@
 // (an atomic ticket, no waiting), after every CTA has read the old value.
 #include "common.cuh"
 #include "internal.h"
+#include "kvq8.cuh"
 
 namespace duo {
 namespace {
@@ -83,10 +84,78 @@ __global__ void __launch_bounds__(256) append_kernel(const LayerArgs a, const Ca
     }
 }
 
+// ------------------------------------------------------------------------
+// 8-bit full cache: one warp per (token, KV head, K|V) row.  A retrieval row
+// is quantized and stored in the 8-bit layouts (kvq8.cuh); a streaming row is
+// copied into the ring as in the plain kernel.
+
+__global__ void __launch_bounds__(256) append_q8_kernel(const LayerArgs a, const CacheArgs c,
+                                                        const __nv_bfloat16* __restrict__ k_new,
+                                                        const __nv_bfloat16* __restrict__ v_new, const int T) {
+    const int lane = threadIdx.x & 31;
+    const long rows = (long)a.B * T * a.Hkv;             // input rows per tensor
+    const long warps = (long)gridDim.x * (blockDim.x >> 5);
+    for (long x = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); x < 2 * rows; x += warps) {
+        const int kv = x >= rows;                         // 0: K, 1: V
+        const long r = x - kv * rows;
+        const int h_in = (int)(r % a.Hkv);
+        const long bt = r / a.Hkv;
+        const int t = (int)(bt % T);
+        const int b = (int)(bt / T);
+        const int slot = a.slot_of[h_in];
+        const int L = c.seq_len[b];
+        const int p = L + t;
+        const __nv_bfloat16* src = (kv ? v_new : k_new) + r * 128;
+        if (slot < a.R) {
+            if (p >= a.capacity || p < 0) {
+                if (lane == 0 && kv == 0) atomicOr(c.status, DUO_DEV_FULL_CACHE_OVERFLOW);
+                continue;
+            }
+            const uint2 w = reinterpret_cast<const uint2*>(src)[lane];
+            const float xv[4] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y)};
+            float scale;
+            const uint32_t codes = q8_quantize(xv, scale);
+            q8_store_row(a, c, kv, b, slot, p, codes, scale, lane);
+        } else {
+            if (p < 0) {
+                if (lane == 0 && kv == 0) atomicOr(c.status, DUO_DEV_BAD_LENGTH);
+                continue;
+            }
+            if (!(p < a.sink || p >= L + T - a.recent)) continue;
+            const int s = slot - a.R;
+            const int rs = ring_slot(p, a.sink, a.recent);
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(kv ? c.v_ring : c.k_ring) + (((long)b * a.S + s) * a.W + rs) * 128;
+            reinterpret_cast<uint2*>(dst)[lane] = reinterpret_cast<const uint2*>(src)[lane];
+            if (s == 0 && lane == 0 && kv == 0) c.ring_pos[(long)b * a.W + rs] = p;
+        }
+    }
+    // the last CTA to finish advances the lengths (every CTA read them first)
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned ticket = atomicAdd(&c.counters[0], 1u);
+        if (ticket == gridDim.x - 1) {
+            __threadfence();
+            for (int b = 0; b < a.B; ++b) c.seq_len[b] += T;
+            c.counters[0] = 0u;
+            __threadfence();
+        }
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_append(const LayerArgs& a, const CacheArgs& c, const void* k_new, const void* v_new, int T,
                           cudaStream_t s) {
+    if (a.kv_int8) {
+        const long warps = 2L * a.B * T * a.Hkv;
+        long blocks = (warps + 7) / 8;
+        if (blocks > 148L * 8) blocks = 148L * 8;
+        if (blocks < 1) blocks = 1;
+        append_q8_kernel<<<(unsigned)blocks, 256, 0, s>>>(a, c, static_cast<const __nv_bfloat16*>(k_new),
+                                                          static_cast<const __nv_bfloat16*>(v_new), T);
+        return cudaGetLastError();
+    }
     const int row_bytes = a.D * (a.dtype == DUO_BF16 ? 2 : 4);
     const long total = 2L * a.B * T * a.Hkv * (row_bytes / 16);
     const int threads = 256;

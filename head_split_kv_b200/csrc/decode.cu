@@ -37,6 +37,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "kvq8.cuh"
 
 namespace duo {
 namespace {
@@ -767,7 +768,7 @@ __global__ void __maxnreg__(200)
     if (threadIdx.x == 0) *s_flag = c.seq_len[b];
     __syncthreads();
     const int L0 = *s_flag;
-    if (fused && threadIdx.x == 0) length_ticket(a, c, d);
+    if (fused && d.grid_ticket && threadIdx.x == 0) length_ticket(a, c, d);
     int len = L0;
     int new_row = -1;
     if (fused) {
@@ -995,7 +996,7 @@ cudaError_t launch_mma_t(const LayerArgs& a, const CacheArgs& c, const DecodeArg
     const uint32_t box3[3] = {64, (uint32_t)kTile, 1};
     CUtensorMap mKf{}, mVf{}, mKr{}, mVr{};
     bool have_f = false, have_r = false;
-    if (a.R > 0) {
+    if (a.R > 0 && d.n_ret_units > 0) {
         if (PAGED) {
             const uint64_t dims[4] = {128, (uint64_t)kTile, (uint64_t)a.R, (uint64_t)a.n_pages};
             const uint64_t st[3] = {row, row * kTile, row * kTile * a.R};
@@ -1085,6 +1086,298 @@ cudaError_t launch_d(const LayerArgs& a, const CacheArgs& c, const DecodeArgs& d
     return cudaErrorInvalidValue;
 }
 
+// ===========================================================================
+// 8-bit full cache: decode_q8_kernel, retrieval heads only (an 8-bit layer's
+// streaming heads run the bf16 kernel in a launch just before, without the
+// length ticket).  Per CTA as decode_mma_kernel -- a TMA producer warp, four
+// consumer warps of 16 keys each, the same split plan and split-K combine --
+// with a 64-token stage of 8 KB of K codes (a row per token, 128-byte
+// swizzle), 8 KB of V codes (transposed, 64-byte swizzle) and the tile's 64 +
+// 64 scales, five stages deep.
+//
+// The contractions run on mma.sync m16n8k16 in fp16 with fp32 accumulation:
+//   S = q . codes: the codes widen to fp16 exactly (kvq8.cuh); the feature
+//     order inside each 16-wide step is permuted the same way for q and K so
+//     that a lane's four features (32 t + 4 kb + 0..3) come from one word of
+//     its key's row; the key's scale multiplies S in fp32;
+//   O += P V: p times the key's V scale, rounded to fp16, is the A operand;
+//     the V layout puts a lane's four keys (2t, 2t+1, 2t+8, 2t+9) in one
+//     word of each feature row.
+// q, p * scale and the codes must fit fp16 (|K|, |V| below 8.3e6, |q| below
+// 65504).
+// ===========================================================================
+
+constexpr int kQ8Stages = 5;
+constexpr uint32_t kQ8Bytes = kTile * 128;          // 8 KB of K or V codes per stage
+constexpr uint32_t kQ8ScBytes = 2 * kTile * 4;      // K and V scales of a stage
+
+constexpr size_t decode_q8_smem_bytes() {
+    return 2 * (size_t)kQ8Stages * kQ8Bytes + kQ8Stages * kQ8ScBytes + (2 * kQ8Stages + 1) * sizeof(uint64_t) + 64;
+}
+
+__device__ __forceinline__ void mma_f16_rows8(float& c0, float& c1, uint32_t a0, uint32_t a2, uint32_t b0,
+                                              uint32_t b1) {
+    float d2, d3;
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%10, %11, %12, %13};"
+        : "=f"(c0), "=f"(c1), "=f"(d2), "=f"(d3)
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(0.f), "f"(0.f));
+}
+
+template <int G>
+__global__ void __maxnreg__(200)
+    decode_q8_kernel(const __grid_constant__ CUtensorMap tmK8, const __grid_constant__ CUtensorMap tmV8,
+                     const LayerArgs a, const CacheArgs c, const DecodeArgs d) {
+    using T = __nv_bfloat16;
+    constexpr int D = 128;
+    constexpr int STAGES = kQ8Stages;
+    constexpr int NW = kMmaWarps;
+    constexpr int kThreads = kMmaThreads;
+    static_assert(G <= 8, "the group must fit the 8 live rows of an m16 tile");
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t* sK8 = smem;
+    uint8_t* sV8 = smem + (size_t)STAGES * kQ8Bytes;
+    float* sSc = reinterpret_cast<float*>(smem + 2 * (size_t)STAGES * kQ8Bytes);
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + 2 * (size_t)STAGES * kQ8Bytes + STAGES * kQ8ScBytes);
+    uint64_t* empty_bar = full_bar + STAGES;
+    uint64_t* comb_bar = empty_bar + STAGES;
+    int* s_flag = reinterpret_cast<int*>(comb_bar + 1);
+    int* s_tile_n = s_flag + 1;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if ((smem_u32(smem) & 1023u) != 0) {  // the swizzled tiles need 1024-byte alignment
+        if (threadIdx.x == 0) atomicOr(c.status, DUO_DEV_BAD_LENGTH);
+        return;
+    }
+
+    // ---------------------------------------------------------- work unit
+    const int split = blockIdx.x % d.nsplit;
+    const int pair = blockIdx.x / d.nsplit;
+    const int slot = pair % a.R;
+    const int b = pair / a.R;
+    const int z = b * a.R + slot;
+    const int tiles_per_head = a.capacity / kTile;
+    const bool fused = d.k_new != nullptr;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], NW);
+        }
+        mbar_init(comb_bar, 1);
+        fence_barrier_init();
+    }
+    if (warp == NW && lane == 0) {
+        prefetch_map(&tmK8);
+        prefetch_map(&tmV8);
+    }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (threadIdx.x == 0) *s_flag = c.seq_len[b];
+    __syncthreads();
+    const int L0 = *s_flag;
+    if (fused && d.grid_ticket && threadIdx.x == 0) length_ticket(a, c, d);
+    int len = L0;
+    int new_row = -1;
+    if (fused) {
+        if (L0 < 0) {
+            if (threadIdx.x == 0) atomicOr(c.status, DUO_DEV_BAD_LENGTH);
+            len = 0;
+        } else if (L0 >= a.capacity) {
+            if (threadIdx.x == 0 && split == 0) atomicOr(c.status, DUO_DEV_FULL_CACHE_OVERFLOW);
+        } else {
+            new_row = L0;
+            len = L0 + 1;
+        }
+    }
+    if (len > a.capacity || len < 0) {
+        if (threadIdx.x == 0 && split == 0) atomicOr(c.status, DUO_DEV_BAD_LENGTH);
+        len = len < 0 ? 0 : a.capacity;
+    }
+    const int per = (len + d.nsplit - 1) / d.nsplit;
+    const int chunk = (per + kTile - 1) / kTile * kTile;
+    const int row_begin = min(len, split * chunk);
+    const int row_end = min(len, row_begin + chunk);
+    const int n_tiles = (row_end - row_begin + kTile - 1) / kTile;
+
+    if (warp == NW) {
+        // ------------------------------------------------------ producer
+        if (new_row >= row_begin && new_row < row_end) {
+            // the new token goes into the 8-bit cache first, quantized; the
+            // tile that holds it is then read back through TMA
+            const int h = a.kv_head[slot];
+            const uint2 kw = reinterpret_cast<const uint2*>(static_cast<const T*>(d.k_new) + ((size_t)b * a.Hkv + h) * D)[lane];
+            const uint2 vw = reinterpret_cast<const uint2*>(static_cast<const T*>(d.v_new) + ((size_t)b * a.Hkv + h) * D)[lane];
+            const float kx[4] = {bf16_lo(kw.x), bf16_hi(kw.x), bf16_lo(kw.y), bf16_hi(kw.y)};
+            const float vx[4] = {bf16_lo(vw.x), bf16_hi(vw.x), bf16_lo(vw.y), bf16_hi(vw.y)};
+            float ks, vs;
+            const uint32_t kc = q8_quantize(kx, ks);
+            const uint32_t vc = q8_quantize(vx, vs);
+            q8_store_row(a, c, 0, b, slot, new_row, kc, ks, lane);
+            q8_store_row(a, c, 1, b, slot, new_row, vc, vs, lane);
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            __syncwarp();
+        }
+        if (lane == 0) {
+            for (int t = 0; t < n_tiles; ++t) {
+                const int st = t % STAGES, round = t / STAGES;
+                if (round > 0 && !mbar_wait(&empty_bar[st], (round - 1) & 1, c.status)) break;
+                const int r0 = row_begin + t * kTile;
+                s_tile_n[st] = min(kTile, row_end - r0);
+                mbar_arrive_expect_tx(&full_bar[st], 2 * kQ8Bytes + kQ8ScBytes);
+                tma_load_3d(smem_u32(sK8 + (size_t)st * kQ8Bytes), &tmK8, 0, r0, z, &full_bar[st]);
+                tma_load_3d(smem_u32(sV8 + (size_t)st * kQ8Bytes), &tmV8, 0, 0, z * tiles_per_head + r0 / kTile,
+                            &full_bar[st]);
+                bulk_g2s(sSc + st * 2 * kTile, c.k_scale + (size_t)z * a.capacity + r0, kTile * 4, &full_bar[st]);
+                bulk_g2s(sSc + st * 2 * kTile + kTile, c.v_scale + (size_t)z * a.capacity + r0, kTile * 4,
+                         &full_bar[st]);
+            }
+        }
+    }
+
+    // ------------------------------------------------------ consumers
+    const int row = lane >> 2;   // query head of the group (rows >= G are padding) / key of an 8-key block
+    const int quad = lane & 3;
+    float o[16][2];
+    float m_run = kNegBig, l_run = 0.f;
+    if (warp < NW) {
+        // q in fp16, features 32 quad + 4 kb + {0, 1} and {2, 3} for step kb
+        uint32_t qa[8][2];
+        {
+            const bool row_ok = row < G;
+            const uint4* qp = reinterpret_cast<const uint4*>(
+                static_cast<const T*>(d.q) + ((size_t)b * a.Hq + a.q_head0[slot] + (row_ok ? row : 0)) * D + 32 * quad);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint4 w = row_ok ? qp[i] : make_uint4(0u, 0u, 0u, 0u);
+                qa[2 * i][0] = f16x2_pack(bf16_lo(w.x), bf16_hi(w.x));
+                qa[2 * i][1] = f16x2_pack(bf16_lo(w.y), bf16_hi(w.y));
+                qa[2 * i + 1][0] = f16x2_pack(bf16_lo(w.z), bf16_hi(w.z));
+                qa[2 * i + 1][1] = f16x2_pack(bf16_lo(w.w), bf16_hi(w.w));
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = 0.f;
+        const float sl = a.scale * kLog2e;
+        const int key_base = warp * 16;
+        for (int t = 0; t < n_tiles; ++t) {
+            const int st = t % STAGES, round = t / STAGES;
+            if (!mbar_wait(&full_bar[st], round & 1, c.status)) break;
+            const int n = s_tile_n[st];
+            const uint8_t* tK = sK8 + (size_t)st * kQ8Bytes;
+            const uint8_t* tV = sV8 + (size_t)st * kQ8Bytes;
+            const float* ksc = sSc + st * 2 * kTile;
+            const float* vsc = ksc + kTile;
+            // S = q . codes for keys key_base + 8 nb + (lane >> 2)
+            float s[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+            for (int nb = 0; nb < 2; ++nb) {
+                const int key = key_base + 8 * nb + row;
+                const uint4 lo = *reinterpret_cast<const uint4*>(tK + key * 128 + (((2 * quad) ^ (key & 7)) << 4));
+                const uint4 hi = *reinterpret_cast<const uint4*>(tK + key * 128 + (((2 * quad + 1) ^ (key & 7)) << 4));
+                const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+                for (int kb = 0; kb < 8; ++kb) {
+                    uint32_t b0, b1;
+                    i8x4_to_f16x2(w[kb], b0, b1);
+                    mma_f16_rows8(s[nb][0], s[nb][1], qa[kb][0], qa[kb][1], b0, b1);
+                }
+            }
+            // this lane's keys: key_base + 2 quad + {0, 1} and + 8
+            const int k0 = key_base + 2 * quad;
+            const float2 ks0 = *reinterpret_cast<const float2*>(ksc + k0);
+            const float2 ks1 = *reinterpret_cast<const float2*>(ksc + k0 + 8);
+            const float sv[4] = {s[0][0] * ks0.x * sl, s[0][1] * ks0.y * sl, s[1][0] * ks1.x * sl,
+                                 s[1][1] * ks1.y * sl};
+            const bool vk[4] = {k0 < n, k0 + 1 < n, k0 + 8 < n, k0 + 9 < n};
+            float mx = kNegBig;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) mx = vk[i] ? fmaxf(mx, sv[i]) : mx;
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float m_new = fmaxf(m_run, mx);
+            const float corr = exp2f(m_run - m_new);
+            float pr[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) pr[i] = vk[i] ? exp2f(sv[i] - m_new) : 0.f;
+            l_run = l_run * corr + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
+            m_run = m_new;
+            // p times the key's V scale, the fp16 A operand of O += P V
+            const float2 vs0 = *reinterpret_cast<const float2*>(vsc + k0);
+            const float2 vs1 = *reinterpret_cast<const float2*>(vsc + k0 + 8);
+            const uint32_t pa0 = f16x2_pack(vk[0] ? pr[0] * vs0.x : 0.f, vk[1] ? pr[1] * vs0.y : 0.f);
+            const uint32_t pa1 = f16x2_pack(vk[2] ? pr[2] * vs1.x : 0.f, vk[3] ? pr[3] * vs1.y : 0.f);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                o[j][0] *= corr;
+                o[j][1] *= corr;
+            }
+            // O += P V: feature row 8 nd + (lane >> 2), this warp's 16-key
+            // group (64-byte swizzle), the lane's four keys in one word
+#pragma unroll
+            for (int nd = 0; nd < 16; ++nd) {
+                const int f = 8 * nd + row;
+                const uint32_t w = *reinterpret_cast<const uint32_t*>(tV + f * 64 + ((warp ^ ((f >> 1) & 3)) << 4) +
+                                                                      4 * quad);
+                uint32_t b0, b1;
+                i8x4_to_f16x2(w, b0, b1);
+                mma_f16_rows8(o[nd][0], o[nd][1], pa0, pa1, b0, b1);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty_bar[st]);
+        }
+        l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+        l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+    }
+    __syncthreads();  // all tiles consumed: the stage buffers are free
+
+    // warp states -> sM[warp][g][STRIDE]: m, l, -, -, o[D]
+    constexpr int STRIDE = D + 4;
+    float* sM = reinterpret_cast<float*>(smem);
+    if (warp < NW && row < G) {
+        float* dst = sM + ((size_t)warp * G + row) * STRIDE;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            dst[4 + 8 * j + 2 * quad] = o[j][0];
+            dst[4 + 8 * j + 2 * quad + 1] = o[j][1];
+        }
+        if (quad == 0) {
+            dst[0] = m_run;
+            dst[1] = l_run;
+        }
+    }
+    __syncthreads();
+    decode_finish<T, D, G, NW, kThreads, 2 * (size_t)STAGES * kQ8Bytes>(sM, comb_bar, s_flag, a, c, d, b, slot, split,
+                                                                      true, fused);
+}
+
+template <int G>
+cudaError_t launch_q8_g(const LayerArgs& a, const CacheArgs& c, const DecodeArgs& d, int grid, cudaStream_t s) {
+    CUtensorMap mK{}, mV{};
+    {
+        const uint64_t dims[3] = {128, (uint64_t)a.capacity, (uint64_t)a.B * a.R};
+        const uint64_t st[2] = {128, 128ull * a.capacity};
+        const uint32_t box[3] = {128, (uint32_t)kTile, 1};
+        if (!encode_tmap(&mK, c.k_full, 3, dims, st, box, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128))
+            return cudaErrorInvalidValue;
+    }
+    {
+        const uint64_t dims[3] = {(uint64_t)kTile, 128, (uint64_t)a.B * a.R * (a.capacity / kTile)};
+        const uint64_t st[2] = {(uint64_t)kTile, 128ull * kTile};
+        const uint32_t box[3] = {(uint32_t)kTile, 128, 1};
+        if (!encode_tmap(&mV, c.v_full, 3, dims, st, box, CU_TENSOR_MAP_DATA_TYPE_UINT8, 64))
+            return cudaErrorInvalidValue;
+    }
+    constexpr size_t smem = decode_q8_smem_bytes();
+    auto kern = decode_q8_kernel<G>;
+    static bool configured = false;  // function attributes are per process, set once
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    return launch_pdl(kern, grid, kMmaThreads, smem, s, mK, mV, a, c, d);
+}
+
 }  // namespace
 
 cudaError_t launch_decode(const LayerArgs& a, const CacheArgs& c, const DecodePlan& plan, const void* q, void* out,
@@ -1102,6 +1395,32 @@ cudaError_t launch_decode(const LayerArgs& a, const CacheArgs& c, const DecodePl
     const long grid = (long)d.n_ret_units + (long)a.B * a.S;
     if (grid == 0) return cudaSuccess;
     if (grid > 0x7fffffffL) return cudaErrorInvalidConfiguration;
+    if (a.kv_int8 && a.R > 0) {
+        // 8-bit full cache: the streaming heads on the bf16 kernel first (no
+        // length ticket), then the retrieval heads, whose last CTA advances
+        // seq_len after both launches have read it
+        if (a.S > 0) {
+            DecodeArgs ds = d;
+            ds.n_ret_units = 0;
+            ds.grid_ticket = nullptr;
+            cudaError_t e = cudaSuccess;
+            switch (a.G) {
+                case 1: e = launch_mma_g<1>(a, c, ds, a.B * a.S, s); break;
+                case 2: e = launch_mma_g<2>(a, c, ds, a.B * a.S, s); break;
+                case 4: e = launch_mma_g<4>(a, c, ds, a.B * a.S, s); break;
+                case 8: e = launch_mma_g<8>(a, c, ds, a.B * a.S, s); break;
+                default: return cudaErrorInvalidValue;
+            }
+            if (e != cudaSuccess) return e;
+        }
+        switch (a.G) {
+            case 1: return launch_q8_g<1>(a, c, d, d.n_ret_units, s);
+            case 2: return launch_q8_g<2>(a, c, d, d.n_ret_units, s);
+            case 4: return launch_q8_g<4>(a, c, d, d.n_ret_units, s);
+            case 8: return launch_q8_g<8>(a, c, d, d.n_ret_units, s);
+        }
+        return cudaErrorInvalidValue;
+    }
     if (a.dtype == DUO_BF16) {
         if (a.D == 128) {
             // bf16, head_dim 128: the tensor-core consumer

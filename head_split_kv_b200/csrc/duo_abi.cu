@@ -63,6 +63,10 @@ duo_status check_desc(const duo_layer_desc* d) {
         return fail(DUO_ERR_INVALID_ARG, "unknown io_order %d", d->io_order);
     if (d->stream_prefill != DUO_STREAM_LAMBDA && d->stream_prefill != DUO_STREAM_CHUNK)
         return fail(DUO_ERR_INVALID_ARG, "unknown stream_prefill %d", d->stream_prefill);
+    if (d->kv_quant != DUO_KV_PLAIN && d->kv_quant != DUO_KV_INT8)
+        return fail(DUO_ERR_INVALID_ARG, "unknown kv_quant %d", d->kv_quant);
+    if (d->kv_quant == DUO_KV_INT8 && (d->dtype != DUO_BF16 || d->head_dim != 128 || d->page_size != 0))
+        return fail(DUO_ERR_UNSUPPORTED, "the 8-bit full cache is built for bf16, head_dim 128, contiguous");
     if (!std::isfinite(d->scale)) return fail(DUO_ERR_INVALID_ARG, "scale is not finite");
     bool seen[DUO_MAX_KV_HEADS] = {};
     for (int i = 0; i < d->n_kv_heads; ++i) {
@@ -88,6 +92,7 @@ void fill_args(const duo_layer_desc* d, duo::LayerArgs& a) {
     a.W = d->sink + d->recent;
     a.dtype = d->dtype;
     a.stream_chunk = d->stream_prefill == DUO_STREAM_CHUNK ? 1 : 0;
+    a.kv_int8 = d->kv_quant == DUO_KV_INT8 ? 1 : 0;
     a.page_size = d->page_size;
     a.capacity = a.max_pages = a.n_pages = 0;
     a.scale = d->scale > 0.f ? d->scale : 1.0f / std::sqrt(static_cast<float>(d->head_dim));
@@ -141,6 +146,14 @@ duo_status check_state(const duo_layer_desc* d, const duo_kv_state* st, duo::Lay
     c.seq_len = st->seq_len;
     c.counters = st->counters;
     c.status = st->status;
+    c.k_scale = st->k_scale;
+    c.v_scale = st->v_scale;
+    if (d->kv_quant == DUO_KV_INT8 && R > 0) {
+        if (!st->k_scale || !st->v_scale) return fail(DUO_ERR_INVALID_ARG, "8-bit cache needs k_scale and v_scale");
+        if (!aligned16(st->k_scale) || !aligned16(st->v_scale))
+            return fail(DUO_ERR_INVALID_ARG, "k_scale / v_scale must be 16-byte aligned");
+        if (st->capacity % 64) return fail(DUO_ERR_SHAPE, "8-bit cache capacity must be a multiple of 64");
+    }
     return DUO_OK;
 }
 
@@ -196,7 +209,7 @@ const char* duo_status_string(duo_status s) {
     return "DUO_ERR_UNKNOWN";
 }
 
-int32_t duo_abi_version(void) { return 2; }
+int32_t duo_abi_version(void) { return 3; }
 
 duo_status duo_partition_heads(const float* alpha, int32_t n_kv_heads, float tau, int32_t target_n_retrieval,
                                uint8_t* gate, int32_t* kv_perm, int32_t* kv_inv_perm, int32_t* n_retrieval) {
@@ -247,6 +260,7 @@ duo_status duo_desc_init(duo_layer_desc* desc, int32_t batch, int32_t n_q_heads,
     desc->n_retrieval = n_retrieval;
     desc->io_order = DUO_ORDER_MODEL;
     desc->stream_prefill = DUO_STREAM_LAMBDA;
+    desc->kv_quant = DUO_KV_PLAIN;
     if (n_kv_heads < 1 || n_kv_heads > DUO_MAX_KV_HEADS)
         return fail(DUO_ERR_INVALID_ARG, "n_kv_heads must be in 1..%d (got %d)", DUO_MAX_KV_HEADS, n_kv_heads);
     for (int i = 0; i < n_kv_heads; ++i) desc->kv_perm[i] = kv_perm[i];
@@ -365,6 +379,8 @@ duo_status duo_prefill_chunk(const duo_layer_desc* desc, const duo_kv_state* st,
         return fail(DUO_ERR_INVALID_ARG, "pre-fill tensors must be 16-byte aligned");
     if (desc->page_size != 0)
         return fail(DUO_ERR_UNSUPPORTED, "duo_prefill_chunk takes a contiguous full cache (page_size 0)");
+    if (desc->kv_quant != DUO_KV_PLAIN)
+        return fail(DUO_ERR_UNSUPPORTED, "duo_prefill_chunk reads a plain full cache, not an 8-bit one");
     cudaError_t e;
     if (a.dtype == DUO_BF16 && a.D == 128) {
         if (!duo::prefill_tc_supported(a))

@@ -17,6 +17,7 @@ struct LayerArgs {
     int B, Hq, Hkv, G, D, R, S, sink, recent, W;
     int dtype, page_size, capacity, max_pages, n_pages;
     int stream_chunk;  // pre-fill: streaming heads see the whole chunk (DUO_STREAM_CHUNK)
+    int kv_int8;       // the full cache holds 8-bit codes + scales (DUO_KV_INT8)
     float scale;       // softmax scale
     // For block slot i (0..Hkv-1): index of its first query head and of its
     // KV head in the caller's q / k / v / out tensors (model or block order).
@@ -36,6 +37,8 @@ struct CacheArgs {
     int32_t* seq_len;
     uint32_t* counters;
     int32_t* status;
+    float* k_scale;    // 8-bit full cache: per-row scales [B][R][capacity]
+    float* v_scale;
 };
 
 // Split-K plan of a decode call: number of splits per (sequence, retrieval
@@ -70,6 +73,9 @@ bool prefill_tc_supported(const LayerArgs& a);
 // cached per (base, dims, strides, box).  False if the driver refuses.
 bool encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                       const uint64_t* strides_bytes, const uint32_t* box);
+// Any element type (a CUtensorMapDataType) and a 32/64/128-byte swizzle (0: none).
+bool encode_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+                 const uint32_t* box, int dtype, int swizzle_bytes);
 
 cudaError_t launch_permute(const void* x, void* y, int64_t rows, int hkv, const int* perm, int heads_per_kv,
                            int64_t head_elems, int elem_bytes, int direction, cudaStream_t s);

@@ -27,6 +27,7 @@ OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_DTYPE, ERR_CAPACITY, ERR_UNSUPPORTED, ERR_CU
 BF16, FP32 = 0, 1
 ORDER_MODEL, ORDER_BLOCK = 0, 1
 STREAM_LAMBDA, STREAM_CHUNK = 0, 1
+KV_PLAIN, KV_INT8 = 0, 1
 MODEL_TO_BLOCK, BLOCK_TO_MODEL = 0, 1
 OP_DECODE, OP_PREFILL = 0, 1
 DEV_FULL_CACHE_OVERFLOW, DEV_BAD_PAGE, DEV_WAIT_TIMEOUT, DEV_BAD_LENGTH = 1, 2, 4, 8
@@ -40,7 +41,7 @@ class LayerDesc(ctypes.Structure):
         ("head_dim", ctypes.c_int32), ("sink", ctypes.c_int32), ("recent", ctypes.c_int32),
         ("dtype", ctypes.c_int32), ("page_size", ctypes.c_int32), ("scale", ctypes.c_float),
         ("n_retrieval", ctypes.c_int32), ("io_order", ctypes.c_int32), ("stream_prefill", ctypes.c_int32),
-        ("kv_perm", ctypes.c_int32 * MAX_KV_HEADS),
+        ("kv_quant", ctypes.c_int32), ("kv_perm", ctypes.c_int32 * MAX_KV_HEADS),
     ]
 
 
@@ -51,6 +52,7 @@ class KVState(ctypes.Structure):
         ("reserved0", ctypes.c_int32),
         ("k_ring", ctypes.c_void_p), ("v_ring", ctypes.c_void_p), ("ring_pos", ctypes.c_void_p),
         ("seq_len", ctypes.c_void_p), ("counters", ctypes.c_void_p), ("status", ctypes.c_void_p),
+        ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
     ]
 
 
@@ -70,7 +72,7 @@ def _fn(name, restype, *argtypes):
 _lib_last_error = _fn("duo_last_error", ctypes.c_char_p)
 _lib_status_string = _fn("duo_status_string", ctypes.c_char_p, ctypes.c_int)
 _lib_abi_version = _fn("duo_abi_version", _I32)
-ABI_VERSION = 2           # the layout of LayerDesc / KVState below
+ABI_VERSION = 3           # the layout of LayerDesc / KVState below
 if _lib_abi_version() != ABI_VERSION:
     raise ImportError(f"{LIB_PATH} has ABI version {_lib_abi_version()}, this binding needs {ABI_VERSION}; rebuild it")
 _lib_partition = _fn("duo_partition_heads", ctypes.c_int, ctypes.POINTER(ctypes.c_float), _I32, ctypes.c_float,
@@ -150,7 +152,8 @@ def partition_heads(alpha, tau: float, target_n_retrieval: int = -1):
 
 
 def desc_init(batch, n_q_heads, n_kv_heads, head_dim, dtype, kv_perm, n_retrieval, *, sink=None, recent=None,
-              page_size=0, io_order=ORDER_MODEL, scale=0.0, stream_prefill=STREAM_LAMBDA) -> LayerDesc:
+              page_size=0, io_order=ORDER_MODEL, scale=0.0, stream_prefill=STREAM_LAMBDA,
+              kv_quant=KV_PLAIN) -> LayerDesc:
     d = LayerDesc()
     perm = (_I32 * max(len(kv_perm), 1))(*[int(p) for p in kv_perm])
     _check(_lib_desc_init(ctypes.byref(d), batch, n_q_heads, n_kv_heads, head_dim, dtype, perm, n_retrieval),
@@ -163,6 +166,7 @@ def desc_init(batch, n_q_heads, n_kv_heads, head_dim, dtype, kv_perm, n_retrieva
     d.io_order = io_order
     d.scale = scale
     d.stream_prefill = stream_prefill
+    d.kv_quant = kv_quant
     _check(_lib_desc_validate(ctypes.byref(d)), "duo_desc_validate")
     return d
 
@@ -240,6 +244,9 @@ class LayerCaches:
     Contiguous full cache: k_full/v_full [B, R, capacity, d].
     Paged full cache: k_full/v_full [n_pages, R, page_size, d] and page_table
     [B, max_pages] int32 (copied from the given host table).
+    8-bit full cache: k_full int8 [B, R, capacity, d], v_full int8
+    [B, R, capacity / 64, d, 64], k_scale/v_scale fp32 [B, R, capacity]
+    (capacity rounded up to a multiple of 64).
     Rings: k_ring/v_ring [B, S, sink + recent, d]; ring_pos [B, W] (-1);
     seq_len [B] (0); counters [4] (0); status [1] (0).
     """
@@ -257,11 +264,22 @@ class LayerCaches:
             self.k_full = torch.zeros((n_pages, R, desc.page_size, d), dtype=dt, device=device)
             self.v_full = torch.zeros_like(self.k_full)
             capacity = max_pages * desc.page_size
+        elif desc.kv_quant == KV_INT8:
+            # 8-bit codes: K row per token, V per 64-token tile transposed; fp32 scale per row
+            max_pages = 0
+            self.page_table = None
+            capacity = (max(capacity, 1) + 63) // 64 * 64
+            self.k_full = torch.zeros((B, R, capacity, d), dtype=torch.int8, device=device)
+            self.v_full = torch.zeros((B, R, capacity // 64, d, 64), dtype=torch.int8, device=device)
+            self.k_scale = torch.zeros((B, R, capacity), dtype=torch.float32, device=device)
+            self.v_scale = torch.zeros_like(self.k_scale)
         else:
             max_pages = 0
             self.page_table = None
             self.k_full = torch.zeros((B, R, max(capacity, 0), d), dtype=dt, device=device)
             self.v_full = torch.zeros_like(self.k_full)
+        if desc.kv_quant != KV_INT8:
+            self.k_scale = self.v_scale = None
         self.capacity = capacity
         self.k_ring = torch.zeros((B, S, W, d), dtype=dt, device=device)
         self.v_ring = torch.zeros_like(self.k_ring)
@@ -273,7 +291,8 @@ class LayerCaches:
             k_full=_ptr(self.k_full), v_full=_ptr(self.v_full), page_table=_ptr(self.page_table),
             capacity=capacity, max_pages=max_pages, n_pages=n_pages, reserved0=0,
             k_ring=_ptr(self.k_ring), v_ring=_ptr(self.v_ring), ring_pos=_ptr(self.ring_pos),
-            seq_len=_ptr(self.seq_len), counters=_ptr(self.counters), status=_ptr(self.status))
+            seq_len=_ptr(self.seq_len), counters=_ptr(self.counters), status=_ptr(self.status),
+            k_scale=_ptr(self.k_scale), v_scale=_ptr(self.v_scale))
 
 
 class Workspace:

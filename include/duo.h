@@ -68,6 +68,11 @@ typedef enum {
 enum { DUO_BF16 = 0, DUO_FP32 = 1 };
 /* head order of q / k / v / out */
 enum { DUO_ORDER_MODEL = 0, DUO_ORDER_BLOCK = 1 };
+/* storage of the retrieval heads' full cache */
+enum {
+    DUO_KV_PLAIN = 0, /* the layer's dtype, as the activations               */
+    DUO_KV_INT8 = 1   /* 8-bit codes + one fp32 scale per row (see duo_kv_state) */
+};
 /* what a streaming head sees in duo_prefill_chunk (decode is the same for both) */
 enum {
     DUO_STREAM_LAMBDA = 0, /* the Lambda mask per query: sinks + its last `recent` tokens */
@@ -102,6 +107,7 @@ typedef struct {
     int32_t n_retrieval;  /* R: retrieval KV heads (block slots 0..R-1)       */
     int32_t io_order;     /* DUO_ORDER_MODEL or DUO_ORDER_BLOCK               */
     int32_t stream_prefill; /* DUO_STREAM_LAMBDA (default) or DUO_STREAM_CHUNK */
+    int32_t kv_quant;     /* DUO_KV_PLAIN (default) or DUO_KV_INT8 (bf16, d 128, contiguous) */
     int32_t kv_perm[DUO_MAX_KV_HEADS]; /* block slot i holds model KV head kv_perm[i] */
 } duo_layer_desc;
 
@@ -120,6 +126,20 @@ typedef struct {
  *   else in slot sink + (p - sink) % recent, evicting the token `recent`
  *   positions older.  ring_pos = [B][W] int32, the position held by each
  *   slot (-1 = empty); all streaming heads of a sequence share it.
+ * 8-bit full cache (desc->kv_quant = DUO_KV_INT8; bf16 activations, d = 128,
+ *   contiguous, capacity a multiple of 64) -- the pages pair the method with a
+ *   quantized KV cache [Review S5 "Decoding performance"] without a scheme;
+ *   this one is per row and symmetric: amax = max |x| over the row's d
+ *   values, code = x * (127 / amax) rounded to nearest even, scale =
+ *   amax / 127, each an fp32 operation (a zero row: scale 0, codes 0);
+ *   attention reads code * scale:
+ *   k_full = int8 [B][R][capacity][d] codes, row per token as above;
+ *   v_full = int8 [B][R][capacity/64][d][64]: per 64-token tile the codes
+ *     transposed (a row of 64 bytes per feature), the 16 tokens of each
+ *     16-token group stored in the order 0 1 8 9 2 3 10 11 4 5 12 13 6 7 14 15;
+ *   k_scale, v_scale = fp32 [B][R][capacity].
+ *   K and V values must stay within +-8.3e6 (the fp16 operands of the
+ *   decode MMAs hold code * 1 and p * scale).
  * seq_len = [B] int32: tokens appended so far per sequence.
  * counters = DUO_STATE_COUNTER_WORDS uint32 words that must be zero before
  *   the first call; every call leaves them zero.
@@ -141,6 +161,8 @@ typedef struct {
     int32_t* seq_len;
     uint32_t* counters;
     int32_t* status;
+    float* k_scale;      /* 8-bit full cache only, else NULL         */
+    float* v_scale;
 } duo_kv_state;
 
 /* ------------------------------------------------------------------------ */
@@ -151,7 +173,8 @@ typedef struct {
 const char* duo_last_error(void);
 /* Name of a status code. */
 const char* duo_status_string(duo_status s);
-/* ABI version: 2 (duo_layer_desc gained stream_prefill). */
+/* ABI version: 3 (duo_layer_desc gained stream_prefill and kv_quant,
+ * duo_kv_state the 8-bit cache's scales). */
 int32_t duo_abi_version(void);
 
 /* ------------------------------------------------------------------------ */
@@ -236,6 +259,8 @@ duo_status duo_permute_heads(const duo_layer_desc* desc, const void* x, void* y,
  * the full cache at p.  Streaming heads: written to the ring only if
  * p < sink or p >= seq_len[b] + T - recent (the tokens that survive), and
  * ring_pos is updated.  seq_len[b] += T once every row is written.
+ * With an 8-bit full cache the retrieval rows are quantized on the way in
+ * (codes and scale as duo_kv_state describes).
  * T == 0 is a no-op.  A row past capacity (or with no page) is not written
  * and sets DUO_DEV_FULL_CACHE_OVERFLOW (DUO_DEV_BAD_PAGE).
  * Errors: DUO_ERR_INVALID_ARG, DUO_ERR_SHAPE, DUO_ERR_CUDA.
@@ -254,7 +279,9 @@ duo_status duo_append_kv(const duo_layer_desc* desc, const duo_kv_state* st, con
  * Retrieval heads: out = softmax(scale q K^T) V over cache rows
  * 0..seq_len[b]-1, split-K across CTAs with a last-CTA combine.  Streaming
  * heads: the same over the min(seq_len[b], W) ring slots.  The G query heads
- * of a KV head share every K/V tile.
+ * of a KV head share every K/V tile.  With an 8-bit full cache the scores
+ * are q . codes * k_scale and the values code * v_scale, the scales applied
+ * per key to the scores and to p (half the bytes per cached token).
  * workspace: >= duo_workspace_bytes(desc, DUO_OP_DECODE, 0) bytes, zeroed once.
  * Concurrent calls must not share a workspace.
  * Errors: DUO_ERR_INVALID_ARG, DUO_ERR_SHAPE, DUO_ERR_CAPACITY (workspace),
@@ -300,7 +327,8 @@ duo_status duo_decode_step(const duo_layer_desc* desc, const duo_kv_state* st, c
  * bf16 with d = 128 runs on the tcgen05 tensor cores (TMA-fed tiles, TMEM
  * accumulators); fp32 and d = 64 run on the CUDA cores.
  * workspace: >= duo_workspace_bytes(desc, DUO_OP_PREFILL, C) bytes (may be 0).
- * The full cache must be contiguous (page_size 0) here.
+ * The full cache must be contiguous (page_size 0) and not 8-bit here
+ * (DUO_ERR_UNSUPPORTED): the pre-fill reads its prior tiles in bf16.
  * Errors: DUO_ERR_INVALID_ARG, DUO_ERR_SHAPE, DUO_ERR_CAPACITY,
  * DUO_ERR_UNSUPPORTED, DUO_ERR_CUDA.
  */

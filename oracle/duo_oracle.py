@@ -317,17 +317,13 @@ def quantize_int8_rows(x) -> tuple:
     float32 [n]).  Every step is one float32 operation as written, so the
     codes are those any IEEE float32 implementation of the same steps gets."""
     x32 = as_f64(x).astype(np.float32)
-    codes = np.zeros(x32.shape, dtype=np.int8)
-    scales = np.zeros(x32.shape[:-1], dtype=np.float32)
-    for i in range(x32.shape[0]):
-        row = x32[i]
-        amax = np.float32(np.max(np.abs(row))) if row.size else np.float32(0)
-        if amax == 0:
-            continue
-        inv = np.float32(127.0) / amax
-        q = np.rint(row * inv)                      # float32 product, round half to even
-        codes[i] = np.clip(q, -127, 127).astype(np.int8)
-        scales[i] = amax / np.float32(127.0)
+    amax = np.abs(x32).max(axis=-1) if x32.shape[-1] else np.zeros(x32.shape[:-1], np.float32)
+    nz = amax > 0
+    inv = np.zeros_like(amax)
+    inv[nz] = np.float32(127.0) / amax[nz]                      # float32 division
+    q = np.rint(x32 * inv[..., None])                           # float32 product, round half to even
+    codes = np.clip(q, -127, 127).astype(np.int8)
+    scales = np.where(nz, amax / np.float32(127.0), np.float32(0)).astype(np.float32)
     return codes, scales
 
 

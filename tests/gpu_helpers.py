@@ -55,7 +55,7 @@ class Layer:
     """One attention layer on the device plus its oracle twin."""
 
     def __init__(self, duo, shape: S.LayerShape, retrieval, batch: int, capacity: int = 0, page_size: int = 0,
-                 page_table=None, n_pages: int = 0, io_order=None, stream_prefill: int = 0):
+                 page_table=None, n_pages: int = 0, io_order=None, stream_prefill: int = 0, kv_quant: int = 0):
         self.duo = duo
         self.shape = shape
         self.B = batch
@@ -68,11 +68,12 @@ class Layer:
         self.desc = duo.desc_init(batch, shape.n_q_heads, hkv, shape.head_dim,
                                   duo.BF16 if shape.dtype == "bf16" else duo.FP32, self.perm, self.R,
                                   sink=shape.sink, recent=shape.recent, page_size=page_size,
-                                  io_order=self.io_order, stream_prefill=stream_prefill)
+                                  io_order=self.io_order, stream_prefill=stream_prefill, kv_quant=kv_quant)
+        self.kv_int8 = kv_quant == duo.KV_INT8
         self.page_table = None if page_table is None else np.asarray(page_table, dtype=np.int32)
         self.caches = duo.LayerCaches(self.desc, capacity, self.page_table, n_pages)
         self.oracle = O.HeadSplitCache(batch, hkv, shape.head_dim, gate=self.gate, sink=shape.sink,
-                                       recent=shape.recent)
+                                       recent=shape.recent, kv_int8=self.kv_int8)
         self.ws = duo.Workspace(self.desc, duo.OP_DECODE, self.caches.capacity)
 
     # -- head order ----------------------------------------------------------
@@ -171,7 +172,23 @@ class Layer:
             L = self.oracle.length[b]
             for h in range(sh.n_kv_heads):
                 slot = self.inv[h]
-                if self.gate[h]:
+                if self.gate[h] and self.kv_int8:
+                    # 8-bit layout: K codes a row per token; V codes per 64-token
+                    # tile, transposed, tokens of a 16-group in the order
+                    # 0 1 8 9 2 3 10 11 4 5 12 13 6 7 14 15
+                    pos, kc, ks, vc, vs = self.oracle.quantized(b, h)
+                    assert np.array_equal(pos, np.arange(L))
+                    k8 = bits(c.k_full)[b, slot, :L]
+                    v8 = bits(c.v_full)[b, slot]
+                    order = [0, 1, 8, 9, 2, 3, 10, 11, 4, 5, 12, 13, 6, 7, 14, 15]
+                    where = np.argsort(order)                          # token -> position in its group
+                    col = (pos % 64) // 16 * 16 + where[pos % 16]
+                    got_v = v8[pos // 64, :, col]                      # [L, d]
+                    assert np.array_equal(k8, kc), f"8-bit K codes b={b} h={h}"
+                    assert np.array_equal(got_v, vc), f"8-bit V codes b={b} h={h}"
+                    assert np.array_equal(bits(c.k_scale)[b, slot, :L], ks), f"K scales b={b} h={h}"
+                    assert np.array_equal(bits(c.v_scale)[b, slot, :L], vs), f"V scales b={b} h={h}"
+                elif self.gate[h]:
                     pos, ko, vo = self.oracle.rows(b, h)
                     if self.page_table is None:
                         gk, gv = kf[b, slot, pos], vf[b, slot, pos]

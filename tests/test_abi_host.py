@@ -64,7 +64,7 @@ int main(void) {
 
 
 def test_abi_version_and_status_strings(duo):
-    assert duo.abi_version() == duo.ABI_VERSION == 2
+    assert duo.abi_version() == duo.ABI_VERSION == 3
     assert duo.status_string(duo.OK) == "DUO_OK"
     assert duo.status_string(duo.ERR_CAPACITY) == "DUO_ERR_CAPACITY"
 
@@ -227,3 +227,36 @@ def test_stream_prefill_mode_is_validated(duo):
     assert duo.desc_init(1, 8, 4, 128, duo.BF16, [0, 1, 2, 3], 2).stream_prefill == duo.STREAM_LAMBDA
     d.stream_prefill = 2
     assert duo.desc_validate(d) == duo.ERR_INVALID_ARG
+
+
+def test_int8_cache_is_validated(duo):
+    perm = [0, 1, 2, 3]
+    d = duo.desc_init(1, 8, 4, 128, duo.BF16, perm, 2, kv_quant=duo.KV_INT8)
+    assert d.kv_quant == duo.KV_INT8
+    with pytest.raises(duo.DuoError) as e:
+        duo.desc_init(1, 8, 4, 64, duo.BF16, perm, 2, kv_quant=duo.KV_INT8)
+    assert e.value.status == duo.ERR_UNSUPPORTED
+    with pytest.raises(duo.DuoError) as e:
+        duo.desc_init(1, 8, 4, 128, duo.FP32, perm, 2, kv_quant=duo.KV_INT8)
+    assert e.value.status == duo.ERR_UNSUPPORTED
+    d.kv_quant = 2
+    assert duo.desc_validate(d) == duo.ERR_INVALID_ARG
+
+
+def test_int8_prefill_is_refused_before_any_launch(duo):
+    d = duo.desc_init(1, 8, 4, 128, duo.BF16, [0, 1, 2, 3], 2, kv_quant=duo.KV_INT8)
+    st = _state(duo)
+    st.k_scale, st.v_scale = 4096, 8192
+    st.capacity = 1024
+    with pytest.raises(duo.DuoError) as e:
+        duo.prefill_chunk(d, st, 256, 512, 768, 16, 1024, stream=0)
+    assert e.value.status == duo.ERR_UNSUPPORTED
+    # the state must carry the scales and a capacity in whole 64-token tiles
+    st.capacity = 1000
+    with pytest.raises(duo.DuoError) as e:
+        duo.append_kv(d, st, 256, 512, 1, stream=0)
+    assert e.value.status == duo.ERR_SHAPE
+    st.capacity, st.k_scale = 1024, None
+    with pytest.raises(duo.DuoError) as e:
+        duo.append_kv(d, st, 256, 512, 1, stream=0)
+    assert e.value.status == duo.ERR_INVALID_ARG
