@@ -1087,9 +1087,9 @@ cudaError_t launch_d(const LayerArgs& a, const CacheArgs& c, const DecodeArgs& d
 }
 
 // ===========================================================================
-// 8-bit full cache: decode_q8_kernel, retrieval heads only (an 8-bit layer's
-// streaming heads run the bf16 kernel in a launch just before, without the
-// length ticket).  Per CTA as decode_mma_kernel -- a TMA producer warp, four
+// 8-bit full cache: decode_q8_kernel.  Streaming CTAs (after the retrieval
+// ones in the grid) read the bf16 ring on the CUDA cores (decode_ring_simt).
+// Per retrieval CTA as decode_mma_kernel -- a TMA producer warp, four
 // consumer warps of 16 keys each, the same split plan and split-K combine --
 // with a 64-token stage of 8 KB of K codes (a row per token, 128-byte
 // swizzle), 8 KB of V codes (transposed, 64-byte swizzle) and the tile's 64 +
@@ -1124,6 +1124,114 @@ __device__ __forceinline__ void mma_f16_rows8(float& c0, float& c1, uint32_t a0,
         : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(0.f), "f"(0.f));
 }
 
+// An 8-bit layer's streaming head in the same launch: the ring's min(len, W)
+// bf16 rows (every one visible to the new token) on the CUDA cores.  The rows
+// are staged in shared memory (rows padded to 272 bytes, so that lanes
+// reading different rows hit different banks), then three passes: the
+// G x n scores, one per thread at a time; the softmax of each head's row of
+// scores, one warp per head; the outputs, one (head, 8 features) per thread.
+// With a fused append the new token is first written to its ring slot.
+constexpr int kRingRowBytes = 272;
+constexpr int kRingMax = 128;        // ring rows this path stages (sink + recent)
+
+template <int G>
+__device__ __forceinline__ void decode_ring_simt(uint8_t* smem, const LayerArgs& a, const CacheArgs& c,
+                                                 const DecodeArgs& d, int b, int slot, int L0, bool fused) {
+    using T = __nv_bfloat16;
+    constexpr int D = 128;
+    const int tid = threadIdx.x, nthr = blockDim.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int s_idx = slot - a.R;
+    T* kr = static_cast<T*>(c.k_ring) + ((size_t)b * a.S + s_idx) * a.W * D;
+    T* vr = static_cast<T*>(c.v_ring) + ((size_t)b * a.S + s_idx) * a.W * D;
+    int len = L0 < 0 ? 0 : L0;
+    if (L0 < 0 && tid == 0) atomicOr(c.status, DUO_DEV_BAD_LENGTH);
+    if (fused && L0 >= 0) {
+        if (warp == 0) {
+            const int rs = ring_slot(L0, a.sink, a.recent);
+            const int h = a.kv_head[slot];
+            const uint2* kn = reinterpret_cast<const uint2*>(static_cast<const T*>(d.k_new) + ((size_t)b * a.Hkv + h) * D);
+            const uint2* vn = reinterpret_cast<const uint2*>(static_cast<const T*>(d.v_new) + ((size_t)b * a.Hkv + h) * D);
+            reinterpret_cast<uint2*>(kr + (size_t)rs * D)[lane] = kn[lane];
+            reinterpret_cast<uint2*>(vr + (size_t)rs * D)[lane] = vn[lane];
+            if (s_idx == 0 && lane == 0) c.ring_pos[(size_t)b * a.W + rs] = L0;
+        }
+        len = L0 + 1;
+    }
+    __syncthreads();
+    const int nk = min(min(len, a.W), kRingMax);
+    uint8_t* sK = smem;                                     // [kRingMax][272]
+    uint8_t* sV = sK + kRingMax * kRingRowBytes;
+    float* sS = reinterpret_cast<float*>(sV + kRingMax * kRingRowBytes);   // [G][kRingMax] scores, then p
+    float* sQ = sS + G * kRingMax;                                          // [G][D] q * scale * log2 e
+    float* sL = sQ + G * D;                                                 // [G] 1 / row sum
+    for (int i = tid; i < nk * 16; i += nthr) {
+        const int j = i >> 4, piece = i & 15;
+        *reinterpret_cast<uint4*>(sK + j * kRingRowBytes + piece * 16) = reinterpret_cast<const uint4*>(kr + (size_t)j * D)[piece];
+        *reinterpret_cast<uint4*>(sV + j * kRingRowBytes + piece * 16) = reinterpret_cast<const uint4*>(vr + (size_t)j * D)[piece];
+    }
+    const float sl = a.scale * kLog2e;
+    for (int i = tid; i < G * D; i += nthr) {
+        const int g = i / D, e = i % D;
+        sQ[i] = __bfloat162float(static_cast<const T*>(d.q)[((size_t)b * a.Hq + a.q_head0[slot] + g) * D + e]) * sl;
+    }
+    __syncthreads();
+    // scores
+    for (int i = tid; i < G * nk; i += nthr) {
+        const int g = i / nk, j = i % nk;
+        const float* q = sQ + g * D;
+        float acc = 0.f;
+#pragma unroll 4
+        for (int piece = 0; piece < 16; ++piece) {
+            float kf[8];
+            load_row_f32<T, 8>(reinterpret_cast<const T*>(sK + j * kRingRowBytes + piece * 16), kf);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc = fmaf(q[piece * 8 + e], kf[e], acc);
+        }
+        sS[g * kRingMax + j] = acc;
+    }
+    __syncthreads();
+    // softmax of each head's scores: p in place, 1 / sum aside
+    for (int g = warp; g < G; g += nthr >> 5) {
+        float m = kNegBig;
+        for (int j = lane; j < nk; j += 32) m = fmaxf(m, sS[g * kRingMax + j]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float l = 0.f;
+        for (int j = lane; j < nk; j += 32) {
+            const float pj = exp2f(sS[g * kRingMax + j] - m);
+            sS[g * kRingMax + j] = pj;
+            l += pj;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        if (lane == 0) sL[g] = l > 0.f ? 1.f / l : 0.f;
+    }
+    __syncthreads();
+    // outputs: (head, 8 consecutive features) per thread
+    for (int i = tid; i < G * 16; i += nthr) {
+        const int g = i >> 4, piece = i & 15;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int j = 0; j < nk; ++j) {
+            const float pj = sS[g * kRingMax + j];
+            float vf[8];
+            load_row_f32<T, 8>(reinterpret_cast<const T*>(sV + j * kRingRowBytes + piece * 16), vf);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = fmaf(pj, vf[e], acc[e]);
+        }
+        const float inv = sL[g];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] *= inv;
+        store_row<T, 8>(static_cast<T*>(d.out) + ((size_t)b * a.Hq + a.q_head0[slot] + g) * D + piece * 8, acc);
+    }
+}
+
+constexpr size_t ring_simt_smem_bytes(int G) {
+    return 2 * (size_t)kRingMax * kRingRowBytes + (size_t)G * kRingMax * 4 + (size_t)G * 128 * 4 + 8 * 4;
+}
+static_assert(ring_simt_smem_bytes(8) <= 2 * (size_t)kQ8Stages * kQ8Bytes + kQ8Stages * kQ8ScBytes,
+              "the ring path must fit below the 8-bit kernel's barriers");
+
 template <int G>
 __global__ void __maxnreg__(200)
     decode_q8_kernel(const __grid_constant__ CUtensorMap tmK8, const __grid_constant__ CUtensorMap tmV8,
@@ -1151,10 +1259,18 @@ __global__ void __maxnreg__(200)
     }
 
     // ---------------------------------------------------------- work unit
-    const int split = blockIdx.x % d.nsplit;
-    const int pair = blockIdx.x / d.nsplit;
-    const int slot = pair % a.R;
-    const int b = pair / a.R;
+    const bool retrieval = (int)blockIdx.x < d.n_ret_units;
+    int split = 0, slot, b;
+    if (retrieval) {
+        split = blockIdx.x % d.nsplit;
+        const int pair = blockIdx.x / d.nsplit;
+        slot = pair % a.R;
+        b = pair / a.R;
+    } else {
+        const int u = blockIdx.x - d.n_ret_units;
+        slot = a.R + u % a.S;
+        b = u / a.S;
+    }
     const int z = b * a.R + slot;
     const int tiles_per_head = a.capacity / kTile;
     const bool fused = d.k_new != nullptr;
@@ -1176,6 +1292,10 @@ __global__ void __maxnreg__(200)
     __syncthreads();
     const int L0 = *s_flag;
     if (fused && d.grid_ticket && threadIdx.x == 0) length_ticket(a, c, d);
+    if (!retrieval) {
+        decode_ring_simt<G>(smem, a, c, d, b, slot, L0, fused);
+        return;
+    }
     int len = L0;
     int new_row = -1;
     if (fused) {
@@ -1396,28 +1516,13 @@ cudaError_t launch_decode(const LayerArgs& a, const CacheArgs& c, const DecodePl
     if (grid == 0) return cudaSuccess;
     if (grid > 0x7fffffffL) return cudaErrorInvalidConfiguration;
     if (a.kv_int8 && a.R > 0) {
-        // 8-bit full cache: the streaming heads on the bf16 kernel first (no
-        // length ticket), then the retrieval heads, whose last CTA advances
-        // seq_len after both launches have read it
-        if (a.S > 0) {
-            DecodeArgs ds = d;
-            ds.n_ret_units = 0;
-            ds.grid_ticket = nullptr;
-            cudaError_t e = cudaSuccess;
-            switch (a.G) {
-                case 1: e = launch_mma_g<1>(a, c, ds, a.B * a.S, s); break;
-                case 2: e = launch_mma_g<2>(a, c, ds, a.B * a.S, s); break;
-                case 4: e = launch_mma_g<4>(a, c, ds, a.B * a.S, s); break;
-                case 8: e = launch_mma_g<8>(a, c, ds, a.B * a.S, s); break;
-                default: return cudaErrorInvalidValue;
-            }
-            if (e != cudaSuccess) return e;
-        }
+        // 8-bit full cache: retrieval CTAs on the int8 tiles, streaming CTAs
+        // over the bf16 ring on the CUDA cores, one launch
         switch (a.G) {
-            case 1: return launch_q8_g<1>(a, c, d, d.n_ret_units, s);
-            case 2: return launch_q8_g<2>(a, c, d, d.n_ret_units, s);
-            case 4: return launch_q8_g<4>(a, c, d, d.n_ret_units, s);
-            case 8: return launch_q8_g<8>(a, c, d, d.n_ret_units, s);
+            case 1: return launch_q8_g<1>(a, c, d, (int)grid, s);
+            case 2: return launch_q8_g<2>(a, c, d, (int)grid, s);
+            case 4: return launch_q8_g<4>(a, c, d, (int)grid, s);
+            case 8: return launch_q8_g<8>(a, c, d, (int)grid, s);
         }
         return cudaErrorInvalidValue;
     }

@@ -65,8 +65,10 @@ duo_status check_desc(const duo_layer_desc* d) {
         return fail(DUO_ERR_INVALID_ARG, "unknown stream_prefill %d", d->stream_prefill);
     if (d->kv_quant != DUO_KV_PLAIN && d->kv_quant != DUO_KV_INT8)
         return fail(DUO_ERR_INVALID_ARG, "unknown kv_quant %d", d->kv_quant);
-    if (d->kv_quant == DUO_KV_INT8 && (d->dtype != DUO_BF16 || d->head_dim != 128 || d->page_size != 0))
-        return fail(DUO_ERR_UNSUPPORTED, "the 8-bit full cache is built for bf16, head_dim 128, contiguous");
+    if (d->kv_quant == DUO_KV_INT8 &&
+        (d->dtype != DUO_BF16 || d->head_dim != 128 || d->page_size != 0 || d->sink + d->recent > 128))
+        return fail(DUO_ERR_UNSUPPORTED,
+                    "the 8-bit full cache is built for bf16, head_dim 128, contiguous, sink + recent <= 128");
     if (!std::isfinite(d->scale)) return fail(DUO_ERR_INVALID_ARG, "scale is not finite");
     bool seen[DUO_MAX_KV_HEADS] = {};
     for (int i = 0; i < d->n_kv_heads; ++i) {

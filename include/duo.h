@@ -107,7 +107,7 @@ typedef struct {
     int32_t n_retrieval;  /* R: retrieval KV heads (block slots 0..R-1)       */
     int32_t io_order;     /* DUO_ORDER_MODEL or DUO_ORDER_BLOCK               */
     int32_t stream_prefill; /* DUO_STREAM_LAMBDA (default) or DUO_STREAM_CHUNK */
-    int32_t kv_quant;     /* DUO_KV_PLAIN (default) or DUO_KV_INT8 (bf16, d 128, contiguous) */
+    int32_t kv_quant;     /* DUO_KV_PLAIN (default) or DUO_KV_INT8 (bf16, d 128, contiguous, sink + recent <= 128) */
     int32_t kv_perm[DUO_MAX_KV_HEADS]; /* block slot i holds model KV head kv_perm[i] */
 } duo_layer_desc;
 
