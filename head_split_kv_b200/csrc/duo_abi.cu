@@ -283,7 +283,12 @@ size_t duo_workspace_bytes(const duo_layer_desc* desc, int32_t op, int32_t max_t
         a.capacity = max_tokens > 0 ? max_tokens : 1;
         return duo::decode_plan(a).bytes;
     }
-    if (op == DUO_OP_PREFILL) return 256;
+    if (op == DUO_OP_PREFILL) {
+        duo::LayerArgs a;
+        fill_args(desc, a);
+        if (a.dtype != DUO_BF16 || a.D != 128) return 256;   // the CUDA-core path needs none
+        return duo::prefill_workspace_bytes(a, max_tokens > 0 ? max_tokens : 1);
+    }
     return 0;
 }
 
@@ -367,8 +372,6 @@ duo_status duo_decode_step(const duo_layer_desc* desc, const duo_kv_state* st, c
 duo_status duo_prefill_chunk(const duo_layer_desc* desc, const duo_kv_state* st, const void* q, const void* k_chunk,
                              const void* v_chunk, int32_t C, void* out, void* workspace, size_t ws_bytes,
                              duo_stream_t stream) {
-    (void)workspace;
-    (void)ws_bytes;
     duo_status s = check_desc(desc);
     if (s != DUO_OK) return s;
     duo::LayerArgs a;
@@ -387,7 +390,7 @@ duo_status duo_prefill_chunk(const duo_layer_desc* desc, const duo_kv_state* st,
     if (a.dtype == DUO_BF16 && a.D == 128) {
         if (!duo::prefill_tc_supported(a))
             return fail(DUO_ERR_UNSUPPORTED, "tensor-core pre-fill cannot take this layer");
-        e = duo::launch_prefill_tc(a, c, q, k_chunk, v_chunk, C, out, (cudaStream_t)stream);
+        e = duo::launch_prefill_tc(a, c, q, k_chunk, v_chunk, C, out, workspace, ws_bytes, (cudaStream_t)stream);
     } else {
         e = duo::launch_simt_attention(a, &c, nullptr, q, k_chunk, v_chunk, C, out, 0, (cudaStream_t)stream);
     }
@@ -436,6 +439,13 @@ duo_status duo_gated_mix_grad_alpha(const duo_layer_desc* desc, const void* q, c
     }
     e = duo::launch_simt_attention(a, nullptr, nullptr, q, k, v, N, nullptr, 2, (cudaStream_t)stream, dout, dalpha);
     return e == cudaSuccess ? ok() : cuda_fail(e, "duo_gated_mix_grad_alpha");
+}
+
+duo_status duo_exp2_fma_probe(const float* x, float* y, int64_t n, duo_stream_t stream) {
+    if (n < 0) return fail(DUO_ERR_INVALID_ARG, "duo_exp2_fma_probe: n must be >= 0 (got %lld)", (long long)n);
+    if (n > 0 && (!x || !y)) return fail(DUO_ERR_INVALID_ARG, "duo_exp2_fma_probe: NULL argument");
+    cudaError_t e = duo::launch_exp2_fma_probe(x, y, n, (cudaStream_t)stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "duo_exp2_fma_probe");
 }
 
 duo_status duo_check_status(const duo_kv_state* st, int32_t* host_status, duo_stream_t stream) {

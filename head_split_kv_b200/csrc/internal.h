@@ -65,8 +65,19 @@ cudaError_t launch_simt_attention(const LayerArgs& a, const CacheArgs* c, const 
                                   const void* dout = nullptr, float* dalpha = nullptr);
 // tcgen05 pre-fill for bf16, d = 128; returns cudaErrorNotSupported when it
 // cannot take the call.
+// Key-range split plan of the tensor-core pre-fill (see prefill_tc.cu).
+struct PrefillPlan {
+    int ns;                 // CTAs per retrieval unit
+    size_t ticket_offset;   // bytes from workspace start to the ticket words
+    size_t bytes;           // workspace bytes the plan needs (256 when ns == 1)
+};
+int sm_count();
+PrefillPlan prefill_plan(const LayerArgs& a, int C, int n_sms);
+size_t prefill_workspace_bytes(const LayerArgs& a, int max_chunk);
 cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void* q, const void* k_chunk,
-                              const void* v_chunk, int C, void* out, cudaStream_t s);
+                              const void* v_chunk, int C, void* out, void* workspace, size_t ws_bytes,
+                              cudaStream_t s);
+cudaError_t launch_exp2_fma_probe(const float* x, float* y, int64_t n, cudaStream_t s);
 bool prefill_tc_supported(const LayerArgs& a);
 // bf16 tensor map of `rank` dims (innermost first), 64-element-wide boxes with
 // the 128-byte swizzle, out-of-range elements read as zero; encodings are

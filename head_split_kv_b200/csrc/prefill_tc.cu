@@ -54,6 +54,12 @@ constexpr uint32_t kTmemCols = 512;
 __device__ __forceinline__ constexpr uint32_t col_s(int i) { return 128u * (uint32_t)i; }       // S_i (and P_i)
 __device__ __forceinline__ constexpr uint32_t col_o(int i) { return 256u + 128u * (uint32_t)i; }  // O_i
 constexpr int kMaxRing = 128;      // sink + recent held by one tile
+constexpr int kMaxSplit = 8;       // key-range splits per retrieval unit
+constexpr int kMinSplitTiles = 16; // no split shorter than 16 key tiles (2,048 keys)
+// One query tile's partial record of one split: the lazily raised row maxima
+// (log2 domain), the row sums, then O unnormalised as [32 column groups][128
+// rows][4], so that a warp's 32 rows write one 512-byte run per group.
+constexpr int kPartFloats = 2 * BM + BM * HD;
 
 constexpr uint32_t kQBytes = BM * HD * 2;      // 32 KB per query tile (two 16 KB halves of d)
 constexpr uint32_t kTileBytes = BN * HD * 2;   // 32 KB per K or V tile (two 16 KB halves of d)
@@ -73,7 +79,11 @@ struct TcArgs {
     LayerArgs a;
     int C;                 // chunk length
     int n_mpairs;          // ceil(C / 256)
-    int n_ret_ctas;        // B * R * G * n_mpairs
+    int n_units;           // retrieval units B * R * G * n_mpairs
+    int ns;                // CTAs per retrieval unit (key-range splits; 1 = none)
+    int n_ret_ctas;        // n_units * ns
+    float* part;           // [n_units][ns][2][kPartFloats] partial records (ns > 1)
+    uint32_t* ticket;      // [n_units] arrivals; the last split merges and resets it
     const int32_t* seq_len;
     int32_t* status;
     void* out;
@@ -220,37 +230,66 @@ __device__ __forceinline__ void visible_columns(const LayerArgs& a, const Sched&
 
 // ------------------------------------------------------------------ softmax
 
-// One row's share of one tile: S (128 columns at s_addr) from TMEM, the
-// running maximum m_ref (log2 domain, lazy: raised only when the tile's
-// maximum exceeds it by more than 2^8) and row sum l_sum updated, and
-// p = 2^(s * scale * log2e - m) written back as packed bf16 over the second
-// half of S for the PV MMA.  Returns the factor by which O must be rescaled
-// (1 unless `need`).
+constexpr int kFmaExpEvery = 8;   // one exp2 pair in 8 on the FMA pipe
+
+// 2^x for a pair of x <= 0 (or -inf) on the FMA pipe, by Cody-Waite range
+// reduction and a polynomial: x = n + f with n = rint(x) (adding 1.5 * 2^23
+// rounds x to an integer held in the low mantissa bits) and f in [-0.5, 0.5];
+// 2^f by a cubic whose coefficients were fitted here to minimise the largest
+// relative error on [-0.5, 0.5] (7.5e-5, far below the 2^-9 half-step of the
+// bf16 p it feeds); 2^n by adding n to the exponent field.  x is clamped at
+// -125 so that the exponent stays normal: a masked key (x = -inf) gets
+// about 2^-125 instead of 0, 1e-38 of the row's largest weight.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+    constexpr float kShift = 12582912.f;  // 1.5 * 2^23
+    constexpr float c0 = 0.9999280571937561f, c1 = 0.6932610273361206f, c2 = 0.24261116981506348f,
+                    c3 = 0.055171627551317215f;
+    x = make_float2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
+    const float2 t = fadd2(x, make_float2(kShift, kShift));
+    const float2 n = fadd2(t, make_float2(-kShift, -kShift));
+    const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
+    float2 q = ffma2(make_float2(c3, c3), f, make_float2(c2, c2));
+    q = ffma2(q, f, make_float2(c1, c1));
+    q = ffma2(q, f, make_float2(c0, c0));
+    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// One row's share of one tile: S (128 columns at s_addr) from TMEM in one
+// round trip, the keys the row does not see set to -inf when `masked` (bit c
+// of vis = column c visible), the running maximum m_ref (log2 domain, lazy:
+// raised only when the tile's maximum exceeds it by more than 2^8) and row sum
+// l_sum updated, and p = 2^(s * scale * log2e - m) written back as packed bf16
+// over the second half of S for the PV MMA (keys 0..63 to columns 64..95,
+// keys 64..127 to columns 96..127).  Returns the factor by which O must be
+// rescaled (1 unless `need`).  The row sum adds the rounded p, so each output
+// is a convex combination of V rows.
 //
-// S is read in two 64-column halves (a whole row would need more registers
-// than three warps per SM sub-partition leave): keys 0..63 for the maximum
-// only, then keys 64..127, which stay in registers; p of keys 64..127 goes to
-// columns 96..127, then keys 0..63 (loaded again) to columns 64..95.  The row
-// sum adds the rounded p, so each output is a convex combination of V rows.
-__device__ __forceinline__ float softmax_tile(uint32_t s_addr, float sl, float& m_ref, float& l_sum, bool& need) {
-    // maximum of 64 raw scores: three-input max, 4 chains
-    auto max_half = [](const float (&v)[64]) {
-        float m4[4] = {v[0], v[1], v[2], v[3]};
+// The exponentials: one tile costs a softmax warp 128 exp2 per row, as many
+// cycles on the SFU as the tile's two MMAs take on the tensor core, so the
+// SFU is the co-bottleneck.  One pair in kFmaExpEvery is computed on the FMA
+// pipe instead (exp2_fma2): 2 % faster than SFU-only on the 131K prompt, and
+// faster than one pair in 4.
+__device__ __forceinline__ float softmax_tile(uint32_t s_addr, float sl, bool masked, const uint32_t (&vis)[4],
+                                              float& m_ref, float& l_sum, bool& need) {
+    float s[128];
+    tmem_ld128(s_addr, s);
+    if (masked) {
 #pragma unroll
-        for (int c = 4; c < 60; c += 8) {
+        for (int c = 0; c < 128; ++c)
+            if (!((vis[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
+    }
+    // maximum of the raw scores: three-input max, 4 chains
+    float m4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) m4[i] = fmax3(m4[i], v[c + i], v[c + 4 + i]);
-        }
+    for (int c = 4; c < 124; c += 8) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) m4[i] = fmaxf(m4[i], v[60 + i]);
-        return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-    };
-    float s[64];
-    tmem_ld64(s_addr, s);
-    float mx = max_half(s);
-    tmem_ld64(s_addr + 64, s);
+        for (int i = 0; i < 4; ++i) m4[i] = fmax3(m4[i], s[c + i], s[c + 4 + i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m4[i] = fmaxf(m4[i], s[124 + i]);
     // into the log2 domain: the scale is positive, so it commutes with max
-    mx = fmaxf(mx, max_half(s)) * sl;
+    const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl;
     const float m_new = fmaxf(m_ref, mx);
     need = m_new > m_ref + 8.f;                           // lazy rescale threshold: 2^8
     const float m_use = need ? m_new : m_ref;
@@ -258,53 +297,24 @@ __device__ __forceinline__ float softmax_tile(uint32_t s_addr, float sl, float& 
     const float corr = need ? exp2_approx(m_ref - m_use) : 1.f;
     const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(-m_safe, -m_safe);
     float2 rs2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-    auto exp_half = [&](const float (&v)[64], uint32_t taddr) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
         uint32_t pk[32];
 #pragma unroll
         for (int c2 = 0; c2 < 32; ++c2) {
-            const float2 x = ffma2(make_float2(v[2 * c2], v[2 * c2 + 1]), sl2, nm2);
-            const float2 e = make_float2(exp2_approx(x.x), exp2_approx(x.y));
+            const float2 x = ffma2(make_float2(s[64 * h + 2 * c2], s[64 * h + 2 * c2 + 1]), sl2, nm2);
+            const float2 e = (c2 % kFmaExpEvery == kFmaExpEvery - 1) ? exp2_fma2(x)
+                                                                  : make_float2(exp2_approx(x.x), exp2_approx(x.y));
             __nv_bfloat162 hb = __floats2bfloat162_rn(e.x, e.y);
             pk[c2] = *reinterpret_cast<uint32_t*>(&hb);
             rs2[c2 & 3] = fadd2(rs2[c2 & 3], make_float2(bf16_lo(pk[c2]), bf16_hi(pk[c2])));
         }
-        tmem_st32(taddr, pk);
-    };
-    exp_half(s, s_addr + 96);
-    tmem_ld64(s_addr, s);
-    exp_half(s, s_addr + 64);
+        tmem_st32(s_addr + 64 + 32 * h, pk);
+    }
     const float rs = ((rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y)) + ((rs2[2].x + rs2[2].y) + (rs2[3].x + rs2[3].y));
     l_sum = l_sum * corr + rs;
     m_ref = m_use;
     return corr;
-}
-
-// A masked tile (diagonal, first prior tile, streaming tiles): this row's
-// invisible scores are overwritten with -inf in TMEM, so the softmax itself
-// never tests a mask and keeps no mask state across its loop.  Costs one more
-// TMEM round trip on the few masked tiles of a query tile; a streaming tile
-// is 6x cheaper than with a per-score position test.
-__device__ __forceinline__ void mask_tile_in_tmem(const LayerArgs& a, const Sched& sc, const Tile& t, int P,
-                                               uint32_t s_addr) {
-    uint32_t vis[4] = {0u, 0u, 0u, 0u};   // the tile's keys this row sees, a bit per column
-    visible_columns(a, sc, t, P, vis);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        float v[64];
-        tmem_ld64(s_addr + 64 * h, v);
-        uint32_t r[32];
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const int col = 64 * h + 32 * half + c;
-                r[c] = ((vis[col >> 5] >> (col & 31)) & 1u) ? __float_as_uint(v[32 * half + c])
-                                                            : __float_as_uint(-INFINITY);
-            }
-            tmem_st32(s_addr + 64 * h + 32 * half, r);
-        }
-    }
-    tmem_wait_st();
 }
 
 // ------------------------------------------------------------------ kernel
@@ -336,7 +346,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------- work item
     const int per_m_ret = a.B * a.R * a.G, per_m_str = a.B * a.S * a.G;
     const bool retrieval = (int)blockIdx.x < p.n_ret_ctas;
-    int idx = retrieval ? (int)blockIdx.x : (int)blockIdx.x - p.n_ret_ctas;
+    const int unit = retrieval ? (int)blockIdx.x / p.ns : 0;
+    const int split = retrieval ? (int)blockIdx.x % p.ns : 0;
+    int idx = retrieval ? unit : (int)blockIdx.x - p.n_ret_ctas;
     const int per_m = retrieval ? per_m_ret : per_m_str;
     const int m = p.n_mpairs - 1 - idx / per_m;        // heaviest query tiles first
     idx %= per_m;
@@ -353,6 +365,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         c0 = a.capacity;
     }
     const Sched sc = make_sched(p, retrieval, c0, m);
+    // Key-range split of a retrieval unit: split `split` of ns_use takes the
+    // unit's tiles [j0, j1); units too short to split run whole, and the CTAs
+    // of splits they do not use leave before any set-up.
+    int ns_use = 1, j0 = 0, j1 = sc.n;
+    if (retrieval && p.ns > 1) {
+        ns_use = min(p.ns, max(1, sc.n / kMinSplitTiles));
+        if (split >= ns_use) return;
+        j0 = split * sc.n / ns_use;
+        j1 = (split + 1) * sc.n / ns_use;
+    }
+    const int nl = j1 - j0;                           // tiles of this CTA for Q1
+    const int nl0 = max(0, min(j1, sc.n0) - j0);      // ... and for Q0
 
     // ------------------------------------------------------- set-up
     if (warp == kMmaWarp) tmem_alloc(holder, kTmemCols);
@@ -384,8 +408,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_4d(sQ + qi * kQBytes + half * (kQBytes / 2), &tmQ, 64 * half, q_idx, BM * (2 * m + qi),
                                 b, q_full);
             const int cache_z = b * a.R + slot, ring_z = b * a.S + (slot - a.R);
-            for (int j = 0; j < sc.n; ++j) {
-                const Tile t = tile_at(sc, j);
+            for (int j = 0; j < nl; ++j) {
+                const Tile t = tile_at(sc, j0 + j);
                 const int st = j & 1;
                 for (int kv = 0; kv < 2; ++kv) {
                     uint64_t* full = kv ? &v_full[st] : &k_full[st];
@@ -413,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(BM, BN, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16(BM, HD, 0, 1);
-            const int n = sc.n, n0 = sc.n0;
+            const int n = nl, n0 = nl0;
             bool ok = mbar_wait(q_full, 0, p.status);
             // S_qi = Q_qi K_j^T: 8 MMAs of K 16 over the two 64-column halves of d
             auto issue_qk = [&](int qi, int j) {
@@ -469,13 +493,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-    } else {
+    } else if (warp < kTmaWarp) {
         // --------------------------------------------------- softmax
         const int qi = warp >> 2;                             // query tile of this warpgroup
         const int row = tid & 127;                            // TMEM lane
         const int crow = BM * (2 * m + qi) + row;             // chunk row
         const int P = c0 + crow;                              // absolute query position
-        const int n_me = qi ? sc.n : sc.n0;
+        const int n_me = qi ? nl : nl0;
         const float sl = a.scale * kLog2e;
         const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         float m_ref = -INFINITY, l_sum = 0.f;
@@ -484,10 +508,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = __all_sync(0xffffffffu, mbar_wait(&s_full[qi], j & 1, p.status));
             if (!ok) break;
             tc_fence_after();
-            const Tile t = tile_at(sc, j);
-            if (needs_mask(sc, t, qi)) mask_tile_in_tmem(a, sc, t, P, lane_base + col_s(qi));
+            const Tile t = tile_at(sc, j0 + j);
+            const bool masked = needs_mask(sc, t, qi);
+            uint32_t vis[4] = {0u, 0u, 0u, 0u};   // the tile's keys this row sees, a bit per column
+            if (masked) visible_columns(a, sc, t, P, vis);
             bool need;
-            const float corr = softmax_tile(lane_base + col_s(qi), sl, m_ref, l_sum, need);
+            const float corr = softmax_tile(lane_base + col_s(qi), sl, masked, vis, m_ref, l_sum, need);
             // O_qi holds every PV up to tile j - 1 (the commit behind s_full
             // covered them); rescale it before PV_qi(j) is issued
             if (j >= 1 && __any_sync(0xffffffffu, need)) {
@@ -507,23 +533,92 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // epilogue: O / l -> bf16
         if (ok && n_me >= 1) ok = __all_sync(0xffffffffu, mbar_wait(&o_done[qi], 0, p.status));
-        if (ok && n_me >= 1) {
-            tc_fence_after();
-            const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-            __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.out) + (((size_t)b * p.C + crow) * a.Hq + q_idx) * HD;
+        __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.out) + (((size_t)b * p.C + crow) * a.Hq + q_idx) * HD;
+        if (ns_use == 1) {
+            if (ok && n_me >= 1) {
+                tc_fence_after();
+                const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    float o[32];
+                    tmem_ld32(lane_base + col_o(qi) + 32 * ch, o);
+                    if (crow < p.C) {
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            float v8[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) v8[e] = o[8 * q4 + e] * inv;
+                            store_row<__nv_bfloat16, 8>(op + 32 * ch + 8 * q4, v8);
+                        }
+                    }
+                }
+            }
+        } else {
+            // (1) this split's record of the query tile: m, l and O unnormalised
+            const bool have = ok && n_me >= 1;               // warp-uniform
+            float* rec = p.part + (((size_t)unit * p.ns + split) * 2 + qi) * kPartFloats;
+            if (have) tc_fence_after();
+            rec[row] = have ? m_ref : -INFINITY;
+            rec[BM + row] = have ? l_sum : 0.f;
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
                 float o[32];
-                tmem_ld32(lane_base + col_o(qi) + 32 * ch, o);
-                if (crow < p.C) {
+                if (have) {
+                    tmem_ld32(lane_base + col_o(qi) + 32 * ch, o);
+                } else {
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        float v8[8];
+                    for (int e = 0; e < 32; ++e) o[e] = 0.f;
+                }
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) v8[e] = o[8 * q4 + e] * inv;
-                        store_row<__nv_bfloat16, 8>(op + 32 * ch + 8 * q4, v8);
+                for (int g4 = 0; g4 < 8; ++g4)
+                    reinterpret_cast<float4*>(rec + 2 * BM)[(8 * ch + g4) * BM + row] =
+                        make_float4(o[4 * g4], o[4 * g4 + 1], o[4 * g4 + 2], o[4 * g4 + 3]);
+            }
+            // (2) a ticket per unit, taken once the 256 softmax threads have
+            // written; the CTA that arrives last merges (no CTA ever waits)
+            __threadfence();
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            if (tid == 0) holder[1] = (atomicAdd(&p.ticket[unit], 1u) == (unsigned)ns_use - 1) ? 1u : 0u;
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            if (holder[1]) {
+                __threadfence();
+                const float* base = p.part + (size_t)unit * p.ns * 2 * kPartFloats + (size_t)qi * kPartFloats;
+                constexpr size_t kSplitStride = 2 * (size_t)kPartFloats;
+                float w[kMaxSplit];
+                float M = -INFINITY, L = 0.f;
+#pragma unroll
+                for (int sp = 0; sp < kMaxSplit; ++sp)
+                    if (sp < ns_use) M = fmaxf(M, __ldcg(base + sp * kSplitStride + row));
+#pragma unroll
+                for (int sp = 0; sp < kMaxSplit; ++sp) {
+                    w[sp] = 0.f;
+                    if (sp < ns_use) {
+                        const float ms = __ldcg(base + sp * kSplitStride + row);
+                        w[sp] = ms == -INFINITY ? 0.f : exp2f(ms - M);
+                        L += w[sp] * __ldcg(base + sp * kSplitStride + BM + row);
                     }
                 }
+                const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll 1
+                for (int g8 = 0; g8 < HD / 8; ++g8) {
+                    float v8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int sp = 0; sp < kMaxSplit; ++sp) {
+                        if (sp < ns_use) {
+                            const float4* o4 = reinterpret_cast<const float4*>(base + sp * kSplitStride + 2 * BM);
+                            const float4 x0 = __ldcg(o4 + (2 * g8) * BM + row);
+                            const float4 x1 = __ldcg(o4 + (2 * g8 + 1) * BM + row);
+                            v8[0] += w[sp] * x0.x; v8[1] += w[sp] * x0.y; v8[2] += w[sp] * x0.z; v8[3] += w[sp] * x0.w;
+                            v8[4] += w[sp] * x1.x; v8[5] += w[sp] * x1.y; v8[6] += w[sp] * x1.z; v8[7] += w[sp] * x1.w;
+                        }
+                    }
+                    if (crow < p.C) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) v8[e] *= inv;
+                        store_row<__nv_bfloat16, 8>(op + 8 * g8, v8);
+                    }
+                }
+                if (tid == 0) p.ticket[unit] = 0u;   // ready for the next launch
             }
         }
     }
@@ -541,8 +636,64 @@ bool prefill_tc_supported(const LayerArgs& a) {
     return a.dtype == DUO_BF16 && a.D == HD && a.page_size == 0 && a.sink <= BN && a.W <= kMaxRing;
 }
 
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+        return 148;
+    return n;
+}
+
+// Key-range splits per retrieval unit for a chunk of C queries.  One CTA fills
+// an SM, so n_units CTAs run in ceil(n_units / n_sms) waves and the last one
+// may leave SMs idle (256 units on 148 SMs: 1.73 waves, 13.5 % of SM time).
+// Splitting every unit's key tiles ns ways makes n_units * ns CTAs of about
+// equal work: take the smallest ns whose waves are at least 95 % full (else
+// the fullest).  The device then uses fewer splits for units shorter than
+// kMinSplitTiles tiles per split (early chunks of a prompt).
+PrefillPlan prefill_plan(const LayerArgs& a, int C, int n_sms) {
+    PrefillPlan pl{};
+    pl.ns = 1;
+    const long units = (long)a.B * a.R * a.G * ((C + 2 * BM - 1) / (2 * BM));
+    if (units > 0 && n_sms > 0) {
+        double best = 0.0;
+        for (int ns = 1; ns <= kMaxSplit; ++ns) {
+            const long items = units * ns;
+            const long waves = (items + n_sms - 1) / n_sms;
+            const double fill = (double)items / ((double)waves * n_sms);
+            if (fill > best + 1e-9) {
+                best = fill;
+                pl.ns = ns;
+            }
+            if (fill >= 0.95) break;
+        }
+    }
+    if (pl.ns > 1) {
+        const size_t part = (size_t)units * pl.ns * 2 * kPartFloats * sizeof(float);
+        pl.ticket_offset = (part + 255) / 256 * 256;
+        pl.bytes = pl.ticket_offset + ((size_t)units * sizeof(uint32_t) + 255) / 256 * 256;
+    } else {
+        pl.ticket_offset = 0;
+        pl.bytes = 256;
+    }
+    return pl;
+}
+
+size_t prefill_workspace_bytes(const LayerArgs& a, int max_chunk) {
+    // the plan depends on the number of 256-query tile pairs; a workspace
+    // sized here serves every chunk length up to max_chunk
+    const int n_sms = sm_count();
+    size_t bytes = 256;
+    for (int mp = 1; mp <= (max_chunk + 2 * BM - 1) / (2 * BM); ++mp) {
+        const size_t b = prefill_plan(a, mp * 2 * BM, n_sms).bytes;
+        if (b > bytes) bytes = b;
+    }
+    return bytes;
+}
+
 cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void* q, const void* k_chunk,
-                              const void* v_chunk, int C, void* out, cudaStream_t s) {
+                              const void* v_chunk, int C, void* out, void* workspace, size_t ws_bytes,
+                              cudaStream_t s) {
     if (!prefill_tc_supported(a)) return cudaErrorNotSupported;
     const uint64_t row = HD * 2;
     CUtensorMap mQ, mKx, mVx, mKc, mVc, mKr, mVr;
@@ -582,11 +733,17 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
     p.a = a;
     p.C = C;
     p.n_mpairs = (C + 2 * BM - 1) / (2 * BM);
-    p.n_ret_ctas = a.B * a.R * a.G * p.n_mpairs;
+    p.n_units = a.B * a.R * a.G * p.n_mpairs;
+    const PrefillPlan plan = prefill_plan(a, C, sm_count());
+    const bool split = plan.ns > 1 && workspace != nullptr && ws_bytes >= plan.bytes;
+    p.ns = split ? plan.ns : 1;
+    p.part = split ? static_cast<float*>(workspace) : nullptr;
+    p.ticket = split ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + plan.ticket_offset) : nullptr;
+    p.n_ret_ctas = p.n_units * p.ns;
     p.seq_len = c.seq_len;
     p.status = c.status;
     p.out = out;
-    const long grid = (long)a.B * a.Hkv * a.G * p.n_mpairs;
+    const long grid = (long)p.n_ret_ctas + (long)a.B * a.S * a.G * p.n_mpairs;
     if (grid == 0) return cudaSuccess;
     if (grid > 0x7fffffffL) return cudaErrorInvalidConfiguration;
     static bool configured = false;  // function attributes are per process, set once
@@ -597,6 +754,28 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
         configured = true;
     }
     prefill_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes + 1024, s>>>(mQ, mKc, mVc, mKx, mVx, mKr, mVr, p);
+    return cudaGetLastError();
+}
+
+namespace {
+
+__global__ void exp2_fma_probe_kernel(const float* x, float* y, int64_t n) {
+    for (int64_t i = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x); i < n;
+         i += 2 * (int64_t)gridDim.x * blockDim.x) {
+        const float x1 = i + 1 < n ? x[i + 1] : 0.f;
+        const float2 e = exp2_fma2(make_float2(x[i], x1));
+        y[i] = e.x;
+        if (i + 1 < n) y[i + 1] = e.y;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_exp2_fma_probe(const float* x, float* y, int64_t n, cudaStream_t s) {
+    if (n <= 0) return cudaSuccess;
+    const int64_t pairs = (n + 1) / 2;
+    const int grid = (int)(pairs < 148 * 8 * 256 ? (pairs + 255) / 256 : 148 * 8);
+    exp2_fma_probe_kernel<<<grid, 256, 0, s>>>(x, y, n);
     return cudaGetLastError();
 }
 

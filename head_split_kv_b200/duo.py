@@ -91,6 +91,7 @@ _lib_mix_grad = _fn("duo_gated_mix_grad_alpha", ctypes.c_int, _DESC, _P, _P, _P,
 _lib_check = _fn("duo_check_status", ctypes.c_int, _STATE, ctypes.POINTER(_I32), _P)
 _lib_decode_step = _fn("duo_decode_step", ctypes.c_int, _DESC, _STATE, _P, _P, _P, _P, _P, ctypes.c_size_t, _P)
 _lib_decode_noalloc = _fn("duo_decode_attn_noalloc", ctypes.c_int, _DESC, _STATE, _P, _P, _P)
+_lib_exp2_probe = _fn("duo_exp2_fma_probe", ctypes.c_int, _P, _P, ctypes.c_int64, _P)
 NOALLOC_SCRATCH_BYTES = 2 << 20
 
 
@@ -225,6 +226,11 @@ def gated_mix(desc, alpha, q, k, v, N: int, out, stream=None) -> None:
 def gated_mix_grad_alpha(desc, q, k, v, N: int, dout, dalpha, stream=None) -> None:
     _check(_lib_mix_grad(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), N, _ptr(dout), _ptr(dalpha),
                          _stream(stream)), "duo_gated_mix_grad_alpha")
+
+
+def exp2_fma_probe(x, y, n: int, stream=None) -> None:
+    """y[:n] = the pre-fill softmax's FMA-pipe 2^x of x[:n] (fp32 device buffers)."""
+    _check(_lib_exp2_probe(_ptr(x), _ptr(y), n, _stream(stream)), "duo_exp2_fma_probe")
 
 
 def check_status(state: KVState, stream=None, raise_on_error: bool = False) -> int:

@@ -326,7 +326,14 @@ duo_status duo_decode_step(const duo_layer_desc* desc, const duo_kv_state* st, c
  *     chunk of a prompt is then causal for every head.
  * bf16 with d = 128 runs on the tcgen05 tensor cores (TMA-fed tiles, TMEM
  * accumulators); fp32 and d = 64 run on the CUDA cores.
- * workspace: >= duo_workspace_bytes(desc, DUO_OP_PREFILL, C) bytes (may be 0).
+ * workspace: duo_workspace_bytes(desc, DUO_OP_PREFILL, C) bytes, zero-filled
+ *   once before its first use (every call leaves its ticket words at zero),
+ *   or NULL / smaller.  With it, the bf16 path splits the key tiles of long
+ *   retrieval query tiles across several CTAs so that the chunk's CTAs fill
+ *   whole waves of SMs; the splits' partial (max, sum, unnormalised output)
+ *   rows go to the workspace and the split that finishes last merges them.
+ *   Without it the kernel runs unsplit (same results up to rounding).
+ *   Concurrent calls must not share a workspace.
  * The full cache must be contiguous (page_size 0) and not 8-bit here
  * (DUO_ERR_UNSUPPORTED): the pre-fill reads its prior tiles in bf16.
  * Errors: DUO_ERR_INVALID_ARG, DUO_ERR_SHAPE, DUO_ERR_CAPACITY,
@@ -403,6 +410,21 @@ duo_status duo_decode_attn_noalloc(const duo_layer_desc* desc, const duo_kv_stat
  */
 duo_status duo_gated_mix_grad_alpha(const duo_layer_desc* desc, const void* q, const void* k, const void* v,
                                     int32_t N, const void* dout, float* dalpha, duo_stream_t stream);
+
+/*
+ * duo_exp2_fma_probe -- y[i] = the pre-fill softmax's FMA-pipe 2^x of x[i]
+ * (Cody-Waite range reduction to x = n + f, f in [-0.5, 0.5], a fitted cubic
+ * for 2^f and n added to the exponent field; inputs below -125, -inf
+ * included, give the value at -125, 2^-125 within the cubic's 7.5e-5).  duo_prefill_chunk computes one exponential pair in
+ * eight this way and the rest on the SFU; this entry point exposes the
+ * routine so that its error can be checked against 2^x.  It is not a step of
+ * the attention path: the paper review's S3 "Core formula" only fixes the
+ * softmax, not how its exponentials are evaluated.
+ * x, y: n fp32 values in device memory (caller-owned; may alias).  n >= 0.
+ * Asynchronous on `stream`.
+ * Errors: DUO_ERR_INVALID_ARG (NULL with n > 0, n < 0), DUO_ERR_CUDA.
+ */
+duo_status duo_exp2_fma_probe(const float* x, float* y, int64_t n, duo_stream_t stream);
 
 /*
  * duo_check_status -- synchronise `stream`, copy the state's device status

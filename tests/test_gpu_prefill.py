@@ -23,12 +23,14 @@ def _cuda():
 
 
 def _run(duo, sh, retrieval, n, chunks, B=1, seed=0, sample_rows=None, check_cache=True, sigma=None,
-         stream_mode="lambda"):
+         stream_mode="lambda", workspace=True):
     """Pre-fill n tokens in the given chunk lengths; compare every output row
-    (or `sample_rows` seeded rows per chunk) with the oracle."""
+    (or `sample_rows` seeded rows per chunk) with the oracle.  With a
+    workspace, long retrieval units split their key tiles across CTAs."""
     t = torch()
     lay = Layer(duo, sh, retrieval, B, capacity=n + 16,
                 stream_prefill=duo.STREAM_CHUNK if stream_mode == "chunk" else duo.STREAM_LAMBDA)
+    ws = duo.Workspace(lay.desc, duo.OP_PREFILL, max(chunks)) if workspace else None
     q, k, v = S.prompt(sh, n, seed=seed, batch=B, sigma=sigma)
     c0 = 0
     rng = S.rng_for(seed, 77)
@@ -39,7 +41,7 @@ def _run(duo, sh, retrieval, n, chunks, B=1, seed=0, sample_rows=None, check_cac
         kd = to_dev(np.ascontiguousarray(k[:, c0:c1]))
         vd = to_dev(np.ascontiguousarray(v[:, c0:c1]))
         out = t.empty_like(qd)
-        duo.prefill_chunk(lay.desc, lay.caches.state, qd, kd, vd, C, out)
+        duo.prefill_chunk(lay.desc, lay.caches.state, qd, kd, vd, C, out, ws and ws.ptr, ws.nbytes if ws else 0)
         duo.append_kv(lay.desc, lay.caches.state, kd, vd, C)
         lay.oracle.append(k[:, c0:c1], v[:, c0:c1])
         got = f64(out)
@@ -82,16 +84,17 @@ def _history(sh, st, b, L, k_new, v_new):
     return k_all, v_all
 
 
-@pytest.mark.parametrize("chunk", [1000, 256])
-def test_prefill_tc_uneven_batch(duo, chunk):
-    """Sequences of one batch at different lengths (0, 1100, 2300 tokens
-    cached) take one chunk together: each sequence's query tiles see their
-    own prior tiles, the first of them partly before position 0 when the
-    length is not a multiple of the tile."""
+@pytest.mark.parametrize("chunk,lengths", [(1000, [0, 1100, 2300]), (256, [0, 1100, 2300]),
+                                          (4096, [0, 5000, 9001])])
+def test_prefill_tc_uneven_batch(duo, chunk, lengths):
+    """Sequences of one batch at different lengths take one chunk together:
+    each sequence's query tiles see their own prior tiles, the first of them
+    partly before position 0 when the length is not a multiple of the tile.
+    With 4,096-token chunks the three sequences split their key tiles 2, 4
+    and 4 ways in the same launch."""
     t = torch()
     sh = S.LayerShape(16, 4, 128, "bf16")
     retrieval = [0, 3]
-    lengths = [0, 1100, 2300]
     B = len(lengths)
     lay = Layer(duo, sh, retrieval, B, capacity=max(lengths) + chunk + 16)
     st = S.decode_state(sh, retrieval, lengths, seed=5)
@@ -101,10 +104,13 @@ def test_prefill_tc_uneven_batch(duo, chunk):
     want = [O.prefill_direct(q[b], *_history(sh, st, b, L, k[b], v[b]), L, np.array(lay.gate), sh.sink, sh.recent,
                              rows=rows) for b, L in enumerate(lengths)]
     out = t.empty((B, chunk, sh.n_q_heads, sh.head_dim), dtype=t.bfloat16, device="cuda")
-    duo.prefill_chunk(lay.desc, lay.caches.state, to_dev(q), to_dev(k), to_dev(v), chunk, out)
-    got = f64(out)
-    for b, L in enumerate(lengths):
-        assert_close(got[b, rows], want[b], "bf16", f"b={b} (cached {L})")
+    ws = duo.Workspace(lay.desc, duo.OP_PREFILL, chunk)
+    for call in range(2):   # the second call reuses the workspace the first left
+        out.zero_()
+        duo.prefill_chunk(lay.desc, lay.caches.state, to_dev(q), to_dev(k), to_dev(v), chunk, out, ws.ptr, ws.nbytes)
+        got = f64(out)
+        for b, L in enumerate(lengths):
+            assert_close(got[b, rows], want[b], "bf16", f"call {call} b={b} (cached {L})")
     assert lay.status() == 0
 
 
@@ -138,10 +144,20 @@ def test_prefill_tc_all_retrieval_and_all_streaming(duo):
     _run(duo, sh, [], 500, [200, 300])
 
 
-def test_prefill_tc_long_prefix(duo):
-    # a 20K-token history, then a 4096 chunk: many prior tiles per query tile
+@pytest.mark.parametrize("workspace", [True, False])
+def test_prefill_tc_long_prefix(duo, workspace):
+    # a 20K-token history, then a 4096 chunk: many prior tiles per query tile,
+    # split 4 ways across CTAs with a workspace, whole without
     sh = S.LayerShape(32, 8, 128, "bf16")
-    _run(duo, sh, S.retrieval_heads_by_seed(8, 4), 24576, [20480, 4096], sample_rows=96, check_cache=False)
+    _run(duo, sh, S.retrieval_heads_by_seed(8, 4), 24576, [20480, 4096], sample_rows=96, check_cache=False,
+         workspace=workspace)
+
+
+def test_prefill_tc_mha_eight_way_split(duo):
+    # MHA with 8 retrieval heads: 128 retrieval units per 4,096 chunk, each
+    # split 8 ways over a 16K history
+    sh = S.LayerShape(32, 32, 128, "bf16")
+    _run(duo, sh, S.retrieval_heads_by_seed(32, 8), 20480, [16384, 4096], sample_rows=64, check_cache=False)
 
 
 @pytest.mark.slow
@@ -150,3 +166,27 @@ def test_prefill_gqa_131k_full(duo):
     sampled rows in every chunk; caches compared at the end."""
     sh = S.LayerShape(32, 8, 128, "bf16")
     _run(duo, sh, S.retrieval_heads_by_seed(8, 4), 131072, [4096] * 32, sample_rows=24)
+
+
+def test_exp2_fma_probe_error_bound(duo):
+    """The FMA-pipe exponential that the pre-fill softmax uses for one pair in
+    eight, against 2^x in float64 over the range the softmax feeds it
+    (x <= 8: the lazily raised row maximum lags the true one by at most 2^8):
+    relative error below 1e-4, far inside the 2^-9 half-step of the bf16
+    probabilities it produces; inputs below -125 (masked keys: -inf) give the
+    value at -125.  An odd count exercises the unpaired last element."""
+    t = torch()
+    rng = np.random.default_rng(5)
+    x = np.concatenate([np.linspace(-125.0, 8.0, 266001), rng.uniform(-125.0, 8.0, 100000),
+                        [-0.5, 0.5, -1.5, 0.0, 8.0, -125.0, -125.5, -126.0, -1000.0, -np.inf]]).astype(np.float32)
+    assert x.size % 2 == 1
+    xd = t.from_numpy(x).cuda()
+    yd = t.full_like(xd, float("nan"))
+    duo.exp2_fma_probe(xd, yd, x.size)
+    y = yd.cpu().numpy().astype(np.float64)
+    inside = x >= -125.0
+    rel = np.abs(y[inside] / np.exp2(x[inside].astype(np.float64)) - 1.0)
+    assert rel.max() < 1e-4, f"max relative error {rel.max():.3e} at x = {x[inside][rel.argmax()]}"
+    # below the clamp every input gives the value at -125: 2^-125 within the same bound
+    assert np.all(y[~inside] == y[x == -125.0][0])
+    assert abs(y[~inside][0] / 2.0 ** -125 - 1.0) < 1e-4
