@@ -496,17 +496,24 @@ def _decode_e2e(duo, env, layers, args, world):
     nl = len(layers)
     n = min(args.steps, 32)
 
-    def pinned(a):
-        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
+    # a step's q, k and v sit back to back in one pinned buffer, so each layer
+    # takes one host->device copy; the views passed to the library start at
+    # 16-byte multiples (each part is a whole number of d-element rows)
+    q_shape, kv_shape = env["qs"][0].shape, env["ks"][0][:, None].shape
+    nq, nk = int(np.prod(q_shape)), int(np.prod(kv_shape))
 
-    h_q = [pinned(env["qs"][i]) for i in range(n)]
-    h_k = [pinned(env["ks"][i][:, None]) for i in range(n)]
-    h_v = [pinned(env["vs"][i][:, None]) for i in range(n)]
-    h_out = [torch.empty_like(h_q[0]).pin_memory() for _ in range(nl)]
-    dq = [torch.empty_like(h_q[0], device="cuda") for _ in range(nl)]
-    dk = [torch.empty_like(h_k[0], device="cuda") for _ in range(nl)]
-    dv = [torch.empty_like(h_v[0], device="cuda") for _ in range(nl)]
-    dout = [torch.empty_like(dq[0]) for _ in range(nl)]
+    def pinned(i):
+        flat = np.concatenate([np.ascontiguousarray(a).reshape(-1) for a in
+                               (env["qs"][i], env["ks"][i], env["vs"][i])])
+        return torch.from_numpy(flat.view(np.int16)).view(torch.bfloat16).pin_memory()
+
+    h_in = [pinned(i) for i in range(n)]
+    h_out = [torch.empty(q_shape, dtype=torch.bfloat16).pin_memory() for _ in range(nl)]
+    d_in = [torch.empty_like(h_in[0], device="cuda") for _ in range(nl)]
+    dq = [x[:nq].view(q_shape) for x in d_in]
+    dk = [x[nq:nq + nk].view(kv_shape) for x in d_in]
+    dv = [x[nq + nk:].view(kv_shape) for x in d_in]
+    dout = [torch.empty(q_shape, dtype=torch.bfloat16, device="cuda") for _ in range(nl)]
     stream = torch.cuda.current_stream()
     sp = int(stream.cuda_stream)
     times = []
@@ -516,9 +523,7 @@ def _decode_e2e(duo, env, layers, args, world):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for l, (caches, ws) in enumerate(layers):
-            dq[l].copy_(h_q[i], non_blocking=True)
-            dk[l].copy_(h_k[i], non_blocking=True)
-            dv[l].copy_(h_v[i], non_blocking=True)
+            d_in[l].copy_(h_in[i], non_blocking=True)
             duo.decode_step(desc, caches.state, dq[l], dk[l], dv[l], dout[l], ws.ptr, ws.nbytes, sp)
             h_out[l].copy_(dout[l], non_blocking=True)
         e1.record(stream)
@@ -526,7 +531,7 @@ def _decode_e2e(duo, env, layers, args, world):
     torch.cuda.synchronize()
     _barrier(world)
     tot = _max_over_ranks(sum(a.elapsed_time(b) for a, b in times), world)
-    h2d = (h_q[0].numel() + h_k[0].numel() + h_v[0].numel()) * 2
+    h2d = h_in[0].numel() * 2
     return {"value": round(tot * 1e3 / (n * nl * world), 3), "unit": "us/step/layer", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": h_out[0].numel() * 2, "steps": n, "note": "bytes per layer and step"}
 

@@ -232,17 +232,23 @@ __device__ __forceinline__ void decode_finish(float* sM, uint64_t* comb_bar, int
         }
     }
     __syncthreads();
-    if (threadIdx.x < G) {
-        const int g = threadIdx.x;
+    // one warp per query head of the group, a lane per split (and per split
+    // + 32, ...): the maximum and the sum are warp reductions, so the weights
+    // take a few steps instead of ns serial exponentials
+    for (int g = warp; g < G; g += kThreads / 32) {
         float M = kNegBig;
-        for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, s_w[sp * G + g]);
+        for (int sp = lane; sp < ns; sp += 32) M = fmaxf(M, s_w[sp * G + g]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
         float L = 0.f;
-        for (int sp = 0; sp < ns; ++sp) {
+        for (int sp = lane; sp < ns; sp += 32) {
             const float w = exp2f(s_w[sp * G + g] - M);
             s_w[sp * G + g] = w;
             L += w * s_l[sp * G + g];
         }
-        s_inv[g] = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        if (lane == 0) s_inv[g] = L > 0.f ? 1.f / L : 0.f;
     }
     __syncthreads();
     constexpr int kOut = (G * D + kThreads - 1) / kThreads;  // outputs per thread
