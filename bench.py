@@ -122,7 +122,7 @@ class ClockSampler:
     """SM clock and clock-event (throttle) reasons of this process's GPU,
     sampled while the timed region runs, from a separate process so that the
     launching thread's hold on the interpreter cannot starve the sampling.
-    Through NVML every 10 ms when the bindings load (the CUDA device is
+    Through NVML every 2 ms when the bindings load (the CUDA device is
     matched to its NVML handle by PCI bus id, so CUDA_VISIBLE_DEVICES cannot
     point it at another GPU), else through `nvidia-smi -lms 200`.  Only
     reads; nothing about the GPU is changed."""
@@ -134,7 +134,7 @@ class ClockSampler:
     # NVML clock-event reason bits
     BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40}
 
-    def __init__(self, gpu_index: int, period_s: float = 0.01):
+    def __init__(self, gpu_index: int, period_s: float = 0.002):
         self.gpu = gpu_index
         self.period = period_s
         self.proc = None
@@ -159,7 +159,7 @@ class ClockSampler:
     def __enter__(self):
         try:
             if self._start_nvml():
-                self.mode = "nvml 10 ms"
+                self.mode = f"nvml {self.period * 1e3:g} ms"
         except Exception:
             self.proc = None
         if self.proc is None:
@@ -181,18 +181,19 @@ class ClockSampler:
 
     def __exit__(self, *exc):
         if self.proc:
-            if self.mode != "nvml 10 ms":
+            if not self.mode.startswith("nvml"):
                 time.sleep(0.25)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+            self.t.join(timeout=5)   # lines still in the pipe belong to the timed region
 
     def summary(self):
         mhz, mx, reasons = [], self.max_mhz, set()
         for ln in list(self.lines):
-            if self.mode == "nvml 10 ms":
+            if self.mode.startswith("nvml"):
                 parts = ln.split()
                 if len(parts) != 2:
                     continue

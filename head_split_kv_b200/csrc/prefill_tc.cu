@@ -6,7 +6,7 @@
 //  full (FlashAttention-style) causal attention; streaming heads run in linear
 //  time and constant memory.]
 //
-// One CTA (one per SM: 193 KB of shared memory, all 512 TMEM columns) owns
+// One CTA (one per SM: 198 KB of shared memory, all 512 TMEM columns) owns
 // 256 query rows of one query head, as two 128-row tiles Q0 (chunk rows
 // 256m .. 256m+127) and Q1 (256m+128 .. 256m+255), and walks 128-key tiles:
 //   retrieval head: every prior key from the full cache (tiles aligned to end
@@ -35,6 +35,11 @@
 // (only when the maximum grows by more than 2^8; the commit that signals S_i
 // also covers the previous PV_i, so O_i is complete when it is rescaled) and
 // at the end divides O by the row sum and stores bf16.
+// Key-range splits: with a workspace, a long retrieval unit (one query-tile
+// pair of one query head) is taken by ns CTAs, each over 1/ns of its key
+// tiles, so that the chunk's CTAs fill whole waves of SMs; each writes its
+// rows' (m, l, O) to the workspace and the CTA that takes the unit's last
+// ticket merges them (prefill_plan picks ns on the host).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -55,7 +60,7 @@ __device__ __forceinline__ constexpr uint32_t col_s(int i) { return 128u * (uint
 __device__ __forceinline__ constexpr uint32_t col_o(int i) { return 256u + 128u * (uint32_t)i; }  // O_i
 constexpr int kMaxRing = 128;      // sink + recent held by one tile
 constexpr int kMaxSplit = 8;       // key-range splits per retrieval unit
-constexpr int kMinSplitTiles = 16; // no split shorter than 16 key tiles (2,048 keys)
+constexpr int kMinSplitTiles = 48; // no split shorter than 48 key tiles (6,144 keys)
 // One query tile's partial record of one split: the lazily raised row maxima
 // (log2 domain), the row sums, then O unnormalised as [32 column groups][128
 // rows][4], so that a warp's 32 rows write one 512-byte run per group.
@@ -230,7 +235,7 @@ __device__ __forceinline__ void visible_columns(const LayerArgs& a, const Sched&
 
 // ------------------------------------------------------------------ softmax
 
-constexpr int kFmaExpEvery = 8;   // one exp2 pair in 8 on the FMA pipe
+constexpr int kFmaExpEvery = 4;   // one exp2 pair in 4 on the FMA pipe
 
 // 2^x for a pair of x <= 0 (or -inf) on the FMA pipe, by Cody-Waite range
 // reduction and a polynomial: x = n + f with n = rint(x) (adding 1.5 * 2^23
@@ -263,13 +268,17 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
 // over the second half of S for the PV MMA (keys 0..63 to columns 64..95,
 // keys 64..127 to columns 96..127).  Returns the factor by which O must be
 // rescaled (1 unless `need`).  The row sum adds the rounded p, so each output
-// is a convex combination of V rows.
+// is a convex combination of V rows (summing the fp32 exponentials instead
+// is two integer operations a pair cheaper, but lets the weights drift from
+// summing to 1 by the bf16 rounding, which put outputs of magnitude 4..8
+// beyond the 2e-2 bound).
 //
 // The exponentials: one tile costs a softmax warp 128 exp2 per row, as many
 // cycles on the SFU as the tile's two MMAs take on the tensor core, so the
 // SFU is the co-bottleneck.  One pair in kFmaExpEvery is computed on the FMA
-// pipe instead (exp2_fma2): 2 % faster than SFU-only on the 131K prompt, and
-// faster than one pair in 4.
+// pipe instead (exp2_fma2).  Measured on the 131K prompt: one pair in 4 or
+// in 8 (equal within run-to-run noise) beat SFU-only by 2-5 %; one in 3 was
+// slower.
 __device__ __forceinline__ float softmax_tile(uint32_t s_addr, float sl, bool masked, const uint32_t (&vis)[4],
                                               float& m_ref, float& l_sum, bool& need) {
     float s[128];
@@ -344,17 +353,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* holder = reinterpret_cast<uint32_t*>(smem + kOffHolder);
 
     // ------------------------------------------------------- work item
-    const int per_m_ret = a.B * a.R * a.G, per_m_str = a.B * a.S * a.G;
     const bool retrieval = (int)blockIdx.x < p.n_ret_ctas;
-    const int unit = retrieval ? (int)blockIdx.x / p.ns : 0;
-    const int split = retrieval ? (int)blockIdx.x % p.ns : 0;
-    int idx = retrieval ? unit : (int)blockIdx.x - p.n_ret_ctas;
-    const int per_m = retrieval ? per_m_ret : per_m_str;
-    const int m = p.n_mpairs - 1 - idx / per_m;        // heaviest query tiles first
-    idx %= per_m;
-    const int g = idx % a.G;
-    const int hs = (idx / a.G) % (retrieval ? a.R : a.S);
-    const int b = idx / (a.G * (retrieval ? a.R : a.S));
+    int unit = 0, split = 0, m, g, hs, b;
+    if (retrieval) {
+        // (sequence, KV head) outermost, then the split, then the query tile
+        // pair (heaviest first) and the query head of the group: the CTAs
+        // that read one KV head's key range run side by side and share its
+        // tiles in L2
+        const int per_group = p.n_mpairs * a.G;
+        const int r = (int)blockIdx.x;
+        const int inner = r % per_group;
+        split = (r / per_group) % p.ns;
+        const int bh = r / (per_group * p.ns);
+        g = inner % a.G;
+        m = p.n_mpairs - 1 - inner / a.G;
+        hs = bh % a.R;
+        b = bh / a.R;
+        unit = (bh * p.n_mpairs + m) * a.G + g;
+    } else {
+        int idx = (int)blockIdx.x - p.n_ret_ctas;
+        const int per_m = a.B * a.S * a.G;
+        m = p.n_mpairs - 1 - idx / per_m;              // heaviest query tiles first
+        idx %= per_m;
+        g = idx % a.G;
+        hs = (idx / a.G) % a.S;
+        b = idx / (a.G * a.S);
+    }
     const int slot = retrieval ? hs : a.R + hs;
     const int q_idx = a.q_head0[slot] + g;
     const int kv_idx = a.kv_head[slot];

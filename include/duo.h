@@ -415,11 +415,12 @@ duo_status duo_gated_mix_grad_alpha(const duo_layer_desc* desc, const void* q, c
  * duo_exp2_fma_probe -- y[i] = the pre-fill softmax's FMA-pipe 2^x of x[i]
  * (Cody-Waite range reduction to x = n + f, f in [-0.5, 0.5], a fitted cubic
  * for 2^f and n added to the exponent field; inputs below -125, -inf
- * included, give the value at -125, 2^-125 within the cubic's 7.5e-5).  duo_prefill_chunk computes one exponential pair in
- * eight this way and the rest on the SFU; this entry point exposes the
- * routine so that its error can be checked against 2^x.  It is not a step of
- * the attention path: the paper review's S3 "Core formula" only fixes the
- * softmax, not how its exponentials are evaluated.
+ * included, give the value at -125, 2^-125 within the cubic's 7.5e-5).
+ * duo_prefill_chunk computes one exponential pair in four this way and the
+ * rest on the SFU; this entry point exposes the routine so that its error
+ * can be checked against 2^x.  It is not a step of the attention path: the
+ * paper review's S3 "Core formula" only fixes the softmax, not how its
+ * exponentials are evaluated.
  * x, y: n fp32 values in device memory (caller-owned; may alias).  n >= 0.
  * Asynchronous on `stream`.
  * Errors: DUO_ERR_INVALID_ARG (NULL with n > 0, n < 0), DUO_ERR_CUDA.

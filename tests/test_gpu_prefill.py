@@ -153,11 +153,20 @@ def test_prefill_tc_long_prefix(duo, workspace):
          workspace=workspace)
 
 
-def test_prefill_tc_mha_eight_way_split(duo):
-    # MHA with 8 retrieval heads: 128 retrieval units per 4,096 chunk, each
-    # split 8 ways over a 16K history
+def test_prefill_tc_mha_split(duo):
+    # MHA with 8 retrieval heads: 128 retrieval units per 4,096 chunk, planned
+    # at 8 splits; over a 16K history a unit has 160 key tiles and takes 3
+    # (no split under 48 tiles)
     sh = S.LayerShape(32, 32, 128, "bf16")
     _run(duo, sh, S.retrieval_heads_by_seed(32, 8), 20480, [16384, 4096], sample_rows=64, check_cache=False)
+
+
+def test_prefill_tc_gqa_eight_way_split(duo):
+    # GQA with 2 of 8 KV heads retrieval: 128 retrieval units per 4,096 chunk,
+    # planned at 8 splits; over a 48K history a unit has 416 key tiles and
+    # takes all 8.  The 49,152-token first chunk runs 2-way splits.
+    sh = S.LayerShape(32, 8, 128, "bf16")
+    _run(duo, sh, [2, 5], 53248, [49152, 4096], sample_rows=48, check_cache=False)
 
 
 @pytest.mark.slow
@@ -170,7 +179,7 @@ def test_prefill_gqa_131k_full(duo):
 
 def test_exp2_fma_probe_error_bound(duo):
     """The FMA-pipe exponential that the pre-fill softmax uses for one pair in
-    eight, against 2^x in float64 over the range the softmax feeds it
+    four, against 2^x in float64 over the range the softmax feeds it
     (x <= 8: the lazily raised row maximum lags the true one by at most 2^8):
     relative error below 1e-4, far inside the 2^-9 half-step of the bf16
     probabilities it produces; inputs below -125 (masked keys: -inf) give the
