@@ -64,6 +64,11 @@ WORKLOADS = {
     "gqa_prefill_128k": dict(kind="prefill", hq=32, hkv=8, d=128, n_ret=4, n=131072, chunk=4096, sigma=False),
     # the same pre-fill on a 32K prompt: a small case for profiler captures
     "gqa_prefill_32k": dict(kind="prefill", hq=32, hkv=8, d=128, n_ret=4, n=32768, chunk=4096, sigma=False),
+    # the gated mix alpha * full + (1 - alpha) * streaming over whole sequences
+    # and its gate gradient: the tiny single-layer MHA case (fp32, d 64, 512
+    # tokens, alpha ~ U(0, 1)) and a Llama-3-8B-shaped GQA layer over 4,096 tokens
+    "gated_mix_pr1": dict(kind="mix", hq=8, hkv=8, d=64, n=512, dtype="fp32", n_ret=2),
+    "gated_mix_gqa_4k": dict(kind="mix", hq=32, hkv=8, d=128, n=4096, dtype="bf16", n_ret=4),
 }
 for _name, _wl in WORKLOADS.items():
     _wl["name"] = _name
@@ -679,6 +684,104 @@ def run_prefill(args, wl, world, rank, steps=None, warmup=None):
 
 
 # ---------------------------------------------------------------------------
+# gated mix (whole sequences, no cache) and its gate gradient
+# ---------------------------------------------------------------------------
+
+# fp32 FMA pipe of the CUDA cores: 148 SMs x 128 lanes x 2 FLOP per clock at
+# the 1,965 MHz maximum SM clock
+ALU_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def _mix_flops(hq, d, n, sink, recent, B):
+    """Algorithmic FLOPs of one gated-mix forward: Q K^T once per causal pair
+    (2*d), P V for the causal softmax over the same pairs (2*d) and for the
+    Lambda softmax over its pairs (2*d), per query head."""
+    return B * hq * (4 * d * (n * (n + 1) // 2) + 2 * d * _lambda_pairs(0, n, sink, recent))
+
+
+def run_mix(args, wl, world, rank):
+    """duo_gated_mix then duo_gated_mix_grad_alpha on one batch of whole
+    sequences; a step is one forward and one gate gradient, L2 flushed (1 GiB
+    write) before each, outside the timed intervals."""
+    import torch
+    from head_split_kv_b200 import duo
+    import oracle as O
+    dt = wl["dtype"]
+    sh = S.LayerShape(wl["hq"], wl["hkv"], wl["d"], dt)
+    n, B = wl["n"], 1
+    if wl["name"] == "gated_mix_pr1":
+        w = S.tiny_prompt()
+        q, k, v, alpha = w["q"][None], w["k"][None], w["v"][None], w["alpha_mix"]
+    else:
+        q, k, v = S.prompt(sh, n, seed=0)
+        alpha = S.rng_for(0, 50).uniform(0.0, 1.0, sh.n_kv_heads).astype(np.float32)
+    dout = S.normal(S.rng_for(0, 61), q.shape, dt)
+    desc = duo.desc_init(B, sh.n_q_heads, sh.n_kv_heads, sh.head_dim, duo.BF16 if dt == "bf16" else duo.FP32,
+                         list(range(sh.n_kv_heads)), 0)
+    qd, kd, vd, dod = _to_dev(q), _to_dev(k), _to_dev(v), _to_dev(dout)
+    ad = torch.from_numpy(alpha).cuda()
+    out = torch.empty_like(qd)
+    dalpha = torch.empty((sh.n_kv_heads,), dtype=torch.float32, device="cuda")
+    flush = torch.empty(1 << 30, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    sp = int(stream.cuda_stream)
+    for _ in range(args.warmup):
+        duo.gated_mix(desc, ad, qd, kd, vd, n, out, sp)
+        duo.gated_mix_grad_alpha(desc, qd, kd, vd, n, dod, dalpha, sp)
+    steps = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    _barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(int(os.environ.get("LOCAL_RANK", "0"))) as clk:
+        for i in range(steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            duo.gated_mix(desc, ad, qd, kd, vd, n, out, sp)
+            ev[i][1].record(stream)
+            flush.zero_()
+            ev[i][2].record(stream)
+            duo.gated_mix_grad_alpha(desc, qd, kd, vd, n, dod, dalpha, sp)
+            ev[i][3].record(stream)
+        torch.cuda.synchronize()
+    _barrier(world)
+    mix_ms = sorted(e[0].elapsed_time(e[1]) for e in ev)
+    grad_ms = sorted(e[2].elapsed_time(e[3]) for e in ev)
+    mix_med = _max_over_ranks(mix_ms[len(mix_ms) // 2], world)
+    grad_med = _max_over_ranks(grad_ms[len(grad_ms) // 2], world)
+    flops = _mix_flops(sh.n_q_heads, sh.head_dim, n, sh.sink, sh.recent, B)
+    tf = flops / (mix_med * 1e-3) / 1e12
+    res = {
+        "metric": METRIC, "value": round(mix_med * 1e3, 2), "unit": "us/call", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": round(mix_med + grad_med, 4), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32" if dt == "fp32" else "bf16", "data": "synthetic",
+        "config": {"workload": wl["name"], "tokens": n, "batch": B, "n_q_heads": sh.n_q_heads,
+                   "n_kv_heads": sh.n_kv_heads, "head_dim": sh.head_dim, "sink": sh.sink, "recent": sh.recent,
+                   "alpha": "U(0, 1) per KV head", "parallelism": f"replicas{world}",
+                   "l2": "flushed (1 GiB write) before every timed call, outside the timed interval"},
+        "roofline": {"bound": "alu", "kernel": "simt_attention_kernel (gated mix)", "achieved": round(tf, 3),
+                     "peak": round(ALU_FP32_TFLOPS, 1), "peak_kind": "derived: fp32 FMA lanes x max SM clock",
+                     "unit": "TFLOP/s", "frac": round(tf / ALU_FP32_TFLOPS, 4), "traffic": None,
+                     "algorithmic_gflop": round(flops / 1e9, 3)},
+        "grad_alpha": {"value": round(grad_med * 1e3, 2), "unit": "us/call",
+                       "achieved_tflops": round(flops / (grad_med * 1e-3) / 1e12, 3)},
+        "gpu_launches": 2 * steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        # the oracle as it stands on the query heads of KV head 0, scaled to all
+        # KV heads (the heads are independent and cost the same)
+        G = sh.group
+        t0 = time.perf_counter()
+        O.gated_mix(q[0][:, :G], k[0][:, :1], v[0][:, :1], alpha[:1].astype(np.float64), sh.sink, sh.recent)
+        dt_s = (time.perf_counter() - t0) * sh.n_kv_heads
+        res["cpu_baseline"] = {"value": round(dt_s * 1e6, 1), "unit": "us/call", "cores": _blas_threads(),
+                               "kind": "oracle",
+                               "sample": f"the gated mix of KV head 0's {G} query heads (fp64 NumPy oracle), "
+                                         f"scaled by the {sh.n_kv_heads} KV heads"}
+    return res
+
+
+# ---------------------------------------------------------------------------
 # reference arm: the oracle, timed on the host cores
 # ---------------------------------------------------------------------------
 
@@ -881,6 +984,8 @@ def main(argv=None):
             res = run_ratio_sweep(args, world, rank)
         elif args.chunk_sweep:
             res = run_chunk_sweep(args, world, rank)
+        elif wl["kind"] == "mix":
+            res = run_mix(args, wl, world, rank)
         elif wl["kind"] == "decode":
             res = run_decode(args, wl, world, rank)
             if not args.no_prefill:

@@ -642,7 +642,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         store_row<__nv_bfloat16, 8>(op + 8 * g8, v8);
                     }
                 }
-                if (tid == 0) p.ticket[unit] = 0u;   // ready for the next launch
             }
         }
     }
@@ -776,6 +775,13 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
                                              (int)(kSmemBytes + 1024));
         if (e != cudaSuccess) return e;
         configured = true;
+    }
+    if (split) {
+        // the ticket words sit after this chunk length's partial records, so
+        // a call with another chunk length may find there what an earlier
+        // call's records left: clear them first
+        const cudaError_t e = cudaMemsetAsync(p.ticket, 0, (size_t)p.n_units * sizeof(uint32_t), s);
+        if (e != cudaSuccess) return e;
     }
     prefill_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes + 1024, s>>>(mQ, mKc, mVc, mKx, mVx, mKr, mVr, p);
     return cudaGetLastError();

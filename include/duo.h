@@ -326,9 +326,9 @@ duo_status duo_decode_step(const duo_layer_desc* desc, const duo_kv_state* st, c
  *     chunk of a prompt is then causal for every head.
  * bf16 with d = 128 runs on the tcgen05 tensor cores (TMA-fed tiles, TMEM
  * accumulators); fp32 and d = 64 run on the CUDA cores.
- * workspace: duo_workspace_bytes(desc, DUO_OP_PREFILL, C) bytes, zero-filled
- *   once before its first use (every call leaves its ticket words at zero),
- *   or NULL / smaller.  With it, the bf16 path splits the key tiles of long
+ * workspace: duo_workspace_bytes(desc, DUO_OP_PREFILL, C) bytes (no
+ *   initialisation needed: each call clears the ticket words it uses), or
+ *   NULL / smaller.  With it, the bf16 path splits the key tiles of long
  *   retrieval query tiles across several CTAs so that the chunk's CTAs fill
  *   whole waves of SMs; the splits' partial (max, sum, unnormalised output)
  *   rows go to the workspace and the split that finishes last merges them.
