@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const LayerArgs& a = p.a;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if ((smem_u32(smem) & 1023u) != 0) {   // the swizzled layouts need 1024-byte alignment
-        if (tid == 0) atomicOr(p.status, DUO_DEV_BAD_LENGTH);
+        if (tid == 0 && p.status) atomicOr(p.status, DUO_DEV_BAD_LENGTH);
         return;
     }
     const uint32_t sQ = smem_u32(smem + kOffQ), sK = smem_u32(smem + kOffK), sV = smem_u32(smem + kOffV);
@@ -382,10 +382,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int slot = retrieval ? hs : a.R + hs;
     const int q_idx = a.q_head0[slot] + g;
     const int kv_idx = a.kv_head[slot];
-    int c0 = p.seq_len[b];
+    int c0 = p.seq_len ? p.seq_len[b] : 0;            // no lengths: whole sequences, no cache
     if (c0 < 0) c0 = 0;
     if (retrieval && c0 > a.capacity) {
-        if (tid == 0 && m == p.n_mpairs - 1) atomicOr(p.status, DUO_DEV_BAD_LENGTH);
+        if (tid == 0 && m == p.n_mpairs - 1 && p.status) atomicOr(p.status, DUO_DEV_BAD_LENGTH);
         c0 = a.capacity;
     }
     const Sched sc = make_sched(p, retrieval, c0, m);
@@ -734,13 +734,13 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
             return cudaErrorInvalidValue;
     }
     const uint32_t bx3[3] = {64, kBox, 1};
-    if (a.R > 0) {
+    if (a.R > 0 && c.k_full != nullptr) {
         const uint64_t d[3] = {HD, (uint64_t)a.capacity, (uint64_t)a.B * a.R};
         const uint64_t st[2] = {row, row * a.capacity};
         if (!encode_tmap_bf16(&mKc, c.k_full, 3, d, st, bx3) || !encode_tmap_bf16(&mVc, c.v_full, 3, d, st, bx3))
             return cudaErrorInvalidValue;
     } else {
-        mKc = mKx;  // never read: there are no retrieval heads
+        mKc = mKx;  // never read: no retrieval heads, or no cache (c0 = 0)
         mVc = mVx;
     }
     if (a.S > 0) {

@@ -318,6 +318,25 @@ def test_gated_mix_bf16_gqa(duo, alpha_kind):
         assert_close(got[b], want, "bf16", f"mix b={b}")
 
 
+@pytest.mark.parametrize("hq,hkv,n,B", [(8, 8, 700, 1), (32, 4, 513, 2), (16, 8, 1031, 1)])
+def test_gated_mix_bf16_tensor_core_path(duo, hq, hkv, n, B):
+    """bf16, d 128: the causal half on the tensor cores, the streaming half and
+    the mix in a second pass; several 256-row query-tile pairs with a ragged
+    tail, MHA, G = 8 and G = 2, alpha ~ U(0, 1) with one gate at each end."""
+    t = torch()
+    sh = S.LayerShape(hq, hkv, 128, "bf16")
+    q, k, v = S.prompt(sh, n, seed=8, batch=B)
+    alpha = S.rng_for(8, 51).uniform(0, 1, hkv).astype(np.float32)
+    alpha[0], alpha[-1] = 1.0, 0.0
+    desc = duo.desc_init(B, hq, hkv, 128, duo.BF16, list(range(hkv)), 0)
+    out = t.empty_like(to_dev(q))
+    duo.gated_mix(desc, t.from_numpy(alpha).cuda(), to_dev(q), to_dev(k), to_dev(v), n, out)
+    got = f64(out)
+    for b in range(B):
+        want = O.gated_mix(q[b], k[b], v[b], alpha.astype(np.float64), sh.sink, sh.recent)
+        assert_close(got[b], want, "bf16", f"mix b={b}")
+
+
 # duo_gated_mix_grad_alpha: each dalpha[kv] sums dout * (full - streaming)
 # over its heads, rows and features, so its error is at most the attention
 # error bound times sum |dout| of those terms: 1e-4 for fp32; for bf16 the
