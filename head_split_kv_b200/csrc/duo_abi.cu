@@ -414,24 +414,28 @@ duo_status duo_gated_mix(const duo_layer_desc* desc, const float* alpha, const v
         a.q_head0[i] = i * a.G;
         a.slot_of[i] = i;
     }
-    if (duo::lambda_mix_supported(a)) {
-        // bf16, d 128: the causal attention of every head on the tensor cores
-        // (the pre-fill kernel over one chunk with no cache and every KV head
-        // in the retrieval block) into out, then one pass that computes the
-        // streaming attention and mixes the two in place
-        duo::LayerArgs ac = a;
-        ac.R = a.Hkv;
-        ac.S = 0;
-        ac.page_size = 0;
-        ac.capacity = 0;
-        ac.stream_chunk = 0;
-        ac.kv_int8 = 0;
-        if (duo::prefill_tc_supported(ac)) {
-            duo::CacheArgs none{};   // no lengths, no caches: every sequence starts at position 0
-            cudaError_t e = duo::launch_prefill_tc(ac, none, q, k, v, N, out, nullptr, 0, (cudaStream_t)stream);
-            if (e == cudaSuccess) e = duo::launch_lambda_mix(a, alpha, q, k, v, N, out, (cudaStream_t)stream);
-            return e == cudaSuccess ? ok() : cuda_fail(e, "duo_gated_mix");
-        }
+    // bf16, d 128: both attentions on the tensor cores, as two launches of
+    // the pre-fill kernel over one chunk with no cache -- every KV head in
+    // the streaming block (Lambda mask) writes the streaming attention to
+    // out, then every KV head in the retrieval block (causal) mixes its
+    // result with it in the epilogue
+    duo::LayerArgs as = a, ac = a;
+    as.R = 0;
+    as.S = a.Hkv;
+    ac.R = a.Hkv;
+    ac.S = 0;
+    for (duo::LayerArgs* x : {&as, &ac}) {
+        x->page_size = 0;
+        x->capacity = 0;
+        x->stream_chunk = 0;
+        x->kv_int8 = 0;
+    }
+    if (duo::prefill_tc_supported(as) && duo::prefill_tc_supported(ac)) {
+        duo::CacheArgs none{};   // no lengths, no caches: every sequence starts at position 0
+        cudaError_t e = duo::launch_prefill_tc(as, none, q, k, v, N, out, nullptr, 0, (cudaStream_t)stream);
+        if (e == cudaSuccess)
+            e = duo::launch_prefill_tc(ac, none, q, k, v, N, out, nullptr, 0, (cudaStream_t)stream, alpha);
+        return e == cudaSuccess ? ok() : cuda_fail(e, "duo_gated_mix");
     }
     const cudaError_t e = duo::launch_simt_attention(a, nullptr, alpha, q, k, v, N, out, 1, (cudaStream_t)stream);
     return e == cudaSuccess ? ok() : cuda_fail(e, "duo_gated_mix");

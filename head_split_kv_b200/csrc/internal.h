@@ -74,15 +74,13 @@ struct PrefillPlan {
 int sm_count();
 PrefillPlan prefill_plan(const LayerArgs& a, int C, int n_sms);
 size_t prefill_workspace_bytes(const LayerArgs& a, int max_chunk);
+// mix_alpha non-NULL (gated mix, no splits): out is read back as the
+// streaming attention and overwritten with alpha * result + (1 - alpha) * out.
 cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void* q, const void* k_chunk,
                               const void* v_chunk, int C, void* out, void* workspace, size_t ws_bytes,
-                              cudaStream_t s);
+                              cudaStream_t s, const float* mix_alpha = nullptr);
 cudaError_t launch_exp2_fma_probe(const float* x, float* y, int64_t n, cudaStream_t s);
-// Gated mix, second pass (bf16, d 128, G in {1, 2, 4, 8}): out holds the
-// causal attention; it becomes alpha * out + (1 - alpha) * streaming attention.
-bool lambda_mix_supported(const LayerArgs& a);
-cudaError_t launch_lambda_mix(const LayerArgs& a, const float* alpha, const void* q, const void* k, const void* v,
-                              int N, void* out, cudaStream_t s);
+
 bool prefill_tc_supported(const LayerArgs& a);
 // bf16 tensor map of `rank` dims (innermost first), 64-element-wide boxes with
 // the 128-byte swizzle, out-of-range elements read as zero; encodings are

@@ -40,6 +40,10 @@
 // tiles, so that the chunk's CTAs fill whole waves of SMs; each writes its
 // rows' (m, l, O) to the workspace and the CTA that takes the unit's last
 // ticket merges them (prefill_plan picks ns on the host).
+// Gated mix: with no length array every sequence starts at position 0 and the
+// launch covers whole sequences; given mix_alpha, the epilogue reads back the
+// streaming attention an earlier launch left in out and stores
+// alpha * (this causal attention) + (1 - alpha) * (that).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -88,7 +92,8 @@ struct TcArgs {
     int ns;                // CTAs per retrieval unit (key-range splits; 1 = none)
     int n_ret_ctas;        // n_units * ns
     float* part;           // [n_units][ns][2][kPartFloats] partial records (ns > 1)
-    uint32_t* ticket;      // [n_units] arrivals; the last split merges and resets it
+    uint32_t* ticket;      // [n_units] arrivals; the last split merges them
+    const float* mix_alpha;  // gated mix: out = alpha[kv] * this attention + (1 - alpha[kv]) * out
     const int32_t* seq_len;
     int32_t* status;
     void* out;
@@ -572,6 +577,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                             float v8[8];
 #pragma unroll
                             for (int e = 0; e < 8; ++e) v8[e] = o[8 * q4 + e] * inv;
+                            if (p.mix_alpha) {
+                                // gated mix: out already holds the streaming attention
+                                const float al = p.mix_alpha[kv_idx];
+                                const uint4 u = *reinterpret_cast<const uint4*>(op + 32 * ch + 8 * q4);
+                                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    v8[2 * e] = al * v8[2 * e] + (1.f - al) * bf16_lo(w[e]);
+                                    v8[2 * e + 1] = al * v8[2 * e + 1] + (1.f - al) * bf16_hi(w[e]);
+                                }
+                            }
                             store_row<__nv_bfloat16, 8>(op + 32 * ch + 8 * q4, v8);
                         }
                     }
@@ -716,7 +732,7 @@ size_t prefill_workspace_bytes(const LayerArgs& a, int max_chunk) {
 
 cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void* q, const void* k_chunk,
                               const void* v_chunk, int C, void* out, void* workspace, size_t ws_bytes,
-                              cudaStream_t s) {
+                              cudaStream_t s, const float* mix_alpha) {
     if (!prefill_tc_supported(a)) return cudaErrorNotSupported;
     const uint64_t row = HD * 2;
     CUtensorMap mQ, mKx, mVx, mKc, mVc, mKr, mVr;
@@ -743,13 +759,13 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
         mKc = mKx;  // never read: no retrieval heads, or no cache (c0 = 0)
         mVc = mVx;
     }
-    if (a.S > 0) {
+    if (a.S > 0 && c.k_ring != nullptr) {
         const uint64_t d[3] = {HD, (uint64_t)a.W, (uint64_t)a.B * a.S};
         const uint64_t st[2] = {row, row * a.W};
         if (!encode_tmap_bf16(&mKr, c.k_ring, 3, d, st, bx3) || !encode_tmap_bf16(&mVr, c.v_ring, 3, d, st, bx3))
             return cudaErrorInvalidValue;
     } else {
-        mKr = mKx;  // never read: there are no streaming heads
+        mKr = mKx;  // never read: no streaming heads, or no cache (c0 = 0)
         mVr = mVx;
     }
     TcArgs p;
@@ -758,7 +774,7 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
     p.n_mpairs = (C + 2 * BM - 1) / (2 * BM);
     p.n_units = a.B * a.R * a.G * p.n_mpairs;
     const PrefillPlan plan = prefill_plan(a, C, sm_count());
-    const bool split = plan.ns > 1 && workspace != nullptr && ws_bytes >= plan.bytes;
+    const bool split = plan.ns > 1 && workspace != nullptr && ws_bytes >= plan.bytes && mix_alpha == nullptr;
     p.ns = split ? plan.ns : 1;
     p.part = split ? static_cast<float*>(workspace) : nullptr;
     p.ticket = split ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + plan.ticket_offset) : nullptr;
@@ -766,6 +782,7 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
     p.seq_len = c.seq_len;
     p.status = c.status;
     p.out = out;
+    p.mix_alpha = mix_alpha;
     const long grid = (long)p.n_ret_ctas + (long)a.B * a.S * a.G * p.n_mpairs;
     if (grid == 0) return cudaSuccess;
     if (grid > 0x7fffffffL) return cudaErrorInvalidConfiguration;
