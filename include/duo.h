@@ -224,8 +224,10 @@ duo_status duo_desc_validate(const duo_layer_desc* desc);
  * duo_workspace_bytes -- device workspace needed by duo_decode_attn
  * (op DUO_OP_DECODE) or duo_prefill_chunk (op DUO_OP_PREFILL, max_tokens =
  * largest chunk).  The workspace holds split-K partial results and ticket
- * words; it must be zero-filled once before its first use, and every call
- * leaves the ticket words zero again.  Returns 0 for an invalid descriptor.
+ * words.  A decode workspace must be zero-filled once before its first use
+ * (every call leaves the ticket words zero again); a pre-fill workspace needs
+ * no initialisation (each call clears the ticket words it uses).  Returns 0
+ * for an invalid descriptor.
  */
 size_t duo_workspace_bytes(const duo_layer_desc* desc, int32_t op, int32_t max_tokens);
 
