@@ -143,6 +143,53 @@ def test_workspace_bytes(duo):
     assert duo.workspace_bytes(d, 99, 0) == 0
 
 
+def _prefill_plan_bytes(units, n_sms=148, max_split=8, part_floats=2 * 128 + 128 * 128):
+    """The pre-fill key-split plan restated: the smallest split count whose
+    units * ns CTAs fill their waves of n_sms to 95 % (else the fullest), and
+    the workspace it needs -- per split and query tile a partial record, then
+    a ticket word per unit, each region rounded up to 256 bytes."""
+    best, ns = 0.0, 1
+    for k in range(1, max_split + 1):
+        items = units * k
+        fill = items / (-(-items // n_sms) * n_sms)
+        if fill > best + 1e-9:
+            best, ns = fill, k
+        if fill >= 0.95:
+            break
+    if ns == 1:
+        return 256
+    part = units * ns * 2 * part_floats * 4
+    return -(-part // 256) * 256 + -(-(units * 4) // 256) * 256
+
+
+@pytest.mark.parametrize("hq,hkv,R,B,chunk", [(32, 8, 4, 1, 4096), (32, 32, 8, 1, 4096), (32, 8, 2, 1, 49152),
+                                              (16, 4, 2, 3, 1000), (8, 8, 8, 64, 4096)])
+def test_prefill_workspace_follows_the_split_plan(duo, hq, hkv, R, B, chunk):
+    # a workspace sized for `chunk` serves every shorter chunk, so it is the
+    # largest plan over 1 .. ceil(chunk / 256) query-tile pairs
+    d = duo.desc_init(B, hq, hkv, 128, duo.BF16, list(range(hkv)), R)
+    want = max(_prefill_plan_bytes(B * R * (hq // hkv) * mp) for mp in range(1, -(-chunk // 256) + 1))
+    assert duo.workspace_bytes(d, duo.OP_PREFILL, chunk) == max(want, 256)
+
+
+def test_prefill_workspace_plans_at_the_bench_shape(duo):
+    # 4,096-token chunks of the GQA layer with 4 of 8 KV heads retrieval: 256
+    # units, 4 splits each (1,024 CTAs in 6.92 waves of 148)
+    assert _prefill_plan_bytes(4 * 4 * 16) == 256 * 4 * 2 * 16640 * 4 + 1024
+    d32 = duo.desc_init(1, 8, 8, 64, duo.FP32, list(range(8)), 2)
+    assert duo.workspace_bytes(d32, duo.OP_PREFILL, 4096) == 256   # the CUDA-core path splits nothing
+
+
+def test_exp2_probe_rejects_bad_arguments(duo):
+    with pytest.raises(duo.DuoError) as e:
+        duo.exp2_fma_probe(0, 0, -1, stream=0)
+    assert e.value.status == duo.ERR_INVALID_ARG
+    with pytest.raises(duo.DuoError) as e:
+        duo.exp2_fma_probe(0, 256, 8, stream=0)
+    assert e.value.status == duo.ERR_INVALID_ARG
+    duo.exp2_fma_probe(0, 0, 0, stream=0)   # nothing to do: no launch
+
+
 # ---------------------------------------------------------------------------
 # Device entry points reject bad arguments on the host, before any launch
 # ---------------------------------------------------------------------------
