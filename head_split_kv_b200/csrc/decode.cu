@@ -1028,12 +1028,9 @@ cudaError_t launch_mma_t(const LayerArgs& a, const CacheArgs& c, const DecodeArg
     if (!have_r) { mKr = mKf; mVr = mVf; }  // never read: there are no streaming heads
     constexpr size_t smem = decode_mma_smem_bytes();
     auto kern = decode_mma_kernel<G, PAGED>;
-    static bool configured = false;  // function attributes are per process, set once
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<unsigned long long> configured{0};
+    const cudaError_t e = smem_limit_once(kern, (int)smem, configured);
+    if (e != cudaSuccess) return e;
     return launch_pdl(kern, grid, kMmaThreads, smem, s, mKf, mVf, mKr, mVr, a, c, d);
 }
 
@@ -1066,12 +1063,9 @@ cudaError_t launch_t(const LayerArgs& a, const CacheArgs& c, const DecodeArgs& d
     constexpr size_t smem = decode_smem_bytes<T, D, G>();
     auto kern = decode_kernel<T, D, G, PAGED>;
     constexpr int kThreads = (consumer_warps(G) + 1) * 32;
-    static bool configured = false;  // function attributes are per process, set once
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<unsigned long long> configured{0};
+    const cudaError_t e = smem_limit_once(kern, (int)smem, configured);
+    if (e != cudaSuccess) return e;
     return launch_pdl(kern, grid, kThreads, smem, s, a, c, d);
 }
 
@@ -1495,12 +1489,9 @@ cudaError_t launch_q8_g(const LayerArgs& a, const CacheArgs& c, const DecodeArgs
     }
     constexpr size_t smem = decode_q8_smem_bytes();
     auto kern = decode_q8_kernel<G>;
-    static bool configured = false;  // function attributes are per process, set once
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<unsigned long long> configured{0};
+    const cudaError_t e = smem_limit_once(kern, (int)smem, configured);
+    if (e != cudaSuccess) return e;
     return launch_pdl(kern, grid, kMmaThreads, smem, s, mK, mV, a, c, d);
 }
 

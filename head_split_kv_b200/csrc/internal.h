@@ -2,6 +2,7 @@
 // and the kernels.  Not part of the public ABI.
 #pragma once
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <cuda.h>
@@ -10,6 +11,22 @@
 #include "duo.h"
 
 namespace duo {
+
+// Raises `kernel`'s dynamic shared memory limit to `bytes` once per device:
+// function attributes belong to a device's context, so a process that
+// launches on several devices sets them on each.  `done` holds a bit per
+// device (ordinal < 64; higher ordinals set the attribute on every call).
+template <typename K>
+inline cudaError_t smem_limit_once(K* kernel, int bytes, std::atomic<unsigned long long>& done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = dev < 64 ? 1ull << dev : 0ull;
+    if (bit && (done.load(std::memory_order_relaxed) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_relaxed);
+    return e;
+}
 
 // Flattened, validated view of a layer descriptor plus state, passed by
 // value to every kernel.

@@ -786,12 +786,10 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
     const long grid = (long)p.n_ret_ctas + (long)a.B * a.S * a.G * p.n_mpairs;
     if (grid == 0) return cudaSuccess;
     if (grid > 0x7fffffffL) return cudaErrorInvalidConfiguration;
-    static bool configured = false;  // function attributes are per process, set once
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)(kSmemBytes + 1024));
+    static std::atomic<unsigned long long> configured{0};
+    {
+        const cudaError_t e = smem_limit_once(prefill_tc_kernel, (int)(kSmemBytes + 1024), configured);
         if (e != cudaSuccess) return e;
-        configured = true;
     }
     if (split) {
         // the ticket words sit after this chunk length's partial records, so
