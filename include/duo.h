@@ -355,8 +355,11 @@ duo_status duo_prefill_chunk(const duo_layer_desc* desc, const duo_kv_state* st,
  *
  * alpha [Hkv] fp32 device, in model KV head order.
  * q [B][N][Hq][d]; k, v [B][N][Hkv][d]; out [B][N][Hq][d]; model head order
- * (kv_perm and io_order are not used).  One pass over QK^T feeds both
- * softmax states.
+ * (kv_perm and io_order are not used).  bf16 with d = 128 runs on the tcgen05
+ * tensor cores in two launches (the streaming attention written to out, then
+ * the causal attention mixed with it as it is stored), so out must not alias
+ * q, k or v; other dtypes and head sizes run on the CUDA cores, one pass over
+ * Q K^T feeding both softmax states.
  * Errors: DUO_ERR_INVALID_ARG, DUO_ERR_SHAPE, DUO_ERR_UNSUPPORTED, DUO_ERR_CUDA.
  */
 duo_status duo_gated_mix(const duo_layer_desc* desc, const float* alpha, const void* q,
