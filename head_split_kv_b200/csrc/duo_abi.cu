@@ -406,6 +406,17 @@ duo_status duo_gated_mix(const duo_layer_desc* desc, const float* alpha, const v
         return fail(DUO_ERR_INVALID_ARG, "duo_gated_mix tensors must be 16-byte aligned");
     if (N < 0) return fail(DUO_ERR_SHAPE, "N must be >= 0 (got %d)", N);
     if (N == 0) return ok();
+    {
+        // out is written while q, k and v are still being read
+        const size_t es = desc->dtype == DUO_BF16 ? 2 : 4;
+        const size_t rows = (size_t)desc->batch * (size_t)N;
+        const size_t nq = rows * desc->n_q_heads * desc->head_dim * es;
+        const size_t nkv = rows * desc->n_kv_heads * desc->head_dim * es;
+        const uintptr_t o = (uintptr_t)out;
+        auto hits = [&](const void* p, size_t n) { return o < (uintptr_t)p + n && (uintptr_t)p < o + nq; };
+        if (hits(q, nq) || hits(k, nkv) || hits(v, nkv))
+            return fail(DUO_ERR_INVALID_ARG, "duo_gated_mix: out overlaps q, k or v");
+    }
     duo::LayerArgs a;
     fill_args(desc, a);
     // the mix runs in model head order over whole sequences

@@ -261,6 +261,18 @@ def test_gated_mix_rejects(duo):
     duo.gated_mix(d, 16, 256, 512, 768, 0, 1024, stream=0)       # N = 0: nothing to do
 
 
+def test_gated_mix_rejects_out_overlapping_an_input(duo):
+    # 32 query / 8 KV heads, d 128, bf16, 10 tokens: q and out are 80 KB, k
+    # and v 20 KB; the check runs on the host, before any launch
+    d = _desc(duo)
+    q, k, v = 1 << 20, 2 << 20, 3 << 20
+    for out in (q, q + 4096, k - 4096, v + 16):
+        with pytest.raises(duo.DuoError) as e:
+            duo.gated_mix(d, 16, q, k, v, 10, out, stream=0)
+        assert e.value.status == duo.ERR_INVALID_ARG
+        assert "overlaps" in duo.last_error()
+
+
 def test_permute_rejects_overlap(duo):
     d = _desc(duo)
     with pytest.raises(duo.DuoError) as e:
