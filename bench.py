@@ -48,19 +48,25 @@ from head_split_kv_b200 import synthetic as S  # noqa: E402
 
 METRIC = "decode attn µs/step/layer & HBM GB/s; chunked-prefill TFLOP/s; % of roofline"
 
+# "layers": attention layers a decode step runs through, each with its own
+# caches (Llama-2-7B and Llama-3-8B have 32; fewer where 32 layers' caches
+# would not leave room on one GPU)
 WORKLOADS = {
-    "mha_decode_32k": dict(kind="decode", hq=32, hkv=32, d=128, n_ret=8, lengths=[32768], steps=256, sigma=False),
-    "gqa_decode_128k": dict(kind="decode", hq=32, hkv=8, d=128, n_ret=4, lengths=[131072], steps=64, sigma=True),
-    "gqa_decode_1m": dict(kind="decode", hq=32, hkv=8, d=128, n_ret=4, lengths=[1048576], steps=64, sigma=True),
+    "mha_decode_32k": dict(kind="decode", hq=32, hkv=32, d=128, n_ret=8, lengths=[32768], steps=256, sigma=False,
+                           layers=32),
+    "gqa_decode_128k": dict(kind="decode", hq=32, hkv=8, d=128, n_ret=4, lengths=[131072], steps=64, sigma=True,
+                            layers=32),
+    "gqa_decode_1m": dict(kind="decode", hq=32, hkv=8, d=128, n_ret=4, lengths=[1048576], steps=64, sigma=True,
+                          layers=16),
     "batch64_paged_decode": dict(kind="decode", hq=32, hkv=32, d=128, n_ret=8, batch=64, lo=4096, hi=32768,
-                                 steps=32, sigma=False, paged=True),
+                                 steps=32, sigma=False, paged=True, layers=8),
     # the same decode workloads over the 8-bit retrieval cache (codes + a scale per row)
     "mha_decode_32k_int8": dict(kind="decode", hq=32, hkv=32, d=128, n_ret=8, lengths=[32768], steps=256,
-                                sigma=False, kv_int8=True),
+                                sigma=False, kv_int8=True, layers=32),
     "gqa_decode_128k_int8": dict(kind="decode", hq=32, hkv=8, d=128, n_ret=4, lengths=[131072], steps=64,
-                                 sigma=True, kv_int8=True),
+                                 sigma=True, kv_int8=True, layers=32),
     "gqa_decode_1m_int8": dict(kind="decode", hq=32, hkv=8, d=128, n_ret=4, lengths=[1048576], steps=64,
-                               sigma=True, kv_int8=True),
+                               sigma=True, kv_int8=True, layers=16),
     "gqa_prefill_128k": dict(kind="prefill", hq=32, hkv=8, d=128, n_ret=4, n=131072, chunk=4096, sigma=False),
     # the same pre-fill on a 32K prompt: a small case for profiler captures
     "gqa_prefill_32k": dict(kind="prefill", hq=32, hkv=8, d=128, n_ret=4, n=32768, chunk=4096, sigma=False),
@@ -70,6 +76,9 @@ WORKLOADS = {
     "gated_mix_pr1": dict(kind="mix", hq=8, hkv=8, d=64, n=512, dtype="fp32", n_ret=2),
     "gated_mix_gqa_4k": dict(kind="mix", hq=32, hkv=8, d=128, n=4096, dtype="bf16", n_ret=4),
 }
+DEFAULT_WORKLOAD = "gqa_decode_128k"
+# decode configurations timed beside the default one, each as its own record
+EXTRA_DECODE = ("mha_decode_32k", "gqa_decode_1m", "batch64_paged_decode")
 for _name, _wl in WORKLOADS.items():
     _wl["name"] = _name
 
@@ -118,8 +127,9 @@ h = nv.nvmlDeviceGetHandleByPciBusId(sys.argv[1])
 period = float(sys.argv[2])
 print("ready", nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM), flush=True)
 while True:
-    print(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), nv.nvmlDeviceGetCurrentClocksEventReasons(h), flush=True)
-    time.sleep(period)
+    t = time.monotonic()
+    print(t, nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), nv.nvmlDeviceGetCurrentClocksEventReasons(h), flush=True)
+    time.sleep(max(0.0, period - (time.monotonic() - t)))
 """
 
 
@@ -127,10 +137,15 @@ class ClockSampler:
     """SM clock and clock-event (throttle) reasons of this process's GPU,
     sampled while the timed region runs, from a separate process so that the
     launching thread's hold on the interpreter cannot starve the sampling.
-    Through NVML every 2 ms when the bindings load (the CUDA device is
+
+    Through NVML every 1 ms when the bindings load (the CUDA device is
     matched to its NVML handle by PCI bus id, so CUDA_VISIBLE_DEVICES cannot
-    point it at another GPU), else through `nvidia-smi -lms 200`.  Only
-    reads; nothing about the GPU is changed."""
+    point it at another GPU), else through `nvidia-smi -lms 100`.  Each NVML
+    sample carries the poller's CLOCK_MONOTONIC time (one clock for every
+    process on the host); entering waits until the first sample has arrived,
+    and the summary keeps the samples taken between entering and leaving --
+    the timed region, which ends with a device synchronisation.  Only reads;
+    nothing about the GPU is changed."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -139,13 +154,15 @@ class ClockSampler:
     # NVML clock-event reason bits
     BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40}
 
-    def __init__(self, gpu_index: int, period_s: float = 0.002):
+    def __init__(self, gpu_index: int, period_s: float = 0.001):
         self.gpu = gpu_index
         self.period = period_s
         self.proc = None
         self.lines = []
         self.mode = None
         self.max_mhz = None
+        self.t_enter = self.t_exit = None
+        self._first = threading.Event()
 
     def _start_nvml(self) -> bool:
         import torch
@@ -171,42 +188,49 @@ class ClockSampler:
             try:
                 self.proc = subprocess.Popen(
                     ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                     "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-                self.mode = "nvidia-smi 200 ms"
+                     "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.mode = "nvidia-smi 100 ms"
             except OSError:
                 self.proc = None
         if self.proc is not None:
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            self._first.wait(timeout=5.0)   # the sampler is running before the region starts
+        self.t_enter = time.monotonic()
         return self
 
     def _read(self):
         for ln in self.proc.stdout:
             self.lines.append(ln.strip())
+            self._first.set()
 
     def __exit__(self, *exc):
+        self.t_exit = time.monotonic()
         if self.proc:
-            if not self.mode.startswith("nvml"):
-                time.sleep(0.25)
+            # let the sample taken across the end of the region arrive
+            time.sleep(0.25 if not self.mode.startswith("nvml") else 3 * self.period)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-            self.t.join(timeout=5)   # lines still in the pipe belong to the timed region
+            self.t.join(timeout=5)
 
     def summary(self):
-        mhz, mx, reasons = [], self.max_mhz, set()
+        mhz, mx, reasons, outside = [], self.max_mhz, set(), 0
         for ln in list(self.lines):
             if self.mode.startswith("nvml"):
                 parts = ln.split()
-                if len(parts) != 2:
+                if len(parts) != 3:
                     continue
                 try:
-                    mhz.append(float(parts[0]))
-                    bits = int(parts[1])
+                    t, f, bits = float(parts[0]), float(parts[1]), int(parts[2])
                 except ValueError:
                     continue
+                if not (self.t_enter <= t <= self.t_exit):
+                    outside += 1
+                    continue
+                mhz.append(f)
                 reasons |= {n for n, bit in self.BITS.items() if bits & bit}
             else:
                 parts = [p.strip() for p in ln.split(",")]
@@ -220,8 +244,11 @@ class ClockSampler:
                 for n, v in zip(self.NAMES, parts[5:9]):
                     if v.lower() == "active":
                         reasons.add(n)
+        region_ms = (self.t_exit - self.t_enter) * 1e3 if self.t_exit else None
         return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(mhz), "sampler": self.mode}
+                "reasons": sorted(reasons), "samples": len(mhz), "sampler": self.mode,
+                "region_ms": round(region_ms, 1) if region_ms is not None else None,
+                "samples_outside_region": outside}
 
 
 # ---------------------------------------------------------------------------
@@ -294,10 +321,7 @@ def _decode_setup(duo, wl, total_steps, seed=0):
                              kv_quant=duo.KV_INT8 if wl.get("kv_int8") else duo.KV_PLAIN)
         caches = duo.LayerCaches(desc, int(lengths.max()) + total_steps)
     st = S.decode_state(sh, retrieval, lengths, seed=seed, sigma=sigma)
-    if wl.get("kv_int8"):
-        _append_decode_state(duo, desc, caches, st, retrieval, sh)
-    else:
-        _load_decode_state(caches, st, inv, R, sh, table)
+    _fill_decode_state(duo, desc, caches, st, inv, R, sh, table, bool(wl.get("kv_int8")))
     ws = duo.Workspace(desc, duo.OP_DECODE, caches.capacity)
     qs, ks, vs = S.decode_steps(sh, B, total_steps, seed=seed, sigma=sigma)
     torch.cuda.synchronize()
@@ -315,63 +339,55 @@ def _to_dev(a):
     return torch.from_numpy(a).cuda()
 
 
-def _load_decode_state(caches, st, inv, R, sh, table):
-    """Write a seeded cache state into the documented device layout."""
-    import torch
-    ring_pos = np.full((caches.ring_pos.shape[0], sh.sink + sh.recent), -1, dtype=np.int32)
-    for (b, h), (k, v) in st["full"].items():
-        r = inv[h]
-        L = k.shape[0]
-        if table is None:
-            caches.k_full[b, r, :L] = _to_dev(k)
-            caches.v_full[b, r, :L] = _to_dev(v)
-        else:
-            pos = np.arange(L)
-            pages = torch.from_numpy(table[b, pos // 64].astype(np.int64)).cuda()
-            rows = torch.from_numpy(pos % 64).cuda()
-            caches.k_full[pages, r, rows] = _to_dev(k)
-            caches.v_full[pages, r, rows] = _to_dev(v)
-    for (b, h), (pos, k, v) in st["stream"].items():
-        s = inv[h] - R
-        slots = np.array([p if p < sh.sink else sh.sink + (p - sh.sink) % sh.recent for p in pos], dtype=np.int64)
-        if len(slots):
-            idx = torch.from_numpy(slots).cuda()
-            caches.k_ring[b, s, idx] = _to_dev(k)
-            caches.v_ring[b, s, idx] = _to_dev(v)
-            ring_pos[b, slots] = pos
-    caches.ring_pos.copy_(torch.from_numpy(ring_pos))
-    caches.seq_len.copy_(torch.from_numpy(st["lengths"].astype(np.int32)))
+def _fill_decode_state(duo, desc, caches, st, inv, R, sh, table, kv_int8, chunk=32768):
+    """Put a seeded prompt state on the device.
 
-
-def _append_decode_state(duo, desc, caches, st, retrieval, sh, chunk=32768):
-    """Fill an 8-bit layer with a seeded state through duo_append_kv, which
-    quantizes the retrieval rows on the device (the streaming heads' rows are
-    zeros there), then install the streaming rings as _load_decode_state does."""
+    Retrieval rows: written straight into the documented cache layout (bf16),
+    or appended through duo_append_kv, which quantizes them (8-bit; the other
+    heads get zero rows there).  Streaming rings: built by the library's own
+    append -- seq_len is set to 0 and the prompt's first W = sink + recent
+    tokens are appended, then seq_len is set to L - W and its last W tokens
+    are appended (every head's rows, so a retrieval head gets its own rows
+    again).  A ring holds at most W tokens, so this leaves it as appending the
+    whole prompt would, without drawing the streaming rows in between."""
     import torch
-    lengths = st["lengths"]
-    B, L = len(lengths), int(lengths.max())
-    assert np.all(lengths == L), "8-bit states are built for equal lengths"
-    for c0 in range(0, L, chunk):
-        T = min(chunk, L - c0)
-        kc = torch.zeros((B, T, sh.n_kv_heads, sh.head_dim), dtype=torch.bfloat16, device="cuda")
-        vc = torch.zeros_like(kc)
-        for (b, h), (k, v) in st["full"].items():
-            kc[b, :, h] = _to_dev(k[c0:c0 + T])
-            vc[b, :, h] = _to_dev(v[c0:c0 + T])
-        duo.append_kv(desc, caches.state, kc, vc, T)
-    inv = {int(h): i for i, h in enumerate(list(desc.kv_perm)[:sh.n_kv_heads])}
-    R = desc.n_retrieval
-    ring_pos = np.full((B, sh.sink + sh.recent), -1, dtype=np.int32)
-    for (b, h), (pos, k, v) in st["stream"].items():
-        s_ = inv[h] - R
-        slots = np.array([p if p < sh.sink else sh.sink + (p - sh.sink) % sh.recent for p in pos], dtype=np.int64)
-        if len(slots):
-            idx = torch.from_numpy(slots).cuda()
-            caches.k_ring[b, s_, idx] = _to_dev(k)
-            caches.v_ring[b, s_, idx] = _to_dev(v)
-            ring_pos[b, slots] = pos
-    caches.ring_pos.copy_(torch.from_numpy(ring_pos))
+    lengths = st.lengths
+    B = len(lengths)
+    W = sh.sink + sh.recent
+    assert int(lengths.min()) >= 2 * W, "bench states are built for prompts of at least 2 (sink + recent) tokens"
+    if kv_int8:
+        L = int(lengths.max())
+        assert np.all(lengths == L), "8-bit states are built for equal lengths"
+        for c0 in range(0, L, chunk):
+            T = min(chunk, L - c0)
+            kc = torch.zeros((B, T, sh.n_kv_heads, sh.head_dim), dtype=torch.bfloat16, device="cuda")
+            vc = torch.zeros_like(kc)
+            for (b, h), (k, v) in st.full.items():
+                kc[b, :, h] = _to_dev(k[c0:c0 + T])
+                vc[b, :, h] = _to_dev(v[c0:c0 + T])
+            duo.append_kv(desc, caches.state, kc, vc, T)
+    else:
+        for (b, h), (k, v) in st.full.items():
+            r = inv[h]
+            L = k.shape[0]
+            if table is None:
+                caches.k_full[b, r, :L] = _to_dev(k)
+                caches.v_full[b, r, :L] = _to_dev(v)
+            else:
+                pos = np.arange(L)
+                pages = torch.from_numpy(table[b, pos // 64].astype(np.int64)).cuda()
+                rows = torch.from_numpy(pos % 64).cuda()
+                caches.k_full[pages, r, rows] = _to_dev(k)
+                caches.v_full[pages, r, rows] = _to_dev(v)
+    for first in (True, False):
+        start = np.zeros(B, dtype=np.int64) if first else lengths - W
+        rows = [st.token_rows(b, np.arange(start[b], start[b] + W)) for b in range(B)]
+        kk = np.stack([r[0] for r in rows])
+        vv = np.stack([r[1] for r in rows])
+        caches.seq_len.copy_(torch.from_numpy(start.astype(np.int32)))
+        duo.append_kv(desc, caches.state, _to_dev(kk), _to_dev(vv), W)
     torch.cuda.synchronize()
+    assert np.array_equal(caches.seq_len.cpu().numpy(), lengths.astype(np.int32))
     assert duo.check_status(caches.state) == 0
 
 
@@ -409,17 +425,18 @@ def _replicate_layers(duo, env, n_layers):
 
 
 def run_decode(args, wl, world, rank):
-    """Decode steps over `layers` layers: per step, every layer's
-    duo_decode_step (append + attend, one launch) runs back to back as in a
-    model's forward pass.  Each layer has its own caches, so a step streams
-    layers x (retrieval cache) bytes -- more than the 126 MB L2 -- and no
-    flush is needed between steps."""
+    """Decode steps: a step is one new token per sequence through every layer
+    of the model's attention -- per layer duo_decode_step (append + attend,
+    one launch), the layers back to back as in a forward pass, each with its
+    own caches.  A step streams layers x (retrieval cache) bytes, far more
+    than the 126 MB L2, so nothing is flushed between steps."""
     import torch
     from head_split_kv_b200 import duo
-    steps, warm, nl = args.steps, args.warmup, args.layers
+    steps, warm = args.steps, args.warmup
+    nl = args.layers or wl["layers"]
     total = warm + steps
-    # capacity for the warm-up, the timed steps and the end-to-end steps
-    env = _decode_setup(duo, wl, max(total + 32, wl["steps"]) + 1)
+    n_e2e = 0 if getattr(args, "no_e2e", False) else min(steps, 32)
+    env = _decode_setup(duo, wl, total + n_e2e + 1)
     sh, desc, B, R = env["sh"], env["desc"], env["B"], env["R"]
     layers = _replicate_layers(duo, env, nl)
     qd = [_to_dev(env["qs"][i]) for i in range(total)]
@@ -461,9 +478,10 @@ def run_decode(args, wl, world, rank):
             raise RuntimeError(f"device status 0x{st_code:x} after the timed steps")
 
     # end to end through the public API with host buffers
-    e2e = None if getattr(args, "no_e2e", False) else _decode_e2e(duo, env, layers, args, world)
+    e2e = _decode_e2e(duo, env, layers, total, n_e2e, world) if n_e2e else None
 
     hbm, _, peak_kind = _peaks()
+    kernel = "decode_q8_kernel" if wl.get("kv_int8") else "decode_mma_kernel"
     bytes_per_launch = statistics.mean(_decode_bytes(sh, R, L, bool(wl.get("kv_int8"))) for L in lengths_seen)
     dec_avg_s = statistics.mean(dec_ms) * 1e-3
     achieved = bytes_per_launch / dec_avg_s / 1e9
@@ -471,7 +489,7 @@ def run_decode(args, wl, world, rank):
         "metric": METRIC, "value": round(us_step, 3), "unit": "us/step/layer", "n_gpus": world, "steps": steps,
         "warmup": warm, "ms_per_step": round(total_ms / steps, 6), "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "batch": B, "n_q_heads": sh.n_q_heads, "n_kv_heads": sh.n_kv_heads,
+        "config": {"workload": wl["name"], "batch": B, "n_q_heads": sh.n_q_heads, "n_kv_heads": sh.n_kv_heads,
                    "head_dim": sh.head_dim, "n_retrieval": R, "sink": sh.sink, "recent": sh.recent,
                    "context": [int(env["lengths"].min()), int(env["lengths"].max())],
                    "paged": bool(wl.get("paged", False)), "layers_per_step": nl,
@@ -479,83 +497,128 @@ def run_decode(args, wl, world, rank):
                    "parallelism": f"replicas{world}",
                    "l2": f"not flushed: inputs larger than L2 (each step streams {nl} layers' caches, "
                          f"{nl * bytes_per_launch / 1e6:.0f} MB > 126 MB)"},
-        "roofline": {"bound": "hbm", "kernel": "decode_mma_kernel", "achieved": round(achieved, 1), "peak": hbm,
+        "roofline": {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 1), "peak": hbm,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / hbm, 4),
-                     "traffic": _traffic("decode_mma_kernel", args.workload),
+                     "traffic": _traffic(kernel, wl["name"]),
                      "algorithmic_bytes_per_launch": int(bytes_per_launch),
-                     "kernel_us": round(statistics.mean(dec_ms) * 1e3, 3)},
+                     "kernel_us": round(statistics.mean(dec_ms) * 1e3, 3),
+                     "timing": "CUDA events on the launching stream around each step; kernel_us = step time / "
+                               "layers (one launch per layer)"},
         "e2e": e2e,
         "gpu_launches": steps * nl,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = _decode_cpu_baseline(env, budget_s=args.cpu_budget)
+    del layers, env
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
     return res
 
 
-def _decode_e2e(duo, env, layers, args, world):
-    """The same steps through the binding with pinned host buffers: per step
-    and layer the new token's q/k/v go host->device and the output comes back
-    device->host, all inside the timed interval."""
+def _decode_e2e(duo, env, layers, first, n, world):
+    """The same decode steps through the binding with pinned host buffers.
+    Per step, every layer's new-token q, k and v go host->device in one copy
+    and every layer's output comes back device->host in one copy, inside the
+    timed interval.  The copies run on their own streams, ordered by events
+    against the compute stream, with two device input and output buffers:
+    step i + 1's inputs arrive and step i - 1's outputs leave while step i's
+    kernels run.  Every layer of a step takes the step's token (as in the
+    device-resident timing)."""
     import torch
     desc = env["desc"]
     nl = len(layers)
-    n = min(args.steps, 32)
-
-    # a step's q, k and v sit back to back in one pinned buffer, so each layer
-    # takes one host->device copy; the views passed to the library start at
-    # 16-byte multiples (each part is a whole number of d-element rows)
     q_shape, kv_shape = env["qs"][0].shape, env["ks"][0][:, None].shape
     nq, nk = int(np.prod(q_shape)), int(np.prod(kv_shape))
+    per = nq + 2 * nk                       # bf16 elements of one layer's q | k | v (whole d-rows each)
 
     def pinned(i):
-        flat = np.concatenate([np.ascontiguousarray(a).reshape(-1) for a in
-                               (env["qs"][i], env["ks"][i], env["vs"][i])])
+        one = np.concatenate([np.ascontiguousarray(a).reshape(-1) for a in
+                              (env["qs"][i], env["ks"][i], env["vs"][i])])
+        flat = np.tile(one, nl)
         return torch.from_numpy(flat.view(np.int16)).view(torch.bfloat16).pin_memory()
 
-    h_in = [pinned(i) for i in range(n)]
-    h_out = [torch.empty(q_shape, dtype=torch.bfloat16).pin_memory() for _ in range(nl)]
-    d_in = [torch.empty_like(h_in[0], device="cuda") for _ in range(nl)]
-    dq = [x[:nq].view(q_shape) for x in d_in]
-    dk = [x[nq:nq + nk].view(kv_shape) for x in d_in]
-    dv = [x[nq + nk:].view(kv_shape) for x in d_in]
-    dout = [torch.empty(q_shape, dtype=torch.bfloat16, device="cuda") for _ in range(nl)]
-    stream = torch.cuda.current_stream()
-    sp = int(stream.cuda_stream)
-    times = []
+    h_in = [pinned(first + i) for i in range(n)]
+    h_out = [torch.empty((nl,) + tuple(q_shape), dtype=torch.bfloat16).pin_memory() for _ in range(n)]
+    d_in = [torch.empty(nl * per, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    d_out = [torch.empty((nl,) + tuple(q_shape), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    views = [[(x[l * per:l * per + nq].view(q_shape), x[l * per + nq:l * per + nq + nk].view(kv_shape),
+               x[l * per + nq + nk:(l + 1) * per].view(kv_shape)) for l in range(nl)] for x in d_in]
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    sp = int(comp.cuda_stream)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(n)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     _barrier(world)
     torch.cuda.synchronize()
+    t0.record(s_in)
+    comp.wait_event(t0)
+    s_out.wait_event(t0)
     for i in range(n):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
+        k = i % 2
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_comp[i - 2])          # d_in[k] is free once step i - 2 ran
+            d_in[k].copy_(h_in[i], non_blocking=True)
+            ev_in[k].record(s_in)
+        comp.wait_event(ev_in[k])
+        if i >= 2:
+            comp.wait_event(ev_out[k])                   # d_out[k] is free once step i - 2's outputs left
         for l, (caches, ws) in enumerate(layers):
-            d_in[l].copy_(h_in[i], non_blocking=True)
-            duo.decode_step(desc, caches.state, dq[l], dk[l], dv[l], dout[l], ws.ptr, ws.nbytes, sp)
-            h_out[l].copy_(dout[l], non_blocking=True)
-        e1.record(stream)
-        times.append((e0, e1))
+            q, kk, vv = views[k][l]
+            duo.decode_step(desc, caches.state, q, kk, vv, d_out[k][l], ws.ptr, ws.nbytes, sp)
+        ev_comp[i].record(comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[i])
+            h_out[i].copy_(d_out[k], non_blocking=True)
+            ev_out[k].record(s_out)
+    comp.wait_event(ev_out[(n - 1) % 2])
+    if n >= 2:
+        comp.wait_event(ev_out[(n - 2) % 2])
+    t1.record(comp)
     torch.cuda.synchronize()
     _barrier(world)
-    tot = _max_over_ranks(sum(a.elapsed_time(b) for a, b in times), world)
-    h2d = h_in[0].numel() * 2
-    return {"value": round(tot * 1e3 / (n * nl * world), 3), "unit": "us/step/layer", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": h_out[0].numel() * 2, "steps": n, "note": "bytes per layer and step"}
+    tot = _max_over_ranks(t0.elapsed_time(t1), world)
+    for caches, _ in layers:
+        st_code = duo.check_status(caches.state)
+        if st_code:
+            raise RuntimeError(f"device status 0x{st_code:x} after the end-to-end steps")
+    assert all(torch.isfinite(h.float()).all().item() for h in h_out)
+    return {"value": round(tot * 1e3 / (n * nl * world), 3), "unit": "us/step/layer",
+            "h2d_bytes_per_step": nl * per * 2, "d2h_bytes_per_step": nl * nq * 2, "steps": n,
+            "note": "bytes per step (all layers); copies on their own streams, double-buffered"}
 
 
-def _decode_cpu_baseline(env, budget_s=15.0):
+def _oracle_cache(O, st, gate, sh, b_list, heads, kv_int8):
+    """The oracle's caches for sequences b_list and KV heads `heads` of a
+    seeded state: retrieval heads hold every prompt row; a streaming head the
+    positions the oracle's own eviction rule keeps, with their seeded rows."""
+    g = np.array([gate[h] for h in heads], dtype=np.uint8)
+    cache = O.HeadSplitCache(len(b_list), len(heads), sh.head_dim, gate=g, sink=sh.sink, recent=sh.recent,
+                             kv_int8=kv_int8)
+    for bi, b in enumerate(b_list):
+        L = int(st.lengths[b])
+        kept = O.streaming_positions(L, sh.sink, sh.recent)
+        for hi, h in enumerate(heads):
+            if gate[h]:
+                k, v = st.full[(b, h)]
+                cache.load_state(bi, hi, np.arange(L), k, v)
+            else:
+                k, v = st.stream_rows(b, h, kept)
+                cache.load_state(bi, hi, kept, k, v)
+        cache.set_length(bi, L)
+    return cache
+
+
+def _decode_cpu_baseline(env, budget_s=8.0):
     """The oracle, as it stands, on this host's cores: decode steps from the
-    same seeded state until the time budget is used."""
+    same seeded state until the time budget is used (at least one)."""
     import oracle as O
     sh, B = env["sh"], env["B"]
-    cache = O.HeadSplitCache(B, sh.n_kv_heads, sh.head_dim, gate=env["gate"], sink=sh.sink, recent=sh.recent,
-                             kv_int8=env.get("kv_int8", False))
-    st = env["state"]
-    for (b, h), (k, v) in st["full"].items():
-        cache.load_state(b, h, np.arange(k.shape[0]), k, v)
-    for (b, h), (pos, k, v) in st["stream"].items():
-        cache.load_state(b, h, pos, k, v)
-    for b, L in enumerate(st["lengths"]):
-        cache.set_length(b, int(L))
+    cache = _oracle_cache(O, env["state"], env["gate"], sh, list(range(B)), list(range(sh.n_kv_heads)),
+                          env.get("kv_int8", False))
     t0 = time.perf_counter()
     n = 0
     while n < len(env["qs"]) and (time.perf_counter() - t0 < budget_s or n < 1):
@@ -563,7 +626,8 @@ def _decode_cpu_baseline(env, budget_s=15.0):
         n += 1
     dt = time.perf_counter() - t0
     return {"value": round(dt * 1e6 / n, 1), "unit": "us/step/layer", "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"{n} decode steps of the same workload from the same seeded state (fp64 NumPy oracle)"}
+            "sample": f"{n} decode steps of one layer of the same workload from the same seeded state "
+                      f"(fp64 NumPy oracle)"}
 
 
 def _blas_threads():
@@ -722,12 +786,13 @@ def run_mix(args, wl, world, rank):
     ad = torch.from_numpy(alpha).cuda()
     out = torch.empty_like(qd)
     dalpha = torch.empty((sh.n_kv_heads,), dtype=torch.float32, device="cuda")
+    status = torch.zeros((1,), dtype=torch.int32, device="cuda")
     flush = torch.empty(1 << 30, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
     sp = int(stream.cuda_stream)
     for _ in range(args.warmup):
-        duo.gated_mix(desc, ad, qd, kd, vd, n, out, sp)
-        duo.gated_mix_grad_alpha(desc, qd, kd, vd, n, dod, dalpha, sp)
+        duo.gated_mix(desc, ad, qd, kd, vd, n, out, status, sp)
+        duo.gated_mix_grad_alpha(desc, qd, kd, vd, n, dod, dalpha, status, sp)
     steps = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
     _barrier(world)
@@ -736,14 +801,16 @@ def run_mix(args, wl, world, rank):
         for i in range(steps):
             flush.zero_()
             ev[i][0].record(stream)
-            duo.gated_mix(desc, ad, qd, kd, vd, n, out, sp)
+            duo.gated_mix(desc, ad, qd, kd, vd, n, out, status, sp)
             ev[i][1].record(stream)
             flush.zero_()
             ev[i][2].record(stream)
-            duo.gated_mix_grad_alpha(desc, qd, kd, vd, n, dod, dalpha, sp)
+            duo.gated_mix_grad_alpha(desc, qd, kd, vd, n, dod, dalpha, status, sp)
             ev[i][3].record(stream)
         torch.cuda.synchronize()
     _barrier(world)
+    if int(status.item()):
+        raise RuntimeError(f"device status 0x{int(status.item()):x} after the gated-mix calls")
     mix_ms = sorted(e[0].elapsed_time(e[1]) for e in ev)
     grad_ms = sorted(e[2].elapsed_time(e[3]) for e in ev)
     mix_med = _max_over_ranks(mix_ms[len(mix_ms) // 2], world)
@@ -815,19 +882,7 @@ def run_reference(args, wl, budget_s: float = 120.0):
     qs, ks, vs = S.decode_steps(sh, B, total, sigma=sigma)
 
     def build(b_list, heads):
-        g = np.array([gate[h] for h in heads], dtype=np.uint8)
-        cache = O.HeadSplitCache(len(b_list), len(heads), sh.head_dim, gate=g, sink=sh.sink, recent=sh.recent,
-                                 kv_int8=bool(wl.get("kv_int8")))
-        for bi, b in enumerate(b_list):
-            for hi, h in enumerate(heads):
-                if gate[h]:
-                    k, v = st["full"][(b, h)]
-                    cache.load_state(bi, hi, np.arange(k.shape[0]), k, v)
-                else:
-                    pos, k, v = st["stream"][(b, h)]
-                    cache.load_state(bi, hi, pos, k, v)
-            cache.set_length(bi, int(lengths[b]))
-        return cache
+        return _oracle_cache(O, st, gate, sh, b_list, heads, bool(wl.get("kv_int8")))
 
     def sl(i, b_list, heads):
         G = sh.group
@@ -953,13 +1008,16 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=256)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="mha_decode_32k", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--cpu-budget", type=float, default=8.0, help="seconds of oracle time per cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the pre-fill measurement of a decode run")
-    ap.add_argument("--layers", type=int, default=4,
-                    help="decode: layers per step, each with its own caches (their total exceeds L2)")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="default run: skip the other decode configurations' records")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end decode measurement")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="decode: layers per step, each with its own caches (default: the workload's)")
     ap.add_argument("--retrieval-ratio-sweep", action="store_true",
                     help="time decode and pre-fill against the share of retrieval heads (one JSON line)")
     ap.add_argument("--chunk-sweep", action="store_true",
@@ -997,6 +1055,13 @@ def main(argv=None):
             res = run_mix(args, wl, world, rank)
         elif wl["kind"] == "decode":
             res = run_decode(args, wl, world, rank)
+            if args.workload == DEFAULT_WORKLOAD and not args.no_extra and args.n_retrieval is None:
+                res["decode_configs"] = {}
+                for name in EXTRA_DECODE:
+                    sub = run_decode(args, WORKLOADS[name], world, rank)
+                    res["decode_configs"][name] = {k: sub[k] for k in (
+                        "value", "unit", "steps", "warmup", "ms_per_step", "config", "roofline", "e2e",
+                        "gpu_launches", "clocks", "cpu_baseline") if k in sub}
             if not args.no_prefill:
                 pre = run_prefill(args, WORKLOADS["gqa_prefill_128k"], world, rank)
                 res["prefill"] = {k: pre[k] for k in ("value", "unit", "steps", "ms_per_step", "config",

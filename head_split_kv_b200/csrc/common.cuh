@@ -74,17 +74,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, ui
     return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
+// Bounded wait for the phase with the given parity to complete: gives up
+// after `limit_ns` of wall time, ORs DUO_DEV_WAIT_TIMEOUT into *status (when
+// given) and returns false.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, int32_t* status, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > DUO_WAIT_TIMEOUT_NS) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             if (status) atomicOr(status, DUO_DEV_WAIT_TIMEOUT);
             return false;
         }
     }
+}
+
+// The kernels' wait: the same, with the library's limit.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
+    return mbar_wait_for(bar, parity, status, DUO_WAIT_TIMEOUT_NS);
 }
 
 // ------------------------------------------------------------- bulk copies

@@ -211,7 +211,7 @@ const char* duo_status_string(duo_status s) {
     return "DUO_ERR_UNKNOWN";
 }
 
-int32_t duo_abi_version(void) { return 3; }
+int32_t duo_abi_version(void) { return 4; }
 
 duo_status duo_partition_heads(const float* alpha, int32_t n_kv_heads, float tau, int32_t target_n_retrieval,
                                uint8_t* gate, int32_t* kv_perm, int32_t* kv_inv_perm, int32_t* n_retrieval) {
@@ -398,10 +398,10 @@ duo_status duo_prefill_chunk(const duo_layer_desc* desc, const duo_kv_state* st,
 }
 
 duo_status duo_gated_mix(const duo_layer_desc* desc, const float* alpha, const void* q, const void* k, const void* v,
-                         int32_t N, void* out, duo_stream_t stream) {
+                         int32_t N, void* out, int32_t* status, duo_stream_t stream) {
     duo_status s = check_desc(desc);
     if (s != DUO_OK) return s;
-    if (!alpha || !q || !k || !v || !out) return fail(DUO_ERR_INVALID_ARG, "duo_gated_mix: NULL argument");
+    if (!alpha || !q || !k || !v || !out || !status) return fail(DUO_ERR_INVALID_ARG, "duo_gated_mix: NULL argument");
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
         return fail(DUO_ERR_INVALID_ARG, "duo_gated_mix tensors must be 16-byte aligned");
     if (N < 0) return fail(DUO_ERR_SHAPE, "N must be >= 0 (got %d)", N);
@@ -443,6 +443,7 @@ duo_status duo_gated_mix(const duo_layer_desc* desc, const float* alpha, const v
     }
     if (duo::prefill_tc_supported(as) && duo::prefill_tc_supported(ac)) {
         duo::CacheArgs none{};   // no lengths, no caches: every sequence starts at position 0
+        none.status = status;    // device conditions (a wait that ran out) are reported here
         cudaError_t e = duo::launch_prefill_tc(as, none, q, k, v, N, out, nullptr, 0, (cudaStream_t)stream);
         if (e == cudaSuccess)
             e = duo::launch_prefill_tc(ac, none, q, k, v, N, out, nullptr, 0, (cudaStream_t)stream, alpha);
@@ -453,10 +454,11 @@ duo_status duo_gated_mix(const duo_layer_desc* desc, const float* alpha, const v
 }
 
 duo_status duo_gated_mix_grad_alpha(const duo_layer_desc* desc, const void* q, const void* k, const void* v,
-                                    int32_t N, const void* dout, float* dalpha, duo_stream_t stream) {
+                                    int32_t N, const void* dout, float* dalpha, int32_t* status,
+                                    duo_stream_t stream) {
     duo_status s = check_desc(desc);
     if (s != DUO_OK) return s;
-    if (!q || !k || !v || !dout || !dalpha)
+    if (!q || !k || !v || !dout || !dalpha || !status)
         return fail(DUO_ERR_INVALID_ARG, "duo_gated_mix_grad_alpha: NULL argument");
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout))
         return fail(DUO_ERR_INVALID_ARG, "duo_gated_mix_grad_alpha tensors must be 16-byte aligned");
@@ -480,6 +482,14 @@ duo_status duo_exp2_fma_probe(const float* x, float* y, int64_t n, duo_stream_t 
     if (n > 0 && (!x || !y)) return fail(DUO_ERR_INVALID_ARG, "duo_exp2_fma_probe: NULL argument");
     cudaError_t e = duo::launch_exp2_fma_probe(x, y, n, (cudaStream_t)stream);
     return e == cudaSuccess ? ok() : cuda_fail(e, "duo_exp2_fma_probe");
+}
+
+duo_status duo_wait_probe(int32_t* status, uint32_t limit_us, duo_stream_t stream) {
+    if (!status) return fail(DUO_ERR_INVALID_ARG, "duo_wait_probe: status is NULL");
+    if (limit_us < 1 || limit_us > 1000000u)
+        return fail(DUO_ERR_INVALID_ARG, "duo_wait_probe: limit_us must be in 1..1000000 (got %u)", limit_us);
+    const cudaError_t e = duo::launch_wait_probe(status, (uint64_t)limit_us * 1000ull, (cudaStream_t)stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "duo_wait_probe");
 }
 
 duo_status duo_check_status(const duo_kv_state* st, int32_t* host_status, duo_stream_t stream) {

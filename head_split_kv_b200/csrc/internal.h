@@ -97,6 +97,8 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
                               const void* v_chunk, int C, void* out, void* workspace, size_t ws_bytes,
                               cudaStream_t s, const float* mix_alpha = nullptr);
 cudaError_t launch_exp2_fma_probe(const float* x, float* y, int64_t n, cudaStream_t s);
+// One warp waits on an mbarrier that never completes, with the given limit.
+cudaError_t launch_wait_probe(int32_t* status, uint64_t limit_ns, cudaStream_t s);
 
 bool prefill_tc_supported(const LayerArgs& a);
 // bf16 tensor map of `rank` dims (innermost first), 64-element-wide boxes with

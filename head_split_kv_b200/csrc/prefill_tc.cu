@@ -240,7 +240,7 @@ __device__ __forceinline__ void visible_columns(const LayerArgs& a, const Sched&
 
 // ------------------------------------------------------------------ softmax
 
-constexpr int kFmaExpEvery = 4;   // one exp2 pair in 4 on the FMA pipe
+constexpr int kFmaExpEvery = 8;   // one exp2 pair in 8 on the FMA pipe (1 in 4 spills at 200 registers)
 
 // 2^x for a pair of x <= 0 (or -inf) on the FMA pipe, by Cody-Waite range
 // reduction and a polynomial: x = n + f with n = rint(x) (adding 1.5 * 2^23
@@ -283,7 +283,8 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
 // SFU is the co-bottleneck.  One pair in kFmaExpEvery is computed on the FMA
 // pipe instead (exp2_fma2).  Measured on the 131K prompt: one pair in 4 or
 // in 8 (equal within run-to-run noise) beat SFU-only by 2-5 %; one in 3 was
-// slower.
+// slower.  One in 8 leaves the kernel without register spills at its
+// 200-register budget (one in 4 spilled 20-30 bytes a thread).
 __device__ __forceinline__ float softmax_tile(uint32_t s_addr, float sl, bool masked, const uint32_t (&vis)[4],
                                               float& m_ref, float& l_sum, bool& need) {
     float s[128];
@@ -333,7 +334,12 @@ __device__ __forceinline__ float softmax_tile(uint32_t s_addr, float sl, bool ma
 
 // ------------------------------------------------------------------ kernel
 
-__global__ void __launch_bounds__(kThreads, 1)
+// MIX: the gated-mix instantiation (its epilogue mixes with what out holds;
+// no key-range splits), so the pre-fill instantiation carries no mix code.
+// 200 registers a thread: 10 warps x 32 x 200 fit the SM's 64K with one CTA
+// per SM.
+template <bool MIX>
+__global__ void __maxnreg__(200)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
                       const __grid_constant__ CUtensorMap tmVc, const __grid_constant__ CUtensorMap tmKx,
                       const __grid_constant__ CUtensorMap tmVx, const __grid_constant__ CUtensorMap tmKr,
@@ -563,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // epilogue: O / l -> bf16
         if (ok && n_me >= 1) ok = __all_sync(0xffffffffu, mbar_wait(&o_done[qi], 0, p.status));
         __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.out) + (((size_t)b * p.C + crow) * a.Hq + q_idx) * HD;
-        if (ns_use == 1) {
+        if (MIX || ns_use == 1) {
             if (ok && n_me >= 1) {
                 tc_fence_after();
                 const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
@@ -577,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             float v8[8];
 #pragma unroll
                             for (int e = 0; e < 8; ++e) v8[e] = o[8 * q4 + e] * inv;
-                            if (p.mix_alpha) {
+                            if constexpr (MIX) {
                                 // gated mix: out already holds the streaming attention
                                 const float al = p.mix_alpha[kv_idx];
                                 const uint4 u = *reinterpret_cast<const uint4*>(op + 32 * ch + 8 * q4);
@@ -593,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-        } else {
+        } else if constexpr (!MIX) {
             // (1) this split's record of the query tile: m, l and O unnormalised
             const bool have = ok && n_me >= 1;               // warp-uniform
             float* rec = p.part + (((size_t)unit * p.ns + split) * 2 + qi) * kPartFloats;
@@ -786,9 +792,10 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
     const long grid = (long)p.n_ret_ctas + (long)a.B * a.S * a.G * p.n_mpairs;
     if (grid == 0) return cudaSuccess;
     if (grid > 0x7fffffffL) return cudaErrorInvalidConfiguration;
-    static std::atomic<unsigned long long> configured{0};
+    static std::atomic<unsigned long long> configured{0}, configured_mix{0};
     {
-        const cudaError_t e = smem_limit_once(prefill_tc_kernel, (int)(kSmemBytes + 1024), configured);
+        const cudaError_t e = mix_alpha ? smem_limit_once(prefill_tc_kernel<true>, (int)(kSmemBytes + 1024), configured_mix)
+                                        : smem_limit_once(prefill_tc_kernel<false>, (int)(kSmemBytes + 1024), configured);
         if (e != cudaSuccess) return e;
     }
     if (split) {
@@ -798,7 +805,10 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
         const cudaError_t e = cudaMemsetAsync(p.ticket, 0, (size_t)p.n_units * sizeof(uint32_t), s);
         if (e != cudaSuccess) return e;
     }
-    prefill_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes + 1024, s>>>(mQ, mKc, mVc, mKx, mVx, mKr, mVr, p);
+    if (mix_alpha)
+        prefill_tc_kernel<true><<<(unsigned)grid, kThreads, kSmemBytes + 1024, s>>>(mQ, mKc, mVc, mKx, mVx, mKr, mVr, p);
+    else
+        prefill_tc_kernel<false><<<(unsigned)grid, kThreads, kSmemBytes + 1024, s>>>(mQ, mKc, mVc, mKx, mVx, mKr, mVr, p);
     return cudaGetLastError();
 }
 

@@ -72,7 +72,7 @@ def _fn(name, restype, *argtypes):
 _lib_last_error = _fn("duo_last_error", ctypes.c_char_p)
 _lib_status_string = _fn("duo_status_string", ctypes.c_char_p, ctypes.c_int)
 _lib_abi_version = _fn("duo_abi_version", _I32)
-ABI_VERSION = 3           # the layout of LayerDesc / KVState below
+ABI_VERSION = 4           # the layout of LayerDesc / KVState and the signatures below
 if _lib_abi_version() != ABI_VERSION:
     raise ImportError(f"{LIB_PATH} has ABI version {_lib_abi_version()}, this binding needs {ABI_VERSION}; rebuild it")
 _lib_partition = _fn("duo_partition_heads", ctypes.c_int, ctypes.POINTER(ctypes.c_float), _I32, ctypes.c_float,
@@ -86,8 +86,9 @@ _lib_permute = _fn("duo_permute_heads", ctypes.c_int, _DESC, _P, _P, ctypes.c_in
 _lib_append = _fn("duo_append_kv", ctypes.c_int, _DESC, _STATE, _P, _P, _I32, _P)
 _lib_decode = _fn("duo_decode_attn", ctypes.c_int, _DESC, _STATE, _P, _P, _P, ctypes.c_size_t, _P)
 _lib_prefill = _fn("duo_prefill_chunk", ctypes.c_int, _DESC, _STATE, _P, _P, _P, _I32, _P, _P, ctypes.c_size_t, _P)
-_lib_mix = _fn("duo_gated_mix", ctypes.c_int, _DESC, _P, _P, _P, _P, _I32, _P, _P)
-_lib_mix_grad = _fn("duo_gated_mix_grad_alpha", ctypes.c_int, _DESC, _P, _P, _P, _I32, _P, _P, _P)
+_lib_mix = _fn("duo_gated_mix", ctypes.c_int, _DESC, _P, _P, _P, _P, _I32, _P, _P, _P)
+_lib_mix_grad = _fn("duo_gated_mix_grad_alpha", ctypes.c_int, _DESC, _P, _P, _P, _I32, _P, _P, _P, _P)
+_lib_wait_probe = _fn("duo_wait_probe", ctypes.c_int, _P, ctypes.c_uint32, _P)
 _lib_check = _fn("duo_check_status", ctypes.c_int, _STATE, ctypes.POINTER(_I32), _P)
 _lib_decode_step = _fn("duo_decode_step", ctypes.c_int, _DESC, _STATE, _P, _P, _P, _P, _P, ctypes.c_size_t, _P)
 _lib_decode_noalloc = _fn("duo_decode_attn_noalloc", ctypes.c_int, _DESC, _STATE, _P, _P, _P)
@@ -218,14 +219,21 @@ def prefill_chunk(desc, state: KVState, q, k_chunk, v_chunk, C: int, out, worksp
                         _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)), "duo_prefill_chunk")
 
 
-def gated_mix(desc, alpha, q, k, v, N: int, out, stream=None) -> None:
-    _check(_lib_mix(ctypes.byref(desc), _ptr(alpha), _ptr(q), _ptr(k), _ptr(v), N, _ptr(out), _stream(stream)),
-           "duo_gated_mix")
+def gated_mix(desc, alpha, q, k, v, N: int, out, status, stream=None) -> None:
+    """status: an int32 device word; DUO_DEV_* bits are ORed into it."""
+    _check(_lib_mix(ctypes.byref(desc), _ptr(alpha), _ptr(q), _ptr(k), _ptr(v), N, _ptr(out), _ptr(status),
+                    _stream(stream)), "duo_gated_mix")
 
 
-def gated_mix_grad_alpha(desc, q, k, v, N: int, dout, dalpha, stream=None) -> None:
-    _check(_lib_mix_grad(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), N, _ptr(dout), _ptr(dalpha),
+def gated_mix_grad_alpha(desc, q, k, v, N: int, dout, dalpha, status, stream=None) -> None:
+    _check(_lib_mix_grad(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), N, _ptr(dout), _ptr(dalpha), _ptr(status),
                          _stream(stream)), "duo_gated_mix_grad_alpha")
+
+
+def wait_probe(status, limit_us: int, stream=None) -> None:
+    """One warp runs the library's bounded device wait on a barrier nothing
+    completes; DUO_DEV_WAIT_TIMEOUT is ORed into the int32 device word `status`."""
+    _check(_lib_wait_probe(_ptr(status), limit_us, _stream(stream)), "duo_wait_probe")
 
 
 def exp2_fma_probe(x, y, n: int, stream=None) -> None:

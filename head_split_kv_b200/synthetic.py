@@ -17,6 +17,8 @@ or datasets are used.
 
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass
 
 import numpy as np
@@ -34,42 +36,65 @@ def rng_for(seed: int, stream: int, *extra: int) -> np.random.Generator:
 
 
 def to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """float32 -> bfloat16 bit patterns (uint16), round to nearest even."""
-    x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    return u.astype(np.uint16)
+    """float32 -> bfloat16 bit patterns (uint16), round to nearest even.
+    For finite values and infinities (the generators draw no NaN) the
+    rounding increment never carries out of 32 bits."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    r = (u >> np.uint32(16)) & np.uint32(1)
+    return ((u + (np.uint32(0x7FFF) + r)) >> np.uint32(16)).astype(np.uint16)
 
 
-def normal(rng: np.random.Generator, shape, dtype: str, block: int = 1 << 24) -> np.ndarray:
-    """N(0, 1) samples as float32 or bf16 bits, generated in blocks to bound
-    host memory."""
+_BLOCK = 1 << 22      # values per generator block
+_pool = None
+
+
+def _threads():
+    global _pool
+    if _pool is None:
+        _pool = ThreadPoolExecutor(max_workers=max(1, min(32, os.cpu_count() or 1)))
+    return _pool
+
+
+def _fill_normal(rng: np.random.Generator, n: int, dtype: str, sigma=None) -> np.ndarray:
+    """n samples of N(0, sigma^2) (sigma = 1 when None), as float32 or bf16
+    bits.  The caller's generator gives one seed; block i of _BLOCK values
+    comes from its own generator seeded (that seed, i), so the blocks are
+    drawn in parallel threads and the result does not depend on how many."""
+    base = int(rng.integers(0, 2 ** 63 - 1))
+    out = np.empty(n, dtype=np.uint16 if dtype == "bf16" else np.float32)
+
+    def fill(i):
+        s, e = i * _BLOCK, min(n, (i + 1) * _BLOCK)
+        x = np.random.default_rng([base, i]).standard_normal(e - s, dtype=np.float32)
+        if sigma is not None:
+            x *= np.float32(sigma)
+        out[s:e] = to_bf16_bits(x) if dtype == "bf16" else x
+
+    nb = (n + _BLOCK - 1) // _BLOCK
+    if nb == 1:
+        fill(0)
+    elif nb > 1:
+        list(_threads().map(fill, range(nb)))
+    return out
+
+
+def normal(rng: np.random.Generator, shape, dtype: str) -> np.ndarray:
+    """N(0, 1) samples of the given shape as float32 or bf16 bits."""
     shape = tuple(int(s) for s in shape)
     n = int(np.prod(shape)) if shape else 1
-    out = np.empty(n, dtype=np.uint16 if dtype == "bf16" else np.float32)
-    for s in range(0, n, block):
-        e = min(n, s + block)
-        x = rng.standard_normal(e - s, dtype=np.float32)
-        out[s:e] = to_bf16_bits(x) if dtype == "bf16" else x
-    return out.reshape(shape)
+    return _fill_normal(rng, n, dtype).reshape(shape)
 
 
 def normal_scaled(rng: np.random.Generator, shape, dtype: str, sigma_per_head: np.ndarray,
-                  head_axis: int, block_rows: int = 1 << 16) -> np.ndarray:
+                  head_axis: int) -> np.ndarray:
     """N(0, sigma_h^2) samples where sigma depends on the index along ``head_axis``."""
     shape = tuple(int(s) for s in shape)
+    rest = tuple(s for i, s in enumerate(shape) if i != head_axis)
+    per = int(np.prod(rest)) if rest else 1
     x = np.empty(shape, dtype=np.uint16 if dtype == "bf16" else np.float32)
     xm = np.moveaxis(x, head_axis, 0)
     for h in range(shape[head_axis]):
-        sub = xm[h]
-        flat = sub.reshape(-1)
-        n = flat.shape[0]
-        blk = block_rows * shape[-1]
-        for s in range(0, n, blk):
-            e = min(n, s + blk)
-            v = rng.standard_normal(e - s, dtype=np.float32) * np.float32(sigma_per_head[h])
-            flat[s:e] = to_bf16_bits(v) if dtype == "bf16" else v
-        xm[h] = flat.reshape(sub.shape)
+        xm[h] = _fill_normal(rng, per, dtype, float(sigma_per_head[h])).reshape(rest)
     return x
 
 
@@ -142,41 +167,77 @@ def context_lengths(batch: int, lo: int, hi: int, seed: int = 0) -> np.ndarray:
     return rng_for(seed, _S_LEN).integers(lo, hi + 1, batch).astype(np.int64)
 
 
-def decode_state(shape: LayerShape, retrieval, lengths, seed: int = 0, sigma=None):
-    """Cache contents after a prompt of ``lengths[b]`` tokens, per model KV head.
+STREAM_BLOCK = 1024   # positions per generator block of a streaming head's rows
 
-    Returns a dict with, for each sequence b and KV head h:
-      full[(b, h)]   = (k [L_b, d], v [L_b, d]) for a retrieval head, positions 0..L_b-1
-      stream[(b, h)] = (pos [n], k [n, d], v [n, d]) for a streaming head, the
-                       surviving positions: 0..min(L, sink)-1 and the last
-                       ``recent`` positions
-    A streaming head never keeps the other tokens, so they are not drawn.
+
+class DecodeState:
+    """Seeded rows of a cache state after a prompt of ``lengths[b]`` tokens.
+
+    ``full[(b, h)] = (k [L_b, d], v [L_b, d])`` for every retrieval KV head h:
+    the rows of positions 0..L_b-1.  A streaming KV head's rows are drawn on
+    demand by ``stream_rows(b, h, positions)``: the row of position p comes
+    from the generator of its block of ``STREAM_BLOCK`` positions, so any set
+    of positions gets the same row for p whichever other positions are asked
+    for.  Which positions a streaming cache still holds is not decided here:
+    that is the method's eviction rule, which each side applies itself.
     """
-    retrieval = set(int(h) for h in retrieval)
-    d = shape.head_dim
-    full, stream = {}, {}
-    for b, L in enumerate(np.asarray(lengths, dtype=np.int64)):
-        L = int(L)
-        for h in range(shape.n_kv_heads):
-            sig = None if sigma is None else np.asarray([sigma[h]], dtype=np.float32)
-            if h in retrieval:
+
+    def __init__(self, shape: LayerShape, retrieval, lengths, seed: int = 0, sigma=None):
+        self.shape = shape
+        self.retrieval = sorted(int(h) for h in retrieval)
+        self.lengths = np.asarray(lengths, dtype=np.int64)
+        self.seed = int(seed)
+        self.sigma = None if sigma is None else np.asarray(sigma, dtype=np.float32)
+        self.full = {}
+        for b, L in enumerate(self.lengths):
+            L = int(L)
+            for h in self.retrieval:
                 rk, rv = rng_for(seed, _S_K, b, h), rng_for(seed, _S_V, b, h)
-                if sig is None:
-                    full[(b, h)] = (normal(rk, (L, d), shape.dtype), normal(rv, (L, d), shape.dtype))
-                else:
-                    full[(b, h)] = (normal_scaled(rk, (1, L, d), shape.dtype, sig, 0)[0],
-                                    normal_scaled(rv, (1, L, d), shape.dtype, sig, 0)[0])
+                self.full[(b, h)] = (self._draw(rk, L, h), self._draw(rv, L, h))
+
+    def _draw(self, rng, n: int, h: int) -> np.ndarray:
+        d = self.shape.head_dim
+        if self.sigma is None:
+            return normal(rng, (n, d), self.shape.dtype)
+        return normal_scaled(rng, (1, n, d), self.shape.dtype, self.sigma[h:h + 1], 0)[0]
+
+    def stream_rows(self, b: int, h: int, positions):
+        """(k [n, d], v [n, d]) of a streaming KV head at the given positions."""
+        pos = np.asarray(positions, dtype=np.int64)
+        d = self.shape.head_dim
+        dt = np.uint16 if self.shape.dtype == "bf16" else np.float32
+        k = np.empty((len(pos), d), dtype=dt)
+        v = np.empty_like(k)
+        for blk in np.unique(pos // STREAM_BLOCK):
+            sel = np.flatnonzero(pos // STREAM_BLOCK == blk)
+            kb = self._draw(rng_for(self.seed, _S_KSTREAM, b, h, int(blk)), STREAM_BLOCK, h)
+            vb = self._draw(rng_for(self.seed, _S_VSTREAM, b, h, int(blk)), STREAM_BLOCK, h)
+            k[sel] = kb[pos[sel] % STREAM_BLOCK]
+            v[sel] = vb[pos[sel] % STREAM_BLOCK]
+        return k, v
+
+    def token_rows(self, b: int, positions):
+        """k, v [n, Hkv, d] of every KV head at the given positions of sequence
+        b (model head order): a retrieval head's cached rows, a streaming
+        head's drawn rows."""
+        pos = np.asarray(positions, dtype=np.int64)
+        sh = self.shape
+        dt = np.uint16 if sh.dtype == "bf16" else np.float32
+        k = np.empty((len(pos), sh.n_kv_heads, sh.head_dim), dtype=dt)
+        v = np.empty_like(k)
+        for h in range(sh.n_kv_heads):
+            if (b, h) in self.full:
+                k[:, h] = self.full[(b, h)][0][pos]
+                v[:, h] = self.full[(b, h)][1][pos]
             else:
-                keep = sorted(set(range(min(L, shape.sink))) | set(range(max(0, L - shape.recent), L)))
-                pos = np.asarray(keep, dtype=np.int64)
-                rk, rv = rng_for(seed, _S_KSTREAM, b, h), rng_for(seed, _S_VSTREAM, b, h)
-                n = len(pos)
-                if sig is None:
-                    stream[(b, h)] = (pos, normal(rk, (n, d), shape.dtype), normal(rv, (n, d), shape.dtype))
-                else:
-                    stream[(b, h)] = (pos, normal_scaled(rk, (1, n, d), shape.dtype, sig, 0)[0],
-                                      normal_scaled(rv, (1, n, d), shape.dtype, sig, 0)[0])
-    return dict(full=full, stream=stream, lengths=np.asarray(lengths, dtype=np.int64))
+                k[:, h], v[:, h] = self.stream_rows(b, h, pos)
+        return k, v
+
+
+def decode_state(shape: LayerShape, retrieval, lengths, seed: int = 0, sigma=None) -> DecodeState:
+    """Rows of a cache state after a prompt of ``lengths[b]`` tokens per
+    sequence (see DecodeState)."""
+    return DecodeState(shape, retrieval, lengths, seed=seed, sigma=sigma)
 
 
 def decode_steps(shape: LayerShape, batch: int, steps: int, seed: int = 0, sigma=None, first: int = 0):

@@ -173,8 +173,9 @@ typedef struct {
 const char* duo_last_error(void);
 /* Name of a status code. */
 const char* duo_status_string(duo_status s);
-/* ABI version: 3 (duo_layer_desc gained stream_prefill and kv_quant,
- * duo_kv_state the 8-bit cache's scales). */
+/* ABI version: 4 (duo_gated_mix and duo_gated_mix_grad_alpha take a device
+ * status word; version 3 added stream_prefill, kv_quant and the 8-bit
+ * cache's scales). */
 int32_t duo_abi_version(void);
 
 /* ------------------------------------------------------------------------ */
@@ -360,10 +361,16 @@ duo_status duo_prefill_chunk(const duo_layer_desc* desc, const duo_kv_state* st,
  * the causal attention mixed with it as it is stored), so out must not alias
  * q, k or v; other dtypes and head sizes run on the CUDA cores, one pass over
  * Q K^T feeding both softmax states.
+ * status: one int32 device word (required), caller-owned; the call only ORs
+ *   DUO_DEV_* bits into it.  A bounded device wait that runs out sets
+ *   DUO_DEV_WAIT_TIMEOUT there and the rows it guarded are not written, so a
+ *   caller that reads the word back after the call (zeroed before it) knows
+ *   whether out is complete.  The call itself does not read it back.
  * Errors: DUO_ERR_INVALID_ARG, DUO_ERR_SHAPE, DUO_ERR_UNSUPPORTED, DUO_ERR_CUDA.
  */
 duo_status duo_gated_mix(const duo_layer_desc* desc, const float* alpha, const void* q,
-                         const void* k, const void* v, int32_t N, void* out, duo_stream_t stream);
+                         const void* k, const void* v, int32_t N, void* out, int32_t* status,
+                         duo_stream_t stream);
 
 /*
  * duo_decode_attn_noalloc -- duo_decode_attn without a caller workspace.
@@ -411,17 +418,19 @@ duo_status duo_decode_attn_noalloc(const duo_layer_desc* desc, const duo_kv_stat
  * model head order as for duo_gated_mix.  dalpha [Hkv] fp32 device: zeroed
  * by the call, then accumulated with atomics (one add per 32 rows), so the
  * last bits vary with the order the CTAs finish in.
+ * status: one int32 device word (required), as for duo_gated_mix.
  * Errors: DUO_ERR_INVALID_ARG, DUO_ERR_SHAPE, DUO_ERR_UNSUPPORTED, DUO_ERR_CUDA.
  */
 duo_status duo_gated_mix_grad_alpha(const duo_layer_desc* desc, const void* q, const void* k, const void* v,
-                                    int32_t N, const void* dout, float* dalpha, duo_stream_t stream);
+                                    int32_t N, const void* dout, float* dalpha, int32_t* status,
+                                    duo_stream_t stream);
 
 /*
  * duo_exp2_fma_probe -- y[i] = the pre-fill softmax's FMA-pipe 2^x of x[i]
  * (Cody-Waite range reduction to x = n + f, f in [-0.5, 0.5], a fitted cubic
  * for 2^f and n added to the exponent field; inputs below -125, -inf
  * included, give the value at -125, 2^-125 within the cubic's 7.5e-5).
- * duo_prefill_chunk computes one exponential pair in four this way and the
+ * duo_prefill_chunk computes one exponential pair in eight this way and the
  * rest on the SFU; this entry point exposes the routine so that its error
  * can be checked against 2^x.  It is not a step of the attention path: the
  * paper review's S3 "Core formula" only fixes the softmax, not how its
@@ -431,6 +440,22 @@ duo_status duo_gated_mix_grad_alpha(const duo_layer_desc* desc, const void* q, c
  * Errors: DUO_ERR_INVALID_ARG (NULL with n > 0, n < 0), DUO_ERR_CUDA.
  */
 duo_status duo_exp2_fma_probe(const float* x, float* y, int64_t n, duo_stream_t stream);
+
+/*
+ * duo_wait_probe -- runs the library's bounded device wait to its limit, so
+ * that its failure path can be observed.  Not a step of the attention path
+ * (the pages describe no device waits): the kernels wait on mbarriers for
+ * their tensor copies and MMAs, each wait bounded in wall time (2 s), after
+ * which it ORs DUO_DEV_WAIT_TIMEOUT into the status word and the kernel
+ * skips what the wait guarded instead of hanging.  This probe launches one
+ * warp that waits, through that same routine, on an mbarrier nothing ever
+ * arrives on, with a limit of limit_us microseconds; nothing else is in
+ * flight, so the kernel then simply returns.
+ * status: one int32 device word, caller-owned; DUO_DEV_WAIT_TIMEOUT is ORed
+ *   into it.  limit_us in 1..1000000.  Asynchronous on `stream`.
+ * Errors: DUO_ERR_INVALID_ARG, DUO_ERR_CUDA.
+ */
+duo_status duo_wait_probe(int32_t* status, uint32_t limit_us, duo_stream_t stream);
 
 /*
  * duo_check_status -- synchronise `stream`, copy the state's device status

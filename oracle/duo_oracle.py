@@ -83,6 +83,7 @@ __all__ = [
     "binarize_gates",
     "partition_heads",
     "ring_slot",
+    "streaming_positions",
     "HeadSplitCache",
     "prefill_direct",
     "decode_direct",
@@ -332,6 +333,29 @@ def dequantize_int8_rows(codes, scales) -> np.ndarray:
     return np.asarray(codes, dtype=np.float64) * np.asarray(scales, dtype=np.float64)[:, None]
 
 
+def _streaming_push(lst: list, entry: tuple, sink: int, recent: int) -> None:
+    """Append one (position, ...) entry to a streaming head's list; when the
+    list grows past sink + recent, evict the oldest token that is not an
+    attention sink [Review S3 "Inference flow": a streaming head keeps only
+    the sink tokens and the recent tokens]."""
+    lst.append(entry)
+    if len(lst) > sink + recent:
+        for e in range(len(lst)):
+            if lst[e][0] >= sink:
+                del lst[e]
+                break
+
+
+def streaming_positions(length: int, sink: int, recent: int) -> np.ndarray:
+    """Positions a streaming head's list holds after tokens 0..length-1 were
+    appended one by one: the same pushes and evictions as
+    ``HeadSplitCache.append``, on positions alone."""
+    lst = []
+    for p in range(int(length)):
+        _streaming_push(lst, (p,), sink, recent)
+    return np.array([e[0] for e in lst], dtype=np.int64)
+
+
 @dataclass
 class HeadSplitCache:
     """Per-layer caches for a batch: full lists for retrieval heads, a
@@ -379,13 +403,8 @@ class HeadSplitCache:
                 else:
                     lst = self.stream[b][h]
                     for i in range(t):
-                        lst.append((int(pos[i]), k_new[b, i, h].copy(), v_new[b, i, h].copy()))
-                        if len(lst) > self.sink + self.recent:
-                            # evict the oldest token that is not an attention sink
-                            for e in range(len(lst)):
-                                if lst[e][0] >= self.sink:
-                                    del lst[e]
-                                    break
+                        _streaming_push(lst, (int(pos[i]), k_new[b, i, h].copy(), v_new[b, i, h].copy()),
+                                        self.sink, self.recent)
             self.length[b] = p0 + t
 
     def load_state(self, b: int, h: int, pos, k, v) -> None:

@@ -92,13 +92,17 @@ class Layer:
         return np.take(x, idx, axis=axis)
 
     # -- state ----------------------------------------------------------------
-    def load_state(self, st: dict) -> None:
-        """Install a synthetic.decode_state() on the device and in the oracle."""
+    def load_state(self, st) -> None:
+        """Install a synthetic.DecodeState on the device and in the oracle.
+        Retrieval heads hold every row of the prompt; a streaming head holds
+        the positions the oracle's eviction rule keeps after the prompt
+        (replayed on positions alone), with their seeded rows, placed in the
+        ring slots by the oracle's slot function."""
         t = torch()
         c = self.caches
         sh = self.shape
         ring_pos = np.full((self.B, sh.sink + sh.recent), -1, dtype=np.int32)
-        for (b, h), (k, v) in st["full"].items():
+        for (b, h), (k, v) in st.full.items():
             r = self.inv[h]
             L = k.shape[0]
             if self.page_table is None:
@@ -111,18 +115,27 @@ class Layer:
                 c.k_full[pages, r, rows] = to_dev(k)
                 c.v_full[pages, r, rows] = to_dev(v)
             self.oracle.load_state(b, h, np.arange(L), k, v)
-        for (b, h), (pos, k, v) in st["stream"].items():
-            s = self.inv[h] - self.R
+        kept = {}
+        for b, L in enumerate(st.lengths):
+            L = int(L)
+            if L not in kept:
+                kept[L] = O.streaming_positions(L, sh.sink, sh.recent)
+            pos = kept[L]
             slots = np.array([O.ring_slot(int(p), sh.sink, sh.recent) for p in pos], dtype=np.int64)
-            if len(slots):
-                idx = t.from_numpy(slots).cuda()
-                c.k_ring[b, s, idx] = to_dev(k)
-                c.v_ring[b, s, idx] = to_dev(v)
-                ring_pos[b, slots] = pos
-            self.oracle.load_state(b, h, pos, k, v)
+            for h in range(sh.n_kv_heads):
+                if self.gate[h]:
+                    continue
+                k, v = st.stream_rows(b, h, pos)
+                s = self.inv[h] - self.R
+                if len(slots):
+                    idx = t.from_numpy(slots).cuda()
+                    c.k_ring[b, s, idx] = to_dev(k)
+                    c.v_ring[b, s, idx] = to_dev(v)
+                    ring_pos[b, slots] = pos
+                self.oracle.load_state(b, h, pos, k, v)
         c.ring_pos.copy_(t.from_numpy(ring_pos))
-        c.seq_len.copy_(t.from_numpy(st["lengths"].astype(np.int32)))
-        for b, L in enumerate(st["lengths"]):
+        c.seq_len.copy_(t.from_numpy(st.lengths.astype(np.int32)))
+        for b, L in enumerate(st.lengths):
             self.oracle.set_length(b, int(L))
 
     # -- calls ------------------------------------------------------------------

@@ -64,7 +64,7 @@ int main(void) {
 
 
 def test_abi_version_and_status_strings(duo):
-    assert duo.abi_version() == duo.ABI_VERSION == 3
+    assert duo.abi_version() == duo.ABI_VERSION == 4
     assert duo.status_string(duo.OK) == "DUO_OK"
     assert duo.status_string(duo.ERR_CAPACITY) == "DUO_ERR_CAPACITY"
 
@@ -256,9 +256,15 @@ def test_prefill_rejects(duo):
 def test_gated_mix_rejects(duo):
     d = _desc(duo)
     with pytest.raises(duo.DuoError) as e:
-        duo.gated_mix(d, None, 256, 512, 768, 10, 1024, stream=0)
+        duo.gated_mix(d, None, 256, 512, 768, 10, 1024, 2048, stream=0)
     assert e.value.status == duo.ERR_INVALID_ARG
-    duo.gated_mix(d, 16, 256, 512, 768, 0, 1024, stream=0)       # N = 0: nothing to do
+    with pytest.raises(duo.DuoError) as e:                          # the status word is required
+        duo.gated_mix(d, 16, 256, 512, 768, 10, 1024, None, stream=0)
+    assert e.value.status == duo.ERR_INVALID_ARG
+    with pytest.raises(duo.DuoError) as e:
+        duo.gated_mix_grad_alpha(d, 256, 512, 768, 10, 1024, 2048, None, stream=0)
+    assert e.value.status == duo.ERR_INVALID_ARG
+    duo.gated_mix(d, 16, 256, 512, 768, 0, 1024, 2048, stream=0)       # N = 0: nothing to do
 
 
 def test_gated_mix_rejects_out_overlapping_an_input(duo):
@@ -268,9 +274,16 @@ def test_gated_mix_rejects_out_overlapping_an_input(duo):
     q, k, v = 1 << 20, 2 << 20, 3 << 20
     for out in (q, q + 4096, k - 4096, v + 16):
         with pytest.raises(duo.DuoError) as e:
-            duo.gated_mix(d, 16, q, k, v, 10, out, stream=0)
+            duo.gated_mix(d, 16, q, k, v, 10, out, 64, stream=0)
         assert e.value.status == duo.ERR_INVALID_ARG
         assert "overlaps" in duo.last_error()
+
+
+def test_wait_probe_rejects(duo):
+    for status, limit in ((None, 10), (64, 0), (64, 1000001)):
+        with pytest.raises(duo.DuoError) as e:
+            duo.wait_probe(status, limit, stream=0)
+        assert e.value.status == duo.ERR_INVALID_ARG
 
 
 def test_permute_rejects_overlap(duo):

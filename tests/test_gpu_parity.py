@@ -219,15 +219,23 @@ def test_decode_mha_32k_full(duo, fused):
 @pytest.mark.slow
 @pytest.mark.parametrize("L0", [131072, 1048576])
 def test_decode_gqa_long_full(duo, L0):
+    """The 128K and 1M GQA decode workloads: outputs against the oracle on
+    sampled steps, then every cache byte (the full caches past 2^20 rows
+    included), the rings, ring positions and lengths against its lists."""
     sh = S.LayerShape(32, 8, 128, "bf16")
-    _decode_run(duo, sh, S.retrieval_heads_by_seed(8, 4), [L0], 64, {0, 31, 63}, sigma=S.head_sigma(8), fused=True)
+    lay, _ = _decode_run(duo, sh, S.retrieval_heads_by_seed(8, 4), [L0], 64, {0, 31, 63}, sigma=S.head_sigma(8),
+                         fused=True)
+    lay.assert_caches_match()
 
 
 @pytest.mark.slow
 def test_decode_batch64_paged_full(duo):
+    """64 sequences of 4K..32K tokens in 64-token pages scattered over the
+    pool: outputs on sampled steps, then every page against the oracle."""
     sh = S.LayerShape(32, 32, 128, "bf16")
     lengths = S.context_lengths(64, 4096, 32768, seed=0)
-    _decode_run(duo, sh, S.retrieval_heads_by_seed(32, 8), lengths, 32, {0, 31}, paged=True, fused=True)
+    lay, _ = _decode_run(duo, sh, S.retrieval_heads_by_seed(32, 8), lengths, 32, {0, 31}, paged=True, fused=True)
+    lay.assert_caches_match()
 
 
 # ---------------------------------------------------------------------------
@@ -297,7 +305,9 @@ def test_gated_mix_tiny_fp32(duo):
     q, k, v = (to_dev(w[x][None]) for x in ("q", "k", "v"))
     out = t.empty_like(q)
     alpha = t.from_numpy(w["alpha_mix"]).cuda()
-    duo.gated_mix(desc, alpha, q, k, v, 512, out)
+    status = t.zeros(1, dtype=t.int32, device="cuda")
+    duo.gated_mix(desc, alpha, q, k, v, 512, out, status)
+    assert status.item() == 0
     want = O.gated_mix(w["q"], w["k"], w["v"], w["alpha_mix"].astype(np.float64), sh.sink, sh.recent)
     assert_close(f64(out)[0], want, "fp32", "gated mix")
 
@@ -311,7 +321,9 @@ def test_gated_mix_bf16_gqa(duo, alpha_kind):
     alpha = alpha.astype(np.float32)
     desc = duo.desc_init(2, 16, 4, 128, duo.BF16, [0, 1, 2, 3], 0)
     out = t.empty_like(to_dev(q))
-    duo.gated_mix(desc, t.from_numpy(alpha).cuda(), to_dev(q), to_dev(k), to_dev(v), 333, out)
+    status = t.zeros(1, dtype=t.int32, device="cuda")
+    duo.gated_mix(desc, t.from_numpy(alpha).cuda(), to_dev(q), to_dev(k), to_dev(v), 333, out, status)
+    assert status.item() == 0
     got = f64(out)
     for b in range(2):
         want = O.gated_mix(q[b], k[b], v[b], alpha.astype(np.float64), sh.sink, sh.recent)
@@ -330,7 +342,9 @@ def test_gated_mix_bf16_tensor_core_path(duo, hq, hkv, n, B):
     alpha[0], alpha[-1] = 1.0, 0.0
     desc = duo.desc_init(B, hq, hkv, 128, duo.BF16, list(range(hkv)), 0)
     out = t.empty_like(to_dev(q))
-    duo.gated_mix(desc, t.from_numpy(alpha).cuda(), to_dev(q), to_dev(k), to_dev(v), n, out)
+    status = t.zeros(1, dtype=t.int32, device="cuda")
+    duo.gated_mix(desc, t.from_numpy(alpha).cuda(), to_dev(q), to_dev(k), to_dev(v), n, out, status)
+    assert status.item() == 0
     got = f64(out)
     for b in range(B):
         want = O.gated_mix(q[b], k[b], v[b], alpha.astype(np.float64), sh.sink, sh.recent)
@@ -357,7 +371,9 @@ def test_gated_mix_grad_alpha_tiny_fp32(duo):
     q, k, v = (to_dev(w[x][None]) for x in ("q", "k", "v"))
     dout = S.rng_for(9, 60).standard_normal((1, 512, 8, 64)).astype(np.float32)
     dalpha = t.full((8,), 7.0, dtype=t.float32, device="cuda")      # overwritten by the call
-    duo.gated_mix_grad_alpha(desc, q, k, v, 512, to_dev(dout), dalpha)
+    status = t.zeros(1, dtype=t.int32, device="cuda")
+    duo.gated_mix_grad_alpha(desc, q, k, v, 512, to_dev(dout), dalpha, status)
+    assert status.item() == 0
     want = O.gated_mix_grad_alpha(w["q"], w["k"], w["v"], dout[0], sh.sink, sh.recent)
     _grad_check(dalpha.cpu().numpy().astype(np.float64), want, dout.astype(np.float64), 1, 1e-4)
 
@@ -369,7 +385,9 @@ def test_gated_mix_grad_alpha_bf16_gqa_batch(duo):
     dout = S.normal(S.rng_for(4, 61), (2, 333, 16, 128), "bf16")
     desc = duo.desc_init(2, 16, 4, 128, duo.BF16, [0, 1, 2, 3], 0)
     dalpha = t.empty((4,), dtype=t.float32, device="cuda")
-    duo.gated_mix_grad_alpha(desc, to_dev(q), to_dev(k), to_dev(v), 333, to_dev(dout), dalpha)
+    status = t.zeros(1, dtype=t.int32, device="cuda")
+    duo.gated_mix_grad_alpha(desc, to_dev(q), to_dev(k), to_dev(v), 333, to_dev(dout), dalpha, status)
+    assert status.item() == 0
     want = sum(O.gated_mix_grad_alpha(q[b], k[b], v[b], dout[b], sh.sink, sh.recent) for b in range(2))
     _grad_check(dalpha.cpu().numpy().astype(np.float64), want, O.as_f64(dout), 4, 2e-3)
 
@@ -383,7 +401,9 @@ def test_gated_mix_grad_alpha_zero_when_window_covers_sequence(duo):
     dout = S.normal(S.rng_for(5, 62), (1, 80, 8, 64), "bf16")
     desc = duo.desc_init(1, 8, 4, 64, duo.BF16, [0, 1, 2, 3], 0)
     dalpha = t.empty((4,), dtype=t.float32, device="cuda")
-    duo.gated_mix_grad_alpha(desc, to_dev(q), to_dev(k), to_dev(v), 80, to_dev(dout), dalpha)
+    status = t.zeros(1, dtype=t.int32, device="cuda")
+    duo.gated_mix_grad_alpha(desc, to_dev(q), to_dev(k), to_dev(v), 80, to_dev(dout), dalpha, status)
+    assert status.item() == 0
     assert t.count_nonzero(dalpha).item() == 0
 
 

@@ -68,18 +68,20 @@ def test_prefill_tc_gqa_chunkings(duo, chunks):
 
 def _history(sh, st, b, L, k_new, v_new):
     """Token history [L + C, Hkv, d] of sequence b: the decode state's rows
-    (zeros where a streaming head kept nothing -- the Lambda mask never reads
-    those positions from a later query) followed by the chunk's rows."""
+    (a streaming head: the positions the oracle's eviction rule keeps, zeros
+    elsewhere -- the Lambda mask never reads those positions from a later
+    query) followed by the chunk's rows."""
     C = k_new.shape[0]
     k_all = np.zeros((L + C, sh.n_kv_heads, sh.head_dim), dtype=np.float64)
     v_all = np.zeros_like(k_all)
+    kept = O.streaming_positions(L, sh.sink, sh.recent)
     for h in range(sh.n_kv_heads):
-        if (b, h) in st["full"]:
-            k, v = st["full"][(b, h)]
+        if (b, h) in st.full:
+            k, v = st.full[(b, h)]
             k_all[:L, h], v_all[:L, h] = O.as_f64(k), O.as_f64(v)
         else:
-            pos, k, v = st["stream"][(b, h)]
-            k_all[pos, h], v_all[pos, h] = O.as_f64(k), O.as_f64(v)
+            k, v = st.stream_rows(b, h, kept)
+            k_all[kept, h], v_all[kept, h] = O.as_f64(k), O.as_f64(v)
     k_all[L:], v_all[L:] = O.as_f64(k_new), O.as_f64(v_new)
     return k_all, v_all
 
@@ -170,11 +172,47 @@ def test_prefill_tc_gqa_eight_way_split(duo):
 
 
 @pytest.mark.slow
-def test_prefill_gqa_131k_full(duo):
-    """The full workload the bench times: 131,072 tokens in 32 chunks of 4,096,
-    sampled rows in every chunk; caches compared at the end."""
+def test_prefill_gqa_131k_full(duo, tmp_path):
+    """The full workload the bench times, in its launch configuration: a
+    131,072-token prompt in 32 chunks of 4,096 with the bench's workspace.
+    Every row of chunks 0, 1 and 31 and 512 seeded rows of every other chunk
+    (plus each chunk's first and last row) are compared with the oracle,
+    whose rows a spawned process pool computes while the GPU runs; the caches
+    are compared byte for byte at the end."""
+    from tests.oracle_pool import PrefillOracle
+    t = torch()
     sh = S.LayerShape(32, 8, 128, "bf16")
-    _run(duo, sh, S.retrieval_heads_by_seed(8, 4), 131072, [4096] * 32, sample_rows=24)
+    n, C = 131072, 4096
+    n_chunks = n // C
+    lay = Layer(duo, sh, S.retrieval_heads_by_seed(8, 4), 1, capacity=n + 16)
+    ws = duo.Workspace(lay.desc, duo.OP_PREFILL, C)
+    q, k, v = S.prompt(sh, n, seed=0)
+    rng = S.rng_for(0, 77)
+    rows = {}
+    for ci in range(n_chunks):
+        if ci in (0, 1, n_chunks - 1):
+            rows[ci] = np.arange(C)
+        else:
+            rows[ci] = np.unique(np.concatenate([[0, C - 1], rng.choice(C, 512, replace=False)]))
+    ora = PrefillOracle(tmp_path, q[0], k[0], v[0], lay.gate, sh.sink, sh.recent)
+    for ci in sorted(rows, key=lambda c: -(c + 1) * len(rows[c])):     # the longest jobs first
+        ora.submit(ci * C, C, rows[ci])
+    got = {}
+    for ci in range(n_chunks):
+        c0 = ci * C
+        qd, kd, vd = (to_dev(np.ascontiguousarray(x[:, c0:c0 + C])) for x in (q, k, v))
+        out = t.empty_like(qd)
+        duo.prefill_chunk(lay.desc, lay.caches.state, qd, kd, vd, C, out, ws.ptr, ws.nbytes)
+        duo.append_kv(lay.desc, lay.caches.state, kd, vd, C)
+        lay.oracle.append(k[:, c0:c0 + C], v[:, c0:c0 + C])
+        got[c0] = f64(out[0].index_select(0, t.from_numpy(rows[ci]).cuda()))
+    assert lay.status() == 0
+    lay.assert_caches_match()
+    want = ora.results()
+    for ci in range(n_chunks):
+        r, w = want[ci * C]
+        assert np.array_equal(r, rows[ci])
+        assert_close(got[ci * C], w, "bf16", f"chunk {ci} ({len(r)} rows)")
 
 
 def test_exp2_fma_probe_error_bound(duo):

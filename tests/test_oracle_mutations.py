@@ -45,6 +45,7 @@ def _pins():
         lambda: P.test_ring_positions_match_hand_table(g),
         lambda: P.test_ring_after_block_append_equals_token_by_token(g),
         lambda: P.test_streaming_cache_stays_constant_size(0),
+        lambda: P.test_streaming_positions_are_the_sinks_and_the_recent_tokens(3, 9),
         P.test_decode_after_prefill_equals_direct_row,
         lambda: P.test_chunked_prefill_from_caches_equals_direct(7),
         P.test_partition_by_threshold,
@@ -152,6 +153,29 @@ def test_planted_mistake_is_caught(monkeypatch, name, fn):
 
 def test_planted_eviction_mistake_is_caught(monkeypatch):
     monkeypatch.setattr(D.HeadSplitCache, "append", _append_evicts_sinks)
+    assert _fails(*_pins())
+
+
+def _push_evicts_sinks(lst, entry, sink, recent):
+    lst.append(entry)
+    if len(lst) > sink + recent:
+        del lst[0]                              # the mistake: sinks are evicted too
+
+
+def _push_keeps_one_too_many(lst, entry, sink, recent):
+    lst.append(entry)
+    if len(lst) > sink + recent + 1:            # the mistake: the window is one token long
+        for e in range(len(lst)):
+            if lst[e][0] >= sink:
+                del lst[e]
+                break
+
+
+@pytest.mark.parametrize("fn", [_push_evicts_sinks, _push_keeps_one_too_many])
+def test_planted_push_mistake_is_caught(monkeypatch, fn):
+    """A mistake in the shared eviction step shows in the appends and in the
+    replayed positions alike."""
+    monkeypatch.setattr(D, "_streaming_push", fn)
     assert _fails(*_pins())
 
 

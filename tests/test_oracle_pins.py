@@ -369,6 +369,8 @@ def test_decode_after_prefill_equals_direct_row():
 
 
 def test_load_state_equals_replayed_prompt():
+    """A state installed from the replayed positions equals the state the
+    appends build, for a retrieval and a streaming head."""
     rng = np.random.default_rng(14)
     n0, hkv, d, s, r = 150, 2, 4, 3, 9
     k = rng.standard_normal((1, n0, hkv, d)).astype(np.float32)
@@ -378,13 +380,30 @@ def test_load_state_equals_replayed_prompt():
     a.append(k, v)
     b = O.HeadSplitCache(1, hkv, d, gate=gate, sink=s, recent=r)
     b.load_state(0, 0, np.arange(n0), k[0, :, 0], v[0, :, 0])
-    keep = sorted(set(range(s)) | set(range(n0 - r, n0)))
+    keep = O.streaming_positions(n0, s, r)
     b.load_state(0, 1, keep, k[0, keep, 1], v[0, keep, 1])
     b.set_length(0, n0)
     for h in range(hkv):
         pa, ka, va = a.rows(0, h)
         pb, kb, vb = b.rows(0, h)
         assert np.array_equal(pa, pb) and np.array_equal(ka, kb) and np.array_equal(va, vb)
+
+
+@pytest.mark.parametrize("s,r", [(16, 64), (3, 9), (0, 5), (4, 1)])
+def test_streaming_positions_are_the_sinks_and_the_recent_tokens(s, r):
+    """After L single-token appends a streaming head holds exactly the first
+    min(L, sink) positions and the last `recent` ones (the pages: sink and
+    recent tokens only), for every L across the boundaries, and the list the
+    appends build holds the same positions."""
+    c = O.HeadSplitCache(1, 1, 1, gate=np.array([0], dtype=np.uint8), sink=s, recent=r)
+    one = np.zeros((1, 1, 1, 1), dtype=np.float32)
+    for L in range(0, 3 * (s + r) + 5):
+        want = sorted(set(range(min(L, s))) | set(range(max(0, L - r), L)))
+        got = O.streaming_positions(L, s, r)
+        assert list(got) == want, (L, list(got), want)
+        assert list(c.rows(0, 0)[0]) == want
+        c.append(one, one)
+    assert len(O.streaming_positions(1 << 16, s, r)) == s + r
 
 
 def test_bf16_widening_is_exact():
@@ -549,3 +568,23 @@ def test_grad_alpha_vanishes_when_the_window_covers_the_sequence():
     dout = rng.standard_normal((n, hq, d))
     assert np.all(np.abs(O.gated_mix_grad_alpha(q, k, v, dout, 8, 32)) < 1e-12)
     assert np.any(np.abs(O.gated_mix_grad_alpha(q, k, v, dout, 2, 5)) > 1e-3)
+
+
+def test_oracle_pool_rows_equal_direct_rows(tmp_path):
+    """The spawned workers the full-size parity test uses return the rows the
+    oracle computes in this process, per chunk and in order (equal up to the
+    fp64 summation order of their single-threaded BLAS)."""
+    from tests.oracle_pool import PrefillOracle
+    sh = S.LayerShape(8, 4, 16, "bf16", sink=3, recent=5)
+    n, C = 96, 32
+    q, k, v = S.prompt(sh, n, seed=2)
+    gate = np.array([1, 0, 0, 1], dtype=np.uint8)
+    ora = PrefillOracle(tmp_path, q[0], k[0], v[0], gate, sh.sink, sh.recent, workers=2)
+    rows = {0: np.arange(C), 32: np.array([0, 5, 31]), 64: np.arange(0, C, 3)}
+    for c0, r in rows.items():
+        ora.submit(c0, C, r, block=4)
+    got = ora.results()
+    for c0, r in rows.items():
+        want = O.prefill_direct(q[0, c0:c0 + C], k[0, :c0 + C], v[0, :c0 + C], c0, gate, sh.sink, sh.recent, rows=r)
+        assert np.array_equal(got[c0][0], r)
+        np.testing.assert_allclose(got[c0][1], want, atol=1e-12, rtol=0)
