@@ -837,10 +837,15 @@ def run_mix(args, wl, world, rank):
                    "l2": "flushed (1 GiB write) before every timed call, outside the timed interval"},
         "roofline": dict(bound, achieved=round(tf, 3), unit="TFLOP/s", frac=round(tf / bound["peak"], 4),
                          traffic=None, algorithmic_gflop=round(flops / 1e9, 3)),
-        "grad_alpha": {"value": round(grad_med * 1e3, 2), "unit": "us/call", "kernel": "simt_attention_kernel",
+        "grad_alpha": {"value": round(grad_med * 1e3, 2), "unit": "us/call",
+                       "kernel": ("prefill_tc_kernel<EPI_DOT> (streaming launch + causal launch)"
+                                  if bound["bound"] == "tensor" else "simt_attention_kernel"),
+                       "achieved_frac_of_bf16_peak": (round(flops / (grad_med * 1e-3) / 1e12 / bound["peak"], 4)
+                                                      if bound["bound"] == "tensor" else None),
                        "achieved_tflops": round(flops / (grad_med * 1e-3) / 1e12, 3),
-                       "frac_of_alu": round(flops / (grad_med * 1e-3) / 1e12 / ALU_FP32_TFLOPS, 4)},
-        "gpu_launches": (3 if bound["bound"] == "tensor" else 2) * steps,
+                       "frac_of_alu": (None if bound["bound"] == "tensor"
+                                       else round(flops / (grad_med * 1e-3) / 1e12 / ALU_FP32_TFLOPS, 4))},
+        "gpu_launches": (4 if bound["bound"] == "tensor" else 2) * steps,
         "clocks": clk.summary(),
     }
     if rank == 0 and not args.no_cpu_baseline:

@@ -444,9 +444,10 @@ duo_status duo_gated_mix(const duo_layer_desc* desc, const float* alpha, const v
     if (duo::prefill_tc_supported(as) && duo::prefill_tc_supported(ac)) {
         duo::CacheArgs none{};   // no lengths, no caches: every sequence starts at position 0
         none.status = status;    // device conditions (a wait that ran out) are reported here
+        const duo::EpiArgs mix{duo::EPI_MIX, alpha, nullptr, nullptr, 0.f};
         cudaError_t e = duo::launch_prefill_tc(as, none, q, k, v, N, out, nullptr, 0, (cudaStream_t)stream);
         if (e == cudaSuccess)
-            e = duo::launch_prefill_tc(ac, none, q, k, v, N, out, nullptr, 0, (cudaStream_t)stream, alpha);
+            e = duo::launch_prefill_tc(ac, none, q, k, v, N, out, nullptr, 0, (cudaStream_t)stream, &mix);
         return e == cudaSuccess ? ok() : cuda_fail(e, "duo_gated_mix");
     }
     const cudaError_t e = duo::launch_simt_attention(a, nullptr, alpha, q, k, v, N, out, 1, (cudaStream_t)stream);
@@ -472,6 +473,31 @@ duo_status duo_gated_mix_grad_alpha(const duo_layer_desc* desc, const void* q, c
         a.kv_head[i] = i;
         a.q_head0[i] = i * a.G;
         a.slot_of[i] = i;
+    }
+    // bf16, d 128: the mix is linear in alpha, so dalpha = <dout, causal> -
+    // <dout, streaming>; each term is one launch of the tensor-core kernel
+    // whose epilogue adds its rows' dot products into dalpha (no attention
+    // is stored, so no scratch is needed)
+    duo::LayerArgs as = a, ac = a;
+    as.R = 0;
+    as.S = a.Hkv;
+    ac.R = a.Hkv;
+    ac.S = 0;
+    for (duo::LayerArgs* x : {&as, &ac}) {
+        x->page_size = 0;
+        x->capacity = 0;
+        x->stream_chunk = 0;
+        x->kv_int8 = 0;
+    }
+    if (duo::prefill_tc_supported(as) && duo::prefill_tc_supported(ac)) {
+        duo::CacheArgs none{};
+        none.status = status;
+        const duo::EpiArgs minus{duo::EPI_DOT, nullptr, dout, dalpha, -1.f};
+        const duo::EpiArgs plus{duo::EPI_DOT, nullptr, dout, dalpha, 1.f};
+        e = duo::launch_prefill_tc(as, none, q, k, v, N, nullptr, nullptr, 0, (cudaStream_t)stream, &minus);
+        if (e == cudaSuccess)
+            e = duo::launch_prefill_tc(ac, none, q, k, v, N, nullptr, nullptr, 0, (cudaStream_t)stream, &plus);
+        return e == cudaSuccess ? ok() : cuda_fail(e, "duo_gated_mix_grad_alpha");
     }
     e = duo::launch_simt_attention(a, nullptr, nullptr, q, k, v, N, nullptr, 2, (cudaStream_t)stream, dout, dalpha);
     return e == cudaSuccess ? ok() : cuda_fail(e, "duo_gated_mix_grad_alpha");
@@ -518,7 +544,25 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[DUO_NOALLOC_SCR
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
+// the array's device address per device ordinal, and the context it was
+// looked up in: a device reset makes a new context, which loads the module
+// again and may place the array elsewhere
 void* g_noalloc_ptr[kMaxDevices] = {};
+CUcontext g_noalloc_ctx[kMaxDevices] = {};
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current() {
+    static CtxGetCurrentFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+    }
+    return fn;
+}
 
 }  // namespace
 
@@ -542,15 +586,23 @@ extern "C" duo_status duo_decode_attn_noalloc(const duo_layer_desc* desc, const 
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "duo_decode_attn_noalloc: cudaGetDevice");
     if (dev < 0 || dev >= kMaxDevices) return fail(DUO_ERR_UNSUPPORTED, "device ordinal %d above %d", dev, kMaxDevices);
+    // the device's current context (cudaGetDevice above made the runtime's
+    // context current)
+    CUcontext ctx = nullptr;
+    const CtxGetCurrentFn get_ctx = ctx_get_current();
+    if (!get_ctx || get_ctx(&ctx) != CUDA_SUCCESS || !ctx)
+        return fail(DUO_ERR_CUDA, "duo_decode_attn_noalloc: cannot read the current CUDA context");
     void* scratch = nullptr;
     {
         std::lock_guard<std::mutex> lock(g_noalloc_mu);
-        if (!g_noalloc_ptr[dev]) {
-            // once per device, with that device current
+        if (!g_noalloc_ptr[dev] || g_noalloc_ctx[dev] != ctx) {
+            // once per device (and again after a reset gave it a new
+            // context), with that device current
             void* p = nullptr;
             e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
             if (e != cudaSuccess) return cuda_fail(e, "duo_decode_attn_noalloc: cudaGetSymbolAddress");
             g_noalloc_ptr[dev] = p;
+            g_noalloc_ctx[dev] = ctx;
         }
         scratch = g_noalloc_ptr[dev];
     }

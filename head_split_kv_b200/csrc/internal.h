@@ -91,11 +91,23 @@ struct PrefillPlan {
 int sm_count();
 PrefillPlan prefill_plan(const LayerArgs& a, int C, int n_sms);
 size_t prefill_workspace_bytes(const LayerArgs& a, int max_chunk);
-// mix_alpha non-NULL (gated mix, no splits): out is read back as the
-// streaming attention and overwritten with alpha * result + (1 - alpha) * out.
+// Epilogues of the tensor-core attention kernel: the pre-fill's store, and
+// the gated mix's two (no key-range splits):
+//   EPI_MIX: out is read back as the streaming attention and overwritten
+//            with alpha[kv] * result + (1 - alpha[kv]) * out;
+//   EPI_DOT: nothing is stored; sign * <dout row, result row> summed over
+//            the rows is added into dalpha[kv] (atomics).
+enum { EPI_STORE = 0, EPI_MIX = 1, EPI_DOT = 2 };
+struct EpiArgs {
+    int mode;
+    const float* alpha;   // EPI_MIX: [Hkv] gates
+    const void* dout;     // EPI_DOT: [B][C][Hq][d] bf16
+    float* dalpha;        // EPI_DOT: [Hkv] accumulated
+    float sign;           // EPI_DOT: +1 or -1
+};
 cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void* q, const void* k_chunk,
                               const void* v_chunk, int C, void* out, void* workspace, size_t ws_bytes,
-                              cudaStream_t s, const float* mix_alpha = nullptr);
+                              cudaStream_t s, const EpiArgs* epi = nullptr);
 cudaError_t launch_exp2_fma_probe(const float* x, float* y, int64_t n, cudaStream_t s);
 // One warp waits on an mbarrier that never completes, with the given limit.
 cudaError_t launch_wait_probe(int32_t* status, uint64_t limit_ns, cudaStream_t s);

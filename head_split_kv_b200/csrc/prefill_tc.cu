@@ -41,9 +41,14 @@
 // rows' (m, l, O) to the workspace and the CTA that takes the unit's last
 // ticket merges them (prefill_plan picks ns on the host).
 // Gated mix: with no length array every sequence starts at position 0 and the
-// launch covers whole sequences; given mix_alpha, the epilogue reads back the
+// launch covers whole sequences.  Two other epilogues serve it (compile-time
+// variants, so the pre-fill carries neither): EPI_MIX reads back the
 // streaming attention an earlier launch left in out and stores
-// alpha * (this causal attention) + (1 - alpha) * (that).
+// alpha * (this causal attention) + (1 - alpha) * (that); EPI_DOT stores
+// nothing and adds sign * <dout row, attention row> over the CTA's rows into
+// dalpha[kv] (the gate gradient, one launch per sign).  Both load the row
+// they combine with before waiting for the last MMAs, so its latency hides
+// behind them.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -79,7 +84,7 @@ constexpr uint32_t kOffK = kOffQ + 2 * kQBytes;
 constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;
 constexpr uint32_t kOffBar = kOffV + 2 * kTileBytes;
 constexpr uint32_t kOffHolder = kOffBar + 16 * 8;
-constexpr uint32_t kSmemBytes = kOffHolder + 16;
+constexpr uint32_t kSmemBytes = kOffHolder + 32;
 static_assert(kSmemBytes + 1024 <= 232448, "one CTA per SM");
 
 enum { SRC_CACHE = 0, SRC_CHUNK = 1, SRC_RING = 2 };
@@ -93,7 +98,7 @@ struct TcArgs {
     int n_ret_ctas;        // n_units * ns
     float* part;           // [n_units][ns][2][kPartFloats] partial records (ns > 1)
     uint32_t* ticket;      // [n_units] arrivals; the last split merges them
-    const float* mix_alpha;  // gated mix: out = alpha[kv] * this attention + (1 - alpha[kv]) * out
+    EpiArgs epi;           // gated-mix epilogues (EPI_MIX, EPI_DOT)
     const int32_t* seq_len;
     int32_t* status;
     void* out;
@@ -240,7 +245,7 @@ __device__ __forceinline__ void visible_columns(const LayerArgs& a, const Sched&
 
 // ------------------------------------------------------------------ softmax
 
-constexpr int kFmaExpEvery = 8;   // one exp2 pair in 8 on the FMA pipe (1 in 4 spills at 200 registers)
+constexpr int kFmaExpEvery = 4;   // one exp2 pair in 4 on the FMA pipe
 
 // 2^x for a pair of x <= 0 (or -inf) on the FMA pipe, by Cody-Waite range
 // reduction and a polynomial: x = n + f with n = rint(x) (adding 1.5 * 2^23
@@ -283,8 +288,7 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
 // SFU is the co-bottleneck.  One pair in kFmaExpEvery is computed on the FMA
 // pipe instead (exp2_fma2).  Measured on the 131K prompt: one pair in 4 or
 // in 8 (equal within run-to-run noise) beat SFU-only by 2-5 %; one in 3 was
-// slower.  One in 8 leaves the kernel without register spills at its
-// 200-register budget (one in 4 spilled 20-30 bytes a thread).
+// slower.
 __device__ __forceinline__ float softmax_tile(uint32_t s_addr, float sl, bool masked, const uint32_t (&vis)[4],
                                               float& m_ref, float& l_sum, bool& need) {
     float s[128];
@@ -332,14 +336,88 @@ __device__ __forceinline__ float softmax_tile(uint32_t s_addr, float sl, bool ma
     return corr;
 }
 
+// ------------------------------------------------------------------ split records
+//
+// One row of a split's record of a query tile: its running maximum, row sum
+// and unnormalised O row (read from TMEM at o_addr; zeros when the split had
+// no tile for it).  Not inlined, like the merge below.
+__device__ __noinline__ void write_split_record(float* rec, int row, bool have, float m_ref, float l_sum,
+                                                uint32_t o_addr) {
+    rec[row] = have ? m_ref : -INFINITY;
+    rec[BM + row] = have ? l_sum : 0.f;
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+        float o[32];
+        if (have) {
+            tmem_ld32(o_addr + 32 * ch, o);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = 0.f;
+        }
+#pragma unroll
+        for (int g4 = 0; g4 < 8; ++g4)
+            reinterpret_cast<float4*>(rec + 2 * BM)[(8 * ch + g4) * BM + row] =
+                make_float4(o[4 * g4], o[4 * g4 + 1], o[4 * g4 + 2], o[4 * g4 + 3]);
+    }
+}
+
+// ------------------------------------------------------------------ split merge
+//
+// The split that arrives last merges the ns_use records of one query tile,
+// row by row (thread = row): the splits' maxima and sums give each record's
+// weight, and the weighted sum of the unnormalised O rows over the total
+// weight is the row's output.  Not inlined, so that its registers do not
+// count against the softmax loop's: the kernel runs at the 168 a thread
+// that ten warps leave (an SM sub-partition holds three of them in its 16K
+// registers).
+__device__ __noinline__ void merge_split_records(const float* base, int ns_use, int row, bool store,
+                                                 __nv_bfloat16* op) {
+    constexpr size_t kSplitStride = 2 * (size_t)kPartFloats;
+    float w[kMaxSplit];
+    float M = -INFINITY, L = 0.f;
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplit; ++sp)
+        if (sp < ns_use) M = fmaxf(M, __ldcg(base + sp * kSplitStride + row));
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplit; ++sp) {
+        w[sp] = 0.f;
+        if (sp < ns_use) {
+            const float ms = __ldcg(base + sp * kSplitStride + row);
+            w[sp] = ms == -INFINITY ? 0.f : exp2f(ms - M);
+            L += w[sp] * __ldcg(base + sp * kSplitStride + BM + row);
+        }
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll 1
+    for (int g8 = 0; g8 < HD / 8; ++g8) {
+        float v8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int sp = 0; sp < kMaxSplit; ++sp) {
+            if (sp < ns_use) {
+                const float4* o4 = reinterpret_cast<const float4*>(base + sp * kSplitStride + 2 * BM);
+                const float4 x0 = __ldcg(o4 + (2 * g8) * BM + row);
+                const float4 x1 = __ldcg(o4 + (2 * g8 + 1) * BM + row);
+                v8[0] += w[sp] * x0.x; v8[1] += w[sp] * x0.y; v8[2] += w[sp] * x0.z; v8[3] += w[sp] * x0.w;
+                v8[4] += w[sp] * x1.x; v8[5] += w[sp] * x1.y; v8[6] += w[sp] * x1.z; v8[7] += w[sp] * x1.w;
+            }
+        }
+        if (store) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v8[e] *= inv;
+            store_row<__nv_bfloat16, 8>(op + 8 * g8, v8);
+        }
+    }
+}
+
 // ------------------------------------------------------------------ kernel
 
-// MIX: the gated-mix instantiation (its epilogue mixes with what out holds;
-// no key-range splits), so the pre-fill instantiation carries no mix code.
-// 200 registers a thread: 10 warps x 32 x 200 fit the SM's 64K with one CTA
-// per SM.
-template <bool MIX>
-__global__ void __maxnreg__(200)
+// EPI: EPI_STORE (pre-fill: store, or key-range split records), EPI_MIX or
+// EPI_DOT (the gated mix's epilogues; no key-range splits).  Ten warps leave
+// 168 registers a thread (three of them share an SM sub-partition's 16K);
+// the split epilogue keeps its indices in shared memory and its record
+// write and merge out of line, so that the softmax loop fits without spills.
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
                       const __grid_constant__ CUtensorMap tmVc, const __grid_constant__ CUtensorMap tmKx,
                       const __grid_constant__ CUtensorMap tmVx, const __grid_constant__ CUtensorMap tmKr,
@@ -416,6 +494,11 @@ __global__ void __maxnreg__(200)
     // ------------------------------------------------------- set-up
     if (warp == kMmaWarp) tmem_alloc(holder, kTmemCols);
     if (tid == 0) {
+        // what the split epilogue needs, parked here instead of in registers
+        // held across the softmax loop
+        holder[2] = (uint32_t)unit;
+        holder[3] = (uint32_t)split;
+        holder[4] = (uint32_t)ns_use;
         mbar_init(q_full, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&k_full[i], 1);
@@ -566,104 +649,77 @@ __global__ void __maxnreg__(200)
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[qi]);          // one arrival per warp
         }
-        // epilogue: O / l -> bf16
+        // epilogue: O / l -> bf16 (or the gated mix's epilogues)
+        const size_t row_off = (((size_t)b * p.C + crow) * a.Hq + q_idx) * HD;
+        uint4 pre[16];   // EPI_MIX / EPI_DOT: this row of out / dout, loaded before the wait below
+        if constexpr (EPI != EPI_STORE) {
+            const uint4* src = reinterpret_cast<const uint4*>(
+                static_cast<const __nv_bfloat16*>(EPI == EPI_MIX ? p.out : p.epi.dout) + row_off);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pre[i] = crow < p.C ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+        }
         if (ok && n_me >= 1) ok = __all_sync(0xffffffffu, mbar_wait(&o_done[qi], 0, p.status));
-        __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.out) + (((size_t)b * p.C + crow) * a.Hq + q_idx) * HD;
-        if (MIX || ns_use == 1) {
+        __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.out) + row_off;
+        if (EPI != EPI_STORE || holder[4] == 1u) {
             if (ok && n_me >= 1) {
                 tc_fence_after();
                 const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+                const float al = EPI == EPI_MIX ? p.epi.alpha[kv_idx] : 0.f;
+                float dot = 0.f;
 #pragma unroll
                 for (int ch = 0; ch < 4; ++ch) {
                     float o[32];
                     tmem_ld32(lane_base + col_o(qi) + 32 * ch, o);
-                    if (crow < p.C) {
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            float v8[8];
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        float v8[8];
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) v8[e] = o[8 * q4 + e] * inv;
-                            if constexpr (MIX) {
-                                // gated mix: out already holds the streaming attention
-                                const float al = p.mix_alpha[kv_idx];
-                                const uint4 u = *reinterpret_cast<const uint4*>(op + 32 * ch + 8 * q4);
-                                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+                        for (int e = 0; e < 8; ++e) v8[e] = o[8 * q4 + e] * inv;
+                        if constexpr (EPI == EPI_STORE) {
+                            if (crow < p.C) store_row<__nv_bfloat16, 8>(op + 32 * ch + 8 * q4, v8);
+                        } else {
+                            const uint4 u = pre[4 * ch + q4];
+                            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+                            if constexpr (EPI == EPI_MIX) {
+                                // out held the streaming attention: mix it in
 #pragma unroll
                                 for (int e = 0; e < 4; ++e) {
                                     v8[2 * e] = al * v8[2 * e] + (1.f - al) * bf16_lo(w[e]);
                                     v8[2 * e + 1] = al * v8[2 * e + 1] + (1.f - al) * bf16_hi(w[e]);
                                 }
+                                if (crow < p.C) store_row<__nv_bfloat16, 8>(op + 32 * ch + 8 * q4, v8);
+                            } else {
+                                // <dout row, attention row>; rows past the sequence hold dout = 0
+#pragma unroll
+                                for (int e = 0; e < 4; ++e)
+                                    dot = fmaf(v8[2 * e], bf16_lo(w[e]), fmaf(v8[2 * e + 1], bf16_hi(w[e]), dot));
                             }
-                            store_row<__nv_bfloat16, 8>(op + 32 * ch + 8 * q4, v8);
                         }
                     }
                 }
+                if constexpr (EPI == EPI_DOT) {
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+                    if (lane == 0) atomicAdd(&p.epi.dalpha[kv_idx], p.epi.sign * dot);
+                }
             }
-        } else if constexpr (!MIX) {
+        } else if constexpr (EPI == EPI_STORE) {
             // (1) this split's record of the query tile: m, l and O unnormalised
             const bool have = ok && n_me >= 1;               // warp-uniform
-            float* rec = p.part + (((size_t)unit * p.ns + split) * 2 + qi) * kPartFloats;
+            const int unit_ = (int)holder[2], split_ = (int)holder[3], ns_use_ = (int)holder[4];
+            float* rec = p.part + (((size_t)unit_ * p.ns + split_) * 2 + qi) * kPartFloats;
             if (have) tc_fence_after();
-            rec[row] = have ? m_ref : -INFINITY;
-            rec[BM + row] = have ? l_sum : 0.f;
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                float o[32];
-                if (have) {
-                    tmem_ld32(lane_base + col_o(qi) + 32 * ch, o);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = 0.f;
-                }
-#pragma unroll
-                for (int g4 = 0; g4 < 8; ++g4)
-                    reinterpret_cast<float4*>(rec + 2 * BM)[(8 * ch + g4) * BM + row] =
-                        make_float4(o[4 * g4], o[4 * g4 + 1], o[4 * g4 + 2], o[4 * g4 + 3]);
-            }
+            write_split_record(rec, row, have, m_ref, l_sum, lane_base + col_o(qi));
             // (2) a ticket per unit, taken once the 256 softmax threads have
             // written; the CTA that arrives last merges (no CTA ever waits)
             __threadfence();
             asm volatile("bar.sync 1, 256;" ::: "memory");
-            if (tid == 0) holder[1] = (atomicAdd(&p.ticket[unit], 1u) == (unsigned)ns_use - 1) ? 1u : 0u;
+            if (tid == 0) holder[1] = (atomicAdd(&p.ticket[unit_], 1u) == (unsigned)ns_use_ - 1) ? 1u : 0u;
             asm volatile("bar.sync 1, 256;" ::: "memory");
             if (holder[1]) {
                 __threadfence();
-                const float* base = p.part + (size_t)unit * p.ns * 2 * kPartFloats + (size_t)qi * kPartFloats;
-                constexpr size_t kSplitStride = 2 * (size_t)kPartFloats;
-                float w[kMaxSplit];
-                float M = -INFINITY, L = 0.f;
-#pragma unroll
-                for (int sp = 0; sp < kMaxSplit; ++sp)
-                    if (sp < ns_use) M = fmaxf(M, __ldcg(base + sp * kSplitStride + row));
-#pragma unroll
-                for (int sp = 0; sp < kMaxSplit; ++sp) {
-                    w[sp] = 0.f;
-                    if (sp < ns_use) {
-                        const float ms = __ldcg(base + sp * kSplitStride + row);
-                        w[sp] = ms == -INFINITY ? 0.f : exp2f(ms - M);
-                        L += w[sp] * __ldcg(base + sp * kSplitStride + BM + row);
-                    }
-                }
-                const float inv = L > 0.f ? 1.f / L : 0.f;
-#pragma unroll 1
-                for (int g8 = 0; g8 < HD / 8; ++g8) {
-                    float v8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int sp = 0; sp < kMaxSplit; ++sp) {
-                        if (sp < ns_use) {
-                            const float4* o4 = reinterpret_cast<const float4*>(base + sp * kSplitStride + 2 * BM);
-                            const float4 x0 = __ldcg(o4 + (2 * g8) * BM + row);
-                            const float4 x1 = __ldcg(o4 + (2 * g8 + 1) * BM + row);
-                            v8[0] += w[sp] * x0.x; v8[1] += w[sp] * x0.y; v8[2] += w[sp] * x0.z; v8[3] += w[sp] * x0.w;
-                            v8[4] += w[sp] * x1.x; v8[5] += w[sp] * x1.y; v8[6] += w[sp] * x1.z; v8[7] += w[sp] * x1.w;
-                        }
-                    }
-                    if (crow < p.C) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) v8[e] *= inv;
-                        store_row<__nv_bfloat16, 8>(op + 8 * g8, v8);
-                    }
-                }
+                merge_split_records(p.part + (size_t)unit_ * p.ns * 2 * kPartFloats + (size_t)qi * kPartFloats,
+                                    ns_use_, row, crow < p.C, op);
             }
         }
     }
@@ -738,7 +794,7 @@ size_t prefill_workspace_bytes(const LayerArgs& a, int max_chunk) {
 
 cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void* q, const void* k_chunk,
                               const void* v_chunk, int C, void* out, void* workspace, size_t ws_bytes,
-                              cudaStream_t s, const float* mix_alpha) {
+                              cudaStream_t s, const EpiArgs* epi) {
     if (!prefill_tc_supported(a)) return cudaErrorNotSupported;
     const uint64_t row = HD * 2;
     CUtensorMap mQ, mKx, mVx, mKc, mVc, mKr, mVr;
@@ -780,7 +836,8 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
     p.n_mpairs = (C + 2 * BM - 1) / (2 * BM);
     p.n_units = a.B * a.R * a.G * p.n_mpairs;
     const PrefillPlan plan = prefill_plan(a, C, sm_count());
-    const bool split = plan.ns > 1 && workspace != nullptr && ws_bytes >= plan.bytes && mix_alpha == nullptr;
+    const int mode = epi ? epi->mode : EPI_STORE;
+    const bool split = plan.ns > 1 && workspace != nullptr && ws_bytes >= plan.bytes && mode == EPI_STORE;
     p.ns = split ? plan.ns : 1;
     p.part = split ? static_cast<float*>(workspace) : nullptr;
     p.ticket = split ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + plan.ticket_offset) : nullptr;
@@ -788,14 +845,16 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
     p.seq_len = c.seq_len;
     p.status = c.status;
     p.out = out;
-    p.mix_alpha = mix_alpha;
+    p.epi = epi ? *epi : EpiArgs{EPI_STORE, nullptr, nullptr, nullptr, 0.f};
     const long grid = (long)p.n_ret_ctas + (long)a.B * a.S * a.G * p.n_mpairs;
     if (grid == 0) return cudaSuccess;
     if (grid > 0x7fffffffL) return cudaErrorInvalidConfiguration;
-    static std::atomic<unsigned long long> configured{0}, configured_mix{0};
+    static std::atomic<unsigned long long> configured[3] = {{0}, {0}, {0}};
     {
-        const cudaError_t e = mix_alpha ? smem_limit_once(prefill_tc_kernel<true>, (int)(kSmemBytes + 1024), configured_mix)
-                                        : smem_limit_once(prefill_tc_kernel<false>, (int)(kSmemBytes + 1024), configured);
+        cudaError_t e = cudaErrorInvalidValue;
+        if (mode == EPI_STORE) e = smem_limit_once(prefill_tc_kernel<EPI_STORE>, (int)(kSmemBytes + 1024), configured[0]);
+        if (mode == EPI_MIX) e = smem_limit_once(prefill_tc_kernel<EPI_MIX>, (int)(kSmemBytes + 1024), configured[1]);
+        if (mode == EPI_DOT) e = smem_limit_once(prefill_tc_kernel<EPI_DOT>, (int)(kSmemBytes + 1024), configured[2]);
         if (e != cudaSuccess) return e;
     }
     if (split) {
@@ -805,10 +864,12 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
         const cudaError_t e = cudaMemsetAsync(p.ticket, 0, (size_t)p.n_units * sizeof(uint32_t), s);
         if (e != cudaSuccess) return e;
     }
-    if (mix_alpha)
-        prefill_tc_kernel<true><<<(unsigned)grid, kThreads, kSmemBytes + 1024, s>>>(mQ, mKc, mVc, mKx, mVx, mKr, mVr, p);
+    if (mode == EPI_MIX)
+        prefill_tc_kernel<EPI_MIX><<<(unsigned)grid, kThreads, kSmemBytes + 1024, s>>>(mQ, mKc, mVc, mKx, mVx, mKr, mVr, p);
+    else if (mode == EPI_DOT)
+        prefill_tc_kernel<EPI_DOT><<<(unsigned)grid, kThreads, kSmemBytes + 1024, s>>>(mQ, mKc, mVc, mKx, mVx, mKr, mVr, p);
     else
-        prefill_tc_kernel<false><<<(unsigned)grid, kThreads, kSmemBytes + 1024, s>>>(mQ, mKc, mVc, mKx, mVx, mKr, mVr, p);
+        prefill_tc_kernel<EPI_STORE><<<(unsigned)grid, kThreads, kSmemBytes + 1024, s>>>(mQ, mKc, mVc, mKx, mVx, mKr, mVr, p);
     return cudaGetLastError();
 }
 

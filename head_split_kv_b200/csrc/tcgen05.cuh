@@ -110,6 +110,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+// registers -> 16 consecutive TMEM columns of this thread's lane (no wait)
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16};" ::"r"(taddr),
+        DUO_W8(0), DUO_W8(8)
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_st32f(uint32_t taddr, const float (&v)[32]) {
     uint32_t r[32];
 #pragma unroll

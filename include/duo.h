@@ -393,7 +393,10 @@ duo_status duo_gated_mix(const duo_layer_desc* desc, const float* alpha, const v
  * Every GPU that loads the library holds the array until the process exits.
  * The first call on each device looks up the array's device address with
  * that device current (cudaGetSymbolAddress); make that first call before
- * any stream capture begins.
+ * any stream capture begins.  The address belongs to the device's context:
+ * after a reset (cudaDeviceReset) the next call finds a new context and looks
+ * the address up again, so the first call after a reset must also come
+ * before any capture.
  * All calls on a device share the one array and it keeps the previous call's
  * contents: each call clears the ticket words it needs on `stream` before the
  * kernel runs.  Calls that can overlap on the GPU (other streams, other host
@@ -417,7 +420,11 @@ duo_status duo_decode_attn_noalloc(const duo_layer_desc* desc, const duo_kv_stat
  * q [B][N][Hq][d]; k, v [B][N][Hkv][d]; dout [B][N][Hq][d] (same dtype);
  * model head order as for duo_gated_mix.  dalpha [Hkv] fp32 device: zeroed
  * by the call, then accumulated with atomics (one add per 32 rows), so the
- * last bits vary with the order the CTAs finish in.
+ * last bits vary with the order the CTAs finish in.  bf16 with d = 128 runs
+ * on the tcgen05 tensor cores in two launches that store no attention: by
+ * linearity dalpha = <dout, full_attn> - <dout, streaming_attn>, and each
+ * launch adds one of the two terms from its epilogue; other dtypes and head
+ * sizes run on the CUDA cores.
  * status: one int32 device word (required), as for duo_gated_mix.
  * Errors: DUO_ERR_INVALID_ARG, DUO_ERR_SHAPE, DUO_ERR_UNSUPPORTED, DUO_ERR_CUDA.
  */
@@ -430,7 +437,7 @@ duo_status duo_gated_mix_grad_alpha(const duo_layer_desc* desc, const void* q, c
  * (Cody-Waite range reduction to x = n + f, f in [-0.5, 0.5], a fitted cubic
  * for 2^f and n added to the exponent field; inputs below -125, -inf
  * included, give the value at -125, 2^-125 within the cubic's 7.5e-5).
- * duo_prefill_chunk computes one exponential pair in eight this way and the
+ * duo_prefill_chunk computes one exponential pair in four this way and the
  * rest on the SFU; this entry point exposes the routine so that its error
  * can be checked against 2^x.  It is not a step of the attention path: the
  * paper review's S3 "Core formula" only fixes the softmax, not how its

@@ -392,6 +392,24 @@ def test_gated_mix_grad_alpha_bf16_gqa_batch(duo):
     _grad_check(dalpha.cpu().numpy().astype(np.float64), want, O.as_f64(dout), 4, 2e-3)
 
 
+@pytest.mark.parametrize("hq,hkv,n,B", [(8, 8, 700, 1), (32, 4, 513, 2), (16, 8, 1031, 1)])
+def test_gated_mix_grad_alpha_bf16_tensor_core_path(duo, hq, hkv, n, B):
+    """bf16, d 128: the gate gradient from the two tensor-core launches (the
+    streaming and the causal attention's dot products with dout); several
+    256-row query-tile pairs with a ragged tail, MHA, G = 8 and G = 2."""
+    t = torch()
+    sh = S.LayerShape(hq, hkv, 128, "bf16")
+    q, k, v = S.prompt(sh, n, seed=10, batch=B)
+    dout = S.normal(S.rng_for(10, 63), (B, n, hq, 128), "bf16")
+    desc = duo.desc_init(B, hq, hkv, 128, duo.BF16, list(range(hkv)), 0)
+    dalpha = t.empty((hkv,), dtype=t.float32, device="cuda")
+    status = t.zeros(1, dtype=t.int32, device="cuda")
+    duo.gated_mix_grad_alpha(desc, to_dev(q), to_dev(k), to_dev(v), n, to_dev(dout), dalpha, status)
+    assert status.item() == 0
+    want = sum(O.gated_mix_grad_alpha(q[b], k[b], v[b], dout[b], sh.sink, sh.recent) for b in range(B))
+    _grad_check(dalpha.cpu().numpy().astype(np.float64), want, O.as_f64(dout), hq // hkv, 2e-3)
+
+
 def test_gated_mix_grad_alpha_zero_when_window_covers_sequence(duo):
     """Both attentions see every key, in the same order: the difference, and
     with it the gradient, is exactly zero."""
