@@ -59,6 +59,10 @@ repository's design notes):
   code = rint(x * (127 / amax)) (round half to even), scale = amax / 127,
   all in float32 as written; a zero row has scale 0 and codes 0.  Attention
   reads code * scale.
+* 4-bit retrieval cache (the paper review's "Quantization combination"
+  pairs 8-bit weights with a 4-bit KV cache, again without a scheme): the
+  same per-row symmetric steps with 7 levels a side, codes -7..7,
+  scale = amax / 7.
 """
 
 from __future__ import annotations
@@ -89,6 +93,7 @@ __all__ = [
     "decode_direct",
     "quantize_int8_rows",
     "dequantize_int8_rows",
+    "quantize_int4_rows",
 ]
 
 
@@ -333,6 +338,24 @@ def dequantize_int8_rows(codes, scales) -> np.ndarray:
     return np.asarray(codes, dtype=np.float64) * np.asarray(scales, dtype=np.float64)[:, None]
 
 
+def quantize_int4_rows(x) -> tuple:
+    """Per-row symmetric 4-bit codes of x [n, d] (bf16 bits, float32 or
+    float64 holding float32 values): the 8-bit scheme's steps with 7 levels
+    a side in place of 127 -- amax = max |x|, code = rint(x * (7 / amax)),
+    scale = amax / 7, each one float32 operation as written; a zero row has
+    scale 0 and codes 0.  Returns (codes int8 [n, d] in -7..7, scales
+    float32 [n])."""
+    x32 = as_f64(x).astype(np.float32)
+    amax = np.abs(x32).max(axis=-1) if x32.shape[-1] else np.zeros(x32.shape[:-1], np.float32)
+    nz = amax > 0
+    inv = np.zeros_like(amax)
+    inv[nz] = np.float32(7.0) / amax[nz]                        # float32 division
+    q = np.rint(x32 * inv[..., None])                           # float32 product, round half to even
+    codes = np.clip(q, -7, 7).astype(np.int8)
+    scales = np.where(nz, amax / np.float32(7.0), np.float32(0)).astype(np.float32)
+    return codes, scales
+
+
 def _streaming_push(lst: list, entry: tuple, sink: int, recent: int) -> None:
     """Append one (position, ...) entry to a streaming head's list; when the
     list grows past sink + recent, evict the oldest token that is not an
@@ -373,6 +396,7 @@ class HeadSplitCache:
     sink: int = 16
     recent: int = 64
     kv_int8: bool = False                # retrieval heads keep int8 codes + a scale per row
+    kv_int4: bool = False                # retrieval heads keep 4-bit codes + a scale per row
     length: list = field(default=None)
     full: list = field(default=None)     # full[b][h] -> list of (pos int64[n], k[n, d], v[n, d]
                                          #   [, k codes, k scales, v codes, v scales] when kv_int8)
@@ -423,17 +447,19 @@ class HeadSplitCache:
         self.length[b] = int(n)
 
     def _full_entry(self, pos, k, v):
-        """A retrieval-head list entry: the rows as given, or (kv_int8) their
-        dequantized values followed by the codes and scales."""
-        if not self.kv_int8:
+        """A retrieval-head list entry: the rows as given, or (kv_int8,
+        kv_int4) their dequantized values followed by the codes and scales."""
+        if not (self.kv_int8 or self.kv_int4):
             return (pos.copy(), k.copy(), v.copy())
-        kc, ks = quantize_int8_rows(k)
-        vc, vs = quantize_int8_rows(v)
+        quantize = quantize_int8_rows if self.kv_int8 else quantize_int4_rows
+        kc, ks = quantize(k)
+        vc, vs = quantize(v)
         return (pos.copy(), dequantize_int8_rows(kc, ks), dequantize_int8_rows(vc, vs), kc, ks, vc, vs)
 
     def quantized(self, b: int, h: int):
-        """A kv_int8 retrieval head's (positions, K codes, K scales, V codes, V scales)."""
-        assert self.kv_int8 and self.gate[h]
+        """A kv_int8 / kv_int4 retrieval head's (positions, K codes, K scales,
+        V codes, V scales)."""
+        assert (self.kv_int8 or self.kv_int4) and self.gate[h]
         ent = self.full[b][h]
         if not ent:
             z8, z32 = np.zeros((0, self.head_dim), np.int8), np.zeros(0, np.float32)

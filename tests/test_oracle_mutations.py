@@ -52,6 +52,9 @@ def _pins():
         P.test_partition_top_k_ties_go_to_lower_index,
         P.test_binarize_uses_greater_or_equal,
         lambda: P.test_int8_codes_match_hand_worked_rows(g),
+        lambda: P.test_int4_codes_match_hand_worked_rows(g),
+        lambda: P.test_int4_round_trip_is_within_half_a_step(0),
+        P.test_int4_cache_decode_equals_direct_on_reconstructed_rows,
         lambda: P.test_int8_round_trip_is_within_half_a_step(0),
         P.test_int8_cache_decode_equals_direct_on_reconstructed_rows,
         lambda: P.test_chunk_streaming_mask_matches_hand_drawn(g),
@@ -219,6 +222,19 @@ def _q8(x, factor_num=127.0, scale_den=127.0, rnd=np.rint, per_tensor=False):
 def test_planted_int8_mistake_is_caught(monkeypatch, mistake):
     _patch(monkeypatch, "quantize_int8_rows", lambda x: _q8(x, **mistake))
     assert _fails(*_pins()), f"no pin caught the planted quantizer mistake {mistake}"
+
+
+@pytest.mark.parametrize("mistake", [
+    dict(factor_num=7.0, scale_den=7.0, rnd=np.floor),                         # rounds down
+    dict(factor_num=7.0, scale_den=7.0, rnd=lambda v: np.floor(v + np.float32(0.5))),   # ties away from even
+    dict(factor_num=8.0, scale_den=8.0),                                       # 8 levels: +8 does not fit
+    dict(factor_num=7.0, scale_den=8.0),                                       # scale from another step
+    dict(factor_num=7.5, scale_den=7.5),                                       # 15 levels over 16 codes
+    dict(factor_num=7.0, scale_den=7.0, per_tensor=True),                      # one scale for all rows
+])
+def test_planted_int4_mistake_is_caught(monkeypatch, mistake):
+    _patch(monkeypatch, "quantize_int4_rows", lambda x: _q8(x, **mistake))
+    assert _fails(*_pins()), f"no pin caught the planted 4-bit quantizer mistake {mistake}"
 
 
 def _chunk_mask_window_short(q_pos, k_pos, c0, sink, recent):

@@ -476,6 +476,60 @@ def test_int8_cache_decode_equals_direct_on_reconstructed_rows():
     assert np.array_equal(pos, np.arange(n)) and kc.shape == (n, 16) and ks.shape == (n,)
 
 
+def test_int4_codes_match_hand_worked_rows(golden):
+    params, _ = golden("int4_rows.txt")
+    for i in range(4):
+        x = np.array([params[f"x{i}"]], dtype=np.float32)
+        codes, scales = O.quantize_int4_rows(x)
+        assert codes.dtype == np.int8 and scales.dtype == np.float32
+        assert codes[0].tolist() == [int(c) for c in params[f"codes{i}"]], i
+        assert scales[0] == np.float32(float(params[f"scale{i}"])), i
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_int4_round_trip_is_within_half_a_step(seed):
+    rng = np.random.default_rng([seed, 92])
+    d = 128
+    x = (rng.standard_normal((64, d)) * np.exp(rng.uniform(-8, 8, (64, 1)))).astype(np.float32)
+    x = (x.view(np.uint32) & np.uint32(0xFFFF0000)).view(np.float32)
+    x[5] = 0.0
+    x[7, :10] = 0.0
+    codes, scales = O.quantize_int4_rows(x)
+    assert np.all(np.abs(codes.astype(np.int32)) <= 7)
+    amax = np.abs(x).max(axis=1)
+    nz = amax > 0
+    assert np.all(np.abs(codes[nz]).max(axis=1) == 7)
+    assert np.all(scales[~nz] == 0) and np.all(codes[~nz] == 0)
+    err = np.abs(x.astype(np.float64) - O.dequantize_int8_rows(codes, scales))
+    assert np.all(err <= scales.astype(np.float64)[:, None] * (0.5 + 1e-5))
+    assert np.all((codes == 0) | (np.sign(codes) == np.sign(x)))
+    again, _ = O.quantize_int4_rows(O.dequantize_int8_rows(codes, scales).astype(np.float32))
+    assert np.array_equal(again, codes)
+
+
+def test_int4_cache_decode_equals_direct_on_reconstructed_rows():
+    """The 4-bit cache, like the 8-bit one, only changes what the retrieval
+    heads' lists hold: a decode from it equals the direct mask definition
+    over the history whose retrieval rows are replaced by code * scale."""
+    sh = S.LayerShape(8, 4, 16, "bf16")
+    gate = np.array([0, 1, 1, 0], dtype=np.uint8)
+    n = 140
+    q, k, v = S.prompt(sh, n, seed=5)
+    c = O.HeadSplitCache(1, 4, 16, gate=gate, kv_int4=True)
+    c.append(k[:, :n - 1], v[:, :n - 1])
+    got = c.decode(q[:, n - 1], k[:, n - 1], v[:, n - 1])[0]
+    k_hat, v_hat = O.as_f64(k[0]), O.as_f64(v[0])
+    for h in (1, 2):
+        kc, ks = O.quantize_int4_rows(k[0, :, h])
+        vc, vs = O.quantize_int4_rows(v[0, :, h])
+        k_hat[:, h] = O.dequantize_int8_rows(kc, ks)
+        v_hat[:, h] = O.dequantize_int8_rows(vc, vs)
+    want = O.decode_direct(q[0, n - 1], k_hat, v_hat, gate, 16, 64)
+    assert np.max(np.abs(got - want)) < 1e-12
+    pos, kc, ks, vc, vs = c.quantized(0, 1)
+    assert np.array_equal(pos, np.arange(n)) and kc.shape == (n, 16) and np.abs(kc).max() <= 7
+
+
 # ---------------------------------------------------------------------------
 # Whole-chunk streaming pre-fill (the second pre-fill mode)
 # ---------------------------------------------------------------------------
