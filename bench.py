@@ -67,6 +67,13 @@ WORKLOADS = {
                                  sigma=True, kv_int8=True, layers=32),
     "gqa_decode_1m_int8": dict(kind="decode", hq=32, hkv=8, d=128, n_ret=4, lengths=[1048576], steps=64,
                                sigma=True, kv_int8=True, layers=16),
+    # ... and over the 4-bit retrieval cache
+    "mha_decode_32k_int4": dict(kind="decode", hq=32, hkv=32, d=128, n_ret=8, lengths=[32768], steps=256,
+                                sigma=False, kv_int4=True, layers=32),
+    "gqa_decode_128k_int4": dict(kind="decode", hq=32, hkv=8, d=128, n_ret=4, lengths=[131072], steps=64,
+                                 sigma=True, kv_int4=True, layers=32),
+    "gqa_decode_1m_int4": dict(kind="decode", hq=32, hkv=8, d=128, n_ret=4, lengths=[1048576], steps=64,
+                               sigma=True, kv_int4=True, layers=16),
     "gqa_prefill_128k": dict(kind="prefill", hq=32, hkv=8, d=128, n_ret=4, n=131072, chunk=4096, sigma=False),
     # the same pre-fill on a 32K prompt: a small case for profiler captures
     "gqa_prefill_32k": dict(kind="prefill", hq=32, hkv=8, d=128, n_ret=4, n=32768, chunk=4096, sigma=False),
@@ -81,6 +88,7 @@ DEFAULT_WORKLOAD = "gqa_decode_128k"
 EXTRA_DECODE = ("mha_decode_32k", "gqa_decode_1m", "batch64_paged_decode")
 for _name, _wl in WORKLOADS.items():
     _wl["name"] = _name
+    _wl["kv_bits"] = 8 if _wl.get("kv_int8") else 4 if _wl.get("kv_int4") else 0
 
 
 def _peaks():
@@ -318,15 +326,15 @@ def _decode_setup(duo, wl, total_steps, seed=0):
     else:
         table = None
         desc = duo.desc_init(B, sh.n_q_heads, sh.n_kv_heads, sh.head_dim, duo.BF16, perm, R,
-                             kv_quant=duo.KV_INT8 if wl.get("kv_int8") else duo.KV_PLAIN)
+                             kv_quant={8: duo.KV_INT8, 4: duo.KV_INT4}.get(wl.get("kv_bits", 0), duo.KV_PLAIN))
         caches = duo.LayerCaches(desc, int(lengths.max()) + total_steps)
     st = S.decode_state(sh, retrieval, lengths, seed=seed, sigma=sigma)
-    _fill_decode_state(duo, desc, caches, st, inv, R, sh, table, bool(wl.get("kv_int8")))
+    _fill_decode_state(duo, desc, caches, st, inv, R, sh, table, wl.get("kv_bits", 0))
     ws = duo.Workspace(desc, duo.OP_DECODE, caches.capacity)
     qs, ks, vs = S.decode_steps(sh, B, total_steps, seed=seed, sigma=sigma)
     torch.cuda.synchronize()
     return dict(sh=sh, desc=desc, caches=caches, ws=ws, qs=qs, ks=ks, vs=vs, lengths=lengths, B=B, R=R,
-                kv_int8=bool(wl.get("kv_int8")),
+                kv_bits=wl.get("kv_bits", 0),
                 retrieval=retrieval, gate=gate, state=st, sigma=sigma, table=table,
                 n_pages=n_pages if paged else 0)
 
@@ -339,12 +347,12 @@ def _to_dev(a):
     return torch.from_numpy(a).cuda()
 
 
-def _fill_decode_state(duo, desc, caches, st, inv, R, sh, table, kv_int8, chunk=32768):
+def _fill_decode_state(duo, desc, caches, st, inv, R, sh, table, kv_bits, chunk=32768):
     """Put a seeded prompt state on the device.
 
     Retrieval rows: written straight into the documented cache layout (bf16),
-    or appended through duo_append_kv, which quantizes them (8-bit; the other
-    heads get zero rows there).  Streaming rings: built by the library's own
+    or appended through duo_append_kv, which quantizes them (8- or 4-bit; the
+    other heads get zero rows there).  Streaming rings: built by the library's own
     append -- seq_len is set to 0 and the prompt's first W = sink + recent
     tokens are appended, then seq_len is set to L - W and its last W tokens
     are appended (every head's rows, so a retrieval head gets its own rows
@@ -355,9 +363,9 @@ def _fill_decode_state(duo, desc, caches, st, inv, R, sh, table, kv_int8, chunk=
     B = len(lengths)
     W = sh.sink + sh.recent
     assert int(lengths.min()) >= 2 * W, "bench states are built for prompts of at least 2 (sink + recent) tokens"
-    if kv_int8:
+    if kv_bits:
         L = int(lengths.max())
-        assert np.all(lengths == L), "8-bit states are built for equal lengths"
+        assert np.all(lengths == L), "quantized states are built for equal lengths"
         for c0 in range(0, L, chunk):
             T = min(chunk, L - c0)
             kc = torch.zeros((B, T, sh.n_kv_heads, sh.head_dim), dtype=torch.bfloat16, device="cuda")
@@ -391,14 +399,14 @@ def _fill_decode_state(duo, desc, caches, st, inv, R, sh, table, kv_int8, chunk=
     assert duo.check_status(caches.state) == 0
 
 
-def _decode_bytes(sh, R, lengths_after, kv_int8=False):
+def _decode_bytes(sh, R, lengths_after, kv_bits=0):
     """Algorithmic HBM bytes of one fused decode step: every cached K/V row of
-    every retrieval head once (8-bit: d codes + a 4-byte scale per row), the
-    ring rows of the streaming heads, q and out, and the new token's K/V rows
-    read once and written once into the caches."""
+    every retrieval head once (8-bit: d code bytes + a 4-byte scale per row;
+    4-bit: d / 2 + 4), the ring rows of the streaming heads, q and out, and
+    the new token's K/V rows read once and written once into the caches."""
     S_ = sh.n_kv_heads - R
     row = sh.head_dim * 2
-    full_row = sh.head_dim + 4 if kv_int8 else row
+    full_row = {8: sh.head_dim + 4, 4: sh.head_dim // 2 + 4}.get(int(kv_bits), row)
     total = 0
     for L in lengths_after:
         total += R * (L - 1) * full_row * 2
@@ -481,8 +489,8 @@ def run_decode(args, wl, world, rank):
     e2e = _decode_e2e(duo, env, layers, total, n_e2e, world) if n_e2e else None
 
     hbm, _, peak_kind = _peaks()
-    kernel = "decode_q8_kernel" if wl.get("kv_int8") else "decode_mma_kernel"
-    bytes_per_launch = statistics.mean(_decode_bytes(sh, R, L, bool(wl.get("kv_int8"))) for L in lengths_seen)
+    kernel = {8: "decode_q8_kernel", 4: "decode_q4_kernel"}.get(wl.get("kv_bits", 0), "decode_mma_kernel")
+    bytes_per_launch = statistics.mean(_decode_bytes(sh, R, L, wl.get("kv_bits", 0)) for L in lengths_seen)
     dec_avg_s = statistics.mean(dec_ms) * 1e-3
     achieved = bytes_per_launch / dec_avg_s / 1e9
     res = {
@@ -493,7 +501,8 @@ def run_decode(args, wl, world, rank):
                    "head_dim": sh.head_dim, "n_retrieval": R, "sink": sh.sink, "recent": sh.recent,
                    "context": [int(env["lengths"].min()), int(env["lengths"].max())],
                    "paged": bool(wl.get("paged", False)), "layers_per_step": nl,
-                   "full_cache": "int8 codes + fp32 scale per row" if wl.get("kv_int8") else "bf16",
+                   "full_cache": {8: "int8 codes + fp32 scale per row", 4: "4-bit codes + fp32 scale per row"}.get(
+                       wl.get("kv_bits", 0), "bf16"),
                    "parallelism": f"replicas{world}",
                    "l2": f"not flushed: inputs larger than L2 (each step streams {nl} layers' caches, "
                          f"{nl * bytes_per_launch / 1e6:.0f} MB > 126 MB)"},
@@ -591,13 +600,13 @@ def _decode_e2e(duo, env, layers, first, n, world):
             "note": "bytes per step (all layers); copies on their own streams, double-buffered"}
 
 
-def _oracle_cache(O, st, gate, sh, b_list, heads, kv_int8):
+def _oracle_cache(O, st, gate, sh, b_list, heads, kv_bits):
     """The oracle's caches for sequences b_list and KV heads `heads` of a
     seeded state: retrieval heads hold every prompt row; a streaming head the
     positions the oracle's own eviction rule keeps, with their seeded rows."""
     g = np.array([gate[h] for h in heads], dtype=np.uint8)
     cache = O.HeadSplitCache(len(b_list), len(heads), sh.head_dim, gate=g, sink=sh.sink, recent=sh.recent,
-                             kv_int8=kv_int8)
+                             kv_int8=kv_bits == 8, kv_int4=kv_bits == 4)
     for bi, b in enumerate(b_list):
         L = int(st.lengths[b])
         kept = O.streaming_positions(L, sh.sink, sh.recent)
@@ -618,7 +627,7 @@ def _decode_cpu_baseline(env, budget_s=8.0):
     import oracle as O
     sh, B = env["sh"], env["B"]
     cache = _oracle_cache(O, env["state"], env["gate"], sh, list(range(B)), list(range(sh.n_kv_heads)),
-                          env.get("kv_int8", False))
+                          env.get("kv_bits", 0))
     t0 = time.perf_counter()
     n = 0
     while n < len(env["qs"]) and (time.perf_counter() - t0 < budget_s or n < 1):
@@ -887,7 +896,7 @@ def run_reference(args, wl, budget_s: float = 120.0):
     qs, ks, vs = S.decode_steps(sh, B, total, sigma=sigma)
 
     def build(b_list, heads):
-        return _oracle_cache(O, st, gate, sh, b_list, heads, bool(wl.get("kv_int8")))
+        return _oracle_cache(O, st, gate, sh, b_list, heads, wl.get("kv_bits", 0))
 
     def sl(i, b_list, heads):
         G = sh.group
@@ -900,7 +909,7 @@ def run_reference(args, wl, budget_s: float = 120.0):
     t0 = time.perf_counter()
     cache.decode(*sl(0, full_b, full_heads))
     t_full = time.perf_counter() - t0
-    bytes_full = _decode_bytes(sh, R, lengths + 1, bool(wl.get("kv_int8")))
+    bytes_full = _decode_bytes(sh, R, lengths + 1, wl.get("kv_bits", 0))
     if total * t_full <= budget_s:
         b_list, heads, scale, sample = full_b, full_heads, 1.0, "full decode steps"
         first = 1
@@ -911,7 +920,7 @@ def run_reference(args, wl, budget_s: float = 120.0):
         b_list = [0]
         sub = S.LayerShape(sh.group * len(heads), len(heads), sh.head_dim, "bf16", sh.sink, sh.recent)
         n_ret = 1 if ret0 is not None else 0
-        bytes_sample = _decode_bytes(sub, n_ret, lengths[:1] + 1, bool(wl.get("kv_int8")))
+        bytes_sample = _decode_bytes(sub, n_ret, lengths[:1] + 1, wl.get("kv_bits", 0))
         scale = bytes_full / bytes_sample
         sample = (f"sequence 0, KV heads {heads} (one retrieval, one streaming) with their query heads; "
                   f"time scaled x{scale:.1f} to the whole step by algorithmic bytes")
@@ -972,7 +981,8 @@ def run_ratio_sweep(args, world, rank):
                     "tflops": res["roofline"]["achieved"]})
     return {"metric": "decode us/step/layer and pre-fill ms vs retrieval-head ratio", "n_gpus": world,
             "data": "synthetic",
-            "decode": {"workload": "mha_decode_32k (32 heads, context 32,768, 4 layers/step, 64 steps)",
+            "decode": {"workload": f"mha_decode_32k (32 heads, context 32,768, "
+                                   f"{args.layers or WORKLOADS['mha_decode_32k']['layers']} layers/step, 64 steps)",
                        "points": dec,
                        "fit_us_vs_ratio": _linear_fit([d["ratio"] for d in dec],
                                                       [d["us_per_step_layer"] for d in dec])},

@@ -11,6 +11,7 @@
 // (an atomic ticket, no waiting), after every CTA has read the old value.
 #include "common.cuh"
 #include "internal.h"
+#include "kvq4.cuh"
 #include "kvq8.cuh"
 
 namespace duo {
@@ -85,13 +86,14 @@ __global__ void __launch_bounds__(256) append_kernel(const LayerArgs a, const Ca
 }
 
 // ------------------------------------------------------------------------
-// 8-bit full cache: one warp per (token, KV head, K|V) row.  A retrieval row
-// is quantized and stored in the 8-bit layouts (kvq8.cuh); a streaming row is
-// copied into the ring as in the plain kernel.
+// 8- and 4-bit full caches: one warp per (token, KV head, K|V) row.  A
+// retrieval row is quantized and stored in the BITS-bit layouts (kvq8.cuh,
+// kvq4.cuh); a streaming row is copied into the ring as in the plain kernel.
 
-__global__ void __launch_bounds__(256) append_q8_kernel(const LayerArgs a, const CacheArgs c,
-                                                        const __nv_bfloat16* __restrict__ k_new,
-                                                        const __nv_bfloat16* __restrict__ v_new, const int T) {
+template <int BITS>
+__global__ void __launch_bounds__(256) append_q_kernel(const LayerArgs a, const CacheArgs c,
+                                                       const __nv_bfloat16* __restrict__ k_new,
+                                                       const __nv_bfloat16* __restrict__ v_new, const int T) {
     const int lane = threadIdx.x & 31;
     const long rows = (long)a.B * T * a.Hkv;             // input rows per tensor
     const long warps = (long)gridDim.x * (blockDim.x >> 5);
@@ -114,8 +116,14 @@ __global__ void __launch_bounds__(256) append_q8_kernel(const LayerArgs a, const
             const uint2 w = reinterpret_cast<const uint2*>(src)[lane];
             const float xv[4] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y)};
             float scale;
-            const uint32_t codes = q8_quantize(xv, scale);
-            q8_store_row(a, c, kv, b, slot, p, codes, scale, lane);
+            if constexpr (BITS == 8) {
+                const uint32_t codes = q8_quantize(xv, scale);
+                q8_store_row(a, c, kv, b, slot, p, codes, scale, lane);
+            } else {
+                int codes[4];
+                q4_quantize(xv, codes, scale);
+                q4_store_row(a, c, kv, b, slot, p, codes, scale, lane);
+            }
         } else {
             if (p < 0) {
                 if (lane == 0 && kv == 0) atomicOr(c.status, DUO_DEV_BAD_LENGTH);
@@ -147,13 +155,17 @@ __global__ void __launch_bounds__(256) append_q8_kernel(const LayerArgs a, const
 
 cudaError_t launch_append(const LayerArgs& a, const CacheArgs& c, const void* k_new, const void* v_new, int T,
                           cudaStream_t s) {
-    if (a.kv_int8) {
+    if (a.kv_bits) {
         const long warps = 2L * a.B * T * a.Hkv;
         long blocks = (warps + 7) / 8;
         if (blocks > 148L * 8) blocks = 148L * 8;
         if (blocks < 1) blocks = 1;
-        append_q8_kernel<<<(unsigned)blocks, 256, 0, s>>>(a, c, static_cast<const __nv_bfloat16*>(k_new),
-                                                          static_cast<const __nv_bfloat16*>(v_new), T);
+        const auto* kn = static_cast<const __nv_bfloat16*>(k_new);
+        const auto* vn = static_cast<const __nv_bfloat16*>(v_new);
+        if (a.kv_bits == 8)
+            append_q_kernel<8><<<(unsigned)blocks, 256, 0, s>>>(a, c, kn, vn, T);
+        else
+            append_q_kernel<4><<<(unsigned)blocks, 256, 0, s>>>(a, c, kn, vn, T);
         return cudaGetLastError();
     }
     const int row_bytes = a.D * (a.dtype == DUO_BF16 ? 2 : 4);

@@ -37,6 +37,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "kvq4.cuh"
 #include "kvq8.cuh"
 
 namespace duo {
@@ -59,6 +60,7 @@ struct DecodeArgs {
     const void* k_new;
     const void* v_new;
     uint32_t* grid_ticket;  // one state counter word: the last CTA advances seq_len
+    uint32_t* tile_ctr;     // [B*R]: tiles handed out past the static ones (tensor-core bf16 kernel)
 };
 
 template <typename T, int D>
@@ -193,99 +195,113 @@ __device__ __forceinline__ void decode_finish(float* sM, uint64_t* comb_bar, int
     }
     __threadfence();
     // This CTA is the last of its (b, r) pair: every split's record is in
-    // global memory (L2).  (1) m and l of all splits into shared memory,
-    // (2) the per-head maximum, each split's weight and 1 / L, (3) the
-    // records themselves stream into the free stage buffers with bulk copies
-    // (the TMA engine moves them at L2 bandwidth), a batch at a time, and each
-    // thread accumulates its outputs from shared memory.
+    // global memory (L2).  (1) The first batch of records starts streaming
+    // into the free stage buffers with a bulk copy (the TMA engine moves
+    // them at L2 bandwidth) while (2) the splits' m and l, read from L2, give
+    // the per-head maximum, each split's weight and 1 / L.  (3) Each thread
+    // accumulates float4 quads of outputs over its share of the splits, a
+    // batch of records at a time; where a group has fewer quads than there
+    // are threads (MHA: 32 quads), the splits are dealt out to TP threads
+    // per quad and their partial sums added at the end.
     const float* all = d.partial + pair * d.nsplit * (size_t)G * STRIDE;
     const int ns = d.nsplit;
     float* s_w = sM;                            // [ns][G] weights (the stage buffers are free)
-    float* s_l = s_w + ns * G;                  // [ns][G]
-    float* s_inv = s_l + ns * G;                // [G] 1 / L
+    float* s_inv = s_w + 128 * G;               // [G] 1 / L (ns <= 128)
     constexpr int kRecFloats = G * STRIDE;      // one split's record
-    constexpr size_t kHead = ((2 * 128 * G + G) * sizeof(float) + 1023) / 1024 * 1024;
+    constexpr size_t kHead = ((128 * G + G) * sizeof(float) + 1023) / 1024 * 1024;
     constexpr int kBatch = (int)((kStageBytes - kHead) / (kRecFloats * sizeof(float)));
     static_assert(kBatch >= 1, "a split-K record must fit in the stage buffers");
     float* stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sM) + kHead);
-    uint32_t phase = 0;
-    const bool one_batch = ns <= kBatch;
-    if (one_batch) {
-        // every record fits: one bulk copy brings m, l and o of all splits
-        if (threadIdx.x == 0) {
-            const uint32_t bytes = (uint32_t)(ns * kRecFloats * sizeof(float));
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(comb_bar, bytes);
-            bulk_g2s(stage, all, bytes, comb_bar);
-        }
-        if (!mbar_wait(comb_bar, phase, c.status)) return;
-        phase ^= 1;
-        for (int i = threadIdx.x; i < ns * G; i += kThreads) {
-            s_w[i] = stage[(size_t)i * STRIDE];
-            s_l[i] = stage[(size_t)i * STRIDE + 1];
-        }
-    } else {
-        for (int i = threadIdx.x; i < ns * G; i += kThreads) {
-            const float* rec = all + (size_t)i * STRIDE;  // records of one split are [G][STRIDE]
-            s_w[i] = __ldcg(rec);
-            s_l[i] = __ldcg(rec + 1);
-        }
-    }
-    __syncthreads();
+    constexpr int kQuads = G * D / 4;                            // float4 outputs of the group
+    constexpr int TP = kQuads >= kThreads ? 1 : kThreads / kQuads;  // threads per quad
+    auto issue_batch = [&](int b0) {
+        const int nb = min(kBatch, ns - b0);
+        const uint32_t bytes = (uint32_t)(nb * kRecFloats * sizeof(float));
+        fence_proxy_async_smem();  // earlier thread accesses of this space before the async-proxy writes
+        mbar_arrive_expect_tx(comb_bar, bytes);
+        bulk_g2s(stage, all + (size_t)b0 * kRecFloats, bytes, comb_bar);
+    };
+    if (threadIdx.x == 0) issue_batch(0);
     // one warp per query head of the group, a lane per split (and per split
-    // + 32, ...): the maximum and the sum are warp reductions, so the weights
-    // take a few steps instead of ns serial exponentials
+    // + 32, ...): the maximum and the sum are warp reductions
     for (int g = warp; g < G; g += kThreads / 32) {
         float M = kNegBig;
-        for (int sp = lane; sp < ns; sp += 32) M = fmaxf(M, s_w[sp * G + g]);
+        for (int sp = lane; sp < ns; sp += 32) M = fmaxf(M, __ldcg(all + (size_t)sp * kRecFloats + g * STRIDE));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
         float L = 0.f;
         for (int sp = lane; sp < ns; sp += 32) {
-            const float w = exp2f(s_w[sp * G + g] - M);
+            const float* rec = all + (size_t)sp * kRecFloats + g * STRIDE;
+            const float w = exp2f(__ldcg(rec) - M);
             s_w[sp * G + g] = w;
-            L += w * s_l[sp * G + g];
+            L += w * __ldcg(rec + 1);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
         if (lane == 0) s_inv[g] = L > 0.f ? 1.f / L : 0.f;
     }
     __syncthreads();
-    constexpr int kOut = (G * D + kThreads - 1) / kThreads;  // outputs per thread
-    float acc[kOut];
+    constexpr int kQPer = (kQuads + kThreads - 1) / kThreads;     // quads per thread (TP == 1)
+    float4 acc[kQPer];
 #pragma unroll
-    for (int k = 0; k < kOut; ++k) acc[k] = 0.f;
+    for (int k = 0; k < kQPer; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int sub = (int)threadIdx.x / kQuads;                    // this thread's share of the splits (TP > 1)
+    uint32_t phase = 0;
     for (int b0 = 0; b0 < ns; b0 += kBatch) {
         const int nb = min(kBatch, ns - b0);
-        if (!one_batch && threadIdx.x == 0) {
-            const uint32_t bytes = (uint32_t)(nb * kRecFloats * sizeof(float));
-            fence_proxy_async_smem();  // earlier thread accesses of this space before the async-proxy writes
-            mbar_arrive_expect_tx(comb_bar, bytes);
-            bulk_g2s(stage, all + (size_t)b0 * kRecFloats, bytes, comb_bar);
-        }
-        if (!one_batch) {
-            if (!mbar_wait(comb_bar, phase, c.status)) break;
-            phase ^= 1;
-        }
+        // a CTA-uniform decision: no thread may leave while others wait at a barrier
+        if (!__syncthreads_and(mbar_wait(comb_bar, phase, c.status))) return;
+        phase ^= 1;
 #pragma unroll
-        for (int k = 0; k < kOut; ++k) {
-            const int i = threadIdx.x + k * kThreads;
-            if (i < G * D) {
-                const int g = i / D, e = i % D;
-                float v = acc[k];
-                for (int sp = 0; sp < nb; ++sp)
-                    v = fmaf(s_w[(b0 + sp) * G + g], stage[sp * kRecFloats + g * STRIDE + 4 + e], v);
+        for (int k = 0; k < kQPer; ++k) {
+            const int qd = TP > 1 ? (int)threadIdx.x % kQuads : (int)threadIdx.x + k * kThreads;
+            if (qd < kQuads && (TP == 1 || sub < TP)) {
+                const int g = (4 * qd) / D, e = (4 * qd) % D;
+                float4 v = acc[k];
+                for (int sp = TP > 1 ? sub : 0; sp < nb; sp += TP) {
+                    const float w = s_w[(b0 + sp) * G + g];
+                    const float4 x = *reinterpret_cast<const float4*>(stage + sp * kRecFloats + g * STRIDE + 4 + e);
+                    v.x = fmaf(w, x.x, v.x);
+                    v.y = fmaf(w, x.y, v.y);
+                    v.z = fmaf(w, x.z, v.z);
+                    v.w = fmaf(w, x.w, v.w);
+                }
                 acc[k] = v;
             }
         }
         __syncthreads();  // the next batch overwrites the staging area
+        if (threadIdx.x == 0 && b0 + kBatch < ns) issue_batch(b0 + kBatch);
+    }
+    if constexpr (TP > 1) {
+        // add the TP partial sums of each quad (the staging area is free)
+        float4* part = reinterpret_cast<float4*>(stage);
+        if (sub < TP) part[sub * kQuads + (int)threadIdx.x % kQuads] = acc[0];
+        __syncthreads();
+        if ((int)threadIdx.x < kQuads) {
+            float4 v = part[threadIdx.x];
+            for (int t = 1; t < TP; ++t) {
+                const float4 x = part[t * kQuads + threadIdx.x];
+                v.x += x.x;
+                v.y += x.y;
+                v.z += x.z;
+                v.w += x.w;
+            }
+            acc[0] = v;
+        }
     }
 #pragma unroll
-    for (int k = 0; k < kOut; ++k) {
-        const int i = threadIdx.x + k * kThreads;
-        if (i < G * D) outp[i] = Elem<T>::from_f32(acc[k] * s_inv[i / D]);
+    for (int k = 0; k < kQPer; ++k) {
+        const int qd = (int)threadIdx.x + k * kThreads;
+        if (qd < kQuads) {
+            const float inv = s_inv[(4 * qd) / D];
+            const float v[4] = {acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv};
+            store_row<T, 4>(outp + 4 * qd, v);
+        }
     }
-    if (threadIdx.x == 0) d.ticket[pair] = 0u;  // leave the workspace ready for the next call
+    if (threadIdx.x == 0) {                     // leave the workspace ready for the next call
+        d.ticket[pair] = 0u;
+        if (d.tile_ctr) d.tile_ctr[pair] = 0u;
+    }
 }
 
 template <typename T, int D, int G, bool PAGED>
@@ -676,6 +692,14 @@ __device__ __forceinline__ uint32_t sw_off(int row, int c16) {
 }
 
 constexpr int kWarmTiles = 2;  // K and V tiles per split brought into L2 before the dependency wait
+// Tiles each split of decode_mma_kernel takes by its index before it draws
+// further tiles from its head's counter: split s takes tiles s, s + nsplit,
+// ..., then nsplit * kStaticTiles + (counter draws).
+constexpr int kStaticTiles = 2;
+
+// The k-th tile split `split` takes when the tiles are not drawn from a
+// counter (one split: all of them in order; otherwise the static ones).
+__device__ __forceinline__ int static_tile(int split, int nsplit, int k) { return split + k * nsplit; }
 
 // Runs before griddepcontrol.wait, while the previous grid on the stream may
 // still be streaming its own caches: asks L2 for the first kWarmTiles K and V
@@ -688,16 +712,12 @@ __device__ __forceinline__ void warm_l2_split(const LayerArgs& a, const CacheArg
     constexpr int kRowBytes = 128 * 2;
     int len = ld_relaxed_gpu(&c.seq_len[b]) + (d.k_new != nullptr ? 1 : 0);
     len = max(0, min(len, a.capacity));
-    const int per = (len + d.nsplit - 1) / d.nsplit;
-    const int chunk = (per + kTile - 1) / kTile * kTile;
-    const int row_begin = min(len, split * chunk);
-    const int row_end = min(len, row_begin + chunk);
-    const int n_tiles = min(kWarmTiles, (row_end - row_begin + kTile - 1) / kTile);
     const uint8_t* kf = static_cast<const uint8_t*>(c.k_full);
     const uint8_t* vf = static_cast<const uint8_t*>(c.v_full);
-    for (int t = 0; t < n_tiles; ++t) {
-        const int r0 = row_begin + t * kTile;
-        const uint32_t bytes = (uint32_t)min(kTile, row_end - r0) * kRowBytes;
+    for (int k = 0; k < kWarmTiles; ++k) {
+        const int r0 = static_tile(split, d.nsplit, k) * kTile;
+        if (r0 >= len) break;
+        const uint32_t bytes = (uint32_t)min(kTile, len - r0) * kRowBytes;
         size_t off;
         if (PAGED) {
             const int pg = ld_relaxed_gpu(&c.page_table[(size_t)b * a.max_pages + r0 / kTile]);
@@ -788,27 +808,29 @@ __global__ void __maxnreg__(200)
             len = L0 + 1;
         }
     }
-    int row_begin = 0, row_end = 0;
+    // Retrieval: the cache rows [0, len) of the (sequence, head) in 64-row
+    // tiles, shared out to the head's splits -- each takes kStaticTiles by
+    // its index, then draws the rest from the head's counter, so that splits
+    // on SMs that stream faster take more tiles and all end together.
+    // Streaming: the min(len, W) ring rows.
+    int rows;
     if (retrieval) {
         if (len > a.capacity || len < 0) {
             if (threadIdx.x == 0 && split == 0) atomicOr(c.status, DUO_DEV_BAD_LENGTH);
             len = len < 0 ? 0 : a.capacity;
         }
-        const int per = (len + d.nsplit - 1) / d.nsplit;
-        const int chunk = (per + kTile - 1) / kTile * kTile;
-        row_begin = min(len, split * chunk);
-        row_end = min(len, row_begin + chunk);
+        rows = len;
     } else {
-        row_end = len < 0 ? 0 : min(len, a.W);
+        rows = len < 0 ? 0 : min(len, a.W);
     }
-    const int n_tiles = (row_end - row_begin + kTile - 1) / kTile;
+    const int total_tiles = (rows + kTile - 1) / kTile;
+    const size_t pair = (size_t)b * a.R + slot;
 
     if (warp == NW) {
         // ------------------------------------------------------ producer
-        const bool owns_new = new_row >= 0 && (!retrieval || (new_row >= row_begin && new_row < row_end));
-        if (owns_new) {
-            // the new token goes into its cache first; the tile that holds it
-            // is then read back through TMA
+        // the new token goes into its cache (whole warp) before the tile
+        // that holds it is read back through TMA
+        auto store_new_row = [&]() {
             const T* kn = static_cast<const T*>(d.k_new) + ((size_t)b * a.Hkv + a.kv_head[slot]) * D;
             const T* vn = static_cast<const T*>(d.v_new) + ((size_t)b * a.Hkv + a.kv_head[slot]) * D;
             T* dk = nullptr;
@@ -840,43 +862,60 @@ __global__ void __maxnreg__(200)
                 asm volatile("fence.proxy.async.global;" ::: "memory");
             }
             __syncwarp();
-        }
-        if (lane == 0) {
-            const CUtensorMap* mk = retrieval ? &tmKf : &tmKr;
-            const CUtensorMap* mv = retrieval ? &tmVf : &tmVr;
-            const int z = retrieval ? b * a.R + slot : b * a.S + (slot - a.R);
-            for (int t = 0; t < n_tiles; ++t) {
-                const int st = t % STAGES, round = t / STAGES;
-                if (round > 0 && !mbar_wait(&empty_bar[st], (round - 1) & 1, c.status)) break;
-                const int r0 = row_begin + t * kTile;
-                const int n = min(kTile, row_end - r0);
+        };
+        if (!retrieval && new_row >= 0) store_new_row();   // the ring's one tile holds every slot
+        const CUtensorMap* mk = retrieval ? &tmKf : &tmKr;
+        const CUtensorMap* mv = retrieval ? &tmVf : &tmVr;
+        const int z = retrieval ? b * a.R + slot : b * a.S + (slot - a.R);
+        const bool draw = retrieval && d.nsplit > 1 && d.tile_ctr != nullptr;
+        uint32_t drawn = 0;   // lane 0: the counter draw for the next tile, made while this one loads
+        for (int i = 0;; ++i) {
+            const int st = i % STAGES, round = i / STAGES;
+            int ok = 1;
+            if (lane == 0 && round > 0) ok = mbar_wait(&empty_bar[st], (round - 1) & 1, c.status) ? 1 : 0;
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            const int t = (draw && i >= kStaticTiles)
+                              ? kStaticTiles * d.nsplit + (int)__shfl_sync(0xffffffffu, drawn, 0)
+                              : (retrieval ? static_tile(split, d.nsplit, i) : i);
+            if (t >= total_tiles) {
+                if (lane == 0) {             // no more tiles: tell the consumers
+                    s_tile_n[st] = -1;
+                    mbar_arrive(&full_bar[st]);
+                }
+                break;
+            }
+            const int r0 = t * kTile;
+            const int n = min(kTile, rows - r0);
+            if (retrieval && new_row >= r0 && new_row < r0 + n) store_new_row();
+            if (lane == 0) {
                 int pg = 0;
-                bool ok = true;
+                bool page_ok = true;
                 if (PAGED && retrieval) {
-                    pg = c.page_table[(size_t)b * a.max_pages + r0 / kTile];
+                    pg = c.page_table[(size_t)b * a.max_pages + t];
                     if (pg < 0 || pg >= a.n_pages) {
                         atomicOr(c.status, DUO_DEV_BAD_PAGE);
-                        ok = false;
+                        page_ok = false;
                     }
                 }
-                s_tile_n[st] = ok ? n : 0;
-                if (!ok) {
+                s_tile_n[st] = page_ok ? n : 0;
+                if (!page_ok) {
                     mbar_arrive(&full_bar[st]);  // an empty tile: every key of it is masked
-                    continue;
-                }
-                mbar_arrive_expect_tx(&full_bar[st], 2 * kMmaTileBytes);
-                const uint32_t dk = smem_u32(sKb + (size_t)st * kMmaTileBytes);
-                const uint32_t dv = smem_u32(sVb + (size_t)st * kMmaTileBytes);
-                for (int h = 0; h < 2; ++h) {
-                    const uint32_t off = h * (kMmaTileBytes / 2);
-                    if (PAGED && retrieval) {
-                        tma_load_4d(dk + off, mk, 64 * h, 0, slot, pg, &full_bar[st]);
-                        tma_load_4d(dv + off, mv, 64 * h, 0, slot, pg, &full_bar[st]);
-                    } else {
-                        tma_load_3d(dk + off, mk, 64 * h, r0, z, &full_bar[st]);
-                        tma_load_3d(dv + off, mv, 64 * h, r0, z, &full_bar[st]);
+                } else {
+                    mbar_arrive_expect_tx(&full_bar[st], 2 * kMmaTileBytes);
+                    const uint32_t dk = smem_u32(sKb + (size_t)st * kMmaTileBytes);
+                    const uint32_t dv = smem_u32(sVb + (size_t)st * kMmaTileBytes);
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t off = h * (kMmaTileBytes / 2);
+                        if (PAGED && retrieval) {
+                            tma_load_4d(dk + off, mk, 64 * h, 0, slot, pg, &full_bar[st]);
+                            tma_load_4d(dv + off, mv, 64 * h, 0, slot, pg, &full_bar[st]);
+                        } else {
+                            tma_load_3d(dk + off, mk, 64 * h, r0, z, &full_bar[st]);
+                            tma_load_3d(dv + off, mv, 64 * h, r0, z, &full_bar[st]);
+                        }
                     }
                 }
+                if (draw && i + 1 >= kStaticTiles) drawn = atomicAdd(&d.tile_ctr[pair], 1u);
             }
         }
     }
@@ -902,10 +941,11 @@ __global__ void __maxnreg__(200)
         for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = 0.f;
         const float sl = a.scale * kLog2e;
         const int key_base = warp * 16;
-        for (int t = 0; t < n_tiles; ++t) {
+        for (int t = 0;; ++t) {
             const int st = t % STAGES, round = t / STAGES;
             if (!mbar_wait(&full_bar[st], round & 1, c.status)) break;
             const int n = s_tile_n[st];
+            if (n < 0) break;                // the producer has no more tiles
             const uint32_t tK = smem_u32(sKb + (size_t)st * kMmaTileBytes);
             uint8_t* tVp = sVb + (size_t)st * kMmaTileBytes;
             const uint32_t tV = smem_u32(tVp);
@@ -1495,6 +1535,266 @@ cudaError_t launch_q8_g(const LayerArgs& a, const CacheArgs& c, const DecodeArgs
     return launch_pdl(kern, grid, kMmaThreads, smem, s, mK, mV, a, c, d);
 }
 
+// ===========================================================================
+// 4-bit full cache: decode_q4_kernel.  The 8-bit kernel's work units,
+// producer/consumer pipeline, streaming path and split-K combine, over the
+// 4-bit layouts of kvq4.cuh: a 64-token stage is 4 KB of K codes and 4 KB of
+// V codes, each one contiguous bulk copy (the layouts are already in the
+// order the consumers read, so no tensor map or swizzle is needed), plus the
+// tile's 64 + 64 scales; ten stages.
+//   S = q . codes: a lane's 16 bytes of a key's row hold its 32 permuted
+//     features; each word gives two k-steps' B fragments by masking nibble
+//     pairs into fp16 (u4x2_to_f16x2); q is permuted as for the 8-bit cache.
+//   O += P V: one word per (feature pair, key quad) gives the B fragments of
+//     feature rows 16 m + r and 16 m + 8 + r for the lane's four keys.
+// ===========================================================================
+
+constexpr int kQ4Stages = 10;
+constexpr uint32_t kQ4ScBytes = 2 * kTile * 4;      // K and V scales of a stage
+
+constexpr size_t decode_q4_smem_bytes() {
+    return 2 * (size_t)kQ4Stages * kQ4TileBytes + kQ4Stages * kQ4ScBytes + (2 * kQ4Stages + 1) * sizeof(uint64_t) + 64;
+}
+static_assert(ring_simt_smem_bytes(8) <= 2 * (size_t)kQ4Stages * kQ4TileBytes + kQ4Stages * kQ4ScBytes,
+              "the ring path must fit below the 4-bit kernel's barriers");
+
+template <int G>
+__global__ void __maxnreg__(200)
+    decode_q4_kernel(const LayerArgs a, const CacheArgs c, const DecodeArgs d) {
+    using T = __nv_bfloat16;
+    constexpr int D = 128;
+    constexpr int STAGES = kQ4Stages;
+    constexpr int NW = kMmaWarps;
+    constexpr int kThreads = kMmaThreads;
+    static_assert(G <= 8, "the group must fit the 8 live rows of an m16 tile");
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t* sK4 = smem;
+    uint8_t* sV4 = smem + (size_t)STAGES * kQ4TileBytes;
+    float* sSc = reinterpret_cast<float*>(smem + 2 * (size_t)STAGES * kQ4TileBytes);
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + 2 * (size_t)STAGES * kQ4TileBytes + STAGES * kQ4ScBytes);
+    uint64_t* empty_bar = full_bar + STAGES;
+    uint64_t* comb_bar = empty_bar + STAGES;
+    int* s_flag = reinterpret_cast<int*>(comb_bar + 1);
+    int* s_tile_n = s_flag + 1;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // ---------------------------------------------------------- work unit
+    const bool retrieval = (int)blockIdx.x < d.n_ret_units;
+    int split = 0, slot, b;
+    if (retrieval) {
+        split = blockIdx.x % d.nsplit;
+        const int pair = blockIdx.x / d.nsplit;
+        slot = pair % a.R;
+        b = pair / a.R;
+    } else {
+        const int u = blockIdx.x - d.n_ret_units;
+        slot = a.R + u % a.S;
+        b = u / a.S;
+    }
+    const size_t z = (size_t)b * a.R + slot;
+    const bool fused = d.k_new != nullptr;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], NW);
+        }
+        mbar_init(comb_bar, 1);
+        fence_barrier_init();
+    }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (threadIdx.x == 0) *s_flag = c.seq_len[b];
+    __syncthreads();
+    const int L0 = *s_flag;
+    if (fused && d.grid_ticket && threadIdx.x == 0) length_ticket(a, c, d);
+    if (!retrieval) {
+        decode_ring_simt<G>(smem, a, c, d, b, slot, L0, fused);
+        return;
+    }
+    int len = L0;
+    int new_row = -1;
+    if (fused) {
+        if (L0 < 0) {
+            if (threadIdx.x == 0) atomicOr(c.status, DUO_DEV_BAD_LENGTH);
+            len = 0;
+        } else if (L0 >= a.capacity) {
+            if (threadIdx.x == 0 && split == 0) atomicOr(c.status, DUO_DEV_FULL_CACHE_OVERFLOW);
+        } else {
+            new_row = L0;
+            len = L0 + 1;
+        }
+    }
+    if (len > a.capacity || len < 0) {
+        if (threadIdx.x == 0 && split == 0) atomicOr(c.status, DUO_DEV_BAD_LENGTH);
+        len = len < 0 ? 0 : a.capacity;
+    }
+    const int per = (len + d.nsplit - 1) / d.nsplit;
+    const int chunk = (per + kTile - 1) / kTile * kTile;
+    const int row_begin = min(len, split * chunk);
+    const int row_end = min(len, row_begin + chunk);
+    const int n_tiles = (row_end - row_begin + kTile - 1) / kTile;
+
+    if (warp == NW) {
+        // ------------------------------------------------------ producer
+        if (new_row >= row_begin && new_row < row_end) {
+            // the new token goes into the 4-bit cache first, quantized; the
+            // tile that holds it is then read back with bulk copies
+            const int h = a.kv_head[slot];
+            const uint2 kw = reinterpret_cast<const uint2*>(static_cast<const T*>(d.k_new) + ((size_t)b * a.Hkv + h) * D)[lane];
+            const uint2 vw = reinterpret_cast<const uint2*>(static_cast<const T*>(d.v_new) + ((size_t)b * a.Hkv + h) * D)[lane];
+            const float kx[4] = {bf16_lo(kw.x), bf16_hi(kw.x), bf16_lo(kw.y), bf16_hi(kw.y)};
+            const float vx[4] = {bf16_lo(vw.x), bf16_hi(vw.x), bf16_lo(vw.y), bf16_hi(vw.y)};
+            int kc[4], vc[4];
+            float ks, vs;
+            q4_quantize(kx, kc, ks);
+            q4_quantize(vx, vc, vs);
+            q4_store_row(a, c, 0, b, slot, new_row, kc, ks, lane);
+            q4_store_row(a, c, 1, b, slot, new_row, vc, vs, lane);
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            __syncwarp();
+        }
+        if (lane == 0) {
+            const uint8_t* kf = static_cast<const uint8_t*>(c.k_full);
+            const uint8_t* vf = static_cast<const uint8_t*>(c.v_full);
+            for (int t = 0; t < n_tiles; ++t) {
+                const int st = t % STAGES, round = t / STAGES;
+                if (round > 0 && !mbar_wait(&empty_bar[st], (round - 1) & 1, c.status)) break;
+                const int r0 = row_begin + t * kTile;
+                s_tile_n[st] = min(kTile, row_end - r0);
+                mbar_arrive_expect_tx(&full_bar[st], 2 * kQ4TileBytes + kQ4ScBytes);
+                // whole 64-token tiles: the capacity is a multiple of 64
+                bulk_g2s(sK4 + (size_t)st * kQ4TileBytes, kf + (z * a.capacity + r0) * kQ4RowBytes, kQ4TileBytes,
+                         &full_bar[st]);
+                bulk_g2s(sV4 + (size_t)st * kQ4TileBytes, vf + (z * (a.capacity / kTile) + r0 / kTile) * kQ4TileBytes,
+                         kQ4TileBytes, &full_bar[st]);
+                bulk_g2s(sSc + st * 2 * kTile, c.k_scale + z * a.capacity + r0, kTile * 4, &full_bar[st]);
+                bulk_g2s(sSc + st * 2 * kTile + kTile, c.v_scale + z * a.capacity + r0, kTile * 4, &full_bar[st]);
+            }
+        }
+    }
+
+    // ------------------------------------------------------ consumers
+    const int row = lane >> 2;   // query head of the group (rows >= G are padding) / key of an 8-key block
+    const int quad = lane & 3;
+    float o[16][2];
+    float m_run = kNegBig, l_run = 0.f;
+    if (warp < NW) {
+        // q in fp16, features 32 quad + 4 kb + {0, 1} and {2, 3} for step kb
+        uint32_t qa[8][2];
+        {
+            const bool row_ok = row < G;
+            const uint4* qp = reinterpret_cast<const uint4*>(
+                static_cast<const T*>(d.q) + ((size_t)b * a.Hq + a.q_head0[slot] + (row_ok ? row : 0)) * D + 32 * quad);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint4 w = row_ok ? qp[i] : make_uint4(0u, 0u, 0u, 0u);
+                qa[2 * i][0] = f16x2_pack(bf16_lo(w.x), bf16_hi(w.x));
+                qa[2 * i][1] = f16x2_pack(bf16_lo(w.y), bf16_hi(w.y));
+                qa[2 * i + 1][0] = f16x2_pack(bf16_lo(w.z), bf16_hi(w.z));
+                qa[2 * i + 1][1] = f16x2_pack(bf16_lo(w.w), bf16_hi(w.w));
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = 0.f;
+        const float sl = a.scale * kLog2e;
+        const int key_base = warp * 16;
+        for (int t = 0; t < n_tiles; ++t) {
+            const int st = t % STAGES, round = t / STAGES;
+            if (!mbar_wait(&full_bar[st], round & 1, c.status)) break;
+            const int n = s_tile_n[st];
+            const uint8_t* tK = sK4 + (size_t)st * kQ4TileBytes;
+            const uint8_t* tV = sV4 + (size_t)st * kQ4TileBytes;
+            const float* ksc = sSc + st * 2 * kTile;
+            const float* vsc = ksc + kTile;
+            // S = q . codes for keys key_base + 8 nb + (lane >> 2)
+            float s[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+            for (int nb = 0; nb < 2; ++nb) {
+                const int key = key_base + 8 * nb + row;
+                const uint4 kw = *reinterpret_cast<const uint4*>(tK + key * kQ4RowBytes + 16 * quad);
+                const uint32_t w[4] = {kw.x, kw.y, kw.z, kw.w};
+#pragma unroll
+                for (int kb = 0; kb < 8; ++kb) {
+                    const uint32_t x = w[kb >> 1] >> (8 * (kb & 1));
+                    mma_f16_rows8(s[nb][0], s[nb][1], qa[kb][0], qa[kb][1], u4x2_to_f16x2(x), u4x2_to_f16x2(x >> 4));
+                }
+            }
+            // this lane's keys: key_base + 2 quad + {0, 1} and + 8
+            const int k0 = key_base + 2 * quad;
+            const float2 ks0 = *reinterpret_cast<const float2*>(ksc + k0);
+            const float2 ks1 = *reinterpret_cast<const float2*>(ksc + k0 + 8);
+            const float sv[4] = {s[0][0] * ks0.x * sl, s[0][1] * ks0.y * sl, s[1][0] * ks1.x * sl,
+                                 s[1][1] * ks1.y * sl};
+            const bool vk[4] = {k0 < n, k0 + 1 < n, k0 + 8 < n, k0 + 9 < n};
+            float mx = kNegBig;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) mx = vk[i] ? fmaxf(mx, sv[i]) : mx;
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float m_new = fmaxf(m_run, mx);
+            const float corr = exp2f(m_run - m_new);
+            float pr[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) pr[i] = vk[i] ? exp2f(sv[i] - m_new) : 0.f;
+            l_run = l_run * corr + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
+            m_run = m_new;
+            // p times the key's V scale, the fp16 A operand of O += P V
+            const float2 vs0 = *reinterpret_cast<const float2*>(vsc + k0);
+            const float2 vs1 = *reinterpret_cast<const float2*>(vsc + k0 + 8);
+            const uint32_t pa0 = f16x2_pack(vk[0] ? pr[0] * vs0.x : 0.f, vk[1] ? pr[1] * vs0.y : 0.f);
+            const uint32_t pa1 = f16x2_pack(vk[2] ? pr[2] * vs1.x : 0.f, vk[3] ? pr[3] * vs1.y : 0.f);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                o[j][0] *= corr;
+                o[j][1] *= corr;
+            }
+            // O += P V: the word of feature pair (16 m + r, 16 m + 8 + r) and
+            // this lane's key quad in the warp's 16-token group
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const uint32_t w = *reinterpret_cast<const uint32_t*>(tV + 1024 * warp + 128 * m + 16 * row + 4 * quad);
+                mma_f16_rows8(o[2 * m][0], o[2 * m][1], pa0, pa1, u4x2_to_f16x2(w), u4x2_to_f16x2(w >> 8));
+                mma_f16_rows8(o[2 * m + 1][0], o[2 * m + 1][1], pa0, pa1, u4x2_to_f16x2(w >> 4), u4x2_to_f16x2(w >> 12));
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty_bar[st]);
+        }
+        l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+        l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+    }
+    __syncthreads();  // all tiles consumed: the stage buffers are free
+
+    // warp states -> sM[warp][g][STRIDE]: m, l, -, -, o[D]
+    constexpr int STRIDE = D + 4;
+    float* sM = reinterpret_cast<float*>(smem);
+    if (warp < NW && row < G) {
+        float* dst = sM + ((size_t)warp * G + row) * STRIDE;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            dst[4 + 8 * j + 2 * quad] = o[j][0];
+            dst[4 + 8 * j + 2 * quad + 1] = o[j][1];
+        }
+        if (quad == 0) {
+            dst[0] = m_run;
+            dst[1] = l_run;
+        }
+    }
+    __syncthreads();
+    decode_finish<T, D, G, NW, kThreads, 2 * (size_t)STAGES * kQ4TileBytes>(sM, comb_bar, s_flag, a, c, d, b, slot,
+                                                                          split, true, fused);
+}
+
+template <int G>
+cudaError_t launch_q4_g(const LayerArgs& a, const CacheArgs& c, const DecodeArgs& d, int grid, cudaStream_t s) {
+    constexpr size_t smem = decode_q4_smem_bytes();
+    auto kern = decode_q4_kernel<G>;
+    static std::atomic<unsigned long long> configured{0};
+    const cudaError_t e = smem_limit_once(kern, (int)smem, configured);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kern, grid, kMmaThreads, smem, s, a, c, d);
+}
+
 }  // namespace
 
 cudaError_t launch_decode(const LayerArgs& a, const CacheArgs& c, const DecodePlan& plan, const void* q, void* out,
@@ -1507,12 +1807,23 @@ cudaError_t launch_decode(const LayerArgs& a, const CacheArgs& c, const DecodePl
     d.out = out;
     d.partial = static_cast<float*>(workspace);
     d.ticket = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + plan.ticket_offset);
+    d.tile_ctr = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + plan.counter_offset);
     d.nsplit = plan.nsplit;
     d.n_ret_units = a.B * a.R * plan.nsplit;
     const long grid = (long)d.n_ret_units + (long)a.B * a.S;
     if (grid == 0) return cudaSuccess;
     if (grid > 0x7fffffffL) return cudaErrorInvalidConfiguration;
-    if (a.kv_int8 && a.R > 0) {
+    if (a.kv_bits == 4 && a.R > 0) {
+        // 4-bit full cache: as the 8-bit path, over nibble codes
+        switch (a.G) {
+            case 1: return launch_q4_g<1>(a, c, d, (int)grid, s);
+            case 2: return launch_q4_g<2>(a, c, d, (int)grid, s);
+            case 4: return launch_q4_g<4>(a, c, d, (int)grid, s);
+            case 8: return launch_q4_g<8>(a, c, d, (int)grid, s);
+        }
+        return cudaErrorInvalidValue;
+    }
+    if (a.kv_bits == 8 && a.R > 0) {
         // 8-bit full cache: retrieval CTAs on the int8 tiles, streaming CTAs
         // over the bf16 ring on the CUDA cores, one launch
         switch (a.G) {

@@ -63,12 +63,12 @@ duo_status check_desc(const duo_layer_desc* d) {
         return fail(DUO_ERR_INVALID_ARG, "unknown io_order %d", d->io_order);
     if (d->stream_prefill != DUO_STREAM_LAMBDA && d->stream_prefill != DUO_STREAM_CHUNK)
         return fail(DUO_ERR_INVALID_ARG, "unknown stream_prefill %d", d->stream_prefill);
-    if (d->kv_quant != DUO_KV_PLAIN && d->kv_quant != DUO_KV_INT8)
+    if (d->kv_quant != DUO_KV_PLAIN && d->kv_quant != DUO_KV_INT8 && d->kv_quant != DUO_KV_INT4)
         return fail(DUO_ERR_INVALID_ARG, "unknown kv_quant %d", d->kv_quant);
-    if (d->kv_quant == DUO_KV_INT8 &&
+    if (d->kv_quant != DUO_KV_PLAIN &&
         (d->dtype != DUO_BF16 || d->head_dim != 128 || d->page_size != 0 || d->sink + d->recent > 128))
         return fail(DUO_ERR_UNSUPPORTED,
-                    "the 8-bit full cache is built for bf16, head_dim 128, contiguous, sink + recent <= 128");
+                    "the 8- and 4-bit full caches are built for bf16, head_dim 128, contiguous, sink + recent <= 128");
     if (!std::isfinite(d->scale)) return fail(DUO_ERR_INVALID_ARG, "scale is not finite");
     bool seen[DUO_MAX_KV_HEADS] = {};
     for (int i = 0; i < d->n_kv_heads; ++i) {
@@ -94,7 +94,7 @@ void fill_args(const duo_layer_desc* d, duo::LayerArgs& a) {
     a.W = d->sink + d->recent;
     a.dtype = d->dtype;
     a.stream_chunk = d->stream_prefill == DUO_STREAM_CHUNK ? 1 : 0;
-    a.kv_int8 = d->kv_quant == DUO_KV_INT8 ? 1 : 0;
+    a.kv_bits = d->kv_quant == DUO_KV_INT8 ? 8 : d->kv_quant == DUO_KV_INT4 ? 4 : 0;
     a.page_size = d->page_size;
     a.capacity = a.max_pages = a.n_pages = 0;
     a.scale = d->scale > 0.f ? d->scale : 1.0f / std::sqrt(static_cast<float>(d->head_dim));
@@ -150,11 +150,12 @@ duo_status check_state(const duo_layer_desc* d, const duo_kv_state* st, duo::Lay
     c.status = st->status;
     c.k_scale = st->k_scale;
     c.v_scale = st->v_scale;
-    if (d->kv_quant == DUO_KV_INT8 && R > 0) {
-        if (!st->k_scale || !st->v_scale) return fail(DUO_ERR_INVALID_ARG, "8-bit cache needs k_scale and v_scale");
+    if (d->kv_quant != DUO_KV_PLAIN && R > 0) {
+        if (!st->k_scale || !st->v_scale)
+            return fail(DUO_ERR_INVALID_ARG, "an 8- or 4-bit cache needs k_scale and v_scale");
         if (!aligned16(st->k_scale) || !aligned16(st->v_scale))
             return fail(DUO_ERR_INVALID_ARG, "k_scale / v_scale must be 16-byte aligned");
-        if (st->capacity % 64) return fail(DUO_ERR_SHAPE, "8-bit cache capacity must be a multiple of 64");
+        if (st->capacity % 64) return fail(DUO_ERR_SHAPE, "an 8- or 4-bit cache's capacity must be a multiple of 64");
     }
     return DUO_OK;
 }
@@ -184,7 +185,8 @@ DecodePlan decode_plan(const LayerArgs& a) {
     p.nsplit = ns;
     p.partial_floats = (size_t)pairs * ns * a.G * (a.D + 4);
     p.ticket_offset = ((p.partial_floats * sizeof(float)) + 255) / 256 * 256;
-    p.bytes = p.ticket_offset + ((size_t)pairs * sizeof(uint32_t) + 255) / 256 * 256;
+    p.counter_offset = p.ticket_offset + ((size_t)pairs * sizeof(uint32_t) + 255) / 256 * 256;
+    p.bytes = p.counter_offset + ((size_t)pairs * sizeof(uint32_t) + 255) / 256 * 256;
     if (pairs == 0) p.bytes = 256;
     return p;
 }
@@ -385,7 +387,7 @@ duo_status duo_prefill_chunk(const duo_layer_desc* desc, const duo_kv_state* st,
     if (desc->page_size != 0)
         return fail(DUO_ERR_UNSUPPORTED, "duo_prefill_chunk takes a contiguous full cache (page_size 0)");
     if (desc->kv_quant != DUO_KV_PLAIN)
-        return fail(DUO_ERR_UNSUPPORTED, "duo_prefill_chunk reads a plain full cache, not an 8-bit one");
+        return fail(DUO_ERR_UNSUPPORTED, "duo_prefill_chunk reads a plain full cache, not an 8- or 4-bit one");
     cudaError_t e;
     if (a.dtype == DUO_BF16 && a.D == 128) {
         if (!duo::prefill_tc_supported(a))
@@ -439,7 +441,7 @@ duo_status duo_gated_mix(const duo_layer_desc* desc, const float* alpha, const v
         x->page_size = 0;
         x->capacity = 0;
         x->stream_chunk = 0;
-        x->kv_int8 = 0;
+        x->kv_bits = 0;
     }
     if (duo::prefill_tc_supported(as) && duo::prefill_tc_supported(ac)) {
         duo::CacheArgs none{};   // no lengths, no caches: every sequence starts at position 0
@@ -487,7 +489,7 @@ duo_status duo_gated_mix_grad_alpha(const duo_layer_desc* desc, const void* q, c
         x->page_size = 0;
         x->capacity = 0;
         x->stream_chunk = 0;
-        x->kv_int8 = 0;
+        x->kv_bits = 0;
     }
     if (duo::prefill_tc_supported(as) && duo::prefill_tc_supported(ac)) {
         duo::CacheArgs none{};

@@ -34,7 +34,7 @@ struct LayerArgs {
     int B, Hq, Hkv, G, D, R, S, sink, recent, W;
     int dtype, page_size, capacity, max_pages, n_pages;
     int stream_chunk;  // pre-fill: streaming heads see the whole chunk (DUO_STREAM_CHUNK)
-    int kv_int8;       // the full cache holds 8-bit codes + scales (DUO_KV_INT8)
+    int kv_bits;       // the full cache holds 8- or 4-bit codes + scales (DUO_KV_INT8 / DUO_KV_INT4); 0: plain
     float scale;       // softmax scale
     // For block slot i (0..Hkv-1): index of its first query head and of its
     // KV head in the caller's q / k / v / out tensors (model or block order).
@@ -54,7 +54,7 @@ struct CacheArgs {
     int32_t* seq_len;
     uint32_t* counters;
     int32_t* status;
-    float* k_scale;    // 8-bit full cache: per-row scales [B][R][capacity]
+    float* k_scale;    // 8- / 4-bit full cache: per-row scales [B][R][capacity]
     float* v_scale;
 };
 
@@ -64,6 +64,7 @@ struct DecodePlan {
     int nsplit;
     size_t partial_floats;  // B * R * nsplit * G * (D + 2)
     size_t ticket_offset;   // bytes from workspace start to the ticket words
+    size_t counter_offset;  // ... to the tile counters (one per pair, after the tickets)
     size_t bytes;           // total workspace bytes
 };
 

@@ -27,7 +27,7 @@ OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_DTYPE, ERR_CAPACITY, ERR_UNSUPPORTED, ERR_CU
 BF16, FP32 = 0, 1
 ORDER_MODEL, ORDER_BLOCK = 0, 1
 STREAM_LAMBDA, STREAM_CHUNK = 0, 1
-KV_PLAIN, KV_INT8 = 0, 1
+KV_PLAIN, KV_INT8, KV_INT4 = 0, 1, 2
 MODEL_TO_BLOCK, BLOCK_TO_MODEL = 0, 1
 OP_DECODE, OP_PREFILL = 0, 1
 DEV_FULL_CACHE_OVERFLOW, DEV_BAD_PAGE, DEV_WAIT_TIMEOUT, DEV_BAD_LENGTH = 1, 2, 4, 8
@@ -261,6 +261,8 @@ class LayerCaches:
     8-bit full cache: k_full int8 [B, R, capacity, d], v_full int8
     [B, R, capacity / 64, d, 64], k_scale/v_scale fp32 [B, R, capacity]
     (capacity rounded up to a multiple of 64).
+    4-bit full cache: k_full uint8 [B, R, capacity, d / 2], v_full uint8
+    [B, R, capacity / 64, 32 d], scales as for 8 bits.
     Rings: k_ring/v_ring [B, S, sink + recent, d]; ring_pos [B, W] (-1);
     seq_len [B] (0); counters [4] (0); status [1] (0).
     """
@@ -287,12 +289,21 @@ class LayerCaches:
             self.v_full = torch.zeros((B, R, capacity // 64, d, 64), dtype=torch.int8, device=device)
             self.k_scale = torch.zeros((B, R, capacity), dtype=torch.float32, device=device)
             self.v_scale = torch.zeros_like(self.k_scale)
+        elif desc.kv_quant == KV_INT4:
+            # 4-bit codes: K 64 bytes per token, V 4 KB per 64-token tile; fp32 scale per row
+            max_pages = 0
+            self.page_table = None
+            capacity = (max(capacity, 1) + 63) // 64 * 64
+            self.k_full = torch.zeros((B, R, capacity, d // 2), dtype=torch.uint8, device=device)
+            self.v_full = torch.zeros((B, R, capacity // 64, 64 * d // 2), dtype=torch.uint8, device=device)
+            self.k_scale = torch.zeros((B, R, capacity), dtype=torch.float32, device=device)
+            self.v_scale = torch.zeros_like(self.k_scale)
         else:
             max_pages = 0
             self.page_table = None
             self.k_full = torch.zeros((B, R, max(capacity, 0), d), dtype=dt, device=device)
             self.v_full = torch.zeros_like(self.k_full)
-        if desc.kv_quant != KV_INT8:
+        if desc.kv_quant not in (KV_INT8, KV_INT4):
             self.k_scale = self.v_scale = None
         self.capacity = capacity
         self.k_ring = torch.zeros((B, S, W, d), dtype=dt, device=device)

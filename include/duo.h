@@ -71,7 +71,8 @@ enum { DUO_ORDER_MODEL = 0, DUO_ORDER_BLOCK = 1 };
 /* storage of the retrieval heads' full cache */
 enum {
     DUO_KV_PLAIN = 0, /* the layer's dtype, as the activations               */
-    DUO_KV_INT8 = 1   /* 8-bit codes + one fp32 scale per row (see duo_kv_state) */
+    DUO_KV_INT8 = 1,  /* 8-bit codes + one fp32 scale per row (see duo_kv_state) */
+    DUO_KV_INT4 = 2   /* 4-bit codes + one fp32 scale per row (see duo_kv_state) */
 };
 /* what a streaming head sees in duo_prefill_chunk (decode is the same for both) */
 enum {
@@ -107,7 +108,7 @@ typedef struct {
     int32_t n_retrieval;  /* R: retrieval KV heads (block slots 0..R-1)       */
     int32_t io_order;     /* DUO_ORDER_MODEL or DUO_ORDER_BLOCK               */
     int32_t stream_prefill; /* DUO_STREAM_LAMBDA (default) or DUO_STREAM_CHUNK */
-    int32_t kv_quant;     /* DUO_KV_PLAIN (default) or DUO_KV_INT8 (bf16, d 128, contiguous, sink + recent <= 128) */
+    int32_t kv_quant;     /* DUO_KV_PLAIN (default), DUO_KV_INT8 or DUO_KV_INT4 (bf16, d 128, contiguous, sink + recent <= 128) */
     int32_t kv_perm[DUO_MAX_KV_HEADS]; /* block slot i holds model KV head kv_perm[i] */
 } duo_layer_desc;
 
@@ -140,6 +141,19 @@ typedef struct {
  *   k_scale, v_scale = fp32 [B][R][capacity].
  *   K and V values must stay within +-8.3e6 (the fp16 operands of the
  *   decode MMAs hold code * 1 and p * scale).
+ * 4-bit full cache (desc->kv_quant = DUO_KV_INT4; the same constraints) --
+ *   the paper review's "Quantization combination" pairs 8-bit weights with a
+ *   4-bit KV cache, again without a scheme; this one is the 8-bit scheme with
+ *   7 levels a side: scale = amax / 7, code = x * (7 / amax) rounded to
+ *   nearest even (-7..7), stored as the nibble code + 8:
+ *   k_full = [B][R][capacity][64] bytes, a row per token; byte 16q + 4j + c
+ *     of a row holds, with e = 32q + 8j, the features (e, e+2), (e+4, e+6),
+ *     (e+1, e+3), (e+5, e+7) for c = 0, 1, 2, 3 (first in the low nibble);
+ *   v_full = [B][R][capacity/64][4096] bytes: per 64-token tile, 16-token
+ *     group g, feature block m, row r (0..7) and key quad k (0..3) a word at
+ *     1024g + 128m + 16r + 4k whose bytes are the group's tokens 2k, 2k+8,
+ *     2k+1, 2k+9, each holding features 16m + r (low) and 16m + 8 + r (high);
+ *   k_scale, v_scale as for the 8-bit cache.
  * seq_len = [B] int32: tokens appended so far per sequence.
  * counters = DUO_STATE_COUNTER_WORDS uint32 words that must be zero before
  *   the first call; every call leaves them zero.

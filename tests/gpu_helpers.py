@@ -51,6 +51,41 @@ def assert_close(got: np.ndarray, want: np.ndarray, dtype: str, what: str = "") 
     return dict(max_abs=mx, mean_abs=mean)
 
 
+# The 4-bit cache's byte layouts, as include/duo.h states them (codes -7..7
+# stored as the nibble code + 8, the first of a byte's pair in its low half).
+
+def q4_k_rows(codes: np.ndarray) -> np.ndarray:
+    """K codes [n, 128] -> the cache's rows [n, 64] bytes: byte 16q + 4j + c
+    holds, with e = 32q + 8j, features (e, e+2), (e+4, e+6), (e+1, e+3),
+    (e+5, e+7) for c = 0..3."""
+    nib = (codes.astype(np.int16) + 8).astype(np.uint8)
+    out = np.zeros((codes.shape[0], 64), dtype=np.uint8)
+    for q in range(4):
+        for j in range(4):
+            e, o = 32 * q + 8 * j, 16 * q + 4 * j
+            for c, (lo, hi) in enumerate([(0, 2), (4, 6), (1, 3), (5, 7)]):
+                out[:, o + c] = nib[:, e + lo] | (nib[:, e + hi] << 4)
+    return out
+
+
+def q4_v_gather(tiles: np.ndarray, n: int) -> np.ndarray:
+    """The V cache's tiles [n_tiles, 4096] bytes -> codes [n, 128] of tokens
+    0..n-1: token t of 16-token group g, key quad k = (t % 8) / 2, byte
+    (t % 2) * 2 + t / 8 of the word at 1024g + 128m + 16r + 4k holds features
+    16m + r (low nibble) and 16m + 8 + r (high nibble)."""
+    p = np.arange(n)
+    t = p % 64
+    g, tt = t // 16, t % 16
+    k, bw = (tt % 8) // 2, (tt % 2) * 2 + tt // 8
+    m, r = np.arange(8)[None, :, None], np.arange(8)[None, None, :]
+    off = 1024 * g[:, None, None] + 128 * m + 16 * r + 4 * k[:, None, None] + bw[:, None, None]   # [n, 8, 8]
+    byte = tiles[(p // 64)[:, None, None], off].astype(np.int16)
+    out = np.zeros((n, 128), dtype=np.int8)
+    out[:, (16 * m + r).reshape(-1)] = ((byte & 15) - 8).reshape(n, -1)
+    out[:, (16 * m + 8 + r).reshape(-1)] = ((byte >> 4) - 8).reshape(n, -1)
+    return out
+
+
 class Layer:
     """One attention layer on the device plus its oracle twin."""
 
@@ -70,10 +105,11 @@ class Layer:
                                   sink=shape.sink, recent=shape.recent, page_size=page_size,
                                   io_order=self.io_order, stream_prefill=stream_prefill, kv_quant=kv_quant)
         self.kv_int8 = kv_quant == duo.KV_INT8
+        self.kv_int4 = kv_quant == duo.KV_INT4
         self.page_table = None if page_table is None else np.asarray(page_table, dtype=np.int32)
         self.caches = duo.LayerCaches(self.desc, capacity, self.page_table, n_pages)
         self.oracle = O.HeadSplitCache(batch, hkv, shape.head_dim, gate=self.gate, sink=shape.sink,
-                                       recent=shape.recent, kv_int8=self.kv_int8)
+                                       recent=shape.recent, kv_int8=self.kv_int8, kv_int4=self.kv_int4)
         self.ws = duo.Workspace(self.desc, duo.OP_DECODE, self.caches.capacity)
 
     # -- head order ----------------------------------------------------------
@@ -185,7 +221,15 @@ class Layer:
             L = self.oracle.length[b]
             for h in range(sh.n_kv_heads):
                 slot = self.inv[h]
-                if self.gate[h] and self.kv_int8:
+                if self.gate[h] and self.kv_int4:
+                    pos, kc, ks, vc, vs = self.oracle.quantized(b, h)
+                    assert np.array_equal(pos, np.arange(L))
+                    assert np.array_equal(bits(c.k_full)[b, slot, :L], q4_k_rows(kc)), f"4-bit K codes b={b} h={h}"
+                    tiles = bits(c.v_full)[b, slot]
+                    assert np.array_equal(q4_v_gather(tiles, L), vc), f"4-bit V codes b={b} h={h}"
+                    assert np.array_equal(bits(c.k_scale)[b, slot, :L], ks), f"K scales b={b} h={h}"
+                    assert np.array_equal(bits(c.v_scale)[b, slot, :L], vs), f"V scales b={b} h={h}"
+                elif self.gate[h] and self.kv_int8:
                     # 8-bit layout: K codes a row per token; V codes per 64-token
                     # tile, transposed, tokens of a 16-group in the order
                     # 0 1 8 9 2 3 10 11 4 5 12 13 6 7 14 15

@@ -311,7 +311,12 @@ def test_int8_cache_is_validated(duo):
     with pytest.raises(duo.DuoError) as e:
         duo.desc_init(1, 8, 4, 128, duo.FP32, perm, 2, kv_quant=duo.KV_INT8)
     assert e.value.status == duo.ERR_UNSUPPORTED
-    d.kv_quant = 2
+    d.kv_quant = duo.KV_INT4
+    assert duo.desc_validate(d) == duo.OK
+    with pytest.raises(duo.DuoError) as e:
+        duo.desc_init(1, 8, 4, 64, duo.BF16, perm, 2, kv_quant=duo.KV_INT4)
+    assert e.value.status == duo.ERR_UNSUPPORTED
+    d.kv_quant = 3
     assert duo.desc_validate(d) == duo.ERR_INVALID_ARG
 
 

@@ -56,8 +56,8 @@ def _rows(cache, b, h):
     return len(cache.stream[b][h])
 
 
-@pytest.mark.parametrize("kv_int8", [False, True])
-def test_decode_bytes_count_the_cached_rows(kv_int8):
+@pytest.mark.parametrize("kv_bits", [0, 8, 4])
+def test_decode_bytes_count_the_cached_rows(kv_bits):
     """One fused decode step (append, then attend) after prompts of several
     lengths: every row the oracle's caches hold after the append except the
     new one is read once (a retrieval row as bf16 K and V, or d codes + a
@@ -81,11 +81,11 @@ def test_decode_bytes_count_the_cached_rows(kv_int8):
             cache.full[b][h], cache.stream[b][h] = one.full[0][h], one.stream[0][h]
         cache.set_length(b, L + 1)
     row = sh.head_dim * 2
-    full_row = sh.head_dim + 4 if kv_int8 else row
+    full_row = {0: row, 8: sh.head_dim + 4, 4: sh.head_dim // 2 + 4}[kv_bits]
     want = 0
     for b in range(B):
         for h in range(sh.n_kv_heads):
             want += (_rows(cache, b, h) - 1) * (full_row if gate[h] else row) * 2
         want += sh.n_kv_heads * row * 2 * 2
         want += sh.n_q_heads * sh.head_dim * 2 * 2
-    assert bench._decode_bytes(sh, R, [L + 1 for L in lengths], kv_int8) == want
+    assert bench._decode_bytes(sh, R, [L + 1 for L in lengths], kv_bits) == want
