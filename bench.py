@@ -3,20 +3,26 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-Default workload ``mha_decode_32k``: a Llama-2-7B-shaped MHA attention layer
-(32 heads, head_dim 128, bf16, batch 1), 8 of 32 heads retrieval (chosen by
-seed), sink 16 / recent 64, context 32,768 tokens, one token appended and
-attended per decode step.  A step is one pass of the path: duo_decode_step,
-the one-launch form of duo_append_kv + duo_decode_attn (both caches, both
-head types, output concatenated in model head order), for each of 4 layers
-with their own caches, back to back as in a forward pass; the value is per
-layer.  Inputs are resident in HBM before timing starts; the 4 layers'
-caches (540 MB) exceed the 126 MB L2, so nothing is flushed between steps.
+Default workload ``gqa_decode_128k``: a Llama-3-8B-shaped GQA attention
+layer (32 query heads over 8 KV heads, head_dim 128, bf16, batch 1), 4 of 8
+KV heads retrieval (chosen by seed), sink 16 / recent 64, context 131,072
+tokens, one token appended and attended per decode step.  A step is one pass
+of the path: duo_decode_step, the one-launch form of duo_append_kv +
+duo_decode_attn (both caches, both head types, output concatenated in model
+head order), for each of 32 layers with their own caches, back to back as in
+a forward pass; the value is per layer.  Inputs are resident in HBM before
+timing starts; the layers' caches (8.6 GB) exceed the 126 MB L2, so nothing
+is flushed between steps.
 
-Other workloads: gqa_decode_128k, gqa_decode_1m (Llama-3-8B-shaped GQA, 4 of
-8 KV heads retrieval), batch64_paged_decode (64 sequences, lengths U[4096,
-32768], 64-token pages), gqa_prefill_128k (one 131,072-token prompt in 32
-chunks of 4,096; a step is one chunk's duo_prefill_chunk + duo_append_kv).
+The default line also carries ``decode_configs``: mha_decode_32k (Llama-2-7B-
+shaped MHA, 8 of 32 heads retrieval, 32 layers), gqa_decode_1m (16 layers)
+and batch64_paged_decode (64 sequences, lengths U[4096, 32768], 64-token
+pages, 8 layers), each with its own roofline, clocks, e2e and CPU baseline
+(--no-extra drops them).  Other workloads: the same decode shapes over 8- or
+4-bit retrieval caches (``*_int8``, ``*_int4``), gqa_prefill_128k (one
+131,072-token prompt in 32 chunks of 4,096; a step is one chunk's
+duo_prefill_chunk + duo_append_kv), gqa_prefill_32k, and the gated mix
+(gated_mix_pr1, gated_mix_gqa_4k: forward and gate gradient).
 
 A decode run also measures the pre-fill workload (unless --no-prefill) and
 reports it under "prefill" in the same line; its TFLOP/s count 4*d FLOPs per
@@ -102,16 +108,17 @@ def _peaks():
 
 def _traffic(kernel: str, workload: str):
     """DRAM bytes (read + write) per launch of `kernel` on `workload` from the
-    committed ncu record profiles/traffic.json -- only while every source file
-    the record lists still has the recorded SHA-256 (a changed kernel has no
-    measured traffic until it is captured again)."""
+    committed ncu record profiles/traffic.json ({kernel: {workload: record}})
+    -- only while every source file the record lists still has the recorded
+    SHA-256 (a changed kernel has no measured traffic until it is captured
+    again)."""
     import hashlib
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            rec = json.load(f).get(kernel)
-    except (OSError, ValueError):
+            rec = (json.load(f).get(kernel) or {}).get(workload)
+    except (OSError, ValueError, AttributeError):
         return None
-    if not rec or rec.get("workload") != workload:
+    if not rec:
         return None
     for rel, digest in rec.get("source_sha256", {}).items():
         try:

@@ -61,6 +61,7 @@ struct DecodeArgs {
     const void* v_new;
     uint32_t* grid_ticket;  // one state counter word: the last CTA advances seq_len
     uint32_t* tile_ctr;     // [B*R]: tiles handed out past the static ones (tensor-core bf16 kernel)
+    int draw;               // draw tiles from tile_ctr: only when the whole grid is resident at once
 };
 
 template <typename T, int D>
@@ -691,11 +692,15 @@ __device__ __forceinline__ uint32_t sw_off(int row, int c16) {
     return (uint32_t)((c16 >> 3) * (kMmaTileBytes / 2) + row * 128 + (((c16 & 7) ^ (row & 7)) << 4));
 }
 
-constexpr int kWarmTiles = 2;  // K and V tiles per split brought into L2 before the dependency wait
 // Tiles each split of decode_mma_kernel takes by its index before it draws
 // further tiles from its head's counter: split s takes tiles s, s + nsplit,
 // ..., then nsplit * kStaticTiles + (counter draws).
 constexpr int kStaticTiles = 2;
+constexpr int kWarmTiles = 3;  // tiles per split asked of L2 (or loaded) before the dependency wait
+// Rows below (a relaxed read of seq_len) - kSpecMargin are loaded before the
+// dependency wait: two earlier decode launches of the same layer may still be
+// writing their new rows just below that length.
+constexpr int kSpecMargin = 2 * kTile;
 
 // The k-th tile split `split` takes when the tiles are not drawn from a
 // counter (one split: all of them in order; otherwise the static ones).
@@ -708,14 +713,16 @@ __device__ __forceinline__ int static_tile(int split, int nsplit, int k) { retur
 // and are clamped to the cache, so a stale value only wastes a prefetch.
 template <bool PAGED>
 __device__ __forceinline__ void warm_l2_split(const LayerArgs& a, const CacheArgs& c, const DecodeArgs& d, int b,
-                                              int slot, int split) {
+                                              int slot, int split, int n_spec) {
     constexpr int kRowBytes = 128 * 2;
     int len = ld_relaxed_gpu(&c.seq_len[b]) + (d.k_new != nullptr ? 1 : 0);
     len = max(0, min(len, a.capacity));
     const uint8_t* kf = static_cast<const uint8_t*>(c.k_full);
     const uint8_t* vf = static_cast<const uint8_t*>(c.v_full);
-    for (int k = 0; k < kWarmTiles; ++k) {
-        const int r0 = static_tile(split, d.nsplit, k) * kTile;
+    for (int k = n_spec; k < kWarmTiles; ++k) {
+        // the static tiles not already loading, then (drawn splits) the
+        // first tile of the counter's range that this split's index points at
+        const int r0 = (k < kStaticTiles ? static_tile(split, d.nsplit, k) : kStaticTiles * d.nsplit + split) * kTile;
         if (r0 >= len) break;
         const uint32_t bytes = (uint32_t)min(kTile, len - r0) * kRowBytes;
         size_t off;
@@ -772,7 +779,15 @@ __global__ void __maxnreg__(200)
     }
     const bool fused = d.k_new != nullptr;
     // Work that reads nothing the previous grid writes: barriers, the tensor
-    // maps (kernel parameters) and the L2 warm-up of this split's first tiles.
+    // maps (kernel parameters), and -- contiguous full cache -- the split's
+    // static tiles that lie at least kSpecMargin rows below the length a
+    // relaxed read of seq_len gives.  The only grid that can still run
+    // before this one's dependency wait is an earlier decode launch (no
+    // other kernel of the library triggers its dependents early); it writes
+    // one new row per sequence, at or past the length it read, and the
+    // lengths only grow, so those rows are final already.  The producer
+    // loads them into the first stages now; past the wait it continues from
+    // there.
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full_bar[s], 1);
@@ -781,10 +796,29 @@ __global__ void __maxnreg__(200)
         mbar_init(comb_bar, 1);
         fence_barrier_init();
     }
+    __syncthreads();
+    int n_spec = 0;   // producer lane: static tiles already loading
     if (warp == NW && lane == 0) {
         prefetch_map(retrieval ? &tmKf : &tmKr);
         prefetch_map(retrieval ? &tmVf : &tmVr);
-        if (retrieval) warm_l2_split<PAGED>(a, c, d, b, slot, split);
+        if (retrieval && !PAGED) {
+            const int safe = min(ld_relaxed_gpu(&c.seq_len[b]), a.capacity) - kSpecMargin;
+            const int z = b * a.R + slot;
+            for (int k = 0; k < kStaticTiles; ++k) {
+                const int t = static_tile(split, d.nsplit, k);
+                if ((t + 1) * kTile > safe) break;
+                s_tile_n[k] = kTile;
+                mbar_arrive_expect_tx(&full_bar[k], 2 * kMmaTileBytes);
+                const uint32_t dk = smem_u32(sKb + (size_t)k * kMmaTileBytes);
+                const uint32_t dv = smem_u32(sVb + (size_t)k * kMmaTileBytes);
+                for (int h = 0; h < 2; ++h) {
+                    tma_load_3d(dk + h * (kMmaTileBytes / 2), &tmKf, 64 * h, t * kTile, z, &full_bar[k]);
+                    tma_load_3d(dv + h * (kMmaTileBytes / 2), &tmVf, 64 * h, t * kTile, z, &full_bar[k]);
+                }
+                ++n_spec;
+            }
+        }
+        if (retrieval) warm_l2_split<PAGED>(a, c, d, b, slot, split, n_spec);
     }
     // launched with programmatic stream serialization: let the next launch's
     // CTAs take SM slots as ours free, and wait for the previous grid before
@@ -867,9 +901,11 @@ __global__ void __maxnreg__(200)
         const CUtensorMap* mk = retrieval ? &tmKf : &tmKr;
         const CUtensorMap* mv = retrieval ? &tmVf : &tmVr;
         const int z = retrieval ? b * a.R + slot : b * a.S + (slot - a.R);
-        const bool draw = retrieval && d.nsplit > 1 && d.tile_ctr != nullptr;
+        const bool draw = retrieval && d.draw && d.nsplit > 1;
+        const int i0 = __shfl_sync(0xffffffffu, n_spec, 0);   // tiles loaded before the wait
         uint32_t drawn = 0;   // lane 0: the counter draw for the next tile, made while this one loads
-        for (int i = 0;; ++i) {
+        if (lane == 0 && draw && i0 >= kStaticTiles) drawn = atomicAdd(&d.tile_ctr[pair], 1u);
+        for (int i = i0;; ++i) {
             const int st = i % STAGES, round = i / STAGES;
             int ok = 1;
             if (lane == 0 && round > 0) ok = mbar_wait(&empty_bar[st], (round - 1) & 1, c.status) ? 1 : 0;
@@ -1155,6 +1191,9 @@ constexpr size_t decode_q8_smem_bytes() {
     return 2 * (size_t)kQ8Stages * kQ8Bytes + kQ8Stages * kQ8ScBytes + (2 * kQ8Stages + 1) * sizeof(uint64_t) + 64;
 }
 
+constexpr uint32_t kF16x2One = 0x3C003C00u;   // (1.0, 1.0) in fp16
+constexpr float kTwo24 = 16777216.f;          // 2^24: undoes the subnormal codes' 2^-24
+
 __device__ __forceinline__ void mma_f16_rows8(float& c0, float& c1, uint32_t a0, uint32_t a2, uint32_t b0,
                                               uint32_t b1) {
     float d2, d3;
@@ -1271,6 +1310,72 @@ constexpr size_t ring_simt_smem_bytes(int G) {
 }
 static_assert(ring_simt_smem_bytes(8) <= 2 * (size_t)kQ8Stages * kQ8Bytes + kQ8Stages * kQ8ScBytes,
               "the ring path must fit below the 8-bit kernel's barriers");
+
+// The scores of a lane's four keys (k0, k0 + 1, k0 + 8, k0 + 9 of the stage)
+// from the MMA sums with the code bias already removed: times the key's K
+// scale and the softmax scale (log2 domain), and the keys' V scales.  Only
+// a split's last tile can be partial (n < 64, the same for the whole warp):
+// there keys at or past n get a score of -inf and a V scale of 0, so that
+// neither a stale score nor a stale scale (whatever the cache holds past the
+// length) reaches the sums.
+__device__ __forceinline__ void quant_scores(float s0, float s1, float s2, float s3, const float* ksc,
+                                             const float* vsc, int k0, int n, float sl, float (&sv)[4],
+                                             float (&vs)[4]) {
+    const float2 ks0 = *reinterpret_cast<const float2*>(ksc + k0);
+    const float2 ks1 = *reinterpret_cast<const float2*>(ksc + k0 + 8);
+    const float2 vs0 = *reinterpret_cast<const float2*>(vsc + k0);
+    const float2 vs1 = *reinterpret_cast<const float2*>(vsc + k0 + 8);
+    sv[0] = s0 * ks0.x * sl;
+    sv[1] = s1 * ks0.y * sl;
+    sv[2] = s2 * ks1.x * sl;
+    sv[3] = s3 * ks1.y * sl;
+    vs[0] = vs0.x;
+    vs[1] = vs0.y;
+    vs[2] = vs1.x;
+    vs[3] = vs1.y;
+    if (n < kTile) {
+        const int kk[4] = {k0, k0 + 1, k0 + 8, k0 + 9};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            sv[i] = kk[i] < n ? sv[i] : -INFINITY;
+            vs[i] = kk[i] < n ? vs[i] : 0.f;
+        }
+    }
+}
+
+// One tile of the online softmax for the lane's row (query head lane / 4,
+// shared by the quad's four lanes): the row maximum over the quad, p =
+// 2^(s - m), the running sum; O, l and the PV bias sums are rescaled only
+// when some row's maximum grew (a warp vote), which over a long cache is
+// rare.  A masked key
+// (-inf) gets p = 0; m starts at a finite -1e30, so a row with no key yet
+// keeps p = 0 and a factor of 1.
+template <int NWS>
+__device__ __forceinline__ void online_softmax_step(const float (&sv)[4], float& m_run, float& l_run, float (&pr)[4],
+                                                    float (&o)[16][2], float (&wsum)[NWS][2]) {
+    float mx = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m_run, mx);
+    if (__any_sync(0xffffffffu, m_new > m_run)) {
+        const float corr = exp2f(m_run - m_new);
+        l_run *= corr;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            o[j][0] *= corr;
+            o[j][1] *= corr;
+        }
+#pragma unroll
+        for (int j = 0; j < NWS; ++j) {
+            wsum[j][0] *= corr;
+            wsum[j][1] *= corr;
+        }
+        m_run = m_new;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) pr[i] = exp2f(sv[i] - m_run);
+    l_run += (pr[0] + pr[1]) + (pr[2] + pr[3]);
+}
 
 template <int G>
 __global__ void __maxnreg__(200)
@@ -1399,9 +1504,14 @@ __global__ void __maxnreg__(200)
     const int quad = lane & 3;
     float o[16][2];
     float m_run = kNegBig, l_run = 0.f;
+    float wsum[1][2] = {{0.f, 0.f}};   // sum of the PV A operand per row (the code bias)
     if (warp < NW) {
-        // q in fp16, features 32 quad + 4 kb + {0, 1} and {2, 3} for step kb
+        // q in fp16, features 32 quad + 4 kb + {0, 1} and {2, 3} for step kb.
+        // The K operands keep the bias of the byte-to-fp16 step (1152 +
+        // code), so a score is the MMA's sum minus 1152 times the row's sum
+        // of q -- a fresh accumulator per tile, so no precision is lost.
         uint32_t qa[8][2];
+        float q_corr = 0.f;
         {
             const bool row_ok = row < G;
             const uint4* qp = reinterpret_cast<const uint4*>(
@@ -1413,7 +1523,17 @@ __global__ void __maxnreg__(200)
                 qa[2 * i][1] = f16x2_pack(bf16_lo(w.y), bf16_hi(w.y));
                 qa[2 * i + 1][0] = f16x2_pack(bf16_lo(w.z), bf16_hi(w.z));
                 qa[2 * i + 1][1] = f16x2_pack(bf16_lo(w.w), bf16_hi(w.w));
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&qa[2 * i + h][e]));
+                        q_corr += f.x + f.y;
+                    }
             }
+            q_corr += __shfl_xor_sync(0xffffffffu, q_corr, 1);
+            q_corr += __shfl_xor_sync(0xffffffffu, q_corr, 2);
+            q_corr *= 1152.f;
         }
 #pragma unroll
         for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = 0.f;
@@ -1438,48 +1558,32 @@ __global__ void __maxnreg__(200)
 #pragma unroll
                 for (int kb = 0; kb < 8; ++kb) {
                     uint32_t b0, b1;
-                    i8x4_to_f16x2(w[kb], b0, b1);
+                    i8x4_to_f16x2_biased(w[kb], b0, b1);
                     mma_f16_rows8(s[nb][0], s[nb][1], qa[kb][0], qa[kb][1], b0, b1);
                 }
             }
             // this lane's keys: key_base + 2 quad + {0, 1} and + 8
             const int k0 = key_base + 2 * quad;
-            const float2 ks0 = *reinterpret_cast<const float2*>(ksc + k0);
-            const float2 ks1 = *reinterpret_cast<const float2*>(ksc + k0 + 8);
-            const float sv[4] = {s[0][0] * ks0.x * sl, s[0][1] * ks0.y * sl, s[1][0] * ks1.x * sl,
-                                 s[1][1] * ks1.y * sl};
-            const bool vk[4] = {k0 < n, k0 + 1 < n, k0 + 8 < n, k0 + 9 < n};
-            float mx = kNegBig;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) mx = vk[i] ? fmaxf(mx, sv[i]) : mx;
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            const float m_new = fmaxf(m_run, mx);
-            const float corr = exp2f(m_run - m_new);
+            float sv[4], vs[4];
+            quant_scores(s[0][0] - q_corr, s[0][1] - q_corr, s[1][0] - q_corr, s[1][1] - q_corr, ksc, vsc, k0, n,
+                         sl, sv, vs);
             float pr[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) pr[i] = vk[i] ? exp2f(sv[i] - m_new) : 0.f;
-            l_run = l_run * corr + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
-            m_run = m_new;
+            online_softmax_step(sv, m_run, l_run, pr, o, wsum);
             // p times the key's V scale, the fp16 A operand of O += P V
-            const float2 vs0 = *reinterpret_cast<const float2*>(vsc + k0);
-            const float2 vs1 = *reinterpret_cast<const float2*>(vsc + k0 + 8);
-            const uint32_t pa0 = f16x2_pack(vk[0] ? pr[0] * vs0.x : 0.f, vk[1] ? pr[1] * vs0.y : 0.f);
-            const uint32_t pa1 = f16x2_pack(vk[2] ? pr[2] * vs1.x : 0.f, vk[3] ? pr[3] * vs1.y : 0.f);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                o[j][0] *= corr;
-                o[j][1] *= corr;
-            }
-            // O += P V: feature row 8 nd + (lane >> 2), this warp's 16-key
-            // group (64-byte swizzle), the lane's four keys in one word
+            const uint32_t pa0 = f16x2_pack(pr[0] * vs[0], pr[1] * vs[1]);
+            const uint32_t pa1 = f16x2_pack(pr[2] * vs[2], pr[3] * vs[3]);
+            // O' += P U with U = (code + 128) 2^-24 (exact fp16 subnormals),
+            // and the bias sum W += P 1 through the same MMA: O = 2^24 O' -
+            // 128 W at the end.  Feature row 8 nd + (lane >> 2), this warp's
+            // 16-key group (64-byte swizzle), the lane's four keys in one word
+            mma_f16_rows8(wsum[0][0], wsum[0][1], pa0, pa1, kF16x2One, kF16x2One);
 #pragma unroll
             for (int nd = 0; nd < 16; ++nd) {
                 const int f = 8 * nd + row;
                 const uint32_t w = *reinterpret_cast<const uint32_t*>(tV + f * 64 + ((warp ^ ((f >> 1) & 3)) << 4) +
                                                                       4 * quad);
                 uint32_t b0, b1;
-                i8x4_to_f16x2(w, b0, b1);
+                i8x4_to_f16x2_sub(w, b0, b1);
                 mma_f16_rows8(o[nd][0], o[nd][1], pa0, pa1, b0, b1);
             }
             __syncwarp();
@@ -1495,10 +1599,11 @@ __global__ void __maxnreg__(200)
     float* sM = reinterpret_cast<float*>(smem);
     if (warp < NW && row < G) {
         float* dst = sM + ((size_t)warp * G + row) * STRIDE;
+        const float bias = 128.f * wsum[0][0];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-            dst[4 + 8 * j + 2 * quad] = o[j][0];
-            dst[4 + 8 * j + 2 * quad + 1] = o[j][1];
+            dst[4 + 8 * j + 2 * quad] = fmaf(o[j][0], kTwo24, -bias);
+            dst[4 + 8 * j + 2 * quad + 1] = fmaf(o[j][1], kTwo24, -bias);
         }
         if (quad == 0) {
             dst[0] = m_run;
@@ -1541,7 +1646,7 @@ cudaError_t launch_q8_g(const LayerArgs& a, const CacheArgs& c, const DecodeArgs
 // 4-bit layouts of kvq4.cuh: a 64-token stage is 4 KB of K codes and 4 KB of
 // V codes, each one contiguous bulk copy (the layouts are already in the
 // order the consumers read, so no tensor map or swizzle is needed), plus the
-// tile's 64 + 64 scales; ten stages.
+// tile's 64 + 64 scales; eight stages, two CTAs to an SM.
 //   S = q . codes: a lane's 16 bytes of a key's row hold its 32 permuted
 //     features; each word gives two k-steps' B fragments by masking nibble
 //     pairs into fp16 (u4x2_to_f16x2); q is permuted as for the 8-bit cache.
@@ -1549,14 +1654,25 @@ cudaError_t launch_q8_g(const LayerArgs& a, const CacheArgs& c, const DecodeArgs
 //     feature rows 16 m + r and 16 m + 8 + r for the lane's four keys.
 // ===========================================================================
 
-constexpr int kQ4Stages = 10;
+constexpr int kQ4Stages = 8;
 constexpr uint32_t kQ4ScBytes = 2 * kTile * 4;      // K and V scales of a stage
 
-constexpr size_t decode_q4_smem_bytes() {
-    return 2 * (size_t)kQ4Stages * kQ4TileBytes + kQ4Stages * kQ4ScBytes + (2 * kQ4Stages + 1) * sizeof(uint64_t) + 64;
+// The barriers sit above both the stage buffers of a retrieval CTA and the
+// ring staging of a streaming CTA (which needs more for a group of 8).
+template <int G>
+constexpr size_t q4_bar_offset() {
+    constexpr size_t stages = 2 * (size_t)kQ4Stages * kQ4TileBytes + kQ4Stages * kQ4ScBytes;
+    constexpr size_t ring = (ring_simt_smem_bytes(G) + 15) / 16 * 16;
+    return stages > ring ? stages : ring;
 }
-static_assert(ring_simt_smem_bytes(8) <= 2 * (size_t)kQ4Stages * kQ4TileBytes + kQ4Stages * kQ4ScBytes,
-              "the ring path must fit below the 4-bit kernel's barriers");
+template <int G>
+constexpr size_t decode_q4_smem_bytes() {
+    return q4_bar_offset<G>() + (2 * kQ4Stages + 1) * sizeof(uint64_t) + 64;
+}
+// two CTAs to an SM (227 KB, 1 KB of it reserved per CTA).  Three (at most
+// 128 registers, eight stages) were measured: no faster at 1M tokens and
+// slower at 128K, the register cap costing spills.
+static_assert(2 * (decode_q4_smem_bytes<8>() + 1024) <= 232448, "two 4-bit CTAs per SM");
 
 template <int G>
 __global__ void __maxnreg__(200)
@@ -1572,7 +1688,7 @@ __global__ void __maxnreg__(200)
     uint8_t* sK4 = smem;
     uint8_t* sV4 = smem + (size_t)STAGES * kQ4TileBytes;
     float* sSc = reinterpret_cast<float*>(smem + 2 * (size_t)STAGES * kQ4TileBytes);
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + 2 * (size_t)STAGES * kQ4TileBytes + STAGES * kQ4ScBytes);
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + q4_bar_offset<G>());
     uint64_t* empty_bar = full_bar + STAGES;
     uint64_t* comb_bar = empty_bar + STAGES;
     int* s_flag = reinterpret_cast<int*>(comb_bar + 1);
@@ -1675,30 +1791,58 @@ __global__ void __maxnreg__(200)
     }
 
     // ------------------------------------------------------ consumers
+    // Nibbles are not shifted down one by one: a mask-and-or puts a word's
+    // nibbles n at bits 0-3 / 16-19 under the fp16 exponent of 1024 (the
+    // values 1024 + n) and those at bits 4-7 / 20-23 likewise (1024 + 16 n);
+    // the MMA partner of a 16 n operand is pre-divided by 16 (exact in fp16).
+    // q . K keeps the bias: every product is 1024 q + q n or 64 q' + q' n
+    // (q' = q / 16), and since code = n - 8 the score is the MMA's sum minus
+    // a per-row constant, 1032 (1152) times the sum of the partners -- a
+    // fresh accumulator per tile, so the cancellation costs no precision.
+    // P V accumulates over the whole cache, so its operands are un-biased
+    // exactly instead: 1024 + n - 1032 = code, 1024 + 16 n - 1152 = 16 code.
     const int row = lane >> 2;   // query head of the group (rows >= G are padding) / key of an 8-key block
     const int quad = lane & 3;
     float o[16][2];
     float m_run = kNegBig, l_run = 0.f;
+    float wsum[2][2] = {{0.f, 0.f}, {0.f, 0.f}};   // PV A operand sums per row: p vs, p vs / 16
     if (warp < NW) {
-        // q in fp16, features 32 quad + 4 kb + {0, 1} and {2, 3} for step kb
+        // q in fp16, features 32 quad + 4 kb + {0, 1} (partners of the low
+        // nibbles) and {2, 3} (partners of the high nibbles, divided by 16)
         uint32_t qa[8][2];
+        float q_corr = 0.f;
         {
             const bool row_ok = row < G;
             const uint4* qp = reinterpret_cast<const uint4*>(
                 static_cast<const T*>(d.q) + ((size_t)b * a.Hq + a.q_head0[slot] + (row_ok ? row : 0)) * D + 32 * quad);
+            const __half2 sixteenth = __float2half2_rn(0.0625f);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const uint4 w = row_ok ? qp[i] : make_uint4(0u, 0u, 0u, 0u);
-                qa[2 * i][0] = f16x2_pack(bf16_lo(w.x), bf16_hi(w.x));
-                qa[2 * i][1] = f16x2_pack(bf16_lo(w.y), bf16_hi(w.y));
-                qa[2 * i + 1][0] = f16x2_pack(bf16_lo(w.z), bf16_hi(w.z));
-                qa[2 * i + 1][1] = f16x2_pack(bf16_lo(w.w), bf16_hi(w.w));
+                const uint32_t lo0 = f16x2_pack(bf16_lo(w.x), bf16_hi(w.x));
+                const uint32_t lo1 = f16x2_pack(bf16_lo(w.z), bf16_hi(w.z));
+                const uint32_t t0 = f16x2_pack(bf16_lo(w.y), bf16_hi(w.y));
+                const uint32_t t1 = f16x2_pack(bf16_lo(w.w), bf16_hi(w.w));
+                const __half2 hi0 = __hmul2(*reinterpret_cast<const __half2*>(&t0), sixteenth);
+                const __half2 hi1 = __hmul2(*reinterpret_cast<const __half2*>(&t1), sixteenth);
+                qa[2 * i][0] = lo0;
+                qa[2 * i][1] = *reinterpret_cast<const uint32_t*>(&hi0);
+                qa[2 * i + 1][0] = lo1;
+                qa[2 * i + 1][1] = *reinterpret_cast<const uint32_t*>(&hi1);
+                const float2 l0 = __half22float2(*reinterpret_cast<const __half2*>(&lo0));
+                const float2 l1 = __half22float2(*reinterpret_cast<const __half2*>(&lo1));
+                const float2 h0 = __half22float2(hi0), h1 = __half22float2(hi1);
+                q_corr += 1032.f * ((l0.x + l0.y) + (l1.x + l1.y)) + 1152.f * ((h0.x + h0.y) + (h1.x + h1.y));
             }
+            // the row's constant over all 128 features (the quad's four lanes)
+            q_corr += __shfl_xor_sync(0xffffffffu, q_corr, 1);
+            q_corr += __shfl_xor_sync(0xffffffffu, q_corr, 2);
         }
 #pragma unroll
         for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = 0.f;
         const float sl = a.scale * kLog2e;
         const int key_base = warp * 16;
+        const __half2 sixteenth = __float2half2_rn(0.0625f);
         for (int t = 0; t < n_tiles; ++t) {
             const int st = t % STAGES, round = t / STAGES;
             if (!mbar_wait(&full_bar[st], round & 1, c.status)) break;
@@ -1707,55 +1851,52 @@ __global__ void __maxnreg__(200)
             const uint8_t* tV = sV4 + (size_t)st * kQ4TileBytes;
             const float* ksc = sSc + st * 2 * kTile;
             const float* vsc = ksc + kTile;
-            // S = q . codes for keys key_base + 8 nb + (lane >> 2)
-            float s[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+            // S' = q . (biased codes) for keys key_base + 8 nb + (lane >> 2),
+            // even and odd k-steps in separate accumulators
+            float s[2][2][2] = {{{0.f, 0.f}, {0.f, 0.f}}, {{0.f, 0.f}, {0.f, 0.f}}};
 #pragma unroll
             for (int nb = 0; nb < 2; ++nb) {
                 const int key = key_base + 8 * nb + row;
                 const uint4 kw = *reinterpret_cast<const uint4*>(tK + key * kQ4RowBytes + 16 * quad);
                 const uint32_t w[4] = {kw.x, kw.y, kw.z, kw.w};
 #pragma unroll
-                for (int kb = 0; kb < 8; ++kb) {
-                    const uint32_t x = w[kb >> 1] >> (8 * (kb & 1));
-                    mma_f16_rows8(s[nb][0], s[nb][1], qa[kb][0], qa[kb][1], u4x2_to_f16x2(x), u4x2_to_f16x2(x >> 4));
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t w8 = w[j] >> 8;
+                    mma_f16_rows8(s[nb][0][0], s[nb][0][1], qa[2 * j][0], qa[2 * j][1], u4_lo_f16x2(w[j]),
+                                  u4_hi_f16x2(w[j]));
+                    mma_f16_rows8(s[nb][1][0], s[nb][1][1], qa[2 * j + 1][0], qa[2 * j + 1][1], u4_lo_f16x2(w8),
+                                  u4_hi_f16x2(w8));
                 }
             }
             // this lane's keys: key_base + 2 quad + {0, 1} and + 8
             const int k0 = key_base + 2 * quad;
-            const float2 ks0 = *reinterpret_cast<const float2*>(ksc + k0);
-            const float2 ks1 = *reinterpret_cast<const float2*>(ksc + k0 + 8);
-            const float sv[4] = {s[0][0] * ks0.x * sl, s[0][1] * ks0.y * sl, s[1][0] * ks1.x * sl,
-                                 s[1][1] * ks1.y * sl};
-            const bool vk[4] = {k0 < n, k0 + 1 < n, k0 + 8 < n, k0 + 9 < n};
-            float mx = kNegBig;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) mx = vk[i] ? fmaxf(mx, sv[i]) : mx;
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            const float m_new = fmaxf(m_run, mx);
-            const float corr = exp2f(m_run - m_new);
+            float sv[4], vs[4];
+            quant_scores(s[0][0][0] + s[0][1][0] - q_corr, s[0][0][1] + s[0][1][1] - q_corr,
+                         s[1][0][0] + s[1][1][0] - q_corr, s[1][0][1] + s[1][1][1] - q_corr, ksc, vsc, k0, n, sl, sv,
+                         vs);
             float pr[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) pr[i] = vk[i] ? exp2f(sv[i] - m_new) : 0.f;
-            l_run = l_run * corr + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
-            m_run = m_new;
-            // p times the key's V scale, the fp16 A operand of O += P V
-            const float2 vs0 = *reinterpret_cast<const float2*>(vsc + k0);
-            const float2 vs1 = *reinterpret_cast<const float2*>(vsc + k0 + 8);
-            const uint32_t pa0 = f16x2_pack(vk[0] ? pr[0] * vs0.x : 0.f, vk[1] ? pr[1] * vs0.y : 0.f);
-            const uint32_t pa1 = f16x2_pack(vk[2] ? pr[2] * vs1.x : 0.f, vk[3] ? pr[3] * vs1.y : 0.f);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                o[j][0] *= corr;
-                o[j][1] *= corr;
-            }
-            // O += P V: the word of feature pair (16 m + r, 16 m + 8 + r) and
-            // this lane's key quad in the warp's 16-token group
+            online_softmax_step(sv, m_run, l_run, pr, o, wsum);
+            // p times the key's V scale, the fp16 A operand of O += P V, and
+            // the same divided by 16 for the high-nibble feature rows
+            const uint32_t pa0 = f16x2_pack(pr[0] * vs[0], pr[1] * vs[1]);
+            const uint32_t pa1 = f16x2_pack(pr[2] * vs[2], pr[3] * vs[3]);
+            const __half2 ph0 = __hmul2(*reinterpret_cast<const __half2*>(&pa0), sixteenth);
+            const __half2 ph1 = __hmul2(*reinterpret_cast<const __half2*>(&pa1), sixteenth);
+            const uint32_t pb0 = *reinterpret_cast<const uint32_t*>(&ph0);
+            const uint32_t pb1 = *reinterpret_cast<const uint32_t*>(&ph1);
+            // O' += P U: the word of feature pair (16 m + r, 16 m + 8 + r) and
+            // this lane's key quad in the warp's 16-token group, its nibbles
+            // taken as exact fp16 subnormals n 2^-24 (low) and 16 n 2^-24
+            // (high, against p / 16); the bias sums W += P 1 ride on the same
+            // MMA, and O = 2^24 O' - 8 W (low) or - 128 W (high) at the end
+            mma_f16_rows8(wsum[0][0], wsum[0][1], pa0, pa1, kF16x2One, kF16x2One);
+            mma_f16_rows8(wsum[1][0], wsum[1][1], pb0, pb1, kF16x2One, kF16x2One);
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
                 const uint32_t w = *reinterpret_cast<const uint32_t*>(tV + 1024 * warp + 128 * m + 16 * row + 4 * quad);
-                mma_f16_rows8(o[2 * m][0], o[2 * m][1], pa0, pa1, u4x2_to_f16x2(w), u4x2_to_f16x2(w >> 8));
-                mma_f16_rows8(o[2 * m + 1][0], o[2 * m + 1][1], pa0, pa1, u4x2_to_f16x2(w >> 4), u4x2_to_f16x2(w >> 12));
+                const uint32_t w8 = w >> 8;
+                mma_f16_rows8(o[2 * m][0], o[2 * m][1], pa0, pa1, u4_lo_sub(w), u4_lo_sub(w8));
+                mma_f16_rows8(o[2 * m + 1][0], o[2 * m + 1][1], pb0, pb1, u4_hi_sub(w), u4_hi_sub(w8));
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty_bar[st]);
@@ -1770,10 +1911,14 @@ __global__ void __maxnreg__(200)
     float* sM = reinterpret_cast<float*>(smem);
     if (warp < NW && row < G) {
         float* dst = sM + ((size_t)warp * G + row) * STRIDE;
+        // even n-tiles are low-nibble feature rows (bias 8 p vs), odd ones
+        // high-nibble rows (bias 8 * 16 * p vs / 16)
+        const float bias_lo = 8.f * wsum[0][0], bias_hi = 128.f * wsum[1][0];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-            dst[4 + 8 * j + 2 * quad] = o[j][0];
-            dst[4 + 8 * j + 2 * quad + 1] = o[j][1];
+            const float bias = (j & 1) ? bias_hi : bias_lo;
+            dst[4 + 8 * j + 2 * quad] = fmaf(o[j][0], kTwo24, -bias);
+            dst[4 + 8 * j + 2 * quad + 1] = fmaf(o[j][1], kTwo24, -bias);
         }
         if (quad == 0) {
             dst[0] = m_run;
@@ -1787,7 +1932,7 @@ __global__ void __maxnreg__(200)
 
 template <int G>
 cudaError_t launch_q4_g(const LayerArgs& a, const CacheArgs& c, const DecodeArgs& d, int grid, cudaStream_t s) {
-    constexpr size_t smem = decode_q4_smem_bytes();
+    constexpr size_t smem = decode_q4_smem_bytes<G>();
     auto kern = decode_q4_kernel<G>;
     static std::atomic<unsigned long long> configured{0};
     const cudaError_t e = smem_limit_once(kern, (int)smem, configured);
@@ -1812,6 +1957,11 @@ cudaError_t launch_decode(const LayerArgs& a, const CacheArgs& c, const DecodePl
     d.n_ret_units = a.B * a.R * plan.nsplit;
     const long grid = (long)d.n_ret_units + (long)a.B * a.S;
     if (grid == 0) return cudaSuccess;
+    // Drawing tiles balances a head's splits when they all run at once (one
+    // wave of two CTAs per SM); in a grid of several waves a split that runs
+    // early would drain its head's counter while its siblings wait for a
+    // slot, so the splits keep their static share there.
+    d.draw = grid <= 2L * sm_count() ? 1 : 0;
     if (grid > 0x7fffffffL) return cudaErrorInvalidConfiguration;
     if (a.kv_bits == 4 && a.R > 0) {
         // 4-bit full cache: as the 8-bit path, over nibble codes

@@ -294,6 +294,17 @@ size_t duo_workspace_bytes(const duo_layer_desc* desc, int32_t op, int32_t max_t
     return 0;
 }
 
+size_t duo_prefill_workspace_bytes(const duo_layer_desc* desc, const duo_kv_state* st, int32_t max_chunk) {
+    if (check_desc(desc) != DUO_OK || !st) return 0;
+    duo::LayerArgs a;
+    duo::CacheArgs c;
+    fill_args(desc, a);
+    if (check_state(desc, st, a, c) != DUO_OK) return 0;
+    size_t bytes = duo_workspace_bytes(desc, DUO_OP_PREFILL, max_chunk);
+    if (a.kv_bits && a.R > 0) bytes += (duo::dequant_staging_bytes(a) + 255) / 256 * 256;
+    return bytes;
+}
+
 duo_status duo_permute_heads(const duo_layer_desc* desc, const void* x, void* y, int64_t rows,
                              int32_t heads_per_kv, int64_t head_elems, int32_t elem_bytes, int32_t direction,
                              duo_stream_t stream) {
@@ -386,10 +397,35 @@ duo_status duo_prefill_chunk(const duo_layer_desc* desc, const duo_kv_state* st,
         return fail(DUO_ERR_INVALID_ARG, "pre-fill tensors must be 16-byte aligned");
     if (desc->page_size != 0)
         return fail(DUO_ERR_UNSUPPORTED, "duo_prefill_chunk takes a contiguous full cache (page_size 0)");
-    if (desc->kv_quant != DUO_KV_PLAIN)
-        return fail(DUO_ERR_UNSUPPORTED, "duo_prefill_chunk reads a plain full cache, not an 8- or 4-bit one");
     cudaError_t e;
-    if (a.dtype == DUO_BF16 && a.D == 128) {
+    if (a.kv_bits && a.R > 0) {
+        // an 8- or 4-bit full cache: its rows below seq_len are staged in
+        // the workspace -- the codes as bf16 values and each row's scales --
+        // and the tensor-core pre-fill reads the codes as its cache and
+        // applies the scales to the scores and to p; the rest of the
+        // workspace serves the key-range splits
+        const size_t staging = (duo::dequant_staging_bytes(a) + 255) / 256 * 256;
+        if (!workspace || ws_bytes < staging)
+            return fail(DUO_ERR_CAPACITY,
+                        "an 8- or 4-bit layer's pre-fill needs a workspace of duo_prefill_workspace_bytes (at least "
+                        "%zu bytes; given %zu)", staging, workspace ? ws_bytes : (size_t)0);
+        if (!aligned16(workspace)) return fail(DUO_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+        duo::LayerArgs ap = a;
+        ap.kv_bits = 0;
+        if (!duo::prefill_tc_supported(ap))
+            return fail(DUO_ERR_UNSUPPORTED, "tensor-core pre-fill cannot take this layer");
+        e = duo::launch_dequant(a, c, workspace, (cudaStream_t)stream);
+        if (e == cudaSuccess) {
+            const size_t code_bytes = (size_t)a.B * a.R * a.capacity * 128 * 2;   // one of K, V
+            duo::CacheArgs cp = c;
+            cp.k_full = workspace;
+            cp.v_full = static_cast<uint8_t*>(workspace) + code_bytes;
+            cp.k_scale = cp.v_scale = nullptr;
+            const float* qscale = reinterpret_cast<const float*>(static_cast<uint8_t*>(workspace) + 2 * code_bytes);
+            e = duo::launch_prefill_tc(ap, cp, q, k_chunk, v_chunk, C, out, static_cast<uint8_t*>(workspace) + staging,
+                                       ws_bytes - staging, (cudaStream_t)stream, nullptr, qscale);
+        }
+    } else if (a.dtype == DUO_BF16 && a.D == 128) {
         if (!duo::prefill_tc_supported(a))
             return fail(DUO_ERR_UNSUPPORTED, "tensor-core pre-fill cannot take this layer");
         e = duo::launch_prefill_tc(a, c, q, k_chunk, v_chunk, C, out, workspace, ws_bytes, (cudaStream_t)stream);

@@ -106,10 +106,19 @@ struct EpiArgs {
     float* dalpha;        // EPI_DOT: [Hkv] accumulated
     float sign;           // EPI_DOT: +1 or -1
 };
+// qscale non-NULL: the full cache holds 8- or 4-bit codes (as bf16 values)
+// and qscale [B][R][capacity][4] fp32 the (k scale, v scale, -, -) of each
+// row, applied to the scores and to p.
 cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void* q, const void* k_chunk,
                               const void* v_chunk, int C, void* out, void* workspace, size_t ws_bytes,
-                              cudaStream_t s, const EpiArgs* epi = nullptr);
+                              cudaStream_t s, const EpiArgs* epi = nullptr, const float* qscale = nullptr);
 cudaError_t launch_exp2_fma_probe(const float* x, float* y, int64_t n, cudaStream_t s);
+// An 8- or 4-bit layer's cached rows (below seq_len) staged for the
+// tensor-core pre-fill: the codes as bf16 values (exact) in a contiguous
+// [B][R][capacity][128] K area, the same for V, then [B][R][capacity][4]
+// fp32 (k scale, v scale, 0, 0).
+size_t dequant_staging_bytes(const LayerArgs& a);
+cudaError_t launch_dequant(const LayerArgs& a, const CacheArgs& c, void* staging, cudaStream_t s);
 // One warp waits on an mbarrier that never completes, with the given limit.
 cudaError_t launch_wait_probe(int32_t* status, uint64_t limit_ns, cudaStream_t s);
 

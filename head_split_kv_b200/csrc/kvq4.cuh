@@ -98,6 +98,16 @@ __device__ __forceinline__ void q4_store_row(const LayerArgs& a, const CacheArgs
     }
 }
 
+// Nibbles at bits 0-3 and 16-19 of w -> the fp16 pair (1024 + n0, 1024 + n1).
+__device__ __forceinline__ uint32_t u4_lo_f16x2(uint32_t w) { return (w & 0x000F000Fu) | 0x64006400u; }
+// Nibbles at bits 4-7 and 20-23 of w -> the fp16 pair (1024 + 16 n0, 1024 + 16 n1).
+__device__ __forceinline__ uint32_t u4_hi_f16x2(uint32_t w) { return (w & 0x00F000F0u) | 0x64006400u; }
+
+// Nibbles at bits 0-3 / 16-19 of w as fp16 subnormals n * 2^-24, and those
+// at bits 4-7 / 20-23 as 16 n * 2^-24, exactly (zero exponent).
+__device__ __forceinline__ uint32_t u4_lo_sub(uint32_t w) { return w & 0x000F000Fu; }
+__device__ __forceinline__ uint32_t u4_hi_sub(uint32_t w) { return w & 0x00F000F0u; }
+
 // Nibbles 0 and 4 of w (bits 0-3 and 16-19) -> two fp16 values nibble - 8,
 // exactly: a nibble n under the fp16 exponent of 1024 is the number 1024 + n,
 // and subtracting 1032 leaves n - 8.

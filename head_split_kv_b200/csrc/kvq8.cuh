@@ -84,6 +84,24 @@ __device__ __forceinline__ void i8x4_to_f16x2(uint32_t w, uint32_t& lo, uint32_t
     hi = *reinterpret_cast<const uint32_t*>(&r1);
 }
 
+// The same without the subtraction: (1152 + code 0, 1152 + code 1) and
+// (1152 + code 2, 1152 + code 3), for products whose bias is removed later.
+__device__ __forceinline__ void i8x4_to_f16x2_biased(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    const uint32_t u = w ^ 0x80808080u;
+    lo = __byte_perm(u, 0x64646464u, 0x4140);
+    hi = __byte_perm(u, 0x64646464u, 0x4342);
+}
+
+// Codes 0..3 of w as fp16 subnormals: (code + 128) * 2^-24 in each half,
+// exactly (the offset code fills bits 0-7 of the half under a zero
+// exponent).  For products whose bias, 128 times the sum of the partners,
+// is removed once at the end.
+__device__ __forceinline__ void i8x4_to_f16x2_sub(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    const uint32_t u = w ^ 0x80808080u;
+    lo = __byte_perm(u, 0u, 0x4140);
+    hi = __byte_perm(u, 0u, 0x4342);
+}
+
 __device__ __forceinline__ uint32_t f16x2_pack(float a, float b) {
     const __half2 h = __floats2half2_rn(a, b);
     return *reinterpret_cast<const uint32_t*>(&h);

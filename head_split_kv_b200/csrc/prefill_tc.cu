@@ -84,8 +84,15 @@ constexpr uint32_t kOffK = kOffQ + 2 * kQBytes;
 constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;
 constexpr uint32_t kOffBar = kOffV + 2 * kTileBytes;
 constexpr uint32_t kOffHolder = kOffBar + 16 * 8;
-constexpr uint32_t kSmemBytes = kOffHolder + 32;
+// quantized prior tiles: (k scale, v scale / 16, -, -) per key, four tiles
+// deep (a K stage is refilled after its QK MMAs, while the softmax may still
+// be on that tile; four slots outlast it -- see the producer)
+constexpr uint32_t kScaleTileBytes = BN * 16;
+constexpr uint32_t kOffScale = kOffHolder + 128;  // a tensor copy's shared destination is 128-byte aligned
+constexpr uint32_t kSmemBytes = kOffScale + 4 * kScaleTileBytes;
 static_assert(kSmemBytes + 1024 <= 232448, "one CTA per SM");
+static_assert(kOffQ % 1024 == 0 && kOffK % 1024 == 0 && kOffV % 1024 == 0, "swizzled TMA destinations");
+static_assert(kOffScale % 128 == 0 && kScaleTileBytes % 128 == 0, "TMA destinations");
 
 enum { SRC_CACHE = 0, SRC_CHUNK = 1, SRC_RING = 2 };
 
@@ -289,10 +296,24 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
 // pipe instead (exp2_fma2).  Measured on the 131K prompt: one pair in 4 or
 // in 8 (equal within run-to-run noise) beat SFU-only by 2-5 %; one in 3 was
 // slower.
+//
+// qsc (a quantized layer's prior tile, else NULL): the tile's keys are
+// codes, and qsc holds (k scale, v scale / 16, -, -) per key: the scores are multiplied by
+// the k scales before anything else, and p by v scale / 16 on the way to the
+// PV operand, which is fp16 for these tiles (the V codes are staged times 16
+// in fp16, exactly): fp16's 11-bit significand keeps the rounding of p times
+// the scale, which the row sum (of the unscaled fp32 p) cannot absorb, at
+// 2^-11 of the value.  p <= 2^8 (the lazy rescale) keeps p v_scale / 16
+// within fp16 for v scales up to 4095.  Other tiles: P in bf16, the row sum
+// of the rounded P.
 __device__ __forceinline__ float softmax_tile(uint32_t s_addr, float sl, bool masked, const uint32_t (&vis)[4],
-                                              float& m_ref, float& l_sum, bool& need) {
+                                              float& m_ref, float& l_sum, bool& need, const float* qsc) {
     float s[128];
     tmem_ld128(s_addr, s);
+    if (qsc) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) s[c] *= qsc[4 * c];
+    }
     if (masked) {
 #pragma unroll
         for (int c = 0; c < 128; ++c)
@@ -324,9 +345,16 @@ __device__ __forceinline__ float softmax_tile(uint32_t s_addr, float sl, bool ma
             const float2 x = ffma2(make_float2(s[64 * h + 2 * c2], s[64 * h + 2 * c2 + 1]), sl2, nm2);
             const float2 e = (c2 % kFmaExpEvery == kFmaExpEvery - 1) ? exp2_fma2(x)
                                                                   : make_float2(exp2_approx(x.x), exp2_approx(x.y));
-            __nv_bfloat162 hb = __floats2bfloat162_rn(e.x, e.y);
-            pk[c2] = *reinterpret_cast<uint32_t*>(&hb);
-            rs2[c2 & 3] = fadd2(rs2[c2 & 3], make_float2(bf16_lo(pk[c2]), bf16_hi(pk[c2])));
+            if (qsc) {
+                const int c = 64 * h + 2 * c2;
+                __half2 hh = __floats2half2_rn(e.x * qsc[4 * c + 1], e.y * qsc[4 * c + 5]);
+                pk[c2] = *reinterpret_cast<uint32_t*>(&hh);
+                rs2[c2 & 3] = fadd2(rs2[c2 & 3], e);
+            } else {
+                __nv_bfloat162 hb = __floats2bfloat162_rn(e.x, e.y);
+                pk[c2] = *reinterpret_cast<uint32_t*>(&hb);
+                rs2[c2 & 3] = fadd2(rs2[c2 & 3], make_float2(bf16_lo(pk[c2]), bf16_hi(pk[c2])));
+            }
         }
         tmem_st32(s_addr + 64 + 32 * h, pk);
     }
@@ -416,12 +444,17 @@ __device__ __noinline__ void merge_split_records(const float* base, int ns_use, 
 // 168 registers a thread (three of them share an SM sub-partition's 16K);
 // the split epilogue keeps its indices in shared memory and its record
 // write and merge out of line, so that the softmax loop fits without spills.
-template <int EPI>
+// QS: the full cache is a quantized layer's staging area -- K codes in bf16,
+// V codes times 16 in fp16, both exact -- and tmS its per-row (k scale,
+// v scale / 16) pairs, applied in the softmax; the PV MMAs of those tiles
+// run in fp16.
+template <int EPI, bool QS>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
                       const __grid_constant__ CUtensorMap tmVc, const __grid_constant__ CUtensorMap tmKx,
                       const __grid_constant__ CUtensorMap tmVx, const __grid_constant__ CUtensorMap tmKr,
-                      const __grid_constant__ CUtensorMap tmVr, const TcArgs p) {
+                      const __grid_constant__ CUtensorMap tmVr, const __grid_constant__ CUtensorMap tmS,
+                      const TcArgs p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const LayerArgs& a = p.a;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -533,7 +566,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint64_t* full = kv ? &v_full[st] : &k_full[st];
                     uint64_t* empty = kv ? &v_empty[st] : &k_empty[st];
                     if (j >= 2 && !mbar_wait(empty, ((j >> 1) - 1) & 1, p.status)) goto producer_done;
-                    mbar_arrive_expect_tx(full, kTileBytes);
+                    // a quantized prior tile's scales ride with its K tile, into
+                    // slot j % 4: the K stage of tile j + 4 is free once QK(j + 2)
+                    // is done, which comes after the softmax of tile j + 1
+                    const bool scales = QS && kv == 0 && t.src == SRC_CACHE;
+                    mbar_arrive_expect_tx(full, kTileBytes + (scales ? kScaleTileBytes : 0u));
+                    if (scales)
+                        tma_load_3d(smem_u32(smem + kOffScale) + (j & 3) * kScaleTileBytes, &tmS, 0, t.row, cache_z,
+                                    full);
                     const uint32_t dst = (kv ? sV : sK) + st * kTileBytes;
                     for (int half = 0; half < 2; ++half)
                         for (int rh = 0; rh < 2; ++rh) {
@@ -555,6 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(BM, BN, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16(BM, HD, 0, 1);
+            constexpr uint32_t idesc_pv16 = idesc_f16(BM, HD, 0, 1);   // a quantized prior tile: fp16 P and V
             const int n = nl, n0 = nl0;
             bool ok = mbar_wait(q_full, 0, p.status);
             // S_qi = Q_qi K_j^T: 8 MMAs of K 16 over the two 64-column halves of d
@@ -574,10 +615,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             // read MN-major
             auto issue_pv = [&](int qi, int j) {
                 const int st = j & 1;
+                const uint32_t idesc = QS && tile_at(sc, j0 + j).src == SRC_CACHE ? idesc_pv16 : idesc_pv;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
                     const uint64_t bd = sw128_desc(sV + st * kTileBytes + kk * 2048, kHalfBytes, 1024);
-                    tc_mma_ta(tmem + col_o(qi), tmem + col_s(qi) + 64 + 8 * kk, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                    tc_mma_ta(tmem + col_o(qi), tmem + col_s(qi) + 64 + 8 * kk, bd, idesc, (j > 0 || kk > 0) ? 1u : 0u);
                 }
             };
             ok = ok && mbar_wait(&k_full[0], 0, p.status);
@@ -631,7 +673,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t vis[4] = {0u, 0u, 0u, 0u};   // the tile's keys this row sees, a bit per column
             if (masked) visible_columns(a, sc, t, P, vis);
             bool need;
-            const float corr = softmax_tile(lane_base + col_s(qi), sl, masked, vis, m_ref, l_sum, need);
+            const float* qsc = QS && t.src == SRC_CACHE
+                                   ? reinterpret_cast<const float*>(smem + kOffScale + (j & 3) * kScaleTileBytes)
+                                   : nullptr;
+            const float corr = softmax_tile(lane_base + col_s(qi), sl, masked, vis, m_ref, l_sum, need, qsc);
             // O_qi holds every PV up to tile j - 1 (the commit behind s_full
             // covered them); rescale it before PV_qi(j) is issued
             if (j >= 1 && __any_sync(0xffffffffu, need)) {
@@ -794,7 +839,7 @@ size_t prefill_workspace_bytes(const LayerArgs& a, int max_chunk) {
 
 cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void* q, const void* k_chunk,
                               const void* v_chunk, int C, void* out, void* workspace, size_t ws_bytes,
-                              cudaStream_t s, const EpiArgs* epi) {
+                              cudaStream_t s, const EpiArgs* epi, const float* qscale) {
     if (!prefill_tc_supported(a)) return cudaErrorNotSupported;
     const uint64_t row = HD * 2;
     CUtensorMap mQ, mKx, mVx, mKc, mVc, mKr, mVr;
@@ -830,6 +875,15 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
         mKr = mKx;  // never read: no streaming heads, or no cache (c0 = 0)
         mVr = mVx;
     }
+    CUtensorMap mS = mKx;   // never read unless the cache holds codes
+    if (qscale != nullptr) {
+        // (k scale, v scale, -, -) per row: 16-byte rows, so the box's inner
+        // extent is one whole row and its first coordinate always 0
+        const uint64_t d[3] = {4, (uint64_t)a.capacity, (uint64_t)a.B * a.R};
+        const uint64_t st[2] = {16, 16ull * a.capacity};
+        const uint32_t bx[3] = {4, BN, 1};
+        if (!encode_tmap(&mS, qscale, 3, d, st, bx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 0)) return cudaErrorInvalidValue;
+    }
     TcArgs p;
     p.a = a;
     p.C = C;
@@ -849,12 +903,16 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
     const long grid = (long)p.n_ret_ctas + (long)a.B * a.S * a.G * p.n_mpairs;
     if (grid == 0) return cudaSuccess;
     if (grid > 0x7fffffffL) return cudaErrorInvalidConfiguration;
-    static std::atomic<unsigned long long> configured[3] = {{0}, {0}, {0}};
+    static std::atomic<unsigned long long> configured[4] = {{0}, {0}, {0}, {0}};
+    const bool qs = qscale != nullptr;
+    if (qs && mode != EPI_STORE) return cudaErrorInvalidValue;
     {
         cudaError_t e = cudaErrorInvalidValue;
-        if (mode == EPI_STORE) e = smem_limit_once(prefill_tc_kernel<EPI_STORE>, (int)(kSmemBytes + 1024), configured[0]);
-        if (mode == EPI_MIX) e = smem_limit_once(prefill_tc_kernel<EPI_MIX>, (int)(kSmemBytes + 1024), configured[1]);
-        if (mode == EPI_DOT) e = smem_limit_once(prefill_tc_kernel<EPI_DOT>, (int)(kSmemBytes + 1024), configured[2]);
+        constexpr int kS = (int)(kSmemBytes + 1024);
+        if (mode == EPI_STORE && !qs) e = smem_limit_once(prefill_tc_kernel<EPI_STORE, false>, kS, configured[0]);
+        if (mode == EPI_STORE && qs) e = smem_limit_once(prefill_tc_kernel<EPI_STORE, true>, kS, configured[3]);
+        if (mode == EPI_MIX) e = smem_limit_once(prefill_tc_kernel<EPI_MIX, false>, kS, configured[1]);
+        if (mode == EPI_DOT) e = smem_limit_once(prefill_tc_kernel<EPI_DOT, false>, kS, configured[2]);
         if (e != cudaSuccess) return e;
     }
     if (split) {
@@ -864,12 +922,16 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
         const cudaError_t e = cudaMemsetAsync(p.ticket, 0, (size_t)p.n_units * sizeof(uint32_t), s);
         if (e != cudaSuccess) return e;
     }
+    const unsigned g = (unsigned)grid;
+    constexpr size_t kS = kSmemBytes + 1024;
     if (mode == EPI_MIX)
-        prefill_tc_kernel<EPI_MIX><<<(unsigned)grid, kThreads, kSmemBytes + 1024, s>>>(mQ, mKc, mVc, mKx, mVx, mKr, mVr, p);
+        prefill_tc_kernel<EPI_MIX, false><<<g, kThreads, kS, s>>>(mQ, mKc, mVc, mKx, mVx, mKr, mVr, mS, p);
     else if (mode == EPI_DOT)
-        prefill_tc_kernel<EPI_DOT><<<(unsigned)grid, kThreads, kSmemBytes + 1024, s>>>(mQ, mKc, mVc, mKx, mVx, mKr, mVr, p);
+        prefill_tc_kernel<EPI_DOT, false><<<g, kThreads, kS, s>>>(mQ, mKc, mVc, mKx, mVx, mKr, mVr, mS, p);
+    else if (qs)
+        prefill_tc_kernel<EPI_STORE, true><<<g, kThreads, kS, s>>>(mQ, mKc, mVc, mKx, mVx, mKr, mVr, mS, p);
     else
-        prefill_tc_kernel<EPI_STORE><<<(unsigned)grid, kThreads, kSmemBytes + 1024, s>>>(mQ, mKc, mVc, mKx, mVx, mKr, mVr, p);
+        prefill_tc_kernel<EPI_STORE, false><<<g, kThreads, kS, s>>>(mQ, mKc, mVc, mKx, mVx, mKr, mVr, mS, p);
     return cudaGetLastError();
 }
 

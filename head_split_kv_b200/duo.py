@@ -81,6 +81,7 @@ _lib_partition = _fn("duo_partition_heads", ctypes.c_int, ctypes.POINTER(ctypes.
 _lib_desc_init = _fn("duo_desc_init", ctypes.c_int, _DESC, _I32, _I32, _I32, _I32, _I32, ctypes.POINTER(_I32), _I32)
 _lib_desc_validate = _fn("duo_desc_validate", ctypes.c_int, _DESC)
 _lib_ws_bytes = _fn("duo_workspace_bytes", ctypes.c_size_t, _DESC, _I32, _I32)
+_lib_pf_ws_bytes = _fn("duo_prefill_workspace_bytes", ctypes.c_size_t, _DESC, _STATE, _I32)
 _lib_permute = _fn("duo_permute_heads", ctypes.c_int, _DESC, _P, _P, ctypes.c_int64, _I32, ctypes.c_int64, _I32,
                    _I32, _P)
 _lib_append = _fn("duo_append_kv", ctypes.c_int, _DESC, _STATE, _P, _P, _I32, _P)
@@ -179,6 +180,10 @@ def desc_validate(desc: LayerDesc) -> int:
 
 def workspace_bytes(desc: LayerDesc, op: int, max_tokens: int) -> int:
     return int(_lib_ws_bytes(ctypes.byref(desc), op, max_tokens))
+
+
+def prefill_workspace_bytes(desc: LayerDesc, state: KVState, max_chunk: int) -> int:
+    return int(_lib_pf_ws_bytes(ctypes.byref(desc), ctypes.byref(state), max_chunk))
 
 
 # ------------------------------------------------------------ device calls
@@ -321,11 +326,16 @@ class LayerCaches:
 
 
 class Workspace:
-    """A zero-filled device workspace of the size the library asks for."""
+    """A zero-filled device workspace of the size the library asks for
+    (pre-fill: pass the layer's state, so that an 8- or 4-bit layer gets its
+    staging area too)."""
 
-    def __init__(self, desc: LayerDesc, op: int, max_tokens: int, device="cuda"):
+    def __init__(self, desc: LayerDesc, op: int, max_tokens: int, device="cuda", state: KVState = None):
         import torch
-        self.nbytes = workspace_bytes(desc, op, max_tokens)
+        if op == OP_PREFILL and state is not None:
+            self.nbytes = prefill_workspace_bytes(desc, state, max_tokens)
+        else:
+            self.nbytes = workspace_bytes(desc, op, max_tokens)
         self.buf = torch.zeros((max(self.nbytes, 16),), dtype=torch.uint8, device=device)
 
     @property

@@ -246,6 +246,16 @@ duo_status duo_desc_validate(const duo_layer_desc* desc);
  */
 size_t duo_workspace_bytes(const duo_layer_desc* desc, int32_t op, int32_t max_tokens);
 
+/*
+ * duo_prefill_workspace_bytes -- the workspace duo_prefill_chunk takes for
+ * chunks of up to max_chunk tokens on this layer and state: what
+ * duo_workspace_bytes(desc, DUO_OP_PREFILL, max_chunk) gives, plus, for an
+ * 8- or 4-bit full cache, the staging area of its cached rows
+ * (B * R * capacity * 528 bytes, which depends on the state's capacity).  st: host pointer to the state (only its sizes are read).
+ * Returns 0 for an invalid descriptor or state.
+ */
+size_t duo_prefill_workspace_bytes(const duo_layer_desc* desc, const duo_kv_state* st, int32_t max_chunk);
+
 /* ------------------------------------------------------------------------ */
 /* Device entry points                                                      */
 /* ------------------------------------------------------------------------ */
@@ -301,6 +311,15 @@ duo_status duo_append_kv(const duo_layer_desc* desc, const duo_kv_state* st, con
  * per key to the scores and to p (half the bytes per cached token).
  * workspace: >= duo_workspace_bytes(desc, DUO_OP_DECODE, 0) bytes, zeroed once.
  * Concurrent calls must not share a workspace.
+ * Launch overlap: the bf16 / d 128 decode is launched with programmatic
+ * dependent launch, so it can start while the kernel before it on the stream
+ * finishes, and with a contiguous full cache it loads its first cache tiles
+ * that lie at least 128 rows below seq_len before waiting for that kernel.
+ * Every other kernel of the library lets dependents start only when it
+ * completes, and the decode kernels write nothing there, so library calls
+ * need no care; a caller kernel launched just before it on the same stream
+ * that triggers programmatic launch completion early must not write those
+ * rows, nor lower seq_len, before it completes.
  * Errors: DUO_ERR_INVALID_ARG, DUO_ERR_SHAPE, DUO_ERR_CAPACITY (workspace),
  * DUO_ERR_UNSUPPORTED, DUO_ERR_CUDA.
  */
@@ -351,8 +370,19 @@ duo_status duo_decode_step(const duo_layer_desc* desc, const duo_kv_state* st, c
  *   rows go to the workspace and the split that finishes last merges them.
  *   Without it the kernel runs unsplit (same results up to rounding).
  *   Concurrent calls must not share a workspace.
- * The full cache must be contiguous (page_size 0) and not 8-bit here
- * (DUO_ERR_UNSUPPORTED): the pre-fill reads its prior tiles in bf16.
+ * The full cache must be contiguous (page_size 0).  With an 8- or 4-bit
+ * full cache the call first stages the cached rows below seq_len at the
+ * start of the workspace -- the K codes as bf16 values, the V codes times
+ * 16 as fp16 values (both exact), and each row's k and v scales -- and the
+ * pre-fill reads its prior tiles from there, multiplying each score by its
+ * key's k scale and each p by its v scale (so code * scale is never rounded
+ * to bf16); for those tiles p * v_scale / 16 is the fp16 operand of the PV
+ * product (rounded at 2^-11 of its value), which holds v scales up to 4095
+ * (|V| up to 520,000 for 8-bit codes, 28,000 for 4-bit); the workspace is
+ * then required: duo_prefill_workspace_bytes(desc, st, C) bytes (the staging
+ * area, 528 bytes per token of the capacity and retrieval head, then the
+ * split records; DUO_ERR_CAPACITY when it is missing or smaller than the
+ * staging area).
  * Errors: DUO_ERR_INVALID_ARG, DUO_ERR_SHAPE, DUO_ERR_CAPACITY,
  * DUO_ERR_UNSUPPORTED, DUO_ERR_CUDA.
  */

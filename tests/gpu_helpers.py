@@ -261,3 +261,43 @@ class Layer:
                     valid = po >= 0
                     assert np.array_equal(kr[b, s][valid], ko[valid]), f"ring K b={b} h={h}"
                     assert np.array_equal(vr[b, s][valid], vo[valid]), f"ring V b={b} h={h}"
+
+
+def prefill_run(lay, chunks, seed, sigma=None, rows_per_chunk=None):
+    """Pre-fill a prompt chunk by chunk through duo_prefill_chunk (with the
+    layer's pre-fill workspace) and duo_append_kv.  Each chunk's output rows
+    (all, or rows_per_chunk seeded ones) are compared with the oracle's
+    direct definition over the history its caches hold before the chunk
+    (for an 8- or 4-bit layer the retrieval rows as code * scale; a
+    streaming head's evicted positions as zeros, which no query of the chunk
+    sees) followed by the chunk's rows as given; the oracle's caches then
+    take the chunk."""
+    t = torch()
+    duo, sh, B = lay.duo, lay.shape, lay.B
+    n = sum(chunks)
+    q, k, v = S.prompt(sh, n, seed=seed, batch=B, sigma=sigma)
+    ws = duo.Workspace(lay.desc, duo.OP_PREFILL, max(chunks), state=lay.caches.state)
+    rng = S.rng_for(seed, 79)
+    c0 = 0
+    for ci, C in enumerate(chunks):
+        sl = slice(c0, c0 + C)
+        qd, kd, vd = (to_dev(np.ascontiguousarray(x[:, sl])) for x in (q, k, v))
+        out = t.empty_like(qd)
+        duo.prefill_chunk(lay.desc, lay.caches.state, qd, kd, vd, C, out, ws.ptr, ws.nbytes)
+        duo.append_kv(lay.desc, lay.caches.state, kd, vd, C)
+        rows = np.arange(C) if rows_per_chunk is None or C <= rows_per_chunk else \
+            np.unique(rng.choice(C, rows_per_chunk, replace=False))
+        got = f64(out)
+        for b in range(B):
+            k_all = np.zeros((c0 + C, sh.n_kv_heads, sh.head_dim))
+            v_all = np.zeros_like(k_all)
+            for h in range(sh.n_kv_heads):
+                pos, kh, vh = lay.oracle.rows(b, h)
+                if len(pos):
+                    k_all[pos, h], v_all[pos, h] = O.as_f64(kh), O.as_f64(vh)
+            k_all[c0:], v_all[c0:] = O.as_f64(k[b, sl]), O.as_f64(v[b, sl])
+            want = O.prefill_direct(q[b, sl], k_all, v_all, c0, np.array(lay.gate), sh.sink, sh.recent, rows=rows)
+            assert_close(got[b, rows], want, sh.dtype, f"chunk {ci} (c0={c0}) b={b}")
+        lay.oracle.append(k[:, sl], v[:, sl])
+        c0 += C
+    assert lay.status() == 0

@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 
 from head_split_kv_b200 import synthetic as S
-from tests.gpu_helpers import Layer, assert_close, torch
+from tests.gpu_helpers import Layer, assert_close, prefill_run, torch
 
 pytestmark = pytest.mark.gpu
 
@@ -98,3 +98,17 @@ def test_int4_decode_1m_full(duo):
         if check:
             assert_close(got, want, "bf16", f"step {i}")
     assert lay.status() == 0
+
+
+@pytest.mark.parametrize("chunks", [[300, 300, 100], [128] * 5 + [60], [4096, 4096]])
+def test_int4_prefill_reads_the_quantized_cache(duo, chunks):
+    """duo_prefill_chunk on a layer with a 4-bit full cache: the prior
+    rows widened to bf16 code * scale in the workspace's staging area, the
+    chunk's own rows as given -- against the oracle's pre-fill from its
+    4-bit caches; the caches filled by the appends stay byte-exact."""
+    sh = S.LayerShape(32, 8, 128, "bf16")
+    retrieval = S.retrieval_heads_by_seed(8, 4)
+    n = sum(chunks)
+    lay = _layer(duo, sh, retrieval, 1, n + 64)
+    prefill_run(lay, chunks, seed=34, sigma=S.head_sigma(8), rows_per_chunk=256)
+    lay.assert_caches_match()
