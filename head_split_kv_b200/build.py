@@ -1,10 +1,16 @@
 """Build step for libduo.so (the C-ABI library) with nvcc for sm_100a.
 
-    python -m head_split_kv_b200.build [--force] [--verbose]
+    python -m head_split_kv_b200.build [--force] [--verbose] [--debug-bounds]
 
 Every ``csrc/*.cu`` file is compiled to an object under ``_build/`` (in
 parallel) and linked into ``head_split_kv_b200/libduo.so``.  Nothing is
 rebuilt when the library is newer than every source and header.
+
+``--debug-bounds`` builds the same sources with ``-DDUO_DEBUG_BOUNDS`` into
+``head_split_kv_b200/libduo_debug.so`` (objects under ``_build_debug/``):
+device index checks that set DUO_DEV_BOUNDS in the status word and skip the
+access instead of faulting.  The binding loads it when the environment has
+``DUO_DEBUG_BOUNDS=1``.
 """
 
 from __future__ import annotations
@@ -23,6 +29,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libduo.so")
+BUILD_DEBUG = os.path.join(ROOT, "_build_debug")
+LIB_DEBUG = os.path.join(PKG, "libduo_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O3", "--expt-relaxed-constexpr",
@@ -45,16 +53,18 @@ def _deps():
         glob.glob(os.path.join(INCLUDE, "*.h")) + [os.path.abspath(__file__)]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def _compile(src: str, verbose: bool, ptxas_verbose: bool) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+def _compile(src: str, verbose: bool, ptxas_verbose: bool, debug_bounds: bool = False) -> str:
+    obj = os.path.join(BUILD_DEBUG if debug_bounds else BUILD, os.path.basename(src)[:-3] + ".o")
     cmd = [nvcc(), *ARCH, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
+    if debug_bounds:
+        cmd += ["-DDUO_DEBUG_BOUNDS"]
     if ptxas_verbose:
         cmd += ["-Xptxas", "-v"]
     if verbose:
@@ -67,23 +77,26 @@ def _compile(src: str, verbose: bool, ptxas_verbose: bool) -> str:
     return obj
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False) -> str:
-    """Compile and link libduo.so; returns its path."""
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False,
+          debug_bounds: bool = False) -> str:
+    """Compile and link libduo.so (libduo_debug.so with debug_bounds);
+    returns its path."""
+    lib = LIB_DEBUG if debug_bounds else LIB
+    if not force and up_to_date(lib):
+        return lib
+    os.makedirs(BUILD_DEBUG if debug_bounds else BUILD, exist_ok=True)
     srcs = _sources()
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose, ptxas_verbose), srcs))
-    tmp = LIB + ".tmp"
+        objs = list(ex.map(lambda s: _compile(s, verbose, ptxas_verbose, debug_bounds), srcs))
+    tmp = lib + ".tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs]
     if verbose:
         print(" ".join(cmd), flush=True)
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 def main(argv=None) -> int:
@@ -91,8 +104,11 @@ def main(argv=None) -> int:
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-verbose", action="store_true", help="print registers / spills / shared memory")
+    ap.add_argument("--debug-bounds", action="store_true",
+                    help="build libduo_debug.so with the device index checks (DUO_DEBUG_BOUNDS)")
     args = ap.parse_args(argv)
-    print(build(force=args.force, verbose=args.verbose, ptxas_verbose=args.ptxas_verbose))
+    print(build(force=args.force, verbose=args.verbose, ptxas_verbose=args.ptxas_verbose,
+                debug_bounds=args.debug_bounds))
     return 0
 
 

@@ -34,6 +34,7 @@ __global__ void __launch_bounds__(256) append_kernel(const LayerArgs a, const Ca
         const int t = (int)(bt % T);
         const int b = (int)(bt / T);
         const int slot = a.slot_of[h_in];
+        if (!bounds_ok(slot >= 0 && slot < a.R + a.S, c.status)) continue;
         const int L = c.seq_len[b];
         const int p = L + t;
         const uint4 val = (tensor ? v_new : k_new)[xr];
@@ -64,6 +65,7 @@ __global__ void __launch_bounds__(256) append_kernel(const LayerArgs a, const Ca
             if (!(p < a.sink || p >= L + T - a.recent)) continue;
             const int s = slot - a.R;
             const int rs = ring_slot(p, a.sink, a.recent);
+            if (!bounds_ok(rs >= 0 && rs < a.W, c.status)) continue;
             const long dst_row = ((long)b * a.S + s) * a.W + rs;
             uint4* dst = reinterpret_cast<uint4*>(tensor ? c.v_ring : c.k_ring);
             dst[dst_row * cpr + piece] = val;
@@ -105,6 +107,7 @@ __global__ void __launch_bounds__(256) append_q_kernel(const LayerArgs a, const 
         const int t = (int)(bt % T);
         const int b = (int)(bt / T);
         const int slot = a.slot_of[h_in];
+        if (!bounds_ok(slot >= 0 && slot < a.R + a.S, c.status)) continue;
         const int L = c.seq_len[b];
         const int p = L + t;
         const __nv_bfloat16* src = (kv ? v_new : k_new) + r * 128;
@@ -132,6 +135,7 @@ __global__ void __launch_bounds__(256) append_q_kernel(const LayerArgs a, const 
             if (!(p < a.sink || p >= L + T - a.recent)) continue;
             const int s = slot - a.R;
             const int rs = ring_slot(p, a.sink, a.recent);
+            if (!bounds_ok(rs >= 0 && rs < a.W, c.status)) continue;
             __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(kv ? c.v_ring : c.k_ring) + (((long)b * a.S + s) * a.W + rs) * 128;
             reinterpret_cast<uint2*>(dst)[lane] = reinterpret_cast<const uint2*>(src)[lane];
             if (s == 0 && lane == 0 && kv == 0) c.ring_pos[(long)b * a.W + rs] = p;

@@ -24,6 +24,24 @@ constexpr float kLog2e = 1.4426950408889634f;
 // and (sentinel - sentinel) is 0, so no NaN can arise.
 constexpr float kNegBig = -1.0e30f;
 
+// Index checks of the debug build (compiled with -DDUO_DEBUG_BOUNDS into
+// libduo_debug.so): a check that fails ORs DUO_DEV_BOUNDS into the status word
+// and the caller skips the access it guards -- never a trap.  In the release
+// build every check is the constant true and compiles away.  The checks sit
+// at the writes whose addresses come from computed indices (outputs, cache
+// rows, ring slots, split records) and at the untiled bulk reads; tensor-map
+// copies are bounds-checked by the TMA unit itself.
+__device__ __forceinline__ bool bounds_ok(bool ok, int32_t* status) {
+#ifdef DUO_DEBUG_BOUNDS
+    if (!ok && status != nullptr) atomicOr(status, (int32_t)DUO_DEV_BOUNDS);
+    return ok;
+#else
+    (void)ok;
+    (void)status;
+    return true;
+#endif
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

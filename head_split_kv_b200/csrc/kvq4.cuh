@@ -68,6 +68,7 @@ __device__ __forceinline__ uint8_t q4_byte(int lo, int hi) {
 // lane 0 stores the scale.
 __device__ __forceinline__ void q4_store_row(const LayerArgs& a, const CacheArgs& c, int kv, int b, int slot, int p,
                                              const int (&code)[4], float scale, int lane) {
+    if (!bounds_ok(slot >= 0 && slot < a.R && p >= 0 && p < a.capacity, c.status)) return;  // warp-uniform
     const size_t z = (size_t)b * a.R + slot;
     if (kv == 0) {
         // lane l: features 4l + i = 32 q + 4 kb + i with q = l / 8, kb = l % 8;

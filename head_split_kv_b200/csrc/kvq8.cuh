@@ -56,6 +56,7 @@ __device__ __forceinline__ uint32_t q8_quantize(const float (&x)[4], float& scal
 // byte in each of the tile's feature rows; lane 0 stores the scale.
 __device__ __forceinline__ void q8_store_row(const LayerArgs& a, const CacheArgs& c, int kv, int b, int slot, int p,
                                              uint32_t codes, float scale, int lane) {
+    if (!bounds_ok(slot >= 0 && slot < a.R && p >= 0 && p < a.capacity, c.status)) return;  // warp-uniform
     const size_t z = (size_t)b * a.R + slot;
     if (kv == 0) {
         reinterpret_cast<uint32_t*>(static_cast<int8_t*>(c.k_full) + (z * a.capacity + p) * 128)[lane] = codes;

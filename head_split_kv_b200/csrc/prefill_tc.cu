@@ -696,16 +696,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // epilogue: O / l -> bf16 (or the gated mix's epilogues)
         const size_t row_off = (((size_t)b * p.C + crow) * a.Hq + q_idx) * HD;
+        // the output row (and the record of a split) exist: CTA-uniform
+        const bool out_ok = bounds_ok(b < a.B && q_idx >= 0 && q_idx < a.Hq, p.status);
         uint4 pre[16];   // EPI_MIX / EPI_DOT: this row of out / dout, loaded before the wait below
         if constexpr (EPI != EPI_STORE) {
             const uint4* src = reinterpret_cast<const uint4*>(
                 static_cast<const __nv_bfloat16*>(EPI == EPI_MIX ? p.out : p.epi.dout) + row_off);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) pre[i] = crow < p.C ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+            for (int i = 0; i < 16; ++i) pre[i] = crow < p.C && out_ok ? src[i] : make_uint4(0u, 0u, 0u, 0u);
         }
         if (ok && n_me >= 1) ok = __all_sync(0xffffffffu, mbar_wait(&o_done[qi], 0, p.status));
         __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.out) + row_off;
-        if (EPI != EPI_STORE || holder[4] == 1u) {
+        if (!out_ok) {
+            // debug build: the check failed, nothing is written
+        } else if (EPI != EPI_STORE || holder[4] == 1u) {
             if (ok && n_me >= 1) {
                 tc_fence_after();
                 const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
@@ -748,7 +752,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (lane == 0) atomicAdd(&p.epi.dalpha[kv_idx], p.epi.sign * dot);
                 }
             }
-        } else if constexpr (EPI == EPI_STORE) {
+        } else if (EPI == EPI_STORE &&
+                   bounds_ok((int)holder[2] < p.n_units && (int)holder[3] < p.ns && (int)holder[4] <= p.ns, p.status)) {
             // (1) this split's record of the query tile: m, l and O unnormalised
             const bool have = ok && n_me >= 1;               // warp-uniform
             const int unit_ = (int)holder[2], split_ = (int)holder[3], ns_use_ = (int)holder[4];

@@ -53,6 +53,8 @@ __global__ void __launch_bounds__(kThreadsSimt) simt_attention_kernel(const Laye
     const int slot = qh_blk / a.G, g = qh_blk % a.G;
     const int q_idx = a.q_head0[slot] + g;         // caller's query-head index
     const int kv_idx = a.kv_head[slot];            // caller's KV-head index
+    if (!bounds_ok(b < a.B && q_idx >= 0 && q_idx < a.Hq && kv_idx >= 0 && kv_idx < a.Hkv, c.status))
+        return;                                    // debug build only; the same for the whole CTA
     const int r0 = blockIdx.x * kRows;
     const int row = r0 + (threadIdx.x >> 2);
     const int quarter = threadIdx.x & 3;

@@ -6,7 +6,11 @@ objects with ``data_ptr()`` (torch tensors); streams are raw ``cudaStream_t``
 values, torch streams, or None for torch's current stream.
 
 Importing this module fails with ImportError when libduo.so has not been
-built; there is no other implementation to fall back to.
+built; there is no other implementation to fall back to.  With
+``DUO_DEBUG_BOUNDS=1`` in the environment it loads libduo_debug.so instead:
+the same kernels built with device index checks, which set DEV_BOUNDS in the
+status word and skip the access rather than fault
+(``python -m head_split_kv_b200.build --debug-bounds``).
 """
 
 from __future__ import annotations
@@ -15,10 +19,12 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libduo.so")
+DEBUG_BOUNDS = os.environ.get("DUO_DEBUG_BOUNDS", "0") not in ("", "0")
+LIB_PATH = os.path.join(_HERE, "libduo_debug.so" if DEBUG_BOUNDS else "libduo.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is not built; run `python -m head_split_kv_b200.build`")
+    raise ImportError(f"{LIB_PATH} is not built; run `python -m head_split_kv_b200.build"
+                      f"{' --debug-bounds' if DEBUG_BOUNDS else ''}`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -30,7 +36,7 @@ STREAM_LAMBDA, STREAM_CHUNK = 0, 1
 KV_PLAIN, KV_INT8, KV_INT4 = 0, 1, 2
 MODEL_TO_BLOCK, BLOCK_TO_MODEL = 0, 1
 OP_DECODE, OP_PREFILL = 0, 1
-DEV_FULL_CACHE_OVERFLOW, DEV_BAD_PAGE, DEV_WAIT_TIMEOUT, DEV_BAD_LENGTH = 1, 2, 4, 8
+DEV_FULL_CACHE_OVERFLOW, DEV_BAD_PAGE, DEV_WAIT_TIMEOUT, DEV_BAD_LENGTH, DEV_BOUNDS = 1, 2, 4, 8, 16
 MAX_KV_HEADS = 64
 STATE_COUNTER_WORDS = 4
 

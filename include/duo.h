@@ -88,7 +88,10 @@ enum {
     DUO_DEV_FULL_CACHE_OVERFLOW = 1, /* append past capacity: row not written */
     DUO_DEV_BAD_PAGE = 2,            /* page table entry missing / out of pool */
     DUO_DEV_WAIT_TIMEOUT = 4,        /* a bounded device wait ran out          */
-    DUO_DEV_BAD_LENGTH = 8           /* a sequence length outside [0, capacity] */
+    DUO_DEV_BAD_LENGTH = 8,          /* a sequence length outside [0, capacity] */
+    DUO_DEV_BOUNDS = 16              /* debug build only (libduo_debug.so, built with
+                                        DUO_DEBUG_BOUNDS): an index check failed and
+                                        the access it guarded was skipped           */
 };
 
 #define DUO_MAX_KV_HEADS 64

@@ -40,6 +40,23 @@ def test_library_exports_every_declared_symbol(duo):
         assert hasattr(lib, n)
 
 
+def test_debug_bounds_library_exports_the_same_symbols(duo):
+    """libduo_debug.so (the build with device index checks, built beside
+    libduo.so) exports every declared entry point too, and the binding loads
+    it in a process whose environment asks for it."""
+    debug = os.path.join(os.path.dirname(duo.LIB_PATH), "libduo_debug.so")
+    assert os.path.exists(debug), "build both libraries: python -m head_split_kv_b200.build [--debug-bounds]"
+    out = subprocess.run(["nm", "-D", "--defined-only", debug], capture_output=True, text=True, check=True)
+    exported = set(re.findall(r"\s[TW]\s(duo_\w+)", out.stdout))
+    missing = [n for n in _declared_functions() if n not in exported]
+    assert not missing, f"declared in duo.h but not exported by the debug build: {missing}"
+    probe = ("import head_split_kv_b200.duo as d; "
+             "print(d.LIB_PATH.endswith('libduo_debug.so'), d.abi_version(), d.DEV_BOUNDS)")
+    r = subprocess.run([os.sys.executable, "-c", probe], cwd=ROOT, capture_output=True, text=True, check=True,
+                       env={**os.environ, "DUO_DEBUG_BOUNDS": "1"})
+    assert r.stdout.split() == ["True", str(duo.ABI_VERSION), "16"]
+
+
 def test_struct_layouts_match_the_c_compiler(duo, tmp_path):
     src = tmp_path / "layout.c"
     src.write_text("""
