@@ -1351,16 +1351,14 @@ __device__ __forceinline__ void quant_scores(float s0, float s1, float s2, float
 }
 
 // One tile of the online softmax for the lane's row (query head lane / 4,
-// shared by the quad's four lanes), in two parts, so that a caller can put
-// independent work (the next tile's q . K) between the branches of the first
-// and the straight-line code of the second.  softmax_max_rescale takes the
-// row maximum over the quad and rescales O, l and the PV bias sums only when
-// some row's maximum grew (a warp vote), which over a long cache is rare;
-// softmax_exp forms p = 2^(s - m) and adds it to the row sum.  A masked key
+// shared by the quad's four lanes): the row maximum over the quad, p =
+// 2^(s - m), the running sum; O, l and the PV bias sums are rescaled only
+// when some row's maximum grew (a warp vote), which over a long cache is
+// rare.  A masked key
 // (-inf) gets p = 0; m starts at a finite -1e30, so a row with no key yet
 // keeps p = 0 and a factor of 1.
 template <int NWS>
-__device__ __forceinline__ void softmax_max_rescale(const float (&sv)[4], float& m_run, float& l_run,
+__device__ __forceinline__ void online_softmax_step(const float (&sv)[4], float& m_run, float& l_run, float (&pr)[4],
                                                     float (&o)[16][2], float (&wsum)[NWS][2]) {
     float mx = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
@@ -1381,9 +1379,6 @@ __device__ __forceinline__ void softmax_max_rescale(const float (&sv)[4], float&
         }
         m_run = m_new;
     }
-}
-
-__device__ __forceinline__ void softmax_exp(const float (&sv)[4], float m_run, float& l_run, float (&pr)[4]) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) pr[i] = exp2f(sv[i] - m_run);
     l_run += (pr[0] + pr[1]) + (pr[2] + pr[3]);
@@ -1556,10 +1551,15 @@ __global__ void __maxnreg__(200)
         for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = 0.f;
         const float sl = a.scale * kLog2e;
         const int key_base = warp * 16;
-        // S = q . codes for the lane's keys key_base + 8 nb + (lane >> 2) of
-        // stage st, less the bias constant
-        auto qk_tile = [&](int st, float (&sr)[4]) {
+        for (int t = 0; t < n_tiles; ++t) {
+            const int st = t % STAGES, round = t / STAGES;
+            if (!mbar_wait(&full_bar[st], round & 1, c.status)) break;
+            const int n = s_tile_n[st];
             const uint8_t* tK = sK8 + (size_t)st * kQ8Bytes;
+            const uint8_t* tV = sV8 + (size_t)st * kQ8Bytes;
+            const float* ksc = sSc + st * 2 * kTile;
+            const float* vsc = ksc + kTile;
+            // S = q . codes for keys key_base + 8 nb + (lane >> 2)
             float s[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
             for (int nb = 0; nb < 2; ++nb) {
@@ -1574,36 +1574,13 @@ __global__ void __maxnreg__(200)
                     mma_f16_rows8(s[nb][0], s[nb][1], qa[kb][0], qa[kb][1], b0, b1);
                 }
             }
-            sr[0] = s[0][0] - q_corr;
-            sr[1] = s[0][1] - q_corr;
-            sr[2] = s[1][0] - q_corr;
-            sr[3] = s[1][1] - q_corr;
-        };
-        // Software-pipelined as in the 4-bit kernel: the q . K of tile t + 1
-        // shares a straight-line block with the exponentials and P V of tile t.
-        float s_cur[4] = {0.f, 0.f, 0.f, 0.f};
-        bool ok = n_tiles > 0 && mbar_wait(&full_bar[0], 0, c.status);
-        if (ok) qk_tile(0, s_cur);
-        for (int t = 0; t < n_tiles && ok; ++t) {
-            const int st = t % STAGES;
-            const int n = s_tile_n[st];
-            const uint8_t* tV = sV8 + (size_t)st * kQ8Bytes;
-            const float* ksc = sSc + st * 2 * kTile;
-            const float* vsc = ksc + kTile;
             // this lane's keys: key_base + 2 quad + {0, 1} and + 8
             const int k0 = key_base + 2 * quad;
             float sv[4], vs[4];
-            quant_scores(s_cur[0], s_cur[1], s_cur[2], s_cur[3], ksc, vsc, k0, n, sl, sv, vs);
-            softmax_max_rescale(sv, m_run, l_run, o, wsum);
-            int st_next = st;
-            if (t + 1 < n_tiles) {
-                st_next = (t + 1) % STAGES;
-                ok = mbar_wait(&full_bar[st_next], ((t + 1) / STAGES) & 1, c.status);
-                if (!ok) st_next = st;
-            }
-            qk_tile(st_next, s_cur);
+            quant_scores(s[0][0] - q_corr, s[0][1] - q_corr, s[1][0] - q_corr, s[1][1] - q_corr, ksc, vsc, k0, n,
+                         sl, sv, vs);
             float pr[4];
-            softmax_exp(sv, m_run, l_run, pr);
+            online_softmax_step(sv, m_run, l_run, pr, o, wsum);
             // p times the key's V scale, the fp16 A operand of O += P V
             const uint32_t pa0 = f16x2_pack(pr[0] * vs[0], pr[1] * vs[1]);
             const uint32_t pa1 = f16x2_pack(pr[2] * vs[2], pr[3] * vs[3]);
@@ -1883,11 +1860,16 @@ __global__ void __maxnreg__(200)
         const float sl = a.scale * kLog2e;
         const int key_base = warp * 16;
         const __half2 sixteenth = __float2half2_rn(0.0625f);
-        // S' = q . (biased codes) for the lane's keys key_base + 8 nb + (lane
-        // >> 2) of stage st, even and odd k-steps in separate accumulators,
-        // less the bias constant
-        auto qk_tile = [&](int st, float (&sr)[4]) {
+        for (int t = 0; t < n_tiles; ++t) {
+            const int st = t % STAGES, round = t / STAGES;
+            if (!mbar_wait(&full_bar[st], round & 1, c.status)) break;
+            const int n = s_tile_n[st];
             const uint8_t* tK = sK4 + (size_t)st * kQ4TileBytes;
+            const uint8_t* tV = sV4 + (size_t)st * kQ4TileBytes;
+            const float* ksc = sSc + st * 2 * kTile;
+            const float* vsc = ksc + kTile;
+            // S' = q . (biased codes) for keys key_base + 8 nb + (lane >> 2),
+            // even and odd k-steps in separate accumulators
             float s[2][2][2] = {{{0.f, 0.f}, {0.f, 0.f}}, {{0.f, 0.f}, {0.f, 0.f}}};
 #pragma unroll
             for (int nb = 0; nb < 2; ++nb) {
@@ -1903,40 +1885,14 @@ __global__ void __maxnreg__(200)
                                   u4_hi_f16x2(w8));
                 }
             }
-            sr[0] = s[0][0][0] + s[0][1][0] - q_corr;
-            sr[1] = s[0][0][1] + s[0][1][1] - q_corr;
-            sr[2] = s[1][0][0] + s[1][1][0] - q_corr;
-            sr[3] = s[1][0][1] + s[1][1][1] - q_corr;
-        };
-        // Software-pipelined over tiles: the q . K of tile t + 1 is issued in
-        // the same straight-line block as the exponentials and the P V of
-        // tile t, so the two dependency chains overlap (a warp has little
-        // else to hide latency with: two CTAs of four consumer warps per SM).
-        // On the last tile the look-ahead reads the current stage again and
-        // is discarded.
-        float s_cur[4] = {0.f, 0.f, 0.f, 0.f};
-        bool ok = n_tiles > 0 && mbar_wait(&full_bar[0], 0, c.status);
-        if (ok) qk_tile(0, s_cur);
-        for (int t = 0; t < n_tiles && ok; ++t) {
-            const int st = t % STAGES;
-            const int n = s_tile_n[st];
-            const uint8_t* tV = sV4 + (size_t)st * kQ4TileBytes;
-            const float* ksc = sSc + st * 2 * kTile;
-            const float* vsc = ksc + kTile;
             // this lane's keys: key_base + 2 quad + {0, 1} and + 8
             const int k0 = key_base + 2 * quad;
             float sv[4], vs[4];
-            quant_scores(s_cur[0], s_cur[1], s_cur[2], s_cur[3], ksc, vsc, k0, n, sl, sv, vs);
-            softmax_max_rescale(sv, m_run, l_run, o, wsum);
-            int st_next = st;
-            if (t + 1 < n_tiles) {
-                st_next = (t + 1) % STAGES;
-                ok = mbar_wait(&full_bar[st_next], ((t + 1) / STAGES) & 1, c.status);
-                if (!ok) st_next = st;
-            }
-            qk_tile(st_next, s_cur);
+            quant_scores(s[0][0][0] + s[0][1][0] - q_corr, s[0][0][1] + s[0][1][1] - q_corr,
+                         s[1][0][0] + s[1][1][0] - q_corr, s[1][0][1] + s[1][1][1] - q_corr, ksc, vsc, k0, n, sl, sv,
+                         vs);
             float pr[4];
-            softmax_exp(sv, m_run, l_run, pr);
+            online_softmax_step(sv, m_run, l_run, pr, o, wsum);
             // p times the key's V scale, the fp16 A operand of O += P V, and
             // the same divided by 16 for the high-nibble feature rows
             const uint32_t pa0 = f16x2_pack(pr[0] * vs[0], pr[1] * vs[1]);

@@ -8,11 +8,12 @@ the binding bound to the debug library) over small cases that reach every
 kernel -- tensor-core and CUDA-core pre-fill, the pre-fill key-range splits,
 appends to contiguous and paged caches, the fused decode step over bf16, 8-
 and 4-bit caches, the gated mix and its gradient -- no check fires (the
-status words stay 0), the caches are byte-identical, and the outputs agree
-with the release build's: to within one bf16 unit in the last place for
-attention outputs (the decode's drawn tiles change which split sums which
-keys from run to run, so the rounding order is not fixed) and to 1e-5 for
-the gate gradient (float atomics).
+status words stay 0), the caches match the oracle byte for byte, the pre-fill and
+gated-mix outputs are bit-identical to the release build's (their reduction
+order is fixed), the decode outputs of both builds are within the parity
+bound of the oracle (the decode's drawn tiles change which split holds which
+keys from run to run, and with it each p's bf16 rounding), and the gate
+gradients agree to 1e-5 (float atomics).
 
 Making a check fire on purpose would need an out-of-range index on the GPU,
 and a check that failed to catch it would fault; the checks are therefore
@@ -26,7 +27,7 @@ import numpy as np
 import pytest
 
 from head_split_kv_b200 import synthetic as S
-from gpu_helpers import Layer, bits, f64, to_dev, torch
+from gpu_helpers import Layer, assert_close, bits, f64, to_dev, torch
 
 pytestmark = pytest.mark.gpu
 
@@ -55,14 +56,6 @@ def duo_debug():
     t.cuda.synchronize()
 
 
-def _same_to_an_ulp(a: np.ndarray, b: np.ndarray, what: str) -> None:
-    """bf16 results equal up to one unit in the last place (8-bit significand)."""
-    a, b = a.astype(np.float64), b.astype(np.float64)
-    tol = np.maximum(np.abs(a), np.abs(b)) * 2.0 ** -7 + 1e-30
-    bad = np.abs(a - b) > tol
-    assert not bad.any(), f"{what}: {int(bad.sum())} values differ by more than one ulp"
-
-
 # (name, shape, retrieval KV heads, batch, pre-fill chunks, decode steps,
 #  paged, 8/4-bit cache)
 CASES = [
@@ -78,8 +71,9 @@ CASES = [
 
 
 def _run_case(duo, case, seed):
-    """Pre-fill and append the chunks, then fused decode steps; returns the
-    outputs (float64) after checking the caches against the oracle twin."""
+    """Pre-fill and append the chunks, then fused decode steps, each checked
+    against the oracle; returns the pre-fill outputs (float64) and the status
+    word after checking the caches against the oracle twin."""
     t = torch()
     name, sh, retrieval, B, chunks, steps, paged, bits_ = case
     n = sum(chunks)
@@ -106,8 +100,8 @@ def _run_case(duo, case, seed):
     else:
         lay.append(k[:, :n], v[:, :n])
     for i in range(steps):
-        got, _ = lay.decode(q[:, n + i], k[:, n + i], v[:, n + i], check_oracle=False, fused=True)
-        outs.append(got)
+        got, want = lay.decode(q[:, n + i], k[:, n + i], v[:, n + i], fused=True)
+        assert_close(got, want, sh.dtype, f"{name}: decode step {i} ({os.path.basename(duo.LIB_PATH)})")
     t.cuda.synchronize()
     status = lay.status()
     lay.assert_caches_match()
@@ -122,7 +116,7 @@ def test_debug_build_checks_do_not_fire_and_change_nothing(duo, duo_debug, case)
     assert st_dbg == 0, f"debug build status 0x{st_dbg:x} (DUO_DEV_BOUNDS = {duo.DEV_BOUNDS})"
     assert len(rel) == len(dbg)
     for i, (a, b) in enumerate(zip(rel, dbg)):
-        _same_to_an_ulp(a, b, f"{case[0]}: output {i}")
+        assert np.array_equal(a, b), f"{case[0]}: pre-fill chunk {i} differs between the builds"
 
 
 @pytest.mark.parametrize("dtype,hq,hkv,d,n", [("bf16", 16, 4, 128, 700), ("fp32", 8, 8, 64, 300)])
@@ -145,8 +139,5 @@ def test_debug_build_gated_mix_and_gradient(duo, duo_debug, dtype, hq, hkv, d, n
         assert status.item() == 0, f"{mod.LIB_PATH}: status 0x{status.item():x}"
         res.append((f64(out), bits(dalpha).astype(np.float64)))
     (o_rel, g_rel), (o_dbg, g_dbg) = res
-    if dtype == "bf16":
-        _same_to_an_ulp(o_rel, o_dbg, "gated mix")
-    else:
-        assert np.array_equal(o_rel, o_dbg), "gated mix (fp32, fixed order)"
+    assert np.array_equal(o_rel, o_dbg), "gated mix differs between the builds"
     assert np.allclose(g_rel, g_dbg, rtol=1e-5, atol=1e-5 * np.abs(g_rel).max()), (g_rel, g_dbg)
