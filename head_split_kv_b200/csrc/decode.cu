@@ -1350,17 +1350,40 @@ __device__ __forceinline__ void quant_scores(float s0, float s1, float s2, float
     }
 }
 
-// One tile of the online softmax for the lane's row (query head lane / 4,
-// shared by the quad's four lanes): the row maximum over the quad, p =
-// 2^(s - m), the running sum; O, l and the PV bias sums are rescaled only
-// when some row's maximum grew (a warp vote), which over a long cache is
-// rare.  A masked key
-// (-inf) gets p = 0; m starts at a finite -1e30, so a row with no key yet
-// keeps p = 0 and a factor of 1.
+// Runs before griddepcontrol.wait in the 8- and 4-bit kernels: asks L2 for
+// the first kWarmTiles tiles of this split's contiguous row range (codes and
+// scales), computed from a relaxed read of seq_len, so that the first loads
+// after the wait hit L2.  A stale length only moves or wastes a prefetch;
+// the rows are clamped to the cache and nothing is written.
+__device__ __forceinline__ void warm_l2_quant_split(const LayerArgs& a, const CacheArgs& c, const DecodeArgs& d,
+                                                    int b, int slot, int split, uint32_t k_row_bytes,
+                                                    uint32_t v_tile_bytes) {
+    int len = ld_relaxed_gpu(&c.seq_len[b]) + (d.k_new != nullptr ? 1 : 0);
+    len = max(0, min(len, a.capacity));
+    const int per = (len + d.nsplit - 1) / d.nsplit;
+    const int chunk = (per + kTile - 1) / kTile * kTile;
+    const int row_begin = min(len, split * chunk);
+    const int row_end = min(len, row_begin + chunk);
+    const size_t z = (size_t)b * a.R + slot;
+    const uint8_t* kf = static_cast<const uint8_t*>(c.k_full);
+    const uint8_t* vf = static_cast<const uint8_t*>(c.v_full);
+    for (int k = 0; k < kWarmTiles; ++k) {
+        const int r0 = row_begin + k * kTile;
+        if (r0 >= row_end) break;
+        bulk_prefetch_l2(kf + (z * a.capacity + r0) * k_row_bytes, kTile * k_row_bytes);
+        bulk_prefetch_l2(vf + (z * (a.capacity / kTile) + r0 / kTile) * v_tile_bytes, v_tile_bytes);
+        bulk_prefetch_l2(c.k_scale + z * a.capacity + r0, kTile * 4);
+        bulk_prefetch_l2(c.v_scale + z * a.capacity + r0, kTile * 4);
+    }
+}
+
+// The online softmax over one or more tiles in two parts: rescale_to_max
+// takes the row maximum of this lane's scores (mx) over the quad and
+// rescales O, l and the PV bias sums only when some row's maximum grew (a
+// warp vote); softmax_exp forms p = 2^(s - m) and adds it to the row sum.
 template <int NWS>
-__device__ __forceinline__ void online_softmax_step(const float (&sv)[4], float& m_run, float& l_run, float (&pr)[4],
-                                                    float (&o)[16][2], float (&wsum)[NWS][2]) {
-    float mx = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
+__device__ __forceinline__ void rescale_to_max(float mx, float& m_run, float& l_run, float (&o)[16][2],
+                                               float (&wsum)[NWS][2]) {
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
     const float m_new = fmaxf(m_run, mx);
@@ -1379,6 +1402,9 @@ __device__ __forceinline__ void online_softmax_step(const float (&sv)[4], float&
         }
         m_run = m_new;
     }
+}
+
+__device__ __forceinline__ void softmax_exp(const float (&sv)[4], float m_run, float& l_run, float (&pr)[4]) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) pr[i] = exp2f(sv[i] - m_run);
     l_run += (pr[0] + pr[1]) + (pr[2] + pr[3]);
@@ -1437,6 +1463,7 @@ __global__ void __maxnreg__(200)
     if (warp == NW && lane == 0) {
         prefetch_map(&tmK8);
         prefetch_map(&tmV8);
+        if (retrieval) warm_l2_quant_split(a, c, d, b, slot, split, 128, kQ8Bytes);
     }
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -1551,56 +1578,80 @@ __global__ void __maxnreg__(200)
         for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = 0.f;
         const float sl = a.scale * kLog2e;
         const int key_base = warp * 16;
-        for (int t = 0; t < n_tiles; ++t) {
-            const int st = t % STAGES, round = t / STAGES;
-            if (!mbar_wait(&full_bar[st], round & 1, c.status)) break;
-            const int n = s_tile_n[st];
-            const uint8_t* tK = sK8 + (size_t)st * kQ8Bytes;
-            const uint8_t* tV = sV8 + (size_t)st * kQ8Bytes;
-            const float* ksc = sSc + st * 2 * kTile;
-            const float* vsc = ksc + kTile;
-            // S = q . codes for keys key_base + 8 nb + (lane >> 2)
-            float s[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+        // one pass over NT (1 or 2) consecutive tiles, as in the 4-bit kernel
+        auto pass = [&](int t, auto nt_c) -> bool {
+            constexpr int NT = decltype(nt_c)::value;
+            int st[NT];
+            bool ok = true;
 #pragma unroll
-            for (int nb = 0; nb < 2; ++nb) {
-                const int key = key_base + 8 * nb + row;
-                const uint4 lo = *reinterpret_cast<const uint4*>(tK + key * 128 + (((2 * quad) ^ (key & 7)) << 4));
-                const uint4 hi = *reinterpret_cast<const uint4*>(tK + key * 128 + (((2 * quad + 1) ^ (key & 7)) << 4));
-                const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-#pragma unroll
-                for (int kb = 0; kb < 8; ++kb) {
-                    uint32_t b0, b1;
-                    i8x4_to_f16x2_biased(w[kb], b0, b1);
-                    mma_f16_rows8(s[nb][0], s[nb][1], qa[kb][0], qa[kb][1], b0, b1);
-                }
+            for (int i = 0; i < NT; ++i) {
+                st[i] = (t + i) % STAGES;
+                ok = ok && mbar_wait(&full_bar[st[i]], ((t + i) / STAGES) & 1, c.status);
             }
+            if (!ok) return false;
             // this lane's keys: key_base + 2 quad + {0, 1} and + 8
             const int k0 = key_base + 2 * quad;
-            float sv[4], vs[4];
-            quant_scores(s[0][0] - q_corr, s[0][1] - q_corr, s[1][0] - q_corr, s[1][1] - q_corr, ksc, vsc, k0, n,
-                         sl, sv, vs);
-            float pr[4];
-            online_softmax_step(sv, m_run, l_run, pr, o, wsum);
-            // p times the key's V scale, the fp16 A operand of O += P V
-            const uint32_t pa0 = f16x2_pack(pr[0] * vs[0], pr[1] * vs[1]);
-            const uint32_t pa1 = f16x2_pack(pr[2] * vs[2], pr[3] * vs[3]);
-            // O' += P U with U = (code + 128) 2^-24 (exact fp16 subnormals),
-            // and the bias sum W += P 1 through the same MMA: O = 2^24 O' -
-            // 128 W at the end.  Feature row 8 nd + (lane >> 2), this warp's
-            // 16-key group (64-byte swizzle), the lane's four keys in one word
-            mma_f16_rows8(wsum[0][0], wsum[0][1], pa0, pa1, kF16x2One, kF16x2One);
+            float sv[NT][4], vs[NT][4];
 #pragma unroll
-            for (int nd = 0; nd < 16; ++nd) {
-                const int f = 8 * nd + row;
-                const uint32_t w = *reinterpret_cast<const uint32_t*>(tV + f * 64 + ((warp ^ ((f >> 1) & 3)) << 4) +
-                                                                      4 * quad);
-                uint32_t b0, b1;
-                i8x4_to_f16x2_sub(w, b0, b1);
-                mma_f16_rows8(o[nd][0], o[nd][1], pa0, pa1, b0, b1);
+            for (int i = 0; i < NT; ++i) {
+                // S = q . codes for keys key_base + 8 nb + (lane >> 2)
+                const uint8_t* tK = sK8 + (size_t)st[i] * kQ8Bytes;
+                float s[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+                for (int nb = 0; nb < 2; ++nb) {
+                    const int key = key_base + 8 * nb + row;
+                    const uint4 lo = *reinterpret_cast<const uint4*>(tK + key * 128 + (((2 * quad) ^ (key & 7)) << 4));
+                    const uint4 hi = *reinterpret_cast<const uint4*>(tK + key * 128 + (((2 * quad + 1) ^ (key & 7)) << 4));
+                    const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+                    for (int kb = 0; kb < 8; ++kb) {
+                        uint32_t b0, b1;
+                        i8x4_to_f16x2_biased(w[kb], b0, b1);
+                        mma_f16_rows8(s[nb][0], s[nb][1], qa[kb][0], qa[kb][1], b0, b1);
+                    }
+                }
+                const float* ksc = sSc + st[i] * 2 * kTile;
+                quant_scores(s[0][0] - q_corr, s[0][1] - q_corr, s[1][0] - q_corr, s[1][1] - q_corr, ksc,
+                             ksc + kTile, k0, s_tile_n[st[i]], sl, sv[i], vs[i]);
+            }
+            float mx = kNegBig;
+#pragma unroll
+            for (int i = 0; i < NT; ++i) mx = fmaxf(mx, fmaxf(fmaxf(sv[i][0], sv[i][1]), fmaxf(sv[i][2], sv[i][3])));
+            rescale_to_max(mx, m_run, l_run, o, wsum);
+#pragma unroll
+            for (int i = 0; i < NT; ++i) {
+                float pr[4];
+                softmax_exp(sv[i], m_run, l_run, pr);
+                // p times the key's V scale, the fp16 A operand of O += P V
+                const uint32_t pa0 = f16x2_pack(pr[0] * vs[i][0], pr[1] * vs[i][1]);
+                const uint32_t pa1 = f16x2_pack(pr[2] * vs[i][2], pr[3] * vs[i][3]);
+                // O' += P U with U = (code + 128) 2^-24 (exact fp16 subnormals),
+                // and the bias sum W += P 1 through the same MMA: O = 2^24 O' -
+                // 128 W at the end.  Feature row 8 nd + (lane >> 2), this warp's
+                // 16-key group (64-byte swizzle), the lane's four keys in one word
+                mma_f16_rows8(wsum[0][0], wsum[0][1], pa0, pa1, kF16x2One, kF16x2One);
+                const uint8_t* tV = sV8 + (size_t)st[i] * kQ8Bytes;
+#pragma unroll
+                for (int nd = 0; nd < 16; ++nd) {
+                    const int f = 8 * nd + row;
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(tV + f * 64 + ((warp ^ ((f >> 1) & 3)) << 4) +
+                                                                          4 * quad);
+                    uint32_t b0, b1;
+                    i8x4_to_f16x2_sub(w, b0, b1);
+                    mma_f16_rows8(o[nd][0], o[nd][1], pa0, pa1, b0, b1);
+                }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty_bar[st]);
-        }
+            if (lane == 0) {
+#pragma unroll
+                for (int i = 0; i < NT; ++i) mbar_arrive(&empty_bar[st[i]]);
+            }
+            return true;
+        };
+        int t = 0;
+        bool ok = true;
+        for (; ok && t + 1 < n_tiles; t += 2) ok = pass(t, std::integral_constant<int, 2>{});
+        if (ok && t < n_tiles) pass(t, std::integral_constant<int, 1>{});
         l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
         l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
     }
@@ -1730,6 +1781,7 @@ __global__ void __maxnreg__(200)
         mbar_init(comb_bar, 1);
         fence_barrier_init();
     }
+    if (retrieval && warp == NW && lane == 0) warm_l2_quant_split(a, c, d, b, slot, split, kQ4RowBytes, kQ4TileBytes);
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (threadIdx.x == 0) *s_flag = c.seq_len[b];
@@ -1860,64 +1912,93 @@ __global__ void __maxnreg__(200)
         const float sl = a.scale * kLog2e;
         const int key_base = warp * 16;
         const __half2 sixteenth = __float2half2_rn(0.0625f);
-        for (int t = 0; t < n_tiles; ++t) {
-            const int st = t % STAGES, round = t / STAGES;
-            if (!mbar_wait(&full_bar[st], round & 1, c.status)) break;
-            const int n = s_tile_n[st];
-            const uint8_t* tK = sK4 + (size_t)st * kQ4TileBytes;
-            const uint8_t* tV = sV4 + (size_t)st * kQ4TileBytes;
-            const float* ksc = sSc + st * 2 * kTile;
-            const float* vsc = ksc + kTile;
-            // S' = q . (biased codes) for keys key_base + 8 nb + (lane >> 2),
-            // even and odd k-steps in separate accumulators
-            float s[2][2][2] = {{{0.f, 0.f}, {0.f, 0.f}}, {{0.f, 0.f}, {0.f, 0.f}}};
+        // One pass over NT (1 or 2) consecutive tiles: both full-barrier waits
+        // first, then one straight-line block -- the tiles' q . K, one joint
+        // row maximum (two shuffles and one rescale vote for both), their
+        // exponentials and P V -- so that the two tiles' independent chains
+        // interleave (a warp has little else to hide latency with: two CTAs
+        // of four consumer warps per SM).  Returns false when a wait ran out.
+        auto pass = [&](int t, auto nt_c) -> bool {
+            constexpr int NT = decltype(nt_c)::value;
+            int st[NT];
+            bool ok = true;
 #pragma unroll
-            for (int nb = 0; nb < 2; ++nb) {
-                const int key = key_base + 8 * nb + row;
-                const uint4 kw = *reinterpret_cast<const uint4*>(tK + key * kQ4RowBytes + 16 * quad);
-                const uint32_t w[4] = {kw.x, kw.y, kw.z, kw.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t w8 = w[j] >> 8;
-                    mma_f16_rows8(s[nb][0][0], s[nb][0][1], qa[2 * j][0], qa[2 * j][1], u4_lo_f16x2(w[j]),
-                                  u4_hi_f16x2(w[j]));
-                    mma_f16_rows8(s[nb][1][0], s[nb][1][1], qa[2 * j + 1][0], qa[2 * j + 1][1], u4_lo_f16x2(w8),
-                                  u4_hi_f16x2(w8));
-                }
+            for (int i = 0; i < NT; ++i) {
+                st[i] = (t + i) % STAGES;
+                ok = ok && mbar_wait(&full_bar[st[i]], ((t + i) / STAGES) & 1, c.status);
             }
+            if (!ok) return false;
             // this lane's keys: key_base + 2 quad + {0, 1} and + 8
             const int k0 = key_base + 2 * quad;
-            float sv[4], vs[4];
-            quant_scores(s[0][0][0] + s[0][1][0] - q_corr, s[0][0][1] + s[0][1][1] - q_corr,
-                         s[1][0][0] + s[1][1][0] - q_corr, s[1][0][1] + s[1][1][1] - q_corr, ksc, vsc, k0, n, sl, sv,
-                         vs);
-            float pr[4];
-            online_softmax_step(sv, m_run, l_run, pr, o, wsum);
-            // p times the key's V scale, the fp16 A operand of O += P V, and
-            // the same divided by 16 for the high-nibble feature rows
-            const uint32_t pa0 = f16x2_pack(pr[0] * vs[0], pr[1] * vs[1]);
-            const uint32_t pa1 = f16x2_pack(pr[2] * vs[2], pr[3] * vs[3]);
-            const __half2 ph0 = __hmul2(*reinterpret_cast<const __half2*>(&pa0), sixteenth);
-            const __half2 ph1 = __hmul2(*reinterpret_cast<const __half2*>(&pa1), sixteenth);
-            const uint32_t pb0 = *reinterpret_cast<const uint32_t*>(&ph0);
-            const uint32_t pb1 = *reinterpret_cast<const uint32_t*>(&ph1);
-            // O' += P U: the word of feature pair (16 m + r, 16 m + 8 + r) and
-            // this lane's key quad in the warp's 16-token group, its nibbles
-            // taken as exact fp16 subnormals n 2^-24 (low) and 16 n 2^-24
-            // (high, against p / 16); the bias sums W += P 1 ride on the same
-            // MMA, and O = 2^24 O' - 8 W (low) or - 128 W (high) at the end
-            mma_f16_rows8(wsum[0][0], wsum[0][1], pa0, pa1, kF16x2One, kF16x2One);
-            mma_f16_rows8(wsum[1][0], wsum[1][1], pb0, pb1, kF16x2One, kF16x2One);
+            float sv[NT][4], vs[NT][4];
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const uint32_t w = *reinterpret_cast<const uint32_t*>(tV + 1024 * warp + 128 * m + 16 * row + 4 * quad);
-                const uint32_t w8 = w >> 8;
-                mma_f16_rows8(o[2 * m][0], o[2 * m][1], pa0, pa1, u4_lo_sub(w), u4_lo_sub(w8));
-                mma_f16_rows8(o[2 * m + 1][0], o[2 * m + 1][1], pb0, pb1, u4_hi_sub(w), u4_hi_sub(w8));
+            for (int i = 0; i < NT; ++i) {
+                // S' = q . (biased codes) for keys key_base + 8 nb + (lane >> 2),
+                // even and odd k-steps in separate accumulators
+                const uint8_t* tK = sK4 + (size_t)st[i] * kQ4TileBytes;
+                float s[2][2][2] = {{{0.f, 0.f}, {0.f, 0.f}}, {{0.f, 0.f}, {0.f, 0.f}}};
+#pragma unroll
+                for (int nb = 0; nb < 2; ++nb) {
+                    const int key = key_base + 8 * nb + row;
+                    const uint4 kw = *reinterpret_cast<const uint4*>(tK + key * kQ4RowBytes + 16 * quad);
+                    const uint32_t w[4] = {kw.x, kw.y, kw.z, kw.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t w8 = w[j] >> 8;
+                        mma_f16_rows8(s[nb][0][0], s[nb][0][1], qa[2 * j][0], qa[2 * j][1], u4_lo_f16x2(w[j]),
+                                      u4_hi_f16x2(w[j]));
+                        mma_f16_rows8(s[nb][1][0], s[nb][1][1], qa[2 * j + 1][0], qa[2 * j + 1][1], u4_lo_f16x2(w8),
+                                      u4_hi_f16x2(w8));
+                    }
+                }
+                const float* ksc = sSc + st[i] * 2 * kTile;
+                quant_scores(s[0][0][0] + s[0][1][0] - q_corr, s[0][0][1] + s[0][1][1] - q_corr,
+                             s[1][0][0] + s[1][1][0] - q_corr, s[1][0][1] + s[1][1][1] - q_corr, ksc, ksc + kTile,
+                             k0, s_tile_n[st[i]], sl, sv[i], vs[i]);
+            }
+            float mx = kNegBig;
+#pragma unroll
+            for (int i = 0; i < NT; ++i) mx = fmaxf(mx, fmaxf(fmaxf(sv[i][0], sv[i][1]), fmaxf(sv[i][2], sv[i][3])));
+            rescale_to_max(mx, m_run, l_run, o, wsum);
+#pragma unroll
+            for (int i = 0; i < NT; ++i) {
+                float pr[4];
+                softmax_exp(sv[i], m_run, l_run, pr);
+                // p times the key's V scale, the fp16 A operand of O += P V, and
+                // the same divided by 16 for the high-nibble feature rows
+                const uint32_t pa0 = f16x2_pack(pr[0] * vs[i][0], pr[1] * vs[i][1]);
+                const uint32_t pa1 = f16x2_pack(pr[2] * vs[i][2], pr[3] * vs[i][3]);
+                const __half2 ph0 = __hmul2(*reinterpret_cast<const __half2*>(&pa0), sixteenth);
+                const __half2 ph1 = __hmul2(*reinterpret_cast<const __half2*>(&pa1), sixteenth);
+                const uint32_t pb0 = *reinterpret_cast<const uint32_t*>(&ph0);
+                const uint32_t pb1 = *reinterpret_cast<const uint32_t*>(&ph1);
+                // O' += P U: the word of feature pair (16 m + r, 16 m + 8 + r) and
+                // this lane's key quad in the warp's 16-token group, its nibbles
+                // taken as exact fp16 subnormals n 2^-24 (low) and 16 n 2^-24
+                // (high, against p / 16); the bias sums W += P 1 ride on the same
+                // MMA, and O = 2^24 O' - 8 W (low) or - 128 W (high) at the end
+                mma_f16_rows8(wsum[0][0], wsum[0][1], pa0, pa1, kF16x2One, kF16x2One);
+                mma_f16_rows8(wsum[1][0], wsum[1][1], pb0, pb1, kF16x2One, kF16x2One);
+                const uint8_t* tV = sV4 + (size_t)st[i] * kQ4TileBytes;
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(tV + 1024 * warp + 128 * m + 16 * row + 4 * quad);
+                    const uint32_t w8 = w >> 8;
+                    mma_f16_rows8(o[2 * m][0], o[2 * m][1], pa0, pa1, u4_lo_sub(w), u4_lo_sub(w8));
+                    mma_f16_rows8(o[2 * m + 1][0], o[2 * m + 1][1], pb0, pb1, u4_hi_sub(w), u4_hi_sub(w8));
+                }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty_bar[st]);
-        }
+            if (lane == 0) {
+#pragma unroll
+                for (int i = 0; i < NT; ++i) mbar_arrive(&empty_bar[st[i]]);
+            }
+            return true;
+        };
+        int t = 0;
+        bool ok = true;
+        for (; ok && t + 1 < n_tiles; t += 2) ok = pass(t, std::integral_constant<int, 2>{});
+        if (ok && t < n_tiles) pass(t, std::integral_constant<int, 1>{});
         l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
         l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
     }
