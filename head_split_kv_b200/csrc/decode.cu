@@ -1594,10 +1594,9 @@ __global__ void __maxnreg__(200)
             float sv[NT][4], vs[NT][4];
 #pragma unroll
             for (int i = 0; i < NT; ++i) {
-                // S = q . codes for keys key_base + 8 nb + (lane >> 2), the k-steps
-                // in four accumulators (dependency chains of two MMAs)
+                // S = q . codes for keys key_base + 8 nb + (lane >> 2)
                 const uint8_t* tK = sK8 + (size_t)st[i] * kQ8Bytes;
-                float s[2][4][2] = {};
+                float s[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
                 for (int nb = 0; nb < 2; ++nb) {
                     const int key = key_base + 8 * nb + row;
@@ -1608,18 +1607,12 @@ __global__ void __maxnreg__(200)
                     for (int kb = 0; kb < 8; ++kb) {
                         uint32_t b0, b1;
                         i8x4_to_f16x2_biased(w[kb], b0, b1);
-                        mma_f16_rows8(s[nb][kb & 3][0], s[nb][kb & 3][1], qa[kb][0], qa[kb][1], b0, b1);
+                        mma_f16_rows8(s[nb][0], s[nb][1], qa[kb][0], qa[kb][1], b0, b1);
                     }
                 }
-                float sr[2][2];
-#pragma unroll
-                for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-                    for (int e = 0; e < 2; ++e)
-                        sr[nb][e] = ((s[nb][0][e] + s[nb][1][e]) + (s[nb][2][e] + s[nb][3][e])) - q_corr;
                 const float* ksc = sSc + st[i] * 2 * kTile;
-                quant_scores(sr[0][0], sr[0][1], sr[1][0], sr[1][1], ksc, ksc + kTile, k0, s_tile_n[st[i]], sl, sv[i],
-                             vs[i]);
+                quant_scores(s[0][0] - q_corr, s[0][1] - q_corr, s[1][0] - q_corr, s[1][1] - q_corr, ksc,
+                             ksc + kTile, k0, s_tile_n[st[i]], sl, sv[i], vs[i]);
             }
             float mx = kNegBig;
 #pragma unroll
@@ -1940,9 +1933,10 @@ __global__ void __maxnreg__(200)
             float sv[NT][4], vs[NT][4];
 #pragma unroll
             for (int i = 0; i < NT; ++i) {
-                // S' = q . (biased codes) for keys key_base + 8 nb + (lane >> 2)
+                // S' = q . (biased codes) for keys key_base + 8 nb + (lane >> 2),
+                // even and odd k-steps in separate accumulators
                 const uint8_t* tK = sK4 + (size_t)st[i] * kQ4TileBytes;
-                float s[2][4][2] = {};   // [nb][k-step mod 4][2]: dependency chains of two MMAs
+                float s[2][2][2] = {{{0.f, 0.f}, {0.f, 0.f}}, {{0.f, 0.f}, {0.f, 0.f}}};
 #pragma unroll
                 for (int nb = 0; nb < 2; ++nb) {
                     const int key = key_base + 8 * nb + row;
@@ -1951,22 +1945,16 @@ __global__ void __maxnreg__(200)
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const uint32_t w8 = w[j] >> 8;
-                        const int c0 = (2 * j) & 3, c1 = (2 * j + 1) & 3;
-                        mma_f16_rows8(s[nb][c0][0], s[nb][c0][1], qa[2 * j][0], qa[2 * j][1], u4_lo_f16x2(w[j]),
+                        mma_f16_rows8(s[nb][0][0], s[nb][0][1], qa[2 * j][0], qa[2 * j][1], u4_lo_f16x2(w[j]),
                                       u4_hi_f16x2(w[j]));
-                        mma_f16_rows8(s[nb][c1][0], s[nb][c1][1], qa[2 * j + 1][0], qa[2 * j + 1][1], u4_lo_f16x2(w8),
+                        mma_f16_rows8(s[nb][1][0], s[nb][1][1], qa[2 * j + 1][0], qa[2 * j + 1][1], u4_lo_f16x2(w8),
                                       u4_hi_f16x2(w8));
                     }
                 }
-                float sr[2][2];
-#pragma unroll
-                for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-                    for (int e = 0; e < 2; ++e)
-                        sr[nb][e] = ((s[nb][0][e] + s[nb][1][e]) + (s[nb][2][e] + s[nb][3][e])) - q_corr;
                 const float* ksc = sSc + st[i] * 2 * kTile;
-                quant_scores(sr[0][0], sr[0][1], sr[1][0], sr[1][1], ksc, ksc + kTile, k0, s_tile_n[st[i]], sl, sv[i],
-                             vs[i]);
+                quant_scores(s[0][0][0] + s[0][1][0] - q_corr, s[0][0][1] + s[0][1][1] - q_corr,
+                             s[1][0][0] + s[1][1][0] - q_corr, s[1][0][1] + s[1][1][1] - q_corr, ksc, ksc + kTile,
+                             k0, s_tile_n[st[i]], sl, sv[i], vs[i]);
             }
             float mx = kNegBig;
 #pragma unroll
