@@ -89,3 +89,24 @@ def test_decode_bytes_count_the_cached_rows(kv_bits):
         want += sh.n_kv_heads * row * 2 * 2
         want += sh.n_q_heads * sh.head_dim * 2 * 2
     assert bench._decode_bytes(sh, R, [L + 1 for L in lengths], kv_bits) == want
+
+
+def test_traffic_record_is_used_only_while_its_sources_are_unchanged(tmp_path, monkeypatch):
+    """roofline.traffic comes from profiles/traffic.json ({kernel: {workload:
+    record}}) only while every source file the record lists still has the
+    recorded SHA-256; a changed kernel reports null until it is captured
+    again."""
+    import hashlib
+    import json
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1\n")
+    (tmp_path / "profiles").mkdir()
+    rec = {"dram_bytes_read": 1000, "dram_bytes_write": 24,
+           "source_sha256": {"k.cu": hashlib.sha256(src.read_bytes()).hexdigest()}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps({"kern": {"wl": rec}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench._traffic("kern", "wl") == 1024
+    assert bench._traffic("kern", "other workload") is None
+    assert bench._traffic("other kernel", "wl") is None
+    src.write_text("kernel v2\n")
+    assert bench._traffic("kern", "wl") is None
