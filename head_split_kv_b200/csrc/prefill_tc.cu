@@ -399,7 +399,7 @@ __device__ __noinline__ void write_split_record(float* rec, int row, bool have, 
 // that ten warps leave (an SM sub-partition holds three of them in its 16K
 // registers).
 __device__ __noinline__ void merge_split_records(const float* base, int ns_use, int row, bool store,
-                                                 __nv_bfloat16* op) {
+                                                 __nv_bfloat16* op, int bar_id) {
     constexpr size_t kSplitStride = 2 * (size_t)kPartFloats;
     float w[kMaxSplit];
     float M = -INFINITY, L = 0.f;
@@ -435,6 +435,17 @@ __device__ __noinline__ void merge_split_records(const float* base, int ns_use, 
             store_row<__nv_bfloat16, 8>(op + 8 * g8, v8);
         }
     }
+    // The records are dead once the warpgroup has read them (only this, the
+    // last split of the unit, reads them; every writer took its ticket after
+    // a fence): drop their lines from L2 without writing them back, so the
+    // splits cost L2 traffic, not DRAM writes.  A record is 520 whole
+    // 128-byte lines at a 128-byte-aligned offset of the workspace.
+    static_assert(kPartFloats * sizeof(float) % 128 == 0, "records are whole L2 lines");
+    constexpr int kLines = (int)(kPartFloats * sizeof(float) / 128);
+    asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
+    for (int sp = 0; sp < ns_use; ++sp)
+        for (int ln = row; ln < kLines; ln += BM)
+            asm volatile("discard.global.L2 [%0], 128;" ::"l"(base + sp * kSplitStride + (size_t)ln * 32) : "memory");
 }
 
 // ------------------------------------------------------------------ kernel
@@ -769,7 +780,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (holder[1]) {
                 __threadfence();
                 merge_split_records(p.part + (size_t)unit_ * p.ns * 2 * kPartFloats + (size_t)qi * kPartFloats,
-                                    ns_use_, row, crow < p.C, op);
+                                    ns_use_, row, crow < p.C, op, 2 + qi);
             }
         }
     }
