@@ -400,7 +400,7 @@ duo_status duo_prefill_chunk(const duo_layer_desc* desc, const duo_kv_state* st,
     cudaError_t e;
     if (a.kv_bits && a.R > 0) {
         // an 8- or 4-bit full cache: its rows below seq_len are staged in
-        // the workspace -- the codes as bf16 values and each row's scales --
+        // the workspace -- K codes as bf16, V codes x16 as fp16, each row's scales --
         // and the tensor-core pre-fill reads the codes as its cache and
         // applies the scales to the scores and to p; the rest of the
         // workspace serves the key-range splits

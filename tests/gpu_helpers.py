@@ -100,6 +100,7 @@ class Layer:
         og, op, oi, on = O.partition_heads(alpha.astype(np.float64), 0.5)
         assert self.gate == list(og) and self.perm == list(op) and self.R == on
         self.io_order = duo.ORDER_MODEL if io_order is None else io_order
+        self.stream_prefill = stream_prefill
         self.desc = duo.desc_init(batch, shape.n_q_heads, hkv, shape.head_dim,
                                   duo.BF16 if shape.dtype == "bf16" else duo.FP32, self.perm, self.R,
                                   sink=shape.sink, recent=shape.recent, page_size=page_size,
@@ -270,8 +271,9 @@ def prefill_run(lay, chunks, seed, sigma=None, rows_per_chunk=None):
     direct definition over the history its caches hold before the chunk
     (for an 8- or 4-bit layer the retrieval rows as code * scale; a
     streaming head's evicted positions as zeros, which no query of the chunk
-    sees) followed by the chunk's rows as given; the oracle's caches then
-    take the chunk."""
+    sees) followed by the chunk's rows as given, through the layer's
+    streaming pre-fill mode; tensors go to the device in the layer's head
+    order.  The oracle's caches then take the chunk."""
     t = torch()
     duo, sh, B = lay.duo, lay.shape, lay.B
     n = sum(chunks)
@@ -279,15 +281,18 @@ def prefill_run(lay, chunks, seed, sigma=None, rows_per_chunk=None):
     ws = duo.Workspace(lay.desc, duo.OP_PREFILL, max(chunks), state=lay.caches.state)
     rng = S.rng_for(seed, 79)
     c0 = 0
+    g = sh.group
+    mode = "chunk" if lay.stream_prefill == duo.STREAM_CHUNK else "lambda"
     for ci, C in enumerate(chunks):
         sl = slice(c0, c0 + C)
-        qd, kd, vd = (to_dev(np.ascontiguousarray(x[:, sl])) for x in (q, k, v))
+        qd = to_dev(np.ascontiguousarray(lay.to_io(q[:, sl], 2, g)))
+        kd, vd = (to_dev(np.ascontiguousarray(lay.to_io(x[:, sl], 2, 1))) for x in (k, v))
         out = t.empty_like(qd)
         duo.prefill_chunk(lay.desc, lay.caches.state, qd, kd, vd, C, out, ws.ptr, ws.nbytes)
         duo.append_kv(lay.desc, lay.caches.state, kd, vd, C)
         rows = np.arange(C) if rows_per_chunk is None or C <= rows_per_chunk else \
             np.unique(rng.choice(C, rows_per_chunk, replace=False))
-        got = f64(out)
+        got = lay.from_io(f64(out), 2, g)
         for b in range(B):
             k_all = np.zeros((c0 + C, sh.n_kv_heads, sh.head_dim))
             v_all = np.zeros_like(k_all)
@@ -296,7 +301,8 @@ def prefill_run(lay, chunks, seed, sigma=None, rows_per_chunk=None):
                 if len(pos):
                     k_all[pos, h], v_all[pos, h] = O.as_f64(kh), O.as_f64(vh)
             k_all[c0:], v_all[c0:] = O.as_f64(k[b, sl]), O.as_f64(v[b, sl])
-            want = O.prefill_direct(q[b, sl], k_all, v_all, c0, np.array(lay.gate), sh.sink, sh.recent, rows=rows)
+            want = O.prefill_direct(q[b, sl], k_all, v_all, c0, np.array(lay.gate), sh.sink, sh.recent, rows=rows,
+                                    stream_mode=mode)
             assert_close(got[b, rows], want, sh.dtype, f"chunk {ci} (c0={c0}) b={b}")
         lay.oracle.append(k[:, sl], v[:, sl])
         c0 += C
