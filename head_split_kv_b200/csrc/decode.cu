@@ -1199,13 +1199,15 @@ constexpr size_t decode_q8_smem_bytes() {
 constexpr uint32_t kF16x2One = 0x3C003C00u;   // (1.0, 1.0) in fp16
 constexpr float kTwo24 = 16777216.f;          // 2^24: undoes the subnormal codes' 2^-24
 
-__device__ __forceinline__ void mma_f16_rows8(float& c0, float& c1, uint32_t a0, uint32_t a2, uint32_t b0,
-                                              uint32_t b1) {
-    float d2, d3;
+// O (16 x 8, fp32) += A (16 x 16, fp16) B (16 x 8, fp16) with the group's
+// query heads in rows 0-7 of A and rows 8-15 zero, accumulating in place into
+// all four accumulator registers: rows 8-15 of C stay zero (their rows of A
+// are zero), so the pair c[2], c[3] is carried, never re-materialised.
+__device__ __forceinline__ void mma_f16_rows8_acc(float (&c)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
     asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-        "{%10, %11, %12, %13};"
-        : "=f"(c0), "=f"(c1), "=f"(d2), "=f"(d3)
-        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(0.f), "f"(0.f));
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
 }
 
 // An 8-bit layer's streaming head in the same launch: the ring's min(len, W)
@@ -1381,9 +1383,9 @@ __device__ __forceinline__ void warm_l2_quant_split(const LayerArgs& a, const Ca
 // takes the row maximum of this lane's scores (mx) over the quad and
 // rescales O, l and the PV bias sums only when some row's maximum grew (a
 // warp vote); softmax_exp forms p = 2^(s - m) and adds it to the row sum.
-template <int NWS>
-__device__ __forceinline__ void rescale_to_max(float mx, float& m_run, float& l_run, float (&o)[16][2],
-                                               float (&wsum)[NWS][2]) {
+template <int NWS, int OW>
+__device__ __forceinline__ void rescale_to_max(float mx, float& m_run, float& l_run, float (&o)[16][OW],
+                                               float (&wsum)[NWS][OW]) {
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
     const float m_new = fmaxf(m_run, mx);
@@ -1541,9 +1543,9 @@ __global__ void __maxnreg__(200)
     // ------------------------------------------------------ consumers
     const int row = lane >> 2;   // query head of the group (rows >= G are padding) / key of an 8-key block
     const int quad = lane & 3;
-    float o[16][2];
+    float o[16][4];   // rows 8-15 of each accumulator stay zero
     float m_run = kNegBig, l_run = 0.f;
-    float wsum[1][2] = {{0.f, 0.f}};   // sum of the PV A operand per row (the code bias)
+    float wsum[1][4] = {};   // sum of the PV A operand per row (the code bias)
     if (warp < NW) {
         // q in fp16, features 32 quad + 4 kb + {0, 1} and {2, 3} for step kb.
         // The K operands keep the bias of the byte-to-fp16 step (1152 +
@@ -1575,7 +1577,7 @@ __global__ void __maxnreg__(200)
             q_corr *= 1152.f;
         }
 #pragma unroll
-        for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = 0.f;
+        for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
         const float sl = a.scale * kLog2e;
         const int key_base = warp * 16;
         // one pass over NT (1 or 2) consecutive tiles, as in the 4-bit kernel
@@ -1596,7 +1598,7 @@ __global__ void __maxnreg__(200)
             for (int i = 0; i < NT; ++i) {
                 // S = q . codes for keys key_base + 8 nb + (lane >> 2)
                 const uint8_t* tK = sK8 + (size_t)st[i] * kQ8Bytes;
-                float s[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+                float s[2][4] = {};
 #pragma unroll
                 for (int nb = 0; nb < 2; ++nb) {
                     const int key = key_base + 8 * nb + row;
@@ -1607,7 +1609,7 @@ __global__ void __maxnreg__(200)
                     for (int kb = 0; kb < 8; ++kb) {
                         uint32_t b0, b1;
                         i8x4_to_f16x2_biased(w[kb], b0, b1);
-                        mma_f16_rows8(s[nb][0], s[nb][1], qa[kb][0], qa[kb][1], b0, b1);
+                        mma_f16_rows8_acc(s[nb], qa[kb][0], qa[kb][1], b0, b1);
                     }
                 }
                 const float* ksc = sSc + st[i] * 2 * kTile;
@@ -1629,7 +1631,7 @@ __global__ void __maxnreg__(200)
                 // and the bias sum W += P 1 through the same MMA: O = 2^24 O' -
                 // 128 W at the end.  Feature row 8 nd + (lane >> 2), this warp's
                 // 16-key group (64-byte swizzle), the lane's four keys in one word
-                mma_f16_rows8(wsum[0][0], wsum[0][1], pa0, pa1, kF16x2One, kF16x2One);
+                mma_f16_rows8_acc(wsum[0], pa0, pa1, kF16x2One, kF16x2One);
                 const uint8_t* tV = sV8 + (size_t)st[i] * kQ8Bytes;
 #pragma unroll
                 for (int nd = 0; nd < 16; ++nd) {
@@ -1638,7 +1640,7 @@ __global__ void __maxnreg__(200)
                                                                           4 * quad);
                     uint32_t b0, b1;
                     i8x4_to_f16x2_sub(w, b0, b1);
-                    mma_f16_rows8(o[nd][0], o[nd][1], pa0, pa1, b0, b1);
+                    mma_f16_rows8_acc(o[nd], pa0, pa1, b0, b1);
                 }
             }
             __syncwarp();
@@ -1872,9 +1874,9 @@ __global__ void __maxnreg__(200)
     // exactly instead: 1024 + n - 1032 = code, 1024 + 16 n - 1152 = 16 code.
     const int row = lane >> 2;   // query head of the group (rows >= G are padding) / key of an 8-key block
     const int quad = lane & 3;
-    float o[16][2];
+    float o[16][4];   // rows 8-15 of each accumulator stay zero
     float m_run = kNegBig, l_run = 0.f;
-    float wsum[2][2] = {{0.f, 0.f}, {0.f, 0.f}};   // PV A operand sums per row: p vs, p vs / 16
+    float wsum[2][4] = {};   // PV A operand sums per row: p vs, p vs / 16
     if (warp < NW) {
         // q in fp16, features 32 quad + 4 kb + {0, 1} (partners of the low
         // nibbles) and {2, 3} (partners of the high nibbles, divided by 16)
@@ -1908,7 +1910,7 @@ __global__ void __maxnreg__(200)
             q_corr += __shfl_xor_sync(0xffffffffu, q_corr, 2);
         }
 #pragma unroll
-        for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = 0.f;
+        for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
         const float sl = a.scale * kLog2e;
         const int key_base = warp * 16;
         const __half2 sixteenth = __float2half2_rn(0.0625f);
@@ -1936,7 +1938,7 @@ __global__ void __maxnreg__(200)
                 // S' = q . (biased codes) for keys key_base + 8 nb + (lane >> 2),
                 // even and odd k-steps in separate accumulators
                 const uint8_t* tK = sK4 + (size_t)st[i] * kQ4TileBytes;
-                float s[2][2][2] = {{{0.f, 0.f}, {0.f, 0.f}}, {{0.f, 0.f}, {0.f, 0.f}}};
+                float s[2][2][4] = {};
 #pragma unroll
                 for (int nb = 0; nb < 2; ++nb) {
                     const int key = key_base + 8 * nb + row;
@@ -1945,10 +1947,8 @@ __global__ void __maxnreg__(200)
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const uint32_t w8 = w[j] >> 8;
-                        mma_f16_rows8(s[nb][0][0], s[nb][0][1], qa[2 * j][0], qa[2 * j][1], u4_lo_f16x2(w[j]),
-                                      u4_hi_f16x2(w[j]));
-                        mma_f16_rows8(s[nb][1][0], s[nb][1][1], qa[2 * j + 1][0], qa[2 * j + 1][1], u4_lo_f16x2(w8),
-                                      u4_hi_f16x2(w8));
+                        mma_f16_rows8_acc(s[nb][0], qa[2 * j][0], qa[2 * j][1], u4_lo_f16x2(w[j]), u4_hi_f16x2(w[j]));
+                        mma_f16_rows8_acc(s[nb][1], qa[2 * j + 1][0], qa[2 * j + 1][1], u4_lo_f16x2(w8), u4_hi_f16x2(w8));
                     }
                 }
                 const float* ksc = sSc + st[i] * 2 * kTile;
@@ -1977,15 +1977,15 @@ __global__ void __maxnreg__(200)
                 // taken as exact fp16 subnormals n 2^-24 (low) and 16 n 2^-24
                 // (high, against p / 16); the bias sums W += P 1 ride on the same
                 // MMA, and O = 2^24 O' - 8 W (low) or - 128 W (high) at the end
-                mma_f16_rows8(wsum[0][0], wsum[0][1], pa0, pa1, kF16x2One, kF16x2One);
-                mma_f16_rows8(wsum[1][0], wsum[1][1], pb0, pb1, kF16x2One, kF16x2One);
+                mma_f16_rows8_acc(wsum[0], pa0, pa1, kF16x2One, kF16x2One);
+                mma_f16_rows8_acc(wsum[1], pb0, pb1, kF16x2One, kF16x2One);
                 const uint8_t* tV = sV4 + (size_t)st[i] * kQ4TileBytes;
 #pragma unroll
                 for (int m = 0; m < 8; ++m) {
                     const uint32_t w = *reinterpret_cast<const uint32_t*>(tV + 1024 * warp + 128 * m + 16 * row + 4 * quad);
                     const uint32_t w8 = w >> 8;
-                    mma_f16_rows8(o[2 * m][0], o[2 * m][1], pa0, pa1, u4_lo_sub(w), u4_lo_sub(w8));
-                    mma_f16_rows8(o[2 * m + 1][0], o[2 * m + 1][1], pb0, pb1, u4_hi_sub(w), u4_hi_sub(w8));
+                    mma_f16_rows8_acc(o[2 * m], pa0, pa1, u4_lo_sub(w), u4_lo_sub(w8));
+                    mma_f16_rows8_acc(o[2 * m + 1], pb0, pb1, u4_hi_sub(w), u4_hi_sub(w8));
                 }
             }
             __syncwarp();
