@@ -680,14 +680,14 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                  : "memory");
 }
 
-// D = A (16 x 16, rows 8..15 zero) * B (16 x 8) + C with C rows 8..15 zero;
-// returns the two accumulators of rows 0..7 this lane holds.
-__device__ __forceinline__ void mma_rows8(float& c0, float& c1, uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
-    float d2, d3;
+// D = A (16 x 16, rows 8..15 zero) * B (16 x 8) + C, in place in all four
+// accumulator registers: rows 8..15 of C stay zero (their rows of A are
+// zero), so c[2], c[3] are carried, never re-materialised before an MMA.
+__device__ __forceinline__ void mma_rows8(float (&c)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
     asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-        "{%10, %11, %12, %13};"
-        : "=f"(c0), "=f"(c1), "=f"(d2), "=f"(d3)
-        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(0.f), "f"(0.f));
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
 }
 
 // byte offset of (row, 16-byte chunk c16 of the 256-byte row) in a tile made
@@ -964,7 +964,7 @@ __global__ void __maxnreg__(200)
     // ------------------------------------------------------ consumers
     const int row = lane >> 2;   // query head of the group for this lane (rows >= G are padding)
     const int quad = lane & 3;
-    float o[16][2];
+    float o[16][4];   // rows 8-15 of each accumulator stay zero
     float m_run = kNegBig, l_run = 0.f;
     if (warp < NW) {
         uint32_t qa[8][2];
@@ -979,7 +979,7 @@ __global__ void __maxnreg__(200)
             }
         }
 #pragma unroll
-        for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = 0.f;
+        for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
         const float sl = a.scale * kLog2e;
         const int key_base = warp * 16;
         for (int t = 0;; ++t) {
@@ -1003,15 +1003,15 @@ __global__ void __maxnreg__(200)
                 __syncwarp();
             }
             // S = Q K^T for keys key_base .. key_base + 15
-            float s0[2] = {0.f, 0.f}, s1[2] = {0.f, 0.f};
+            float s0[4] = {}, s1[4] = {};
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const int key = key_base + (lane & 7) + ((lane >> 4) & 1) * 8;
                 const int c16 = 2 * ks + ((lane >> 3) & 1);
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4(tK + sw_off(key, c16), b0, b1, b2, b3);
-                mma_rows8(s0[0], s0[1], qa[ks][0], qa[ks][1], b0, b1);
-                mma_rows8(s1[0], s1[1], qa[ks][0], qa[ks][1], b2, b3);
+                mma_rows8(s0, qa[ks][0], qa[ks][1], b0, b1);
+                mma_rows8(s1, qa[ks][0], qa[ks][1], b2, b3);
             }
             // this lane's keys: key_base + 2 quad + {0, 1} and + 8
             const int k0 = key_base + 2 * quad;
@@ -1023,21 +1023,26 @@ __global__ void __maxnreg__(200)
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
             const float m_new = fmaxf(m_run, mx);
-            const float corr = exp2f(m_run - m_new);
+            // O and l are rescaled only when some row's maximum grew (a warp
+            // vote), which over a long cache is rare
+            if (__any_sync(0xffffffffu, m_new > m_run)) {
+                const float corr = exp2f(m_run - m_new);
+                l_run *= corr;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    o[j][0] *= corr;
+                    o[j][1] *= corr;
+                }
+                m_run = m_new;
+            }
             // P rounded to bf16 for the PV MMA; the row sum uses the rounded values
-            __nv_bfloat162 p01 = __floats2bfloat162_rn(vk[0] ? exp2f(sv[0] - m_new) : 0.f,
-                                                       vk[1] ? exp2f(sv[1] - m_new) : 0.f);
-            __nv_bfloat162 p23 = __floats2bfloat162_rn(vk[2] ? exp2f(sv[2] - m_new) : 0.f,
-                                                       vk[3] ? exp2f(sv[3] - m_new) : 0.f);
+            __nv_bfloat162 p01 = __floats2bfloat162_rn(vk[0] ? exp2f(sv[0] - m_run) : 0.f,
+                                                       vk[1] ? exp2f(sv[1] - m_run) : 0.f);
+            __nv_bfloat162 p23 = __floats2bfloat162_rn(vk[2] ? exp2f(sv[2] - m_run) : 0.f,
+                                                       vk[3] ? exp2f(sv[3] - m_run) : 0.f);
             const uint32_t pa0 = *reinterpret_cast<uint32_t*>(&p01);
             const uint32_t pa1 = *reinterpret_cast<uint32_t*>(&p23);
-            l_run = l_run * corr + (bf16_lo(pa0) + bf16_hi(pa0)) + (bf16_lo(pa1) + bf16_hi(pa1));
-            m_run = m_new;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                o[j][0] *= corr;
-                o[j][1] *= corr;
-            }
+            l_run += (bf16_lo(pa0) + bf16_hi(pa0)) + (bf16_lo(pa1) + bf16_hi(pa1));
             // O += P V over the 16 keys, 8 pairs of 8-column blocks of d
 #pragma unroll
             for (int jj = 0; jj < 8; ++jj) {
@@ -1045,8 +1050,8 @@ __global__ void __maxnreg__(200)
                 const int c16 = 2 * jj + (lane >> 4);
                 uint32_t r0, r1, r2, r3;
                 ldsm_x4_t(tV + sw_off(key, c16), r0, r1, r2, r3);
-                mma_rows8(o[2 * jj][0], o[2 * jj][1], pa0, pa1, r0, r1);
-                mma_rows8(o[2 * jj + 1][0], o[2 * jj + 1][1], pa0, pa1, r2, r3);
+                mma_rows8(o[2 * jj], pa0, pa1, r0, r1);
+                mma_rows8(o[2 * jj + 1], pa0, pa1, r2, r3);
             }
             __syncwarp();
             if (partial) fence_proxy_async_smem();  // the zero stores before the next TMA write
