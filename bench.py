@@ -21,7 +21,8 @@ pages, 8 layers), each with its own roofline, clocks, e2e and CPU baseline
 (--no-extra drops them).  Other workloads: the same decode shapes over 8- or
 4-bit retrieval caches (``*_int8``, ``*_int4``), gqa_prefill_128k (one
 131,072-token prompt in 32 chunks of 4,096; a step is one chunk's
-duo_prefill_chunk + duo_append_kv), gqa_prefill_32k, and the gated mix
+duo_prefill_chunk + duo_append_kv) and the same over 8- / 4-bit caches
+(``gqa_prefill_128k_int8``, ``_int4``), gqa_prefill_32k, and the gated mix
 (gated_mix_pr1, gated_mix_gqa_4k: forward and gate gradient).
 
 A decode run also measures the pre-fill workload (unless --no-prefill) and
@@ -81,6 +82,12 @@ WORKLOADS = {
     "gqa_decode_1m_int4": dict(kind="decode", hq=32, hkv=8, d=128, n_ret=4, lengths=[1048576], steps=64,
                                sigma=True, kv_int4=True, layers=16),
     "gqa_prefill_128k": dict(kind="prefill", hq=32, hkv=8, d=128, n_ret=4, n=131072, chunk=4096, sigma=False),
+    # ... over 8- and 4-bit retrieval caches (each chunk stages the prior codes
+    # and scales, then runs the tensor-core pre-fill over them)
+    "gqa_prefill_128k_int8": dict(kind="prefill", hq=32, hkv=8, d=128, n_ret=4, n=131072, chunk=4096, sigma=False,
+                                  kv_int8=True),
+    "gqa_prefill_128k_int4": dict(kind="prefill", hq=32, hkv=8, d=128, n_ret=4, n=131072, chunk=4096, sigma=False,
+                                  kv_int4=True),
     # the same pre-fill on a 32K prompt: a small case for profiler captures
     "gqa_prefill_32k": dict(kind="prefill", hq=32, hkv=8, d=128, n_ret=4, n=32768, chunk=4096, sigma=False),
     # the gated mix alpha * full + (1 - alpha) * streaming over whole sequences
@@ -691,8 +698,10 @@ def run_prefill(args, wl, world, rank, steps=None, warmup=None):
     retrieval = S.retrieval_heads_by_seed(wl["hkv"], wl["n_ret"], seed=1)
     gate, perm, inv, R = duo.partition_heads(S.binary_alpha(wl["hkv"], retrieval), 0.5)
     stream_chunk = wl.get("stream") == "chunk"
+    kv_bits = wl.get("kv_bits", 0)
     desc = duo.desc_init(1, sh.n_q_heads, sh.n_kv_heads, sh.head_dim, duo.BF16, perm, R,
-                         stream_prefill=duo.STREAM_CHUNK if stream_chunk else duo.STREAM_LAMBDA)
+                         stream_prefill=duo.STREAM_CHUNK if stream_chunk else duo.STREAM_LAMBDA,
+                         kv_quant={8: duo.KV_INT8, 4: duo.KV_INT4}.get(kv_bits, duo.KV_PLAIN))
     caches = duo.LayerCaches(desc, n)
     q, k, v = S.prompt(sh, n, seed=0)
     qd, kd, vd = _to_dev(q), _to_dev(k), _to_dev(v)
@@ -709,7 +718,9 @@ def run_prefill(args, wl, world, rank, steps=None, warmup=None):
         return qc, kc, vc
 
     chunks = [chunk(i) for i in range(n_chunks)]
-    ws = duo.Workspace(desc, duo.OP_PREFILL, C)   # lets long retrieval units split their key tiles
+    # lets long retrieval units split their key tiles; for an 8- or 4-bit
+    # layer it also holds the staged codes and scales
+    ws = duo.Workspace(desc, duo.OP_PREFILL, C, state=caches.state)
     for i in range(min(warmup, n_chunks)):
         qc, kc, vc = chunks[i]
         duo.prefill_chunk(desc, caches.state, qc, kc, vc, C, out, ws.ptr, ws.nbytes, sp)
@@ -751,14 +762,19 @@ def run_prefill(args, wl, world, rank, steps=None, warmup=None):
         "config": {"workload": wl["name"], "prompt": n, "chunk": C, "n_q_heads": sh.n_q_heads,
                    "n_kv_heads": sh.n_kv_heads, "head_dim": sh.head_dim, "n_retrieval": R, "sink": sh.sink,
                    "recent": sh.recent, "parallelism": f"replicas{world}", "workspace_bytes": ws.nbytes,
+                   "full_cache": {8: "int8 codes + fp32 scale per row", 4: "4-bit codes + fp32 scale per row"}.get(
+                       kv_bits, "bf16"),
                    "l2": "flushed (1 GiB write) before every timed chunk, outside the timed interval"},
-        "roofline": {"bound": "tensor", "kernel": "prefill_tc_kernel", "achieved": round(achieved, 1),
+        "roofline": {"bound": "tensor",
+                     "kernel": "prefill_tc_kernel" if not kv_bits else
+                               "dequant_kernel (staging) + prefill_tc_kernel (fp16 PV on the prior tiles)",
+                     "achieved": round(achieved, 1),
                      "peak": tf_peak, "peak_kind": peak_kind + " (burst; sustained 1381.5)", "unit": "TFLOP/s",
                      "frac": round(achieved / tf_peak, 4), "traffic": _traffic("prefill_tc_kernel", wl["name"]),
                      "algorithmic_tflop_total": round(sum(flops) / 1e12, 3),
                      "prefill_ms_total": round(sum(pre_ms), 3), "append_ms_total": round(sum(step_ms) - sum(pre_ms), 3),
                      "per_chunk_ms": [round(x, 3) for x in pre_ms]},
-        "gpu_launches": 2 * steps,
+        "gpu_launches": (3 if kv_bits else 2) * steps,
         "clocks": clk.summary(),
     }
 
