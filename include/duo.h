@@ -317,7 +317,9 @@ duo_status duo_append_kv(const duo_layer_desc* desc, const duo_kv_state* st, con
  * Launch overlap: the bf16 / d 128 decode is launched with programmatic
  * dependent launch, so it can start while the kernel before it on the stream
  * finishes, and with a contiguous full cache it loads its first cache tiles
- * that lie at least 128 rows below seq_len before waiting for that kernel.
+ * that lie at least 128 rows below seq_len before waiting for that kernel
+ * (the 8- and 4-bit decodes only ask L2 for their first tiles then: a hint,
+ * whatever the rows hold).
  * Every other kernel of the library lets dependents start only when it
  * completes, and the decode kernels write nothing there, so library calls
  * need no care; a caller kernel launched just before it on the same stream
