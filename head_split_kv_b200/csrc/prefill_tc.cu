@@ -84,10 +84,10 @@ constexpr uint32_t kOffK = kOffQ + 2 * kQBytes;
 constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;
 constexpr uint32_t kOffBar = kOffV + 2 * kTileBytes;
 constexpr uint32_t kOffHolder = kOffBar + 16 * 8;
-// quantized prior tiles: (k scale, v scale / 16, -, -) per key, four tiles
-// deep (a K stage is refilled after its QK MMAs, while the softmax may still
-// be on that tile; four slots outlast it -- see the producer)
-constexpr uint32_t kScaleTileBytes = BN * 16;
+// quantized prior tiles: the tile's 128 k scales, then its 128 v scales / 16,
+// four tiles deep (a K stage is refilled after its QK MMAs, while the softmax
+// may still be on that tile; four slots outlast it -- see the producer)
+constexpr uint32_t kScaleTileBytes = 2 * BN * 4;
 constexpr uint32_t kOffScale = kOffHolder + 128;  // a tensor copy's shared destination is 128-byte aligned
 constexpr uint32_t kSmemBytes = kOffScale + 4 * kScaleTileBytes;
 static_assert(kSmemBytes + 1024 <= 232448, "one CTA per SM");
@@ -298,7 +298,8 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
 // slower.
 //
 // qsc (a quantized layer's prior tile, else NULL): the tile's keys are
-// codes, and qsc holds (k scale, v scale / 16, -, -) per key: the scores are multiplied by
+// codes, and qsc holds the keys' k scales, then their v scales / 16 (read
+// four at a time): the scores are multiplied by
 // the k scales before anything else, and p by v scale / 16 on the way to the
 // PV operand, which is fp16 for these tiles (the V codes are staged times 16
 // in fp16, exactly): fp16's 11-bit significand keeps the rounding of p times
@@ -311,8 +312,17 @@ __device__ __forceinline__ float softmax_tile(uint32_t s_addr, float sl, bool ma
     float s[128];
     tmem_ld128(s_addr, s);
     if (qsc) {
+        const float4* k4 = reinterpret_cast<const float4*>(qsc);
 #pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] *= qsc[4 * c];
+        for (int i = 0; i < 32; ++i) {   // packed fp32 pairs: one instruction per two scores
+            const float4 ks = k4[i];
+            const float2 a = fmul2(make_float2(s[4 * i], s[4 * i + 1]), make_float2(ks.x, ks.y));
+            const float2 b = fmul2(make_float2(s[4 * i + 2], s[4 * i + 3]), make_float2(ks.z, ks.w));
+            s[4 * i] = a.x;
+            s[4 * i + 1] = a.y;
+            s[4 * i + 2] = b.x;
+            s[4 * i + 3] = b.y;
+        }
     }
     if (masked) {
 #pragma unroll
@@ -346,8 +356,9 @@ __device__ __forceinline__ float softmax_tile(uint32_t s_addr, float sl, bool ma
             const float2 e = (c2 % kFmaExpEvery == kFmaExpEvery - 1) ? exp2_fma2(x)
                                                                   : make_float2(exp2_approx(x.x), exp2_approx(x.y));
             if (qsc) {
-                const int c = 64 * h + 2 * c2;
-                __half2 hh = __floats2half2_rn(e.x * qsc[4 * c + 1], e.y * qsc[4 * c + 5]);
+                const float4 vq = reinterpret_cast<const float4*>(qsc + BN)[16 * h + (c2 >> 1)];
+                const float2 pv = fmul2(e, (c2 & 1) ? make_float2(vq.z, vq.w) : make_float2(vq.x, vq.y));
+                __half2 hh = __floats2half2_rn(pv.x, pv.y);
                 pk[c2] = *reinterpret_cast<uint32_t*>(&hh);
                 rs2[c2 & 3] = fadd2(rs2[c2 & 3], e);
             } else {
@@ -582,9 +593,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // is done, which comes after the softmax of tile j + 1
                     const bool scales = QS && kv == 0 && t.src == SRC_CACHE;
                     mbar_arrive_expect_tx(full, kTileBytes + (scales ? kScaleTileBytes : 0u));
-                    if (scales)
-                        tma_load_3d(smem_u32(smem + kOffScale) + (j & 3) * kScaleTileBytes, &tmS, 0, t.row, cache_z,
-                                    full);
+                    if (scales)   // x = t.row + the staging shift: a multiple of four floats
+                        tma_load_3d(smem_u32(smem + kOffScale) + (j & 3) * kScaleTileBytes, &tmS,
+                                    t.row + ((4 - (c0 & 3)) & 3), 0, cache_z, full);
                     const uint32_t dst = (kv ? sV : sK) + st * kTileBytes;
                     for (int half = 0; half < 2; ++half)
                         for (int rh = 0; rh < 2; ++rh) {
@@ -893,11 +904,13 @@ cudaError_t launch_prefill_tc(const LayerArgs& a, const CacheArgs& c, const void
     }
     CUtensorMap mS = mKx;   // never read unless the cache holds codes
     if (qscale != nullptr) {
-        // (k scale, v scale, -, -) per row: 16-byte rows, so the box's inner
-        // extent is one whole row and its first coordinate always 0
-        const uint64_t d[3] = {4, (uint64_t)a.capacity, (uint64_t)a.B * a.R};
-        const uint64_t st[2] = {16, 16ull * a.capacity};
-        const uint32_t bx[3] = {4, BN, 1};
+        // [B * R][2][capacity + 4] fp32: per head a row of k scales and a row
+        // of v scales / 16, shifted by the staging so that every prior tile
+        // starts on a multiple of four floats; a box is a tile's 128 scales of
+        // both rows
+        const uint64_t d[3] = {(uint64_t)a.capacity + 4, 2, (uint64_t)a.B * a.R};
+        const uint64_t st[2] = {4ull * (a.capacity + 4), 8ull * (a.capacity + 4)};
+        const uint32_t bx[3] = {BN, 2, 1};
         if (!encode_tmap(&mS, qscale, 3, d, st, bx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 0)) return cudaErrorInvalidValue;
     }
     TcArgs p;

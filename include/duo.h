@@ -385,7 +385,8 @@ duo_status duo_decode_step(const duo_layer_desc* desc, const duo_kv_state* st, c
  * product (rounded at 2^-11 of its value), which holds v scales up to 4095
  * (|V| up to 520,000 for 8-bit codes, 28,000 for 4-bit); the workspace is
  * then required: duo_prefill_workspace_bytes(desc, st, C) bytes (the staging
- * area, 528 bytes per token of the capacity and retrieval head, then the
+ * area -- 512 bytes of codes per token of the capacity and retrieval head
+ * and two rows of capacity + 4 fp32 scales per retrieval head -- then the
  * split records; DUO_ERR_CAPACITY when it is missing or smaller than the
  * staging area).
  * Errors: DUO_ERR_INVALID_ARG, DUO_ERR_SHAPE, DUO_ERR_CAPACITY,

@@ -338,18 +338,20 @@ def test_int8_cache_is_validated(duo):
 
 
 def test_quantized_prefill_needs_its_staging_workspace(duo):
-    """An 8- or 4-bit layer's pre-fill reads its prior rows from a bf16
-    staging area in the workspace: without one, or with one smaller than the
-    staging area, the call is refused before anything is queued; the size
-    query counts 528 bytes per token of the capacity and retrieval head on
-    top of the plain layer's workspace."""
+    """An 8- or 4-bit layer's pre-fill reads its prior rows from a staging
+    area in the workspace: without one, or with one smaller than the staging
+    area, the call is refused before anything is queued; the size query
+    counts, on top of the plain layer's workspace, 512 bytes of codes per
+    token of the capacity and retrieval head and two rows of capacity + 4
+    fp32 scales per retrieval head, rounded up to 256 bytes."""
     for quant in (duo.KV_INT8, duo.KV_INT4):
         d = duo.desc_init(1, 8, 4, 128, duo.BF16, [0, 1, 2, 3], 2, kv_quant=quant)
         st = _state(duo)
         st.k_scale, st.v_scale = 4096, 8192
         st.capacity = 1024
         plain = duo.workspace_bytes(d, duo.OP_PREFILL, 16)
-        assert duo.prefill_workspace_bytes(d, st, 16) == plain + 1 * 2 * 1024 * (2 * 128 * 2 + 16)
+        staging = 1 * 2 * 1024 * (2 * 128 * 2) + 1 * 2 * 2 * (1024 + 4) * 4
+        assert duo.prefill_workspace_bytes(d, st, 16) == plain + (staging + 255) // 256 * 256
         for ws, nbytes in ((None, 0), (1 << 20, 1 << 19)):
             with pytest.raises(duo.DuoError) as e:
                 duo.prefill_chunk(d, st, 256, 512, 768, 16, 1024, ws, nbytes, stream=0)

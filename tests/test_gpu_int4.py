@@ -100,7 +100,7 @@ def test_int4_decode_1m_full(duo):
     assert lay.status() == 0
 
 
-@pytest.mark.parametrize("chunks", [[300, 300, 100], [128] * 5 + [60], [4096, 4096]])
+@pytest.mark.parametrize("chunks", [[300, 300, 100], [128] * 5 + [60], [4096, 4096], [301, 250, 99, 130]])
 def test_int4_prefill_reads_the_quantized_cache(duo, chunks):
     """duo_prefill_chunk on a layer with a 4-bit full cache: the prior
     rows widened to bf16 code * scale in the workspace's staging area, the
