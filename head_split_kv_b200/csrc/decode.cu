@@ -123,14 +123,29 @@ __host__ __device__ constexpr int decode_max_regs(int G) {
 // broadcast through shared memory) and then takes a grid-wide ticket; the
 // CTA that takes the last ticket knows every CTA has read the old lengths and
 // advances them.  Taken at the start, this stays off the kernel's tail.
+// Atomic add at GPU scope with acquire-release semantics.  The release half
+// orders the calling thread's earlier memory accesses -- and, after a CTA
+// barrier, those of the whole CTA (release is cumulative) -- before the add;
+// the acquire half orders its later accesses after it.  A chain of such adds
+// on one counter therefore hands every earlier adder's writes to the last
+// one, with one round trip to L2 instead of a full fence plus the atomic.
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+// Called by the thread that read seq_len, after it read it: the CTA that
+// takes the last ticket of the grid advances every sequence's length.  The
+// release half of each add orders that CTA's read of seq_len before its
+// ticket; the acquire half of the last add orders the increments after every
+// CTA's read.  The counter is reset for the next launch, which waits for this
+// grid to complete before it reads the counter.
 __device__ __forceinline__ void length_ticket(const LayerArgs& a, const CacheArgs& c, const DecodeArgs& d) {
-    __threadfence();
-    const unsigned tk = atomicAdd(d.grid_ticket, 1u);
+    const unsigned tk = atom_add_acq_rel_gpu(d.grid_ticket, 1u);
     if (tk == gridDim.x - 1) {
-        __threadfence();
         for (int bb = 0; bb < a.B; ++bb) atomicAdd(&c.seq_len[bb], 1);
         *d.grid_ticket = 0u;
-        __threadfence();
     }
 }
 
@@ -187,17 +202,19 @@ __device__ __forceinline__ void decode_finish(float* sM, uint64_t* comb_bar, int
     if (!bounds_ok(pair < (size_t)a.B * a.R && split < d.nsplit && d.nsplit <= 128, c.status)) return;
     float* mine = d.partial + (pair * d.nsplit + split) * (size_t)G * STRIDE;
     for (int i = threadIdx.x; i < G * STRIDE; i += kThreads) mine[i] = cta[i];
-    __threadfence();
+    // The barrier orders every thread's record stores before thread 0's
+    // acquire-release ticket; the CTA that takes the last ticket thus sees
+    // every split's record, and its second barrier passes them on to its
+    // other threads.
     __syncthreads();
     if (threadIdx.x == 0) {
-        const unsigned tk = atomicAdd(&d.ticket[pair], 1u);
+        const unsigned tk = atom_add_acq_rel_gpu(&d.ticket[pair], 1u);
         *s_flag = (tk == (unsigned)d.nsplit - 1);
     }
     __syncthreads();
     if (!*s_flag) {
         return;
     }
-    __threadfence();
     // This CTA is the last of its (b, r) pair: every split's record is in
     // global memory (L2).  (1) The first batch of records starts streaming
     // into the free stage buffers with a bulk copy (the TMA engine moves
@@ -222,23 +239,46 @@ __device__ __forceinline__ void decode_finish(float* sM, uint64_t* comb_bar, int
         const int nb = min(kBatch, ns - b0);
         const uint32_t bytes = (uint32_t)(nb * kRecFloats * sizeof(float));
         fence_proxy_async_smem();  // earlier thread accesses of this space before the async-proxy writes
+        // the records were written through the generic proxy; the bulk copy reads them through the async one
+        asm volatile("fence.proxy.async.global;" ::: "memory");
         mbar_arrive_expect_tx(comb_bar, bytes);
         bulk_g2s(stage, all + (size_t)b0 * kRecFloats, bytes, comb_bar);
     };
     if (threadIdx.x == 0) issue_batch(0);
-    // one warp per query head of the group, a lane per split (and per split
-    // + 32, ...): the maximum and the sum are warp reductions
-    for (int g = warp; g < G; g += kThreads / 32) {
-        float M = kNegBig;
-        for (int sp = lane; sp < ns; sp += 32) M = fmaxf(M, __ldcg(all + (size_t)sp * kRecFloats + g * STRIDE));
+    // one warp per query head of the group (two for the first warps when G
+    // exceeds the warp count), a lane per split and per split + 32, + 64,
+    // + 96: every (m, l) pair the warp needs is loaded at once, so the pass
+    // costs one round trip to L2; the maximum and the sum are warp reductions
+    constexpr int kWarps = kThreads / 32;
+    constexpr int kHPW = (G + kWarps - 1) / kWarps;             // query heads per warp
+    float2 ml[kHPW][4];
+#pragma unroll
+    for (int h = 0; h < kHPW; ++h) {
+        const int g = warp + h * kWarps;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int sp = lane + 32 * j;
+            ml[h][j] = (g < G && sp < ns)
+                           ? __ldcg(reinterpret_cast<const float2*>(all + (size_t)sp * kRecFloats + g * STRIDE))
+                           : make_float2(kNegBig, 0.f);
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < kHPW; ++h) {
+        const int g = warp + h * kWarps;
+        if (g >= G) break;                                      // warp-uniform
+        float M = fmaxf(fmaxf(ml[h][0].x, ml[h][1].x), fmaxf(ml[h][2].x, ml[h][3].x));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
         float L = 0.f;
-        for (int sp = lane; sp < ns; sp += 32) {
-            const float* rec = all + (size_t)sp * kRecFloats + g * STRIDE;
-            const float w = exp2f(__ldcg(rec) - M);
-            s_w[sp * G + g] = w;
-            L += w * __ldcg(rec + 1);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int sp = lane + 32 * j;
+            if (sp < ns) {
+                const float w = exp2f(ml[h][j].x - M);
+                s_w[sp * G + g] = w;
+                L += w * ml[h][j].y;
+            }
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
